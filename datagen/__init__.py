@@ -111,3 +111,22 @@ def uniform_float(seed: int, stream: int, n: int, lo: float, hi: float, start: i
 def gain(seed: int, stream: int, n: int, start: int = 0) -> np.ndarray:
     """Norm gain of the seeded variant: fp32(1 + N(0, 0.1))."""
     return (np.float32(1.0) + normal(seed, stream, n, 0.1, start)).astype(np.float32)
+
+
+def history_stream(kind: str, ordinal: int, kv: int) -> int:
+    """Stream id of the synthetic K/V history of one cache tensor
+    (kind "ring": sliding-layer ordinal; "global": full-layer ordinal)."""
+    return stream_attn((0x1000 if kind == "ring" else 0x2000) + 2 * ordinal + kv)
+
+
+def qk_gain_base(hd: int) -> np.float32:
+    """hd^(-1/4) as the fp32 constant of the C header (unit-variance q.k scores)."""
+    return np.float32({256: 0.25, 512: 0.21022410381342863, 64: 0.35355339059327373,
+                       32: 0.42044820762685725}.get(hd, 1.0))
+
+
+def qk_gain(seed: int, stream: int, hd: int, variant: int) -> np.ndarray:
+    b = qk_gain_base(hd)
+    if not variant:
+        return np.full(hd, b, dtype=np.float32)
+    return (b * gain(seed, stream, hd)).astype(np.float32)

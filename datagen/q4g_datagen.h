@@ -97,6 +97,27 @@ DG_FN float dg_gain(uint64_t key, uint64_t i) {
 #endif
 }
 
+/* Base gain of the per-head q_norm / k_norm of the synthetic decoder: hd^(-1/4),
+ * so that scale-1.0 attention over two unit-RMS vectors has unit-variance scores
+ * (q.k ~ N(0, 1)) instead of standard deviation sqrt(hd). fp32 constants. */
+DG_FN float dg_qk_gain_base(int hd) {
+  return hd == 256 ? 0.25f : hd == 512 ? 0.21022410381342863f : hd == 64 ? 0.35355339059327373f
+       : hd == 32 ? 0.42044820762685725f : 1.0f;
+}
+
+/* q_norm / k_norm gain element i: base, or base * (1 + N(0, 0.1)) in the seeded
+ * variant (one fp32 multiply). */
+DG_FN float dg_qk_gain(uint64_t key, uint64_t i, int hd, int variant) {
+  float b = dg_qk_gain_base(hd);
+  if (!variant) return b;
+#ifdef __CUDA_ARCH__
+  return __fmul_rn(b, dg_gain(key, i));
+#else
+  volatile float g = dg_gain(key, i);
+  return b * g;
+#endif
+}
+
 /*
  * Stream ids of the synthetic workloads. A weight tensor of shape [rows][cols]
  * draws element (r, c) at index r*cols + c.

@@ -1,0 +1,534 @@
+// Split-KV flash-decode attention for the sliding ring and the full layers.
+//
+// Operation ("Gemma 4 12B" page, flash-decode paragraph: GQA decode over the
+// cache, scale 1.0, fp32 online softmax, the KV scan split across cooperating
+// groups; "Gemma-4-12B-CoreAI", v5 section: slot = position mod R, implied
+// position p = q - ((q - j) mod R), window test q - p < W):
+//   o[row] = sum_key softmax_key(q[row] . k[key]) v[key]
+// over the live keys of each query row.
+//
+// Grid (KV head, chunk of keys, group of query rows). The query rows of one KV
+// head -- (verify row j, query head h of the group) -- form the M dimension of
+// tensor-core tiles (mma.sync m16n8k16, fp16 in, fp32 accumulate): the GQA
+// group is folded into the query so every key row is read once for all its
+// query heads. Keys stream through shared memory in tiles of 64 with cp.async.
+// The probabilities enter the P.V product as fp16 hi + lo parts, so P carries
+// ~22 bits. Each CTA writes (m, l, acc) partials; a combine pass (the last CTA
+// of a ring head, or a separate kernel for the full layers) merges them in a
+// fixed order.
+//
+// With the fused QKV epilogue (qkv != NULL) the prologue computes, from the raw
+// projections: per-head RMSNorm of q (learned gains) and RoPE, RMSNorm of k and
+// RoPE, and V = scale-free RMSNorm of the v projection or, on full layers
+// (attention_k_eq_v), of the raw k projection. Chunk 0 writes the block's K/V
+// rows to the cache; every CTA reads this block's own rows from shared memory.
+#include "q4g_common.cuh"
+#include "q4g_internal.h"
+
+namespace q4g {
+
+namespace {
+
+constexpr int TK = 64;   // keys per tile
+constexpr int MROWS = 32;  // query rows per CTA (two m16 tiles)
+
+Q4G_DEV uint32_t saddr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+Q4G_DEV void ldsm_x4(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(saddr(p)));
+}
+Q4G_DEV void ldsm_x2(uint32_t (&r)[2], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(saddr(p)));
+}
+Q4G_DEV void ldsm_x2_t(uint32_t (&r)[2], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(saddr(p)));
+}
+Q4G_DEV void mma16816(float (&c)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+Q4G_DEV void cp_async16(void* dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr(dst)), "l"(src),
+               "r"(valid ? 16 : 0));
+}
+Q4G_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+Q4G_DEV void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+Q4G_DEV int64_t pmod(int64_t a, int64_t m) {
+  int64_t r = a % m;
+  return r < 0 ? r + m : r;
+}
+
+template <int HD>
+struct Smem {
+  static constexpr int LD = HD + 8;  // padded row (halves): conflict-free ldmatrix
+  __half q[MROWS][LD];
+  __half k[TK][LD];
+  __half v[TK][LD];
+  __half phi[MROWS][TK + 8];
+  __half plo[MROWS][TK + 8];
+  __half kloc[kMaxRows][HD];
+  __half vloc[kMaxRows][HD];
+  int64_t kidx[2][TK];  // slot (ring) or position (linear); -1: no key
+  float red[8][MROWS];
+  float m_run[MROWS], l_run[MROWS], scale[MROWS];
+  int ticket;
+};
+
+// Cache row (slot or position) of key `a` of the scan and whether it exists.
+struct KeyRange {
+  int64_t begin, end;  // scan indices [begin, end)
+};
+
+template <int HD>
+__global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  Smem<HD>& sm = *reinterpret_cast<Smem<HD>*>(smem_raw);
+  constexpr int LD = Smem<HD>::LD;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int kv = blockIdx.x, chunk = blockIdx.y, mg = blockIdx.z;
+  const int G = p.n_q / p.n_kv;
+  const int M = p.kr * G;                      // query rows of this KV head
+  const int row0 = mg * MROWS;                 // first query row of this CTA
+  const int nrows = min(MROWS, M - row0);
+
+  pdl_wait();
+  const int64_t pos0 = p.pos_dev ? *p.pos_dev : p.pos0;
+  const int64_t q_last = pos0 + p.kr - 1;
+  const bool fused = p.qkv != nullptr;
+
+  // ---- key scan of this chunk: ring scans ages, linear scans positions ----
+  int64_t nscan;
+  if (p.ring)
+    nscan = min((int64_t)p.window + p.kr - 1, q_last + 1);
+  else
+    nscan = q_last + 1;
+  // chunks are whole tiles; trailing chunks may be empty
+  const int64_t cs = ((nscan + p.n_chunks - 1) / p.n_chunks + TK - 1) / TK * TK;
+  const int64_t a_begin = min(nscan, (int64_t)chunk * cs);
+  const int64_t a_end = min(nscan, a_begin + cs);
+  const int ntiles = (int)((a_end - a_begin + TK - 1) / TK);
+
+  auto key_row = [&](int64_t a) -> int64_t {  // cache row of scan index a
+    return p.ring ? pmod(q_last - a, p.cache_rows) : a;
+  };
+  auto key_is_local = [&](int64_t a) -> int {  // block row index or -1
+    if (!fused) return -1;
+    const int64_t pos = p.ring ? q_last - a : a;
+    return pos >= pos0 ? (int)(pos - pos0) : -1;
+  };
+
+  const __half* kc = p.k_cache + (size_t)kv * p.cache_rows * HD;
+  const __half* vc = p.v_cache + (size_t)kv * p.cache_rows * HD;
+  constexpr int CPR = HD / 8;  // 16-byte chunks per row
+
+  auto load_tile = [&](int t, bool kpart, bool patch_local) {
+    const int buf = t & 1;
+    const int64_t a0 = a_begin + (int64_t)t * TK;
+    if (kpart && tid < TK) {
+      const int64_t a = a0 + tid;
+      sm.kidx[buf][tid] = a < a_end ? key_row(a) : -1;
+    }
+    __half(*dst)[LD] = kpart ? sm.k : sm.v;
+    const __half* src = kpart ? kc : vc;
+    for (int c = tid; c < TK * CPR; c += kThreads) {
+      const int key = c / CPR, part = c - key * CPR;
+      const int64_t a = a0 + key;
+      const bool in = a < a_end;
+      const int loc = in ? key_is_local(a) : -1;
+      if (loc >= 0) {
+        if (patch_local) {
+          const __half* l = kpart ? sm.kloc[loc] : sm.vloc[loc];
+          *reinterpret_cast<uint4*>(&dst[key][part * 8]) =
+              *reinterpret_cast<const uint4*>(l + part * 8);
+        }
+      } else {
+        const __half* s = in ? src + (size_t)key_row(a) * HD + part * 8 : src;
+        cp_async16(&dst[key][part * 8], s, in);
+      }
+    }
+  };
+
+  // first tile's cache rows go out before the prologue
+  if (ntiles > 0) {
+    load_tile(0, true, false);
+    cp_async_commit();
+    load_tile(0, false, false);
+    cp_async_commit();
+  }
+
+  // ---- prologue: queries (and this block's K/V rows) into shared memory ----
+  if (fused) {
+    const int nvec = nrows + 2 * p.kr;
+    constexpr int E = HD / 64;  // elements per lane per half
+    for (int vi = warp; vi < nvec; vi += kThreads / 32) {
+      int j, kind;  // kind 0: q row, 1: k, 2: v
+      const float* src;
+      if (vi < nrows) {
+        const int r = row0 + vi;
+        j = r / G;
+        kind = 0;
+        src = p.qkv + (size_t)j * p.qkv_stride + (size_t)(kv * G + r % G) * HD;
+      } else if (vi < nrows + p.kr) {
+        j = vi - nrows;
+        kind = 1;
+        src = p.qkv + (size_t)j * p.qkv_stride + p.k_off + (size_t)kv * HD;
+      } else {
+        j = vi - nrows - p.kr;
+        kind = 2;
+        src = p.qkv + (size_t)j * p.qkv_stride +
+              (p.v_off >= 0 ? p.v_off + (size_t)kv * HD : p.k_off + (size_t)kv * HD);
+      }
+      float lo[E], hi[E];
+      float ss = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        lo[e] = src[lane * E + e];
+        hi[e] = src[HD / 2 + lane * E + e];
+        ss = fmaf(lo[e], lo[e], ss);
+        ss = fmaf(hi[e], hi[e], ss);
+      }
+      const bool do_norm = kind != 2 || p.v_norm;
+      const float inv = do_norm ? rms_inv(warp_sum(ss), HD, p.eps) : 1.0f;
+      const float* gain = kind == 0 ? p.w_q : kind == 1 ? p.w_k : nullptr;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const int i = lane * E + e;
+        float a = __fmul_rn(lo[e], inv), b = __fmul_rn(hi[e], inv);
+        if (gain) a = __fmul_rn(a, gain[i]), b = __fmul_rn(b, gain[HD / 2 + i]);
+        if (kind != 2 && i < p.rope_pairs) {
+          const float2 cs2 = p.rope[(size_t)j * p.rope_pairs + i];
+          const float ra = a * cs2.x - b * cs2.y;
+          const float rb = b * cs2.x + a * cs2.y;
+          a = ra, b = rb;
+        }
+        __half* dst = kind == 0 ? sm.q[vi] : kind == 1 ? sm.kloc[j] : sm.vloc[j];
+        dst[i] = __float2half_rn(a);
+        dst[HD / 2 + i] = __float2half_rn(b);
+      }
+    }
+  } else {
+    for (int c = tid; c < nrows * CPR; c += kThreads) {
+      const int r = c / CPR, part = c - r * CPR;
+      const int gr = row0 + r;
+      const __half* src = p.q16 + ((size_t)(gr / G) * p.n_q + kv * G + gr % G) * HD + part * 8;
+      *reinterpret_cast<uint4*>(&sm.q[r][part * 8]) = *reinterpret_cast<const uint4*>(src);
+    }
+  }
+  // zero the unused query rows (their results are never written)
+  for (int c = tid; c < (MROWS - nrows) * LD; c += kThreads)
+    sm.q[nrows + c / LD][c % LD] = __float2half_rn(0.f);
+  if (tid < MROWS) sm.m_run[tid] = -INFINITY, sm.l_run[tid] = 0.f;
+  __syncthreads();
+
+  if (fused && p.write_kv && chunk == 0 && mg == 0) {
+    for (int c = tid; c < p.kr * CPR; c += kThreads) {
+      const int j = c / CPR, part = c - j * CPR;
+      const int64_t pos = pos0 + j;
+      const int64_t row = p.ring ? pmod(pos, p.cache_rows) : pos;
+      *reinterpret_cast<uint4*>(p.k_cache + ((size_t)kv * p.cache_rows + row) * HD + part * 8) =
+          *reinterpret_cast<const uint4*>(&sm.kloc[j][part * 8]);
+      *reinterpret_cast<uint4*>(p.v_cache + ((size_t)kv * p.cache_rows + row) * HD + part * 8) =
+          *reinterpret_cast<const uint4*>(&sm.vloc[j][part * 8]);
+    }
+  }
+  pdl_launch_dependents();
+
+  // ---- tile loop ----
+  constexpr int NT_PV = HD / 64;   // 8-dim n-tiles per warp in P.V
+  const int mtiles = (nrows + 15) / 16;
+  float oacc[2][NT_PV][4];
+#pragma unroll
+  for (int a = 0; a < 2; ++a)
+#pragma unroll
+    for (int b = 0; b < NT_PV; ++b)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) oacc[a][b][c] = 0.f;
+
+  const int g4 = lane >> 2, t4 = lane & 3;
+  for (int t = 0; t < ntiles; ++t) {
+    const int buf = t & 1;
+    if (t == 0 && fused) {  // this block's own rows, now that they exist
+      load_tile(0, true, true);
+      load_tile(0, false, true);
+    }
+    cp_async_wait<1>();
+    __syncthreads();
+
+    // scores S[row][key] for key n-tile `warp`
+    float s[2][4];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) s[mt][c] = 0.f;
+      if (mt < mtiles) {
+#pragma unroll 4
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          uint32_t a[4], b[2];
+          ldsm_x4(a, &sm.q[mt * 16 + (lane & 15)][kk * 16 + (lane >> 4) * 8]);
+          ldsm_x2(b, &sm.k[warp * 8 + (lane & 7)][kk * 16 + ((lane >> 3) & 1) * 8]);
+          mma16816(s[mt], a, b);
+        }
+      }
+    }
+    __syncthreads();  // K tile consumed
+    if (t + 1 < ntiles) {
+      load_tile(t + 1, true, true);
+    }
+    cp_async_commit();
+
+    // mask and per-tile row maxima
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int lr = mt * 16 + g4 + hh * 8;  // local query row
+        const int gr = row0 + lr;
+        const int j = gr / G;
+        const int64_t qj = pos0 + j;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int key = warp * 8 + t4 * 2 + e;
+          const int64_t kr_ = sm.kidx[buf][key];
+          bool live = lr < nrows && kr_ >= 0;
+          if (live) {
+            if (p.ring) {
+              const int64_t pp = qj - pmod(qj - kr_, p.cache_rows);
+              live = pp >= 0 && qj - pp < p.window;
+            } else {
+              live = kr_ <= qj;
+            }
+          }
+          float& v = s[mt][hh * 2 + e];
+          v = live ? v : -INFINITY;
+          mx = fmaxf(mx, v);
+        }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        if (t4 == 0) sm.red[warp][lr] = mx;
+      }
+    }
+    __syncthreads();
+    if (tid < MROWS) {
+      float mx = sm.red[0][tid];
+#pragma unroll
+      for (int w = 1; w < 8; ++w) mx = fmaxf(mx, sm.red[w][tid]);
+      const float mold = sm.m_run[tid];
+      const float mnew = fmaxf(mold, mx);
+      sm.scale[tid] = mnew == -INFINITY ? 1.0f : __expf(mold - mnew);
+      sm.m_run[tid] = mnew;
+    }
+    __syncthreads();
+    // probabilities (fp16 hi + lo) and per-tile row sums
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int lr = mt * 16 + g4 + hh * 8;
+        const float mrow = sm.m_run[lr];
+        float sum = 0.f;
+        __half2 ph, pl;
+        float pv[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float v = s[mt][hh * 2 + e];
+          pv[e] = (v == -INFINITY) ? 0.f : __expf(v - mrow);
+          sum += pv[e];
+        }
+        ph = __floats2half2_rn(pv[0], pv[1]);
+        const float2 phf = __half22float2(ph);
+        pl = __floats2half2_rn(pv[0] - phf.x, pv[1] - phf.y);
+        *reinterpret_cast<__half2*>(&sm.phi[lr][warp * 8 + t4 * 2]) = ph;
+        *reinterpret_cast<__half2*>(&sm.plo[lr][warp * 8 + t4 * 2]) = pl;
+        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+        if (t4 == 0) sm.red[warp][lr] = sum;
+      }
+    }
+    cp_async_wait<1>();  // V tile of this step (the next K may still fly)
+    __syncthreads();
+    if (tid < MROWS) {
+      float sum = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) sum += sm.red[w][tid];
+      sm.l_run[tid] = sm.l_run[tid] * sm.scale[tid] + sum;
+    }
+    // O = O * scale + P . V   (warp owns dims [warp*HD/8, (warp+1)*HD/8))
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+      if (mt < mtiles) {
+        const float sc0 = sm.scale[mt * 16 + g4], sc1 = sm.scale[mt * 16 + g4 + 8];
+#pragma unroll
+        for (int nt = 0; nt < NT_PV; ++nt) {
+          oacc[mt][nt][0] *= sc0, oacc[mt][nt][1] *= sc0;
+          oacc[mt][nt][2] *= sc1, oacc[mt][nt][3] *= sc1;
+        }
+#pragma unroll
+        for (int ks = 0; ks < TK / 16; ++ks) {
+          uint32_t ah[4], al[4];
+          ldsm_x4(ah, &sm.phi[mt * 16 + (lane & 15)][ks * 16 + (lane >> 4) * 8]);
+          ldsm_x4(al, &sm.plo[mt * 16 + (lane & 15)][ks * 16 + (lane >> 4) * 8]);
+#pragma unroll
+          for (int nt = 0; nt < NT_PV; ++nt) {
+            uint32_t b[2];
+            ldsm_x2_t(b, &sm.v[ks * 16 + (lane & 15)][warp * (HD / 8) + nt * 8]);
+            mma16816(oacc[mt][nt], ah, b);
+            mma16816(oacc[mt][nt], al, b);
+          }
+        }
+      }
+    }
+    __syncthreads();  // V tile and P consumed
+    if (t + 1 < ntiles) load_tile(t + 1, false, true);
+    cp_async_commit();
+  }
+  cp_async_wait<0>();
+
+  // ---- partials ----
+  const int nq_rows = p.kr * p.n_q;
+  for (int mt = 0; mt < mtiles; ++mt) {
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int lr = mt * 16 + g4 + hh * 8;
+      if (lr < nrows) {
+        const int gr = row0 + lr;
+        const int orow = (gr / G) * p.n_q + kv * G + gr % G;
+        float* acc = p.part_acc + ((size_t)orow * p.n_chunks + chunk) * HD;
+#pragma unroll
+        for (int nt = 0; nt < NT_PV; ++nt) {
+          const int d = warp * (HD / 8) + nt * 8 + t4 * 2;
+          *reinterpret_cast<float2*>(acc + d) = make_float2(oacc[mt][nt][hh * 2], oacc[mt][nt][hh * 2 + 1]);
+        }
+      }
+    }
+  }
+  if (tid < nrows) {
+    const int gr = row0 + tid;
+    const int orow = (gr / G) * p.n_q + kv * G + gr % G;
+    p.part_ml[((size_t)orow * p.n_chunks + chunk) * 2] = sm.m_run[tid];
+    p.part_ml[((size_t)orow * p.n_chunks + chunk) * 2 + 1] = sm.l_run[tid];
+  }
+  (void)nq_rows;
+  if (!p.combine_in_kernel) return;
+
+  // ---- the last CTA of this (KV head, row group) merges the chunks ----
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) sm.ticket = atomicAdd(&p.counters[kv * p.m_groups + mg], 1);
+  __syncthreads();
+  if (sm.ticket != p.n_chunks - 1) return;
+  __threadfence();
+  for (int c = tid; c < nrows * HD; c += kThreads) {
+    const int r = c / HD, d = c - r * HD;
+    const int gr = row0 + r;
+    const int orow = (gr / G) * p.n_q + kv * G + gr % G;
+    const float* ml = p.part_ml + (size_t)orow * p.n_chunks * 2;
+    float mstar = -INFINITY;
+    for (int ch = 0; ch < p.n_chunks; ++ch) mstar = fmaxf(mstar, __ldcg(ml + 2 * ch));
+    float l = 0.f, o = 0.f;
+    for (int ch = 0; ch < p.n_chunks; ++ch) {
+      const float mc = __ldcg(ml + 2 * ch);
+      if (mc == -INFINITY) continue;
+      const float w = __expf(mc - mstar);
+      l = fmaf(__ldcg(ml + 2 * ch + 1), w, l);
+      o = fmaf(__ldcg(p.part_acc + ((size_t)orow * p.n_chunks + ch) * HD + d), w, o);
+    }
+    p.out[(size_t)orow * HD + d] = __float2half_rn(o / l);
+  }
+  if (tid == 0) p.counters[kv * p.m_groups + mg] = 0;
+}
+
+// Separate merge of the chunk partials: one thread per (row, dim).
+template <int HD>
+__global__ void __launch_bounds__(128) attn_combine_kernel(const AttnParams p) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int orow = blockIdx.x;
+  const int d = blockIdx.y * 128 + threadIdx.x;
+  const float* ml = p.part_ml + (size_t)orow * p.n_chunks * 2;
+  float mstar = -INFINITY;
+  for (int ch = 0; ch < p.n_chunks; ++ch) mstar = fmaxf(mstar, ml[2 * ch]);
+  float l = 0.f, o = 0.f;
+  for (int ch = 0; ch < p.n_chunks; ++ch) {
+    const float mc = ml[2 * ch];
+    if (mc == -INFINITY) continue;
+    const float w = __expf(mc - mstar);
+    l = fmaf(ml[2 * ch + 1], w, l);
+    o = fmaf(p.part_acc[((size_t)orow * p.n_chunks + ch) * HD + d], w, o);
+  }
+  p.out[(size_t)orow * HD + d] = __float2half_rn(o / l);
+}
+
+template <int HD>
+cudaError_t launch_attn_t(const AttnParams& p, cudaStream_t st, bool pdl) {
+  static bool configured = false;
+  const size_t smem = sizeof(Smem<HD>);
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(attn_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.n_kv, p.n_chunks, p.m_groups);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, attn_kernel<HD>, p);
+}
+
+template <int HD>
+cudaError_t launch_combine_t(const AttnParams& p, cudaStream_t st, bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.kr * p.n_q, HD / 128);
+  cfg.blockDim = dim3(128);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, attn_combine_kernel<HD>, p);
+}
+
+}  // namespace
+
+size_t attn_smem_bytes(int hd, int) {
+  return hd == 256 ? sizeof(Smem<256>) : sizeof(Smem<512>);
+}
+
+size_t attn_partial_floats(int kr, int n_q, int n_chunks, int hd) {
+  return (size_t)kr * n_q * n_chunks * (size_t)hd;
+}
+
+cudaError_t launch_attention(const AttnParams& p, cudaStream_t st, bool pdl) {
+  if (p.hd == 256) return launch_attn_t<256>(p, st, pdl);
+  if (p.hd == 512) return launch_attn_t<512>(p, st, pdl);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_attn_combine(const AttnParams& p, cudaStream_t st, bool pdl) {
+  if (p.hd == 256) return launch_combine_t<256>(p, st, pdl);
+  if (p.hd == 512) return launch_combine_t<512>(p, st, pdl);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace q4g

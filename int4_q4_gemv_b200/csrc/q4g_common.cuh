@@ -1,0 +1,139 @@
+// Shared device helpers of libq4g (sm_100a).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#define Q4G_DEV __device__ __forceinline__
+
+namespace q4g {
+
+constexpr int kMaxRows = 8;       // verify rows per call
+constexpr int kThreads = 256;     // block size of the GEMV and attention kernels
+constexpr int kUnitRows = 16;     // GEMV rows per unit of work
+constexpr int kSpinLimit = 1 << 22;
+
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch. Without the launch attribute both are no-ops.
+// ---------------------------------------------------------------------------
+Q4G_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+Q4G_DEV void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
+// Loads. Weights are read once per step: stream them past L1.
+// ---------------------------------------------------------------------------
+Q4G_DEV uint4 ld_stream_u4(const void* p) {
+  uint4 r;
+  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+      : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+      : "l"(p));
+  return r;
+}
+
+Q4G_DEV uint16_t ld_stream_u16(const void* p) {
+  uint16_t r;
+  asm("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(r) : "l"(p));
+  return r;
+}
+
+Q4G_DEV uint4 lds_u4(const void* p) {
+  uint4 r;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "r"((uint32_t)__cvta_generic_to_shared(p)));
+  return r;
+}
+
+// ---------------------------------------------------------------------------
+// q4_0 nibble unpacking. A 32-bit word w of a block's 16 code bytes holds, per
+// 16-bit half, the codes of two columns in each nibble. Moving one nibble of
+// each half to bits 4..7 and OR-ing the fp16 pattern 0x5400 (64.0, whose
+// lowest fraction bit weighs 1/16) yields the exact half2 value (64 + c).
+// lop3 immediate 0xEA = (a & b) | c.
+// ---------------------------------------------------------------------------
+Q4G_DEV uint32_t nib_to_h2(uint32_t v) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(v), "n"(0x00F000F0), "n"(0x54005400));
+  return r;
+}
+
+// acc + w.lo * x.lo + w.hi * x.hi with fp16 products accumulated in fp32
+// (mixed-precision fma, products exact).
+Q4G_DEV float fma2_h_f32(uint32_t w2, uint32_t x2, float acc) {
+  float r;
+  asm("{\n\t.reg .b16 wl, wh, xl, xh;\n\t"
+      "mov.b32 {wl, wh}, %1;\n\t"
+      "mov.b32 {xl, xh}, %2;\n\t"
+      "fma.rn.f32.f16 %0, wl, xl, %3;\n\t"
+      "fma.rn.f32.f16 %0, wh, xh, %0;\n\t}"
+      : "=f"(r)
+      : "r"(w2), "r"(x2), "f"(acc));
+  return r;
+}
+
+// Sum over the 32 columns of one block of (64 + c_i) * x_i, split into two
+// accumulators. xq[k] holds the block's x in the order the unpacking of word k
+// produces: {x[4k], x[4k+2]}, {x[4k+16], x[4k+18]}, {x[4k+1], x[4k+3]},
+// {x[4k+17], x[4k+19]}.
+Q4G_DEV void block_dot(const uint4 q, const uint4 (&xq)[4], float& a0, float& a1) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    a0 = fma2_h_f32(nib_to_h2(w[k] << 4), xq[k].x, a0);
+    a1 = fma2_h_f32(nib_to_h2(w[k]), xq[k].y, a1);
+    a0 = fma2_h_f32(nib_to_h2(w[k] >> 4), xq[k].z, a0);
+    a1 = fma2_h_f32(nib_to_h2(w[k] >> 8), xq[k].w, a1);
+  }
+}
+
+// Column order of the x layout above: slot s (0..31) of a block holds column
+// kXPerm[s]; quarter k = slots 8k..8k+7.
+__host__ __device__ constexpr int xperm(int s) {
+  // within a quarter: 0:4k 1:4k+2 2:4k+16 3:4k+18 4:4k+1 5:4k+3 6:4k+17 7:4k+19
+  return 4 * (s >> 3) + ((s & 7) == 0 ? 0 : (s & 7) == 1 ? 2 : (s & 7) == 2 ? 16 : (s & 7) == 3 ? 18
+                       : (s & 7) == 4 ? 1 : (s & 7) == 5 ? 3 : (s & 7) == 6 ? 17 : 19);
+}
+
+// ---------------------------------------------------------------------------
+// Reductions.
+// ---------------------------------------------------------------------------
+Q4G_DEV float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+Q4G_DEV float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Block-wide sum for blockDim.x == kThreads; `red` holds >= 32 floats. All
+// threads receive the result. Summation order is fixed.
+Q4G_DEV float block_sum(float v, float* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v = warp_sum(v);
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float t = 0.f;
+#pragma unroll
+  for (int i = 0; i < kThreads / 32; ++i) t += red[i];
+  return t;
+}
+
+// IEEE division and square root (correctly rounded), so results do not depend
+// on compiler flags.
+Q4G_DEV float rms_inv(float sumsq, int n, float eps) {
+  return __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(sumsq, (float)n), eps)));
+}
+
+Q4G_DEV float gelu_tanh(float g) {
+  const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
+  float inner = k0 * (g + 0.044715f * g * g * g);
+  return 0.5f * g * (1.0f + tanhf(inner));
+}
+
+}  // namespace q4g

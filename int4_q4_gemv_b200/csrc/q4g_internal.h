@@ -1,0 +1,135 @@
+// Internal host-side interfaces between the translation units of libq4g.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace q4g {
+
+// ----------------------------------------------------------------- GEMV ----
+struct GemvSeg {
+  const uint8_t* qs;
+  const uint16_t* sc;
+  int32_t rows;
+};
+
+enum GemvPro { PRO_X16 = 0, PRO_RESID = 1 };
+enum GemvEpi { EPI_STORE = 0, EPI_GEGLU = 1, EPI_HEAD = 2 };
+
+struct GemvParams {
+  GemvSeg seg[3];
+  int32_t nseg;
+  int32_t k;        // columns
+  int32_t n_rows;   // output rows (STORE / HEAD); the last unit may be partial
+  int32_t n_units;  // 16-row units (GEGLU: units of 8 gate + 8 up rows)
+  int32_t kr;       // activation rows (<= template KRM)
+  int32_t pro, epi;
+  // PRO_X16: x [kr][x_stride] fp16
+  const __half* x;
+  int64_t x_stride;
+  // PRO_RESID: r_new = (r_in + rmsnorm(delta) * w_delta) * scale   (delta may be NULL)
+  //            x     = fp16(rmsnorm(r_new) * w_x); block 0 stores r_new to r_out
+  const float* r_in;
+  float* r_out;
+  const float* delta;
+  const float* w_delta;
+  float scale;
+  const float* w_x;
+  float eps;
+  float* dump;  // optional [kr][dump_stride] copy of r_new (block 0)
+  int64_t dump_stride;
+  // EPI_STORE: y [kr][y_stride]
+  float* y;
+  int64_t y_stride;
+  // EPI_GEGLU: act [kr][act_stride] = fp16(gelu_tanh(gate) * up); seg[0] gate, seg[1] up
+  __half* act;
+  int64_t act_stride;
+  // EPI_HEAD: logits [kr][logits_stride] (optional), softcap, argmax
+  float* logits;
+  int64_t logits_stride;
+  float softcap;
+  float* am_val;     // [kMaxRows][grid]
+  int32_t* am_idx;   // [kMaxRows][grid]
+  int32_t* counter;  // one int, zero between launches
+  int32_t* argmax_out;
+};
+
+// Largest number of activation rows one GEMV launch can stage for k columns.
+int gemv_max_rows(int k);
+size_t gemv_smem_bytes(int krm, int k);
+cudaError_t launch_gemv(const GemvParams& p, cudaStream_t st, bool pdl);
+
+// ------------------------------------------------------------ attention ----
+struct AttnParams {
+  // queries: either the fused QKV epilogue (qkv != NULL) or ready fp16 q
+  const float* qkv;      // [kr][qkv_stride] raw projections (q | k | v)
+  int64_t qkv_stride;
+  int32_t k_off, v_off;  // column offsets of k and v (v_off < 0: V from raw k, k_eq_v)
+  const float* w_q;      // q_norm gains [hd]
+  const float* w_k;      // k_norm gains [hd]
+  int32_t v_norm;        // scale-free RMSNorm on V
+  const float2* rope;    // [kr][rope_pairs] (cos, sin), pairs >= rope_pairs untouched
+  int32_t rope_pairs;
+  float eps;
+  const __half* q16;     // standalone: [kr][n_q][hd] fp16
+  // cache
+  __half* k_cache;       // ring: [n_kv][R][hd]; linear: [n_kv][cap][hd]
+  __half* v_cache;
+  int64_t cache_rows;    // R (ring) or capacity (linear)
+  int32_t ring;          // 1: ring addressing with the implied-position window test
+  int64_t window;
+  int64_t pos0;
+  const int64_t* pos_dev;  // if non-NULL, pos0 is read from here (graph replay)
+  int32_t kr;
+  int32_t write_kv;      // chunk 0 writes the block rows to the cache
+  int32_t n_q, n_kv, hd;
+  int32_t n_chunks;
+  int32_t m_groups;
+  // partials [kr*n_q][n_chunks] of (m, l) and acc [kr*n_q][n_chunks][hd]
+  float* part_ml;
+  float* part_acc;
+  int32_t* counters;     // [n_kv] for the in-kernel combine (ring), zero between launches
+  int32_t combine_in_kernel;
+  __half* out;           // [kr][n_q][hd]
+};
+
+size_t attn_smem_bytes(int hd, int m_tiles_per_cta);
+size_t attn_partial_floats(int kr, int n_q, int n_chunks, int hd);
+cudaError_t launch_attention(const AttnParams& p, cudaStream_t st, bool pdl);
+cudaError_t launch_attn_combine(const AttnParams& p, cudaStream_t st, bool pdl);
+
+// --------------------------------------------------------------- misc ----
+cudaError_t launch_pack(const float* w, int64_t rows, int64_t k, uint8_t* qs, uint16_t* sc,
+                        int32_t* bad_flag, cudaStream_t st);
+cudaError_t launch_unpack(const uint8_t* qs, const uint16_t* sc, int64_t rows, int64_t k, float* w,
+                          cudaStream_t st);
+
+struct StepParams {
+  int32_t kr;
+  int64_t pos0;
+  const int32_t* ids_dev;   // [kr] token ids on the device (or NULL)
+  int32_t ids_host[8];      // used when ids_dev == NULL and hidden == NULL
+  const float* hidden;      // [kr][h] replaces the embedding
+  const uint8_t* emb_qs;
+  const uint16_t* emb_sc;
+  int32_t hidden_size, vocab;
+  float embed_scale;
+  float* r_out;             // [kr][h]
+  float* dump;              // optional [kr][dump_stride]
+  int64_t dump_stride;
+  // RoPE tables for this step
+  const double* inv_freq_sl;  // [pairs_sl]
+  const double* inv_freq_gl;  // [pairs_gl]
+  int32_t pairs_sl, pairs_gl;
+  float2* rope_sl;          // [kr][pairs_sl]
+  float2* rope_gl;          // [kr][pairs_gl]
+  int64_t* pos_dev;         // written: pos0
+  int32_t* counters;        // zeroed
+  int32_t n_counters;
+};
+cudaError_t launch_step_init(const StepParams& p, cudaStream_t st);
+
+int device_sm_count();
+
+}  // namespace q4g

@@ -10,6 +10,8 @@ import os
 
 import numpy as np
 
+import datagen as DG
+
 from . import build as _build
 
 _LIB = None
@@ -58,6 +60,7 @@ def lib():
             "or_cache_clone": (vp, [vp]),
             "or_cache_ring": (vp, [vp, C.c_int, C.c_int]),
             "or_cache_global": (vp, [vp, C.c_int, C.c_int]),
+            "or_fill_normal_f16": (None, [vp, i64, u64, u64, C.c_float, i64]),
             "or_verify_block": (C.c_int, [vp, vp, vp, vp, C.c_int, i64, C.c_int, C.c_int,
                                           vp, vp, vp, vp, vp]),
         }
@@ -257,6 +260,29 @@ class Cache:
             self.close()
         except Exception:
             pass
+
+
+def fill_normal_f16(out: np.ndarray, seed: int, stream: int, sigma: float = 1.0, start: int = 0):
+    assert out.dtype == np.uint16 and out.flags["C_CONTIGUOUS"]
+    lib().or_fill_normal_f16(_p(out), out.size, seed, stream, sigma, start)
+
+
+def fill_history(cache: Cache, seed: int = 99):
+    """Seeded N(0, 1) fp16 K/V in every ring slot and every global row (the
+    same streams as the GPU harness: datagen.history_stream)."""
+    cfg = cache.model.cfg
+    n_sl = sum(1 for l in range(cfg["n_layers"]) if not _is_full(cfg, l))
+    n_gl = cfg["n_layers"] - n_sl
+    for i in range(n_sl):
+        for kv in (0, 1):
+            fill_normal_f16(cache.ring(i, kv), seed, DG.history_stream("ring", i, kv))
+    for i in range(n_gl):
+        for kv in (0, 1):
+            fill_normal_f16(cache.global_(i, kv), seed, DG.history_stream("global", i, kv))
+
+
+def _is_full(cfg, l):
+    return cfg["full_every"] > 0 and l % cfg["full_every"] == cfg["full_offset"]
 
 
 def verify_block(model: Model, cache: Cache, pos0: int, ids=None, hidden=None, accepted=None,

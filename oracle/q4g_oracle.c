@@ -347,6 +347,13 @@ static double* make_gain(uint64_t seed, uint64_t stream, int64_t n, int variant)
   return g;
 }
 
+static double* make_qk_gain(uint64_t seed, uint64_t stream, int64_t hd, int variant) {
+  double* g = (double*)malloc(sizeof(double) * (size_t)hd);
+  uint64_t key = dg_key(seed, stream);
+  for (int64_t i = 0; i < hd; ++i) g[i] = (double)dg_qk_gain(key, (uint64_t)i, (int)hd, variant);
+  return g;
+}
+
 or_model* or_model_create(const or_config* cfg, uint64_t seed, int variant, int nthreads) {
 #ifdef _OPENMP
   if (nthreads > 0) omp_set_num_threads(nthreads);
@@ -379,8 +386,8 @@ or_model* or_model_create(const or_config* cfg, uint64_t seed, int variant, int 
     L->n_pa = make_gain(seed, DG_STREAM_LAYER(l, DG_T_NORM_POST_ATTN), H, variant);
     L->n_pf = make_gain(seed, DG_STREAM_LAYER(l, DG_T_NORM_PRE_FFN), H, variant);
     L->n_po = make_gain(seed, DG_STREAM_LAYER(l, DG_T_NORM_POST_FFN), H, variant);
-    L->n_q = make_gain(seed, DG_STREAM_LAYER(l, DG_T_NORM_Q), hd, variant);
-    L->n_k = make_gain(seed, DG_STREAM_LAYER(l, DG_T_NORM_K), hd, variant);
+    L->n_q = make_qk_gain(seed, DG_STREAM_LAYER(l, DG_T_NORM_Q), hd, variant);
+    L->n_k = make_qk_gain(seed, DG_STREAM_LAYER(l, DG_T_NORM_K), hd, variant);
     L->lscalar = variant ? (double)dg_uniform_float(dg_key(seed, DG_STREAM_LAYER(l, DG_T_LAYER_SCALAR)),
                                                     0, 0.5f, 1.5f)
                          : 1.0;
@@ -732,4 +739,14 @@ void or_set_num_threads(int n) {
 #else
   (void)n;
 #endif
+}
+
+/* Seeded N(0, sigma) values rounded to fp16 (datagen definition), for loading
+ * the same synthetic K/V history as the GPU harness. */
+void or_fill_normal_f16(uint16_t* out, int64_t n, uint64_t seed, uint64_t stream, float sigma,
+                        int64_t start) {
+  uint64_t key = dg_key(seed, stream);
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < n; ++i)
+    out[i] = or_f16_from_double((double)dg_normal(key, (uint64_t)(start + i), sigma));
 }

@@ -74,13 +74,19 @@ void or_attn_linear(const uint16_t* q16, int n_q, int n_kv, int hd, const uint16
 /* Live-slot mask of the ring for query position q: mask[j] = implied position or -1. */
 void or_ring_implied_positions(int64_t R, int64_t W, int64_t q, int64_t* out);
 
+/* Seeded N(0, sigma) rounded to fp16 (datagen definition): synthetic history. */
+void or_fill_normal_f16(uint16_t* out, int64_t n, uint64_t seed, uint64_t stream, float sigma,
+                        int64_t start);
+
 /* ---- model ---- */
 typedef struct or_model or_model;
 typedef struct or_cache or_cache;
 
 /* Weights generated from the seeded recipe: linear weights N(0, 0.02) packed
- * to q4_0; norm gains 1 (variant 0) or 1 + N(0, 0.1) (variant 1); layer
- * scalars 1 (variant 0) or U(0.5, 1.5) (variant 1). nthreads <= 0: all. */
+ * to q4_0; residual-stream norm gains 1 (variant 0) or 1 + N(0, 0.1)
+ * (variant 1); q_norm / k_norm gains hd^(-1/4), times 1 + N(0, 0.1) in
+ * variant 1; layer scalars 1 (variant 0) or U(0.5, 1.5) (variant 1).
+ * nthreads <= 0: all. */
 or_model* or_model_create(const or_config* cfg, uint64_t seed, int variant, int nthreads);
 void or_model_destroy(or_model* m);
 /* Packed bytes of one weight tensor, for bit-exact comparison with another packer.

@@ -60,7 +60,9 @@ class TorchDecoder:
                 wg=mat(l, 4), wu=mat(l, 5), wd=mat(l, 6),
                 n_in=gain(s(DG.T_NORM_IN), cfg["hidden"]), n_pa=gain(s(DG.T_NORM_POST_ATTN), cfg["hidden"]),
                 n_pf=gain(s(DG.T_NORM_PRE_FFN), cfg["hidden"]), n_po=gain(s(DG.T_NORM_POST_FFN), cfg["hidden"]),
-                n_q=gain(s(DG.T_NORM_Q), hd), n_k=gain(s(DG.T_NORM_K), hd), scal=scal))
+                n_q=torch.from_numpy(DG.qk_gain(seed, s(DG.T_NORM_Q), hd, variant).astype(np.float64)),
+                n_k=torch.from_numpy(DG.qk_gain(seed, s(DG.T_NORM_K), hd, variant).astype(np.float64)),
+                scal=scal))
         self.embed = torch.from_numpy(O.q4_0_unpack(*om.tensor(-1, 100)))
         self.n_final = gain(DG.STREAM_FINAL_NORM, cfg["hidden"])
         self.K = [[] for _ in range(L)]   # linear history of fp16 K per layer
