@@ -195,10 +195,31 @@ q4g_status q4g_model_check(q4g_model* m, q4g_stream_t stream);
 typedef enum {
   Q4G_OPT_CUDA_GRAPH = 1, /* [1] replay a captured CUDA graph per step shape   */
   Q4G_OPT_PDL = 2,        /* [1] programmatic dependent launch between kernels */
-  Q4G_OPT_DUMP = 3        /* [0] value = device float* [K][n_layers+1][h]: residual
+  Q4G_OPT_DUMP = 3,       /* [0] value = device float* [K][n_layers+1][h]: residual
                                  stream after the embedding and after each layer */
+  Q4G_OPT_PROFILE = 4     /* [0] 1: launch eagerly and bracket every kernel with CUDA
+                                 events on the launching stream (read with
+                                 q4g_model_profile_read) */
 } q4g_option;
 q4g_status q4g_model_set_option(q4g_model* m, q4g_option opt, intptr_t value);
+
+/* One kernel launch recorded in profile mode. kind: 0 step init, 1 QKV GEMV,
+ * 2 sliding attention, 3 full attention, 4 attention combine, 5 O GEMV,
+ * 6 gate|up GEMV, 7 down GEMV, 8 head GEMV. bytes: algorithmic HBM bytes of the
+ * launch (q4_0 weights 0.5625 B/weight + activations; attention: the live K/V
+ * rows, 2 * head_dim * 2 B per key and KV head). */
+typedef struct {
+  int32_t kind;
+  int32_t layer;
+  float ms;
+  double bytes;
+} q4g_launch_record;
+
+/* Synchronises `stream`, copies up to `max` records of the launches made since
+ * the last read into `out` (host), clears them and returns how many there were
+ * (which may exceed max), or -1 on error (see q4g_last_error). */
+int32_t q4g_model_profile_read(q4g_model* m, q4g_launch_record* out, int32_t max,
+                               q4g_stream_t stream);
 
 /* KV cache for up to `capacity` positions: per sliding layer a ring K and V of
  * [sl_kv_heads][ring][sl_head_dim] fp16 (slot = position mod ring); per full

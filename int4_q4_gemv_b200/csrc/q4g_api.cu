@@ -6,6 +6,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -109,6 +110,16 @@ struct q4g_model {
   // options
   bool use_graph = true, use_pdl = true;
   float* dump = nullptr;
+  // profile mode: events around every launch
+  bool profile = false;
+  std::vector<cudaEvent_t> ev_pool;
+  struct Rec {
+    int kind, layer;
+    double bytes;
+    cudaEvent_t a, b;
+  };
+  std::vector<Rec> recs;
+  size_t ev_next = 0;
   // graphs
   cudaStream_t cap_stream = nullptr;
   std::vector<GraphEntry> graphs;
@@ -310,6 +321,7 @@ extern "C" q4g_status q4g_model_create(const q4g_config* cfg, const q4g_weights*
 extern "C" void q4g_model_destroy(q4g_model* m) {
   if (!m) return;
   free_graphs(m);
+  for (cudaEvent_t e : m->ev_pool) cudaEventDestroy(e);
   if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
   cudaFree(m->scratch);
   delete m;
@@ -329,6 +341,7 @@ extern "C" q4g_status q4g_model_set_option(q4g_model* m, q4g_option opt, intptr_
     case Q4G_OPT_CUDA_GRAPH: m->use_graph = value != 0; break;
     case Q4G_OPT_PDL: m->use_pdl = value != 0; break;
     case Q4G_OPT_DUMP: m->dump = (float*)value; break;
+    case Q4G_OPT_PROFILE: m->profile = value != 0; break;
     default: return fail(Q4G_EINVAL, "unknown option %d", (int)opt);
   }
   free_graphs(m);
@@ -571,6 +584,37 @@ __half* ring_v(const q4g_cache* c, int i) { return (__half*)(c->buf + c->view.ri
 __half* glob_k(const q4g_cache* c, int i) { return (__half*)(c->buf + c->view.global_k_offset + i * c->view.global_layer_bytes); }
 __half* glob_v(const q4g_cache* c, int i) { return (__half*)(c->buf + c->view.global_v_offset + i * c->view.global_layer_bytes); }
 
+// Profile mode: an event before and after each launch on the launching stream.
+cudaEvent_t next_event(q4g_model* m) {
+  if (m->ev_next == m->ev_pool.size()) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    m->ev_pool.push_back(e);
+  }
+  return m->ev_pool[m->ev_next++];
+}
+
+struct Prof {
+  q4g_model* m;
+  cudaStream_t st;
+  cudaEvent_t a = nullptr;
+  Prof(q4g_model* m_, cudaStream_t s) : m(m_), st(s) {
+    if (m->profile && (a = next_event(m))) cudaEventRecord(a, st);
+  }
+  cudaError_t done(cudaError_t e, int kind, int layer, double bytes) {
+    if (!a || e != cudaSuccess) return e;
+    cudaEvent_t b = next_event(m);
+    if (!b) return e;
+    cudaEventRecord(b, st);
+    m->recs.push_back({kind, layer, bytes, a, b});
+    return e;
+  }
+};
+
+double gemv_bytes(int64_t rows, int64_t k, int kr, int out_bytes) {
+  return (double)rows * k * 0.5625 + (double)kr * k * 2 + (double)kr * rows * out_bytes;
+}
+
 // Q4G_DEBUG_SYNC=1 (eager mode only): synchronise and report after every launch.
 cudaError_t debug_sync(cudaError_t e, const char* what, int layer, cudaStream_t st) {
   static const bool on = getenv("Q4G_DEBUG_SYNC") != nullptr;
@@ -585,8 +629,8 @@ cudaError_t debug_sync(cudaError_t e, const char* what, int layer, cudaStream_t 
 }
 
 // All kernels of one step after step_init (the part that is captured in a graph).
-cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, float* logits, int32_t* argmax,
-                         cudaStream_t st) {
+cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0, float* logits,
+                         int32_t* argmax, cudaStream_t st) {
   const q4g_config& cf = m->cfg;
   const int H = cf.hidden, L = cf.n_layers;
   const bool pdl = m->use_pdl;
@@ -627,7 +671,9 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, float* logits
       p.epi = EPI_STORE;
       p.y = m->qkv;
       p.y_stride = S.qkv_cols;
-      if ((e = debug_sync(launch_gemv(p, st, pdl), "qkv", l, st)) != cudaSuccess) return e;
+      Prof pr(m, st);
+      e = pr.done(debug_sync(launch_gemv(p, st, pdl), "qkv", l, st), 1, l, gemv_bytes(S.qkv_cols, H, kr, 4));
+      if (e != cudaSuccess) return e;
     }
     // (a4-a6) q/k/v epilogue, cache write, split-KV attention, combine
     {
@@ -660,8 +706,18 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, float* logits
       p.counters = m->counters + 8;
       p.combine_in_kernel = full ? 0 : 1;
       p.out = m->attn;
-      if ((e = debug_sync(launch_attention(p, st, pdl), "attention", l, st)) != cudaSuccess) return e;
-      if (full && (e = debug_sync(launch_attn_combine(p, st, pdl), "combine", l, st)) != cudaSuccess) return e;
+      const int64_t q_last = pos0 + kr - 1;
+      const int64_t keys = full ? q_last + 1 : std::min<int64_t>(q_last + 1, (int64_t)cf.window + kr - 1);
+      const double kv_bytes = (double)S.nkv * (keys + kr) * 2.0 * S.hd * 2.0;
+      Prof pr(m, st);
+      e = pr.done(debug_sync(launch_attention(p, st, pdl), "attention", l, st), full ? 3 : 2, l, kv_bytes);
+      if (e != cudaSuccess) return e;
+      if (full) {
+        Prof pc(m, st);
+        e = pc.done(debug_sync(launch_attn_combine(p, st, pdl), "combine", l, st), 4, l,
+                    (double)kr * cf.n_q_heads * p.n_chunks * (S.hd + 2) * 4.0);
+        if (e != cudaSuccess) return e;
+      }
     }
     // (a7) output projection
     {
@@ -681,7 +737,9 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, float* logits
         p.epi = EPI_STORE;
         p.y = m->o + (size_t)r0 * H;
         p.y_stride = H;
-        if ((e = debug_sync(launch_gemv(p, st, pdl), "o_proj", l, st)) != cudaSuccess) return e;
+        Prof pr(m, st);
+        e = pr.done(debug_sync(launch_gemv(p, st, pdl), "o_proj", l, st), 5, l, gemv_bytes(H, kin, p.kr, 4));
+        if (e != cudaSuccess) return e;
       }
     }
     // (a8-a10) post-attention norm + residual, pre-FFN norm, gate|up, GeGLU
@@ -705,7 +763,9 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, float* logits
       p.epi = EPI_GEGLU;
       p.act = m->act;
       p.act_stride = cf.ffn;
-      if ((e = debug_sync(launch_gemv(p, st, pdl), "gate_up", l, st)) != cudaSuccess) return e;
+      Prof pr(m, st);
+      e = pr.done(debug_sync(launch_gemv(p, st, pdl), "gate_up", l, st), 6, l, gemv_bytes(2 * cf.ffn, H, kr, 1));
+      if (e != cudaSuccess) return e;
     }
     // (a11) down projection
     {
@@ -724,7 +784,9 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, float* logits
         p.epi = EPI_STORE;
         p.y = m->d + (size_t)r0 * H;
         p.y_stride = H;
-        if ((e = debug_sync(launch_gemv(p, st, pdl), "down", l, st)) != cudaSuccess) return e;
+        Prof pr(m, st);
+        e = pr.done(debug_sync(launch_gemv(p, st, pdl), "down", l, st), 7, l, gemv_bytes(H, cf.ffn, p.kr, 4));
+        if (e != cudaSuccess) return e;
       }
     }
   }
@@ -755,7 +817,10 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, float* logits
     p.am_idx = m->am_idx;
     p.counter = m->counters;
     p.argmax_out = argmax ? argmax : m->argmax_buf;
-    if ((e = debug_sync(launch_gemv(p, st, pdl), "head", L, st)) != cudaSuccess) return e;
+    Prof pr(m, st);
+    e = pr.done(debug_sync(launch_gemv(p, st, pdl), "head", L, st), 8, L,
+                gemv_bytes(cf.vocab, H, kr, logits ? 4 : 0));
+    if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
 }
@@ -791,9 +856,12 @@ q4g_status run_step(q4g_model* m, q4g_cache* c, int kr, int64_t pos0, const int3
   sp.pos_dev = m->pos_dev;
   sp.counters = m->counters;
   sp.n_counters = m->n_counters;
-  CK(launch_step_init(sp, st));
-  if (!m->use_graph) {
-    CK(enqueue_body(m, c, kr, logits, argmax, st));
+  {
+    Prof pr(m, st);
+    CK(pr.done(launch_step_init(sp, st), 0, -1, (double)kr * cf.hidden * (4 + 0.5625)));
+  }
+  if (!m->use_graph || m->profile) {
+    CK(enqueue_body(m, c, kr, pos0, logits, argmax, st));
     return Q4G_OK;
   }
   cudaGraphExec_t exec = nullptr;
@@ -804,7 +872,7 @@ q4g_status run_step(q4g_model* m, q4g_cache* c, int kr, int64_t pos0, const int3
     if (m->graphs.size() >= 16) free_graphs(m);
     cudaGraph_t graph = nullptr;
     CK(cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal));
-    cudaError_t e = enqueue_body(m, c, kr, logits, argmax, m->cap_stream);
+    cudaError_t e = enqueue_body(m, c, kr, pos0, logits, argmax, m->cap_stream);
     cudaError_t e2 = cudaStreamEndCapture(m->cap_stream, &graph);
     if (e != cudaSuccess) {
       if (graph) cudaGraphDestroy(graph);
@@ -867,4 +935,27 @@ extern "C" q4g_status q4g_verify_block(q4g_model* m, q4g_cache* c, const int32_t
   if (pos0 < 0 || pos0 + K > c->capacity) return fail(Q4G_ERANGE, "block outside [0, capacity)");
   if (accepted_count < 0 || accepted_count > K) return fail(Q4G_ERANGE, "accepted_count outside [0, K]");
   return run_step(m, c, K, pos0, ids, nullptr, nullptr, logits, argmax, (cudaStream_t)stream);
+}
+
+extern "C" int32_t q4g_model_profile_read(q4g_model* m, q4g_launch_record* out, int32_t max,
+                                          q4g_stream_t stream) {
+  if (!m || (max > 0 && !out)) {
+    fail(Q4G_EINVAL, "NULL argument");
+    return -1;
+  }
+  std::lock_guard<std::mutex> lk(m->mu);
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) {
+    cuda_fail(e, "q4g_model_profile_read");
+    return -1;
+  }
+  const int32_t n = (int32_t)m->recs.size();
+  for (int32_t i = 0; i < n && i < max; ++i) {
+    float ms = 0.f;
+    cudaEventElapsedTime(&ms, m->recs[i].a, m->recs[i].b);
+    out[i] = {m->recs[i].kind, m->recs[i].layer, ms, m->recs[i].bytes};
+  }
+  m->recs.clear();
+  m->ev_next = 0;
+  return n;
 }

@@ -13,7 +13,9 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libq4g.so")
 
 Q4G_OK, Q4G_EINVAL, Q4G_ERANGE, Q4G_ENOMEM, Q4G_ECUDA, Q4G_ETIMEOUT = range(6)
-Q4G_OPT_CUDA_GRAPH, Q4G_OPT_PDL, Q4G_OPT_DUMP = 1, 2, 3
+Q4G_OPT_CUDA_GRAPH, Q4G_OPT_PDL, Q4G_OPT_DUMP, Q4G_OPT_PROFILE = 1, 2, 3, 4
+KIND_NAMES = ["step_init", "qkv_gemv", "attn_sliding", "attn_full", "attn_combine", "o_gemv",
+              "gate_up_gemv", "down_gemv", "head_gemv"]
 
 EXPORTS = [
     "q4g_last_error", "q4g_status_string", "q4g_abi_version",
@@ -22,7 +24,7 @@ EXPORTS = [
     "q4g_model_create", "q4g_model_destroy", "q4g_model_check", "q4g_model_set_option",
     "q4g_cache_bytes", "q4g_cache_init", "q4g_cache_reset", "q4g_cache_destroy", "q4g_cache_layout",
     "q4g_decode_step", "q4g_decode_step_device_token", "q4g_decode_step_hidden",
-    "q4g_decode_step_host", "q4g_verify_block",
+    "q4g_decode_step_host", "q4g_verify_block", "q4g_model_profile_read",
 ]
 
 
@@ -53,6 +55,10 @@ class q4g_layer_weights(C.Structure):
 class q4g_weights(C.Structure):
     _fields_ = [("layers", C.POINTER(q4g_layer_weights)), ("embed", q4g_qtensor),
                 ("norm_final", C.c_void_p)]
+
+
+class q4g_launch_record(C.Structure):
+    _fields_ = [("kind", C.c_int32), ("layer", C.c_int32), ("ms", C.c_float), ("bytes", C.c_double)]
 
 
 class q4g_cache_view(C.Structure):
@@ -99,6 +105,7 @@ def lib() -> C.CDLL:
             "q4g_decode_step_hidden": (C.c_int, [vp, vp, vp, i64, vp, vp, vp]),
             "q4g_decode_step_host": (C.c_int, [vp, vp, i32, i64, vp, vp, vp]),
             "q4g_verify_block": (C.c_int, [vp, vp, vp, i32, i64, i32, vp, vp, vp]),
+            "q4g_model_profile_read": (i32, [vp, C.POINTER(q4g_launch_record), i32, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -212,3 +219,12 @@ def q4g_decode_step_host(model, cache, token, pos, logits_host, argmax_host, str
 
 def q4g_verify_block(model, cache, ids, K, pos0, accepted_count, logits, argmax, stream):
     _call("q4g_verify_block", model, cache, ids, K, pos0, accepted_count, logits, argmax, stream)
+
+
+def q4g_model_profile_read(model, stream, max_records: int = 1 << 16):
+    """Launch records since the last read: list of (kind, layer, ms, bytes)."""
+    buf = (q4g_launch_record * max_records)()
+    n = lib().q4g_model_profile_read(model, buf, max_records, stream)
+    if n < 0:
+        check(Q4G_ECUDA)
+    return [(buf[i].kind, buf[i].layer, buf[i].ms, buf[i].bytes) for i in range(min(n, max_records))]
