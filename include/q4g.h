@@ -122,6 +122,31 @@ q4g_status q4g_flash_decode_linear(const uint16_t* q, int32_t n_q, int32_t n_kv,
                                    const uint16_t* k, const uint16_t* v, int64_t len, uint16_t* out,
                                    void* workspace, size_t workspace_bytes, q4g_stream_t stream);
 
+/* Allocation-free variant of q4g_flash_decode_ring (no counterpart on the pages;
+ * an integration convenience). It is for callers that cannot allocate device
+ * memory at call time -- for example a program whose device memory belongs to a
+ * framework's caching allocator that this library cannot reach, or a process
+ * that reserves its memory budget at start-up and treats a later cudaMalloc as
+ * a failure -- and so cannot provide the workspace the ordinary entry point
+ * takes. Same inputs, outputs and results as q4g_flash_decode_ring; the
+ * split-KV scratch lives in one fixed device array of
+ * Q4G_NOALLOC_SCRATCH_BYTES, which every GPU that loads the library holds until
+ * the process exits. It must hold 256 bytes of counters plus, per query head
+ * and chunk, 8 bytes of (max, sum) and head_dim * 4 bytes of partial output
+ * (chunks = ceil(window / 64) at most); larger requests return Q4G_ERANGE with
+ * a message. The call makes no device allocation or free of any kind; it
+ * clears the counters (an asynchronous memset on `stream`) and launches one
+ * kernel. The first call on a device looks up the array's device address with
+ * that device current; make that first call before any stream capture. All
+ * calls on a device share the array, and it keeps the last call's contents:
+ * calls that overlap on the GPU (other streams, or without ordering between
+ * them) race on it and must be serialised by the caller. */
+#define Q4G_NOALLOC_SCRATCH_BYTES ((size_t)1 << 20)
+q4g_status q4g_flash_decode_ring_noalloc(const uint16_t* q, int32_t n_q, int32_t n_kv,
+                                         int32_t head_dim, const uint16_t* k_ring,
+                                         const uint16_t* v_ring, int64_t ring, int64_t window,
+                                         int64_t pos, uint16_t* out, q4g_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Model and cache.                                                           */
 /* ------------------------------------------------------------------------ */

@@ -51,6 +51,8 @@ struct LayerShape {
 
 extern "C" const char* q4g_last_error(void) { return g_err.c_str(); }
 
+void q4g::set_last_error(const char* msg) { g_err = msg ? msg : ""; }
+
 extern "C" const char* q4g_status_string(q4g_status s) {
   switch (s) {
     case Q4G_OK: return "Q4G_OK";

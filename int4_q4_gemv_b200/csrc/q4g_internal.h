@@ -132,4 +132,7 @@ cudaError_t launch_step_init(const StepParams& p, cudaStream_t st);
 
 int device_sm_count();
 
+// Sets the message q4g_last_error() returns on this thread.
+void set_last_error(const char* msg);
+
 }  // namespace q4g

@@ -25,7 +25,9 @@ EXPORTS = [
     "q4g_cache_bytes", "q4g_cache_init", "q4g_cache_reset", "q4g_cache_destroy", "q4g_cache_layout",
     "q4g_decode_step", "q4g_decode_step_device_token", "q4g_decode_step_hidden",
     "q4g_decode_step_host", "q4g_verify_block", "q4g_model_profile_read",
+    "q4g_flash_decode_ring_noalloc",
 ]
+Q4G_NOALLOC_SCRATCH_BYTES = 1 << 20
 
 
 class Q4GError(RuntimeError):
@@ -106,6 +108,7 @@ def lib() -> C.CDLL:
             "q4g_decode_step_host": (C.c_int, [vp, vp, i32, i64, vp, vp, vp]),
             "q4g_verify_block": (C.c_int, [vp, vp, vp, i32, i64, i32, vp, vp, vp]),
             "q4g_model_profile_read": (i32, [vp, C.POINTER(q4g_launch_record), i32, vp]),
+            "q4g_flash_decode_ring_noalloc": (C.c_int, [vp, i32, i32, i32, vp, vp, i64, i64, i64, vp, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -155,6 +158,11 @@ def q4g_flash_decode_ring(q, n_q, n_kv, head_dim, k_ring, v_ring, ring, window, 
 
 def q4g_flash_decode_linear(q, n_q, n_kv, head_dim, k, v, length, out, ws, ws_bytes, stream):
     _call("q4g_flash_decode_linear", q, n_q, n_kv, head_dim, k, v, length, out, ws, ws_bytes, stream)
+
+
+def q4g_flash_decode_ring_noalloc(q, n_q, n_kv, head_dim, k_ring, v_ring, ring, window, pos, out, stream):
+    _call("q4g_flash_decode_ring_noalloc", q, n_q, n_kv, head_dim, k_ring, v_ring, ring, window, pos, out,
+          stream)
 
 
 def q4g_model_create(cfg: q4g_config, weights: q4g_weights) -> int:
