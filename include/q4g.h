@@ -106,7 +106,8 @@ size_t q4g_flash_decode_workspace_bytes(int32_t n_q_heads, int32_t head_dim);
  * slot = position mod R. For the query at absolute position `pos`, slot j is
  * attended iff p = pos - ((pos - j) mod R) satisfies p >= 0 and pos - p < W.
  * Query head h uses KV head h / (n_q / n_kv). Scale 1.0, fp32 online softmax,
- * fp16 output [n_q][hd]. hd must be 256 or 512; W <= R.
+ * fp16 output [n_q][hd]. hd must be 256 or 512; W <= R <= 2^30 (Q4G_ERANGE
+ * above); pos is any non-negative int64.
  * workspace: device buffer of q4g_flash_decode_workspace_bytes(n_q, hd) bytes,
  * 256-byte aligned, used as scratch by this call (calls that share a workspace
  * must not overlap on the GPU). */
@@ -117,7 +118,7 @@ q4g_status q4g_flash_decode_ring(const uint16_t* q, int32_t n_q, int32_t n_kv, i
 
 /* Flash-decode over a linear cache ("Gemma 4 12B", flash-decode paragraph):
  * K/V [len_capacity][n_kv][hd] fp16, keys 0..len-1 all attended (mask-free,
- * causal by construction). Otherwise as q4g_flash_decode_ring. */
+ * causal by construction), 1 <= len <= 2^30. Otherwise as q4g_flash_decode_ring. */
 q4g_status q4g_flash_decode_linear(const uint16_t* q, int32_t n_q, int32_t n_kv, int32_t head_dim,
                                    const uint16_t* k, const uint16_t* v, int64_t len, uint16_t* out,
                                    void* workspace, size_t workspace_bytes, q4g_stream_t stream);
@@ -157,7 +158,7 @@ q4g_status q4g_flash_decode_ring_noalloc(const uint16_t* q, int32_t n_q, int32_t
  * sliding-window layers. */
 typedef struct {
   int32_t n_layers;        /* [48] */
-  int32_t hidden;          /* h [3840], multiple of 256 */
+  int32_t hidden;          /* h [3840], multiple of 32, at most 8192 */
   int32_t n_q_heads;       /* [16] */
   int32_t ffn;             /* [15360], multiple of 256 */
   int32_t vocab;           /* tied embedding / head rows [262144], multiple of 16 */
@@ -212,8 +213,9 @@ typedef struct q4g_cache q4g_cache;
 q4g_status q4g_model_create(const q4g_config* cfg, const q4g_weights* w, q4g_model** out);
 void q4g_model_destroy(q4g_model* m);
 
-/* Reports (and clears) a device-side error word set by a bounded wait that gave
- * up (Q4G_ETIMEOUT) and any sticky CUDA error (Q4G_ECUDA). Synchronises `stream`. */
+/* Reports (and clears) the device-side error word that a bounded wait sets when
+ * it gives up (Q4G_ETIMEOUT; every wait inside the kernels is limited in time,
+ * 2 s by default) and any sticky CUDA error (Q4G_ECUDA). Synchronises `stream`. */
 q4g_status q4g_model_check(q4g_model* m, q4g_stream_t stream);
 
 /* Options (defaults in brackets): */
@@ -222,9 +224,14 @@ typedef enum {
   Q4G_OPT_PDL = 2,        /* [1] programmatic dependent launch between kernels */
   Q4G_OPT_DUMP = 3,       /* [0] value = device float* [K][n_layers+1][h]: residual
                                  stream after the embedding and after each layer */
-  Q4G_OPT_PROFILE = 4     /* [0] 1: launch eagerly and bracket every kernel with CUDA
+  Q4G_OPT_PROFILE = 4,    /* [0] 1: launch eagerly and bracket every kernel with CUDA
                                  events on the launching stream (read with
                                  q4g_model_profile_read) */
+  Q4G_OPT_TEST_STALL = 5  /* [0] 1: failure-path test. In the next step, one pipeline
+                                 stage of the first GEMV expects 16 bytes that never
+                                 arrive; its bounded wait (20 ms) gives up, the step
+                                 finishes with unspecified results and
+                                 q4g_model_check returns Q4G_ETIMEOUT. One-shot. */
 } q4g_option;
 q4g_status q4g_model_set_option(q4g_model* m, q4g_option opt, intptr_t value);
 
@@ -250,7 +257,8 @@ int32_t q4g_model_profile_read(q4g_model* m, q4g_launch_record* out, int32_t max
  * [sl_kv_heads][ring][sl_head_dim] fp16 (slot = position mod ring); per full
  * layer K and V of [gl_kv_heads][capacity][gl_head_dim] fp16 indexed by absolute
  * position ("Gemma-4-12B-CoreAI": v5 section and "The per-tier cost"). The
- * storage is a caller-owned device buffer of q4g_cache_bytes() bytes. */
+ * storage is a caller-owned device buffer of q4g_cache_bytes() bytes.
+ * 1 <= capacity <= 2^30, else Q4G_ERANGE. */
 q4g_status q4g_cache_bytes(const q4g_model* m, int64_t capacity, size_t* bytes);
 q4g_status q4g_cache_init(const q4g_model* m, int64_t capacity, void* dev_buf, size_t bytes,
                           q4g_cache** out);

@@ -114,6 +114,7 @@ struct q4g_model {
   float* dump = nullptr;
   // profile mode: events around every launch
   bool profile = false;
+  bool stall_next = false;  // test: the next step's first GEMV waits on a stage that never completes
   std::vector<cudaEvent_t> ev_pool;
   struct Rec {
     int kind, layer;
@@ -156,13 +157,15 @@ q4g_status validate_config(const q4g_config* c) {
   if (c->n_layers < 1 || c->hidden < 32 || c->hidden % 32 || c->ffn < 32 || c->ffn % 32 ||
       c->vocab < 1 || c->n_q_heads < 1)
     return fail(Q4G_EINVAL, "hidden and ffn must be positive multiples of 32; layers, heads, vocab >= 1");
+  if (c->hidden > 8192)
+    return fail(Q4G_EINVAL, "hidden must be <= 8192 (the fused residual prologue keeps it in registers)");
   if (c->sl_head_dim != 256 || c->gl_head_dim != 512)
     return fail(Q4G_EINVAL, "head dims must be 256 (sliding) and 512 (full)");
   if (c->sl_kv_heads < 1 || c->gl_kv_heads < 1 || c->n_q_heads % c->sl_kv_heads ||
       c->n_q_heads % c->gl_kv_heads)
     return fail(Q4G_EINVAL, "n_q_heads must be a multiple of both KV head counts");
-  if (c->window < 1 || c->ring < c->window + 1)
-    return fail(Q4G_EINVAL, "need window >= 1 and ring > window");
+  if (c->window < 1 || c->ring < c->window + 1 || c->ring > (1 << 30))
+    return fail(Q4G_EINVAL, "need window >= 1, window < ring <= 2^30");
   if (c->rope_pairs_full < 0 || c->rope_pairs_full > c->gl_head_dim / 2)
     return fail(Q4G_EINVAL, "rope_pairs_full out of range");
   if (!(c->rope_theta_sl > 0) || !(c->rope_theta_gl > 0) || !(c->rms_eps >= 0) || !(c->softcap > 0) ||
@@ -333,6 +336,16 @@ extern "C" q4g_status q4g_model_check(q4g_model* m, q4g_stream_t stream) {
   if (!m) return fail(Q4G_EINVAL, "model is NULL");
   CK(cudaStreamSynchronize((cudaStream_t)stream));
   CK(cudaGetLastError());
+  int32_t* ew = device_error_word();
+  if (!ew) return fail(Q4G_ECUDA, "error word unavailable");
+  int32_t word = 0;
+  CK(cudaMemcpy(&word, ew, sizeof word, cudaMemcpyDeviceToHost));
+  if (word) {
+    const int32_t zero = 0;
+    CK(cudaMemcpy(ew, &zero, sizeof zero, cudaMemcpyHostToDevice));
+    return fail(Q4G_ETIMEOUT, "a bounded device wait gave up (error word 0x%x); results of that step are unspecified",
+                word);
+  }
   return Q4G_OK;
 }
 
@@ -344,6 +357,7 @@ extern "C" q4g_status q4g_model_set_option(q4g_model* m, q4g_option opt, intptr_
     case Q4G_OPT_PDL: m->use_pdl = value != 0; break;
     case Q4G_OPT_DUMP: m->dump = (float*)value; break;
     case Q4G_OPT_PROFILE: m->profile = value != 0; break;
+    case Q4G_OPT_TEST_STALL: m->stall_next = value != 0; break;
     default: return fail(Q4G_EINVAL, "unknown option %d", (int)opt);
   }
   free_graphs(m);
@@ -353,7 +367,7 @@ extern "C" q4g_status q4g_model_set_option(q4g_model* m, q4g_option opt, intptr_
 // --------------------------------------------------------------- cache ------
 extern "C" q4g_status q4g_cache_bytes(const q4g_model* m, int64_t capacity, size_t* bytes) {
   if (!m || !bytes) return fail(Q4G_EINVAL, "NULL argument");
-  if (capacity < 1 || capacity > (int64_t)1 << 31) return fail(Q4G_ERANGE, "capacity out of range");
+  if (capacity < 1 || capacity > (int64_t)1 << 30) return fail(Q4G_ERANGE, "capacity must be in [1, 2^30]");
   const q4g_config& c = m->cfg;
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
   const size_t ring = up((size_t)c.sl_kv_heads * c.ring * c.sl_head_dim * 2);
@@ -563,6 +577,7 @@ extern "C" q4g_status q4g_flash_decode_ring(const uint16_t* q, int32_t n_q, int3
                                             int64_t window, int64_t pos, uint16_t* out, void* workspace,
                                             size_t workspace_bytes, q4g_stream_t stream) {
   if (ring < 1 || window < 1 || window > ring) return fail(Q4G_EINVAL, "need 1 <= window <= ring");
+  if (ring > ((int64_t)1 << 30)) return fail(Q4G_ERANGE, "ring > 2^30");
   if (pos < 0) return fail(Q4G_ERANGE, "pos < 0");
   return flash_standalone(q, n_q, n_kv, head_dim, k_ring, v_ring, ring, true, window, pos, out, workspace,
                           workspace_bytes, (cudaStream_t)stream);
@@ -571,7 +586,7 @@ extern "C" q4g_status q4g_flash_decode_ring(const uint16_t* q, int32_t n_q, int3
 extern "C" q4g_status q4g_flash_decode_linear(const uint16_t* q, int32_t n_q, int32_t n_kv, int32_t head_dim,
                                               const uint16_t* k, const uint16_t* v, int64_t len, uint16_t* out,
                                               void* workspace, size_t workspace_bytes, q4g_stream_t stream) {
-  if (len < 1) return fail(Q4G_ERANGE, "len must be >= 1");
+  if (len < 1 || len > ((int64_t)1 << 30)) return fail(Q4G_ERANGE, "len must be in [1, 2^30]");
   // linear cache [len][n_kv][hd] is addressed as [n_kv][rows][hd] with rows = len only when n_kv == 1
   if (n_kv != 1) return fail(Q4G_EINVAL, "the linear entry point takes one KV head ([len][hd] cache)");
   return flash_standalone(q, n_q, n_kv, head_dim, k, v, len, false, 0, len - 1, out, workspace,
@@ -630,6 +645,18 @@ cudaError_t debug_sync(cudaError_t e, const char* what, int layer, cudaStream_t 
   return e;
 }
 
+// Scale of the fraction of the next GEMV's per-warp ranges a kernel prefetches
+// into L2 once its own loads are in flight (Q4G_L2_PREFETCH, default 0: off;
+// measured slower, the prefetch traffic delays the attention kernels).
+float prefetch_scale() {
+  static float f = -1.f;
+  if (f < 0.f) {
+    const char* e = getenv("Q4G_L2_PREFETCH");
+    f = e ? (float)atof(e) : 0.0f;
+  }
+  return f;
+}
+
 // All kernels of one step after step_init (the part that is captured in a graph).
 cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0, float* logits,
                          int32_t* argmax, cudaStream_t st) {
@@ -637,42 +664,154 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
   const int H = cf.hidden, L = cf.n_layers;
   const bool pdl = m->use_pdl;
   const int64_t dstride = (int64_t)(L + 1) * H;
+  const float pf = prefetch_scale();
   cudaError_t e;
   float* rA = m->r[0];
   float* rB = m->r[1];
+
+  // (a2, a3) pre-attention norm (+ previous layer's post-FFN residual) and QKV
+  auto qkv_params = [&](int l) {
+    const q4g_layer_weights& W = m->layers[l];
+    const bool full = m->full[l];
+    const LayerShape& S = full ? m->gl : m->sl;
+    GemvParams p{};
+    p.seg[0] = {W.wq.qs, W.wq.scales, S.nq_cols};
+    p.seg[1] = {W.wk.qs, W.wk.scales, S.k_cols};
+    p.nseg = 2;
+    if (!full) p.seg[2] = {W.wv.qs, W.wv.scales, S.v_cols}, p.nseg = 3;
+    p.k = H;
+    p.n_rows = S.qkv_cols;
+    p.n_units = S.qkv_cols / 16;
+    p.kr = kr;
+    p.pro = PRO_RESID;
+    p.r_in = rA;
+    p.r_out = rB;
+    if (l > 0) {
+      p.delta = m->d;
+      p.w_delta = m->layers[l - 1].norm_post_ffn;
+      p.scale = m->layers[l - 1].layer_scalar;
+    } else {
+      p.scale = 1.0f;
+    }
+    p.w_x = W.norm_in;
+    p.eps = cf.rms_eps;
+    p.dump = m->dump ? m->dump + (size_t)l * H : nullptr;
+    p.dump_stride = dstride;
+    p.epi = EPI_STORE;
+    p.y = m->qkv;
+    p.y_stride = S.qkv_cols;
+    return p;
+  };
+  // (a7) output projection, activation rows [r0, r0 + maxr)
+  auto o_params = [&](int l, int r0) {
+    const q4g_layer_weights& W = m->layers[l];
+    const LayerShape& S = m->full[l] ? m->gl : m->sl;
+    const int kin = cf.n_q_heads * S.hd;
+    const int maxr = gemv_max_rows(kin);
+    GemvParams p{};
+    p.seg[0] = {W.wo.qs, W.wo.scales, H};
+    p.nseg = 1;
+    p.k = kin;
+    p.n_rows = H;
+    p.n_units = H / 16;
+    p.kr = kr - r0 < maxr ? kr - r0 : maxr;
+    p.pro = PRO_X16;
+    p.x = m->attn + (size_t)r0 * kin;
+    p.x_stride = kin;
+    p.epi = EPI_STORE;
+    p.y = m->o + (size_t)r0 * H;
+    p.y_stride = H;
+    return p;
+  };
+  // (a8-a10) post-attention norm + residual, pre-FFN norm, gate|up, GeGLU
+  auto gate_up_params = [&](int l) {
+    const q4g_layer_weights& W = m->layers[l];
+    GemvParams p{};
+    p.seg[0] = {W.wgate.qs, W.wgate.scales, cf.ffn};
+    p.seg[1] = {W.wup.qs, W.wup.scales, cf.ffn};
+    p.nseg = 2;
+    p.k = H;
+    p.n_rows = 2 * cf.ffn;
+    p.n_units = cf.ffn / 8;
+    p.kr = kr;
+    p.pro = PRO_RESID;
+    p.r_in = rB;
+    p.r_out = rA;
+    p.delta = m->o;
+    p.w_delta = W.norm_post_attn;
+    p.scale = 1.0f;
+    p.w_x = W.norm_pre_ffn;
+    p.eps = cf.rms_eps;
+    p.epi = EPI_GEGLU;
+    p.act = m->act;
+    p.act_stride = cf.ffn;
+    return p;
+  };
+  // (a11) down projection, activation rows [r0, r0 + maxr)
+  auto down_params = [&](int l, int r0) {
+    const q4g_layer_weights& W = m->layers[l];
+    const int maxr = gemv_max_rows(cf.ffn);
+    GemvParams p{};
+    p.seg[0] = {W.wdown.qs, W.wdown.scales, H};
+    p.nseg = 1;
+    p.k = cf.ffn;
+    p.n_rows = H;
+    p.n_units = H / 16;
+    p.kr = kr - r0 < maxr ? kr - r0 : maxr;
+    p.pro = PRO_X16;
+    p.x = m->act + (size_t)r0 * cf.ffn;
+    p.x_stride = cf.ffn;
+    p.epi = EPI_STORE;
+    p.y = m->d + (size_t)r0 * H;
+    p.y_stride = H;
+    return p;
+  };
+  // (a12, a13) last residual + layer scalar, final norm, tied head, softcap, argmax
+  auto head_params = [&]() {
+    GemvParams p{};
+    p.seg[0] = {m->embed.qs, m->embed.scales, cf.vocab};
+    p.nseg = 1;
+    p.k = H;
+    p.n_rows = cf.vocab;
+    p.n_units = (cf.vocab + 15) / 16;
+    p.kr = kr;
+    p.pro = PRO_RESID;
+    p.r_in = rA;
+    p.r_out = rB;
+    p.delta = m->d;
+    p.w_delta = m->layers[L - 1].norm_post_ffn;
+    p.scale = m->layers[L - 1].layer_scalar;
+    p.w_x = m->norm_final;
+    p.eps = cf.rms_eps;
+    p.dump = m->dump ? m->dump + (size_t)L * H : nullptr;
+    p.dump_stride = dstride;
+    p.epi = EPI_HEAD;
+    p.logits = logits;
+    p.logits_stride = cf.vocab;
+    p.softcap = cf.softcap;
+    p.am_val = m->am_val;
+    p.am_idx = m->am_idx;
+    p.counter = m->counters;
+    p.argmax_out = argmax ? argmax : m->argmax_buf;
+    return p;
+  };
+  auto next_of = [&](const GemvParams& q, float frac) {
+    return pf > 0.f ? gemv_next_desc(q, std::min(1.0f, frac * pf)) : NextGemv{};
+  };
+
   for (int l = 0; l < L; ++l) {
     const q4g_layer_weights& W = m->layers[l];
     const bool full = m->full[l];
     const LayerShape& S = full ? m->gl : m->sl;
     const int ord = m->ordinal[l];
-    // (a2, a3) pre-attention norm (+ previous layer's post-FFN residual) and QKV
+    const GemvParams gate_up = gate_up_params(l);
     {
-      GemvParams p{};
-      p.seg[0] = {W.wq.qs, W.wq.scales, S.nq_cols};
-      p.seg[1] = {W.wk.qs, W.wk.scales, S.k_cols};
-      p.nseg = 2;
-      if (!full) p.seg[2] = {W.wv.qs, W.wv.scales, S.v_cols}, p.nseg = 3;
-      p.k = H;
-      p.n_rows = S.qkv_cols;
-      p.n_units = S.qkv_cols / 16;
-      p.kr = kr;
-      p.pro = PRO_RESID;
-      p.r_in = rA;
-      p.r_out = rB;
-      if (l > 0) {
-        p.delta = m->d;
-        p.w_delta = m->layers[l - 1].norm_post_ffn;
-        p.scale = m->layers[l - 1].layer_scalar;
-      } else {
-        p.scale = 1.0f;
+      GemvParams p = qkv_params(l);
+      p.next = next_of(o_params(l, 0), 1.0f);
+      if (l == 0 && m->stall_next) {
+        p.stall_test = 1;
+        p.wait_ns = 20000000ull;  // 20 ms
       }
-      p.w_x = W.norm_in;
-      p.eps = cf.rms_eps;
-      p.dump = m->dump ? m->dump + (size_t)l * H : nullptr;
-      p.dump_stride = dstride;
-      p.epi = EPI_STORE;
-      p.y = m->qkv;
-      p.y_stride = S.qkv_cols;
       Prof pr(m, st);
       e = pr.done(debug_sync(launch_gemv(p, st, pdl), "qkv", l, st), 1, l, gemv_bytes(S.qkv_cols, H, kr, 4));
       if (e != cudaSuccess) return e;
@@ -680,6 +819,7 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
     // (a4-a6) q/k/v epilogue, cache write, split-KV attention, combine
     {
       AttnParams p{};
+      p.next = next_of(gate_up, 0.15f);
       p.qkv = m->qkv;
       p.qkv_stride = S.qkv_cols;
       p.k_off = S.nq_cols;
@@ -715,110 +855,44 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
       e = pr.done(debug_sync(launch_attention(p, st, pdl), "attention", l, st), full ? 3 : 2, l, kv_bytes);
       if (e != cudaSuccess) return e;
       if (full) {
+        p.next = NextGemv{};
         Prof pc(m, st);
         e = pc.done(debug_sync(launch_attn_combine(p, st, pdl), "combine", l, st), 4, l,
                     (double)kr * cf.n_q_heads * p.n_chunks * (S.hd + 2) * 4.0);
         if (e != cudaSuccess) return e;
       }
     }
-    // (a7) output projection
     {
       const int kin = cf.n_q_heads * S.hd;
       const int maxr = gemv_max_rows(kin);
       for (int r0 = 0; r0 < kr; r0 += maxr) {
-        GemvParams p{};
-        p.seg[0] = {W.wo.qs, W.wo.scales, H};
-        p.nseg = 1;
-        p.k = kin;
-        p.n_rows = H;
-        p.n_units = H / 16;
-        p.kr = kr - r0 < maxr ? kr - r0 : maxr;
-        p.pro = PRO_X16;
-        p.x = m->attn + (size_t)r0 * kin;
-        p.x_stride = kin;
-        p.epi = EPI_STORE;
-        p.y = m->o + (size_t)r0 * H;
-        p.y_stride = H;
+        GemvParams p = o_params(l, r0);
+        if (r0 + maxr >= kr) p.next = next_of(gate_up, 0.35f);
         Prof pr(m, st);
         e = pr.done(debug_sync(launch_gemv(p, st, pdl), "o_proj", l, st), 5, l, gemv_bytes(H, kin, p.kr, 4));
         if (e != cudaSuccess) return e;
       }
     }
-    // (a8-a10) post-attention norm + residual, pre-FFN norm, gate|up, GeGLU
     {
-      GemvParams p{};
-      p.seg[0] = {W.wgate.qs, W.wgate.scales, cf.ffn};
-      p.seg[1] = {W.wup.qs, W.wup.scales, cf.ffn};
-      p.nseg = 2;
-      p.k = H;
-      p.n_rows = 2 * cf.ffn;
-      p.n_units = cf.ffn / 8;
-      p.kr = kr;
-      p.pro = PRO_RESID;
-      p.r_in = rB;
-      p.r_out = rA;
-      p.delta = m->o;
-      p.w_delta = W.norm_post_attn;
-      p.scale = 1.0f;
-      p.w_x = W.norm_pre_ffn;
-      p.eps = cf.rms_eps;
-      p.epi = EPI_GEGLU;
-      p.act = m->act;
-      p.act_stride = cf.ffn;
+      GemvParams p = gate_up;
+      p.next = next_of(down_params(l, 0), 0.6f);
       Prof pr(m, st);
       e = pr.done(debug_sync(launch_gemv(p, st, pdl), "gate_up", l, st), 6, l, gemv_bytes(2 * cf.ffn, H, kr, 1));
       if (e != cudaSuccess) return e;
     }
-    // (a11) down projection
     {
       const int maxr = gemv_max_rows(cf.ffn);
       for (int r0 = 0; r0 < kr; r0 += maxr) {
-        GemvParams p{};
-        p.seg[0] = {W.wdown.qs, W.wdown.scales, H};
-        p.nseg = 1;
-        p.k = cf.ffn;
-        p.n_rows = H;
-        p.n_units = H / 16;
-        p.kr = kr - r0 < maxr ? kr - r0 : maxr;
-        p.pro = PRO_X16;
-        p.x = m->act + (size_t)r0 * cf.ffn;
-        p.x_stride = cf.ffn;
-        p.epi = EPI_STORE;
-        p.y = m->d + (size_t)r0 * H;
-        p.y_stride = H;
+        GemvParams p = down_params(l, r0);
+        if (r0 + maxr >= kr) p.next = l + 1 < L ? next_of(qkv_params(l + 1), 1.0f) : next_of(head_params(), 0.05f);
         Prof pr(m, st);
         e = pr.done(debug_sync(launch_gemv(p, st, pdl), "down", l, st), 7, l, gemv_bytes(H, cf.ffn, p.kr, 4));
         if (e != cudaSuccess) return e;
       }
     }
   }
-  // (a12, a13) last residual + layer scalar, final norm, tied head, softcap, argmax
   {
-    GemvParams p{};
-    p.seg[0] = {m->embed.qs, m->embed.scales, cf.vocab};
-    p.nseg = 1;
-    p.k = H;
-    p.n_rows = cf.vocab;
-    p.n_units = (cf.vocab + 15) / 16;
-    p.kr = kr;
-    p.pro = PRO_RESID;
-    p.r_in = rA;
-    p.r_out = rB;
-    p.delta = m->d;
-    p.w_delta = m->layers[L - 1].norm_post_ffn;
-    p.scale = m->layers[L - 1].layer_scalar;
-    p.w_x = m->norm_final;
-    p.eps = cf.rms_eps;
-    p.dump = m->dump ? m->dump + (size_t)L * H : nullptr;
-    p.dump_stride = dstride;
-    p.epi = EPI_HEAD;
-    p.logits = logits;
-    p.logits_stride = cf.vocab;
-    p.softcap = cf.softcap;
-    p.am_val = m->am_val;
-    p.am_idx = m->am_idx;
-    p.counter = m->counters;
-    p.argmax_out = argmax ? argmax : m->argmax_buf;
+    GemvParams p = head_params();
     Prof pr(m, st);
     e = pr.done(debug_sync(launch_gemv(p, st, pdl), "head", L, st), 8, L,
                 gemv_bytes(cf.vocab, H, kr, logits ? 4 : 0));
@@ -862,8 +936,10 @@ q4g_status run_step(q4g_model* m, q4g_cache* c, int kr, int64_t pos0, const int3
     Prof pr(m, st);
     CK(pr.done(launch_step_init(sp, st), 0, -1, (double)kr * cf.hidden * (4 + 0.5625)));
   }
-  if (!m->use_graph || m->profile) {
-    CK(enqueue_body(m, c, kr, pos0, logits, argmax, st));
+  if (!m->use_graph || m->profile || m->stall_next) {
+    cudaError_t e = enqueue_body(m, c, kr, pos0, logits, argmax, st);
+    m->stall_next = false;
+    CK(e);
     return Q4G_OK;
   }
   cudaGraphExec_t exec = nullptr;

@@ -24,6 +24,7 @@
 // rows to the cache; every CTA reads this block's own rows from shared memory.
 #include "q4g_common.cuh"
 #include "q4g_internal.h"
+#include "q4g_prefetch.cuh"
 
 namespace q4g {
 
@@ -66,9 +67,11 @@ Q4G_DEV void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-Q4G_DEV int64_t pmod(int64_t a, int64_t m) {
-  int64_t r = a % m;
-  return r < 0 ? r + m : r;
+// a mod m in [0, m) for 32-bit a, m > 0; the common case (a >= -m) takes one add
+Q4G_DEV int wrap(int a, int m) {
+  if (a >= 0) return a < m ? a : a % m;
+  a += m;
+  return a >= 0 ? a : (a % m + m) % m;
 }
 
 template <int HD>
@@ -81,15 +84,10 @@ struct Smem {
   __half plo[MROWS][TK + 8];
   __half kloc[kMaxRows][HD];
   __half vloc[kMaxRows][HD];
-  int64_t kidx[2][TK];  // slot (ring) or position (linear); -1: no key
+  int32_t kidx[2][TK];  // slot (ring) or position (linear); -1: no key
   float red[8][MROWS];
   float m_run[MROWS], l_run[MROWS], scale[MROWS];
   int ticket;
-};
-
-// Cache row (slot or position) of key `a` of the scan and whether it exists.
-struct KeyRange {
-  int64_t begin, end;  // scan indices [begin, end)
 };
 
 template <int HD>
@@ -108,26 +106,26 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
   const int64_t pos0 = p.pos_dev ? *p.pos_dev : p.pos0;
   const int64_t q_last = pos0 + p.kr - 1;
   const bool fused = p.qkv != nullptr;
+  // 32-bit index arithmetic: the host keeps R, the window and linear positions
+  // below 2^30; ring positions may be any int64, only q_last mod R enters.
+  const int R = (int)p.cache_rows, W = (int)p.window;
+  const int qlm = p.ring ? (int)(q_last % p.cache_rows) : 0;  // slot of the newest key
 
   // ---- key scan of this chunk: ring scans ages, linear scans positions ----
-  int64_t nscan;
-  if (p.ring)
-    nscan = min((int64_t)p.window + p.kr - 1, q_last + 1);
-  else
-    nscan = q_last + 1;
+  const int nscan = p.ring ? (int)min((int64_t)W + p.kr - 1, q_last + 1) : (int)(q_last + 1);
   // chunks are whole tiles; trailing chunks may be empty
-  const int64_t cs = ((nscan + p.n_chunks - 1) / p.n_chunks + TK - 1) / TK * TK;
-  const int64_t a_begin = min(nscan, (int64_t)chunk * cs);
-  const int64_t a_end = min(nscan, a_begin + cs);
-  const int ntiles = (int)((a_end - a_begin + TK - 1) / TK);
+  const int cs = ((nscan + p.n_chunks - 1) / p.n_chunks + TK - 1) / TK * TK;
+  const int a_begin = min(nscan, chunk * cs);
+  const int a_end = min(nscan, a_begin + cs);
+  const int ntiles = (a_end - a_begin + TK - 1) / TK;
 
-  auto key_row = [&](int64_t a) -> int64_t {  // cache row of scan index a
-    return p.ring ? pmod(q_last - a, p.cache_rows) : a;
+  auto key_row = [&](int a) -> int {  // cache row of scan index a (age for the ring)
+    return p.ring ? wrap(qlm - a, R) : a;
   };
-  auto key_is_local = [&](int64_t a) -> int {  // block row index or -1
+  auto key_is_local = [&](int a) -> int {  // block row index or -1
     if (!fused) return -1;
-    const int64_t pos = p.ring ? q_last - a : a;
-    return pos >= pos0 ? (int)(pos - pos0) : -1;
+    if (p.ring) return a < p.kr ? p.kr - 1 - a : -1;
+    return a >= (int)pos0 ? a - (int)pos0 : -1;
   };
 
   const __half* kc = p.k_cache + (size_t)kv * p.cache_rows * HD;
@@ -136,16 +134,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
 
   auto load_tile = [&](int t, bool kpart, bool patch_local) {
     const int buf = t & 1;
-    const int64_t a0 = a_begin + (int64_t)t * TK;
+    const int a0 = a_begin + t * TK;
     if (kpart && tid < TK) {
-      const int64_t a = a0 + tid;
+      const int a = a0 + tid;
       sm.kidx[buf][tid] = a < a_end ? key_row(a) : -1;
     }
     __half(*dst)[LD] = kpart ? sm.k : sm.v;
     const __half* src = kpart ? kc : vc;
     for (int c = tid; c < TK * CPR; c += kThreads) {
       const int key = c / CPR, part = c - key * CPR;
-      const int64_t a = a0 + key;
+      const int a = a0 + key;
       const bool in = a < a_end;
       const int loc = in ? key_is_local(a) : -1;
       if (loc >= 0) {
@@ -168,6 +166,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
     load_tile(0, false, false);
     cp_async_commit();
   }
+  // the next GEMV's first weights towards L2, one slice per CTA
+  if (tid == 0)
+    prefetch_next(p.next, ((long long)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x,
+                  (long long)gridDim.x * gridDim.y * gridDim.z);
 
   // ---- prologue: queries (and this block's K/V rows) into shared memory ----
   if (fused) {
@@ -237,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
     for (int c = tid; c < p.kr * CPR; c += kThreads) {
       const int j = c / CPR, part = c - j * CPR;
       const int64_t pos = pos0 + j;
-      const int64_t row = p.ring ? pmod(pos, p.cache_rows) : pos;
+      const int64_t row = p.ring ? (int64_t)wrap(qlm - (p.kr - 1 - j), R) : pos;
       *reinterpret_cast<uint4*>(p.k_cache + ((size_t)kv * p.cache_rows + row) * HD + part * 8) =
           *reinterpret_cast<const uint4*>(&sm.kloc[j][part * 8]);
       *reinterpret_cast<uint4*>(p.v_cache + ((size_t)kv * p.cache_rows + row) * HD + part * 8) =
@@ -298,18 +300,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
         const int gr = row0 + lr;
         const int j = gr / G;
         const int64_t qj = pos0 + j;
+        // ring: key at slot s has implied position qj - d, d = (qj - s) mod R;
+        // it is live when d < W and qj - d >= 0
+        const int qjm = p.ring ? wrap(qlm - (p.kr - 1 - j), R) : 0;
         float mx = -INFINITY;
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int key = warp * 8 + t4 * 2 + e;
-          const int64_t kr_ = sm.kidx[buf][key];
-          bool live = lr < nrows && kr_ >= 0;
+          const int ks = sm.kidx[buf][key];
+          bool live = lr < nrows && ks >= 0;
           if (live) {
             if (p.ring) {
-              const int64_t pp = qj - pmod(qj - kr_, p.cache_rows);
-              live = pp >= 0 && qj - pp < p.window;
+              const int d = wrap(qjm - ks, R);
+              live = d < W && (int64_t)d <= qj;
             } else {
-              live = kr_ <= qj;
+              live = (int64_t)ks <= qj;
             }
           }
           float& v = s[mt][hh * 2 + e];
@@ -431,45 +436,107 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
   __syncthreads();
   if (sm.ticket != p.n_chunks - 1) return;
   __threadfence();
+  // chunk weights exp(m_c - m*) / l* per row (one warp per row), in the K/V tiles
+  float* wgt = reinterpret_cast<float*>(&sm.k[0][0]);  // [nrows][n_chunks]
+  for (int r = warp; r < nrows; r += kThreads / 32) {
+    const int gr = row0 + r;
+    const int orow = (gr / G) * p.n_q + kv * G + gr % G;
+    const float* ml = p.part_ml + (size_t)orow * p.n_chunks * 2;
+    float mx = -INFINITY;
+    for (int c = lane; c < p.n_chunks; c += 32) mx = fmaxf(mx, __ldcg(ml + 2 * c));
+    mx = warp_max(mx);
+    float l = 0.f;
+    for (int c = lane; c < p.n_chunks; c += 32) {
+      const float mc = __ldcg(ml + 2 * c);
+      const float e = mc == -INFINITY ? 0.f : __expf(mc - mx);
+      wgt[r * p.n_chunks + c] = e;
+      l = fmaf(__ldcg(ml + 2 * c + 1), e, l);
+    }
+    l = warp_sum(l);
+    __syncwarp();
+    for (int c = lane; c < p.n_chunks; c += 32) wgt[r * p.n_chunks + c] /= l;
+  }
+  __syncthreads();
   for (int c = tid; c < nrows * HD; c += kThreads) {
     const int r = c / HD, d = c - r * HD;
     const int gr = row0 + r;
     const int orow = (gr / G) * p.n_q + kv * G + gr % G;
-    const float* ml = p.part_ml + (size_t)orow * p.n_chunks * 2;
-    float mstar = -INFINITY;
-    for (int ch = 0; ch < p.n_chunks; ++ch) mstar = fmaxf(mstar, __ldcg(ml + 2 * ch));
-    float l = 0.f, o = 0.f;
-    for (int ch = 0; ch < p.n_chunks; ++ch) {
-      const float mc = __ldcg(ml + 2 * ch);
-      if (mc == -INFINITY) continue;
-      const float w = __expf(mc - mstar);
-      l = fmaf(__ldcg(ml + 2 * ch + 1), w, l);
-      o = fmaf(__ldcg(p.part_acc + ((size_t)orow * p.n_chunks + ch) * HD + d), w, o);
-    }
-    p.out[(size_t)orow * HD + d] = __float2half_rn(o / l);
+    const float* acc = p.part_acc + (size_t)orow * p.n_chunks * HD + d;
+    const float* w = wgt + r * p.n_chunks;
+    float o = 0.f;
+#pragma unroll 8
+    for (int ch = 0; ch < p.n_chunks; ++ch)
+      if (w[ch] != 0.f) o = fmaf(__ldcg(acc + (size_t)ch * HD), w[ch], o);
+    p.out[(size_t)orow * HD + d] = __float2half_rn(o);
   }
   if (tid == 0) p.counters[kv * p.m_groups + mg] = 0;
 }
 
-// Separate merge of the chunk partials: one thread per (row, dim).
+// Separate merge of the chunk partials: block (output row, 128 dims), 8 warps.
+// The chunk weights exp(m_c - m*) are computed once per block in shared memory;
+// then thread (g, f) sums float4 column f over the chunks g, g + 8, ... (skipping
+// empty chunks), and the 8 group sums are added in a fixed order.
+constexpr int kCombineThreads = 256;
+constexpr int kMaxChunks = 1024;
+
 template <int HD>
-__global__ void __launch_bounds__(128) attn_combine_kernel(const AttnParams p) {
+__global__ void __launch_bounds__(kCombineThreads) attn_combine_kernel(const AttnParams p) {
+  constexpr int F4 = 32;                      // float4 columns per block (128 dims)
+  constexpr int NG = kCombineThreads / F4;    // chunk groups
+  __shared__ float wgt[kMaxChunks];
+  __shared__ float4 part[NG][F4];
+  __shared__ float red[2][kCombineThreads / 32];
   pdl_wait();
   pdl_launch_dependents();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int orow = blockIdx.x;
-  const int d = blockIdx.y * 128 + threadIdx.x;
   const float* ml = p.part_ml + (size_t)orow * p.n_chunks * 2;
-  float mstar = -INFINITY;
-  for (int ch = 0; ch < p.n_chunks; ++ch) mstar = fmaxf(mstar, ml[2 * ch]);
-  float l = 0.f, o = 0.f;
-  for (int ch = 0; ch < p.n_chunks; ++ch) {
-    const float mc = ml[2 * ch];
-    if (mc == -INFINITY) continue;
-    const float w = __expf(mc - mstar);
-    l = fmaf(ml[2 * ch + 1], w, l);
-    o = fmaf(p.part_acc[((size_t)orow * p.n_chunks + ch) * HD + d], w, o);
+  float mx = -INFINITY;
+  for (int c = tid; c < p.n_chunks; c += kCombineThreads) mx = fmaxf(mx, ml[2 * c]);
+  mx = warp_max(mx);
+  if (lane == 0) red[0][warp] = mx;
+  __syncthreads();
+  mx = red[0][0];
+#pragma unroll
+  for (int w = 1; w < kCombineThreads / 32; ++w) mx = fmaxf(mx, red[0][w]);
+  float l = 0.f;
+  for (int c = tid; c < p.n_chunks; c += kCombineThreads) {
+    const float mc = ml[2 * c];
+    const float e = mc == -INFINITY ? 0.f : __expf(mc - mx);
+    wgt[c] = e;
+    l = fmaf(ml[2 * c + 1], e, l);
   }
-  p.out[(size_t)orow * HD + d] = __float2half_rn(o / l);
+  l = warp_sum(l);
+  if (lane == 0) red[1][warp] = l;
+  __syncthreads();
+  l = 0.f;
+#pragma unroll
+  for (int w = 0; w < kCombineThreads / 32; ++w) l += red[1][w];
+  const int g = tid / F4, f = tid % F4;
+  const float4* acc =
+      reinterpret_cast<const float4*>(p.part_acc + (size_t)orow * p.n_chunks * HD) + blockIdx.y * F4 + f;
+  float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+  for (int c = g; c < p.n_chunks; c += NG) {
+    const float w = wgt[c];
+    if (w != 0.f) {
+      const float4 v = acc[(size_t)c * (HD / 4)];
+      o.x = fmaf(v.x, w, o.x), o.y = fmaf(v.y, w, o.y), o.z = fmaf(v.z, w, o.z), o.w = fmaf(v.w, w, o.w);
+    }
+  }
+  part[g][f] = o;
+  __syncthreads();
+  if (tid < F4) {
+    float4 t = part[0][tid];
+#pragma unroll
+    for (int q = 1; q < NG; ++q) {
+      const float4 v = part[q][tid];
+      t.x += v.x, t.y += v.y, t.z += v.z, t.w += v.w;
+    }
+    __half* out = p.out + (size_t)orow * HD + blockIdx.y * 128 + 4 * tid;
+    *reinterpret_cast<__half2*>(out) = __floats2half2_rn(t.x / l, t.y / l);
+    *reinterpret_cast<__half2*>(out + 2) = __floats2half2_rn(t.z / l, t.w / l);
+  }
 }
 
 template <int HD>
@@ -479,6 +546,9 @@ cudaError_t launch_attn_t(const AttnParams& p, cudaStream_t st, bool pdl) {
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(attn_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(attn_kernel<HD>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     configured = true;
   }
@@ -499,7 +569,7 @@ template <int HD>
 cudaError_t launch_combine_t(const AttnParams& p, cudaStream_t st, bool pdl) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.kr * p.n_q, HD / 128);
-  cfg.blockDim = dim3(128);
+  cfg.blockDim = dim3(kCombineThreads);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -87,12 +87,103 @@ Q4G_DEV void block_dot(const uint4 q, const uint4 (&xq)[4], float& a0, float& a1
   }
 }
 
+// 4-way byte dot products with 32-bit accumulation (unsigned x unsigned and
+// unsigned x signed).
+Q4G_DEV int dp4a_uu(uint32_t a, uint32_t b, int c) {
+  int r;
+  asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+Q4G_DEV int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int r;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+
 // Column order of the x layout above: slot s (0..31) of a block holds column
 // kXPerm[s]; quarter k = slots 8k..8k+7.
 __host__ __device__ constexpr int xperm(int s) {
   // within a quarter: 0:4k 1:4k+2 2:4k+16 3:4k+18 4:4k+1 5:4k+3 6:4k+17 7:4k+19
   return 4 * (s >> 3) + ((s & 7) == 0 ? 0 : (s & 7) == 1 ? 2 : (s & 7) == 2 ? 16 : (s & 7) == 3 ? 18
                        : (s & 7) == 4 ? 1 : (s & 7) == 5 ? 3 : (s & 7) == 6 ? 17 : 19);
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier and 1-D bulk copies (TMA engine), sm_90+ PTX.
+// ---------------------------------------------------------------------------
+Q4G_DEV uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+Q4G_DEV void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+Q4G_DEV void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+Q4G_DEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+Q4G_DEV void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// One poll of `phase` of `bar`. With the suspend-time hint the thread sleeps in
+// the instruction until the phase completes or ~0.1 ms pass, instead of spinning.
+Q4G_DEV bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(phase), "r"(100000u)
+      : "memory");
+  return ok != 0;
+}
+// Copy `bytes` (multiple of 16, 16-byte aligned addresses) global -> shared;
+// completion is counted on `bar`.
+Q4G_DEV void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+// As bulk_g2s with an L2 eviction-priority policy (createpolicy) for the source.
+Q4G_DEV void bulk_g2s_hint(void* dst, const void* src, uint32_t bytes, uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], "
+      "%4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+// Weights are read once per step: evict them from L2 first.
+Q4G_DEV uint64_t policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+// Asynchronous L2 prefetch of [p, p + bytes) (p 16-byte aligned; a tail below
+// 16 bytes is skipped). A hint: nothing waits for it.
+Q4G_DEV void l2_prefetch(const void* p, uint64_t bytes) {
+  const char* c = static_cast<const char*>(p);
+  while (bytes >= 16) {
+    const uint32_t n = (uint32_t)(bytes < 32768 ? bytes : 32768) & ~15u;
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(c), "r"(n) : "memory");
+    c += n;
+    bytes -= n;
+  }
+}
+Q4G_DEV uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Wait for `phase` of `bar` for at most `limit_ns`; false if the limit ran out.
+Q4G_DEV bool mbar_wait_bounded(uint64_t* bar, uint32_t phase, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, phase)) return true;
+  const uint64_t t0 = global_ns();
+  for (int it = 0; it < kSpinLimit; ++it) {
+    if (mbar_try_wait(bar, phase)) return true;
+    if (global_ns() - t0 > limit_ns) break;
+  }
+  return false;
 }
 
 // ---------------------------------------------------------------------------
@@ -110,8 +201,9 @@ Q4G_DEV float warp_max(float v) {
   return v;
 }
 
-// Block-wide sum for blockDim.x == kThreads; `red` holds >= 32 floats. All
-// threads receive the result. Summation order is fixed.
+// Block-wide sum for blockDim.x == NT; `red` holds >= 32 floats. All threads
+// receive the result. Summation order is fixed.
+template <int NT = kThreads>
 Q4G_DEV float block_sum(float v, float* red) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   v = warp_sum(v);
@@ -120,7 +212,7 @@ Q4G_DEV float block_sum(float v, float* red) {
   __syncthreads();
   float t = 0.f;
 #pragma unroll
-  for (int i = 0; i < kThreads / 32; ++i) t += red[i];
+  for (int i = 0; i < NT / 32; ++i) t += red[i];
   return t;
 }
 

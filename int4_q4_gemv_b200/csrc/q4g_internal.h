@@ -17,7 +17,22 @@ struct GemvSeg {
 enum GemvPro { PRO_X16 = 0, PRO_RESID = 1 };
 enum GemvEpi { EPI_STORE = 0, EPI_GEGLU = 1, EPI_HEAD = 2 };
 
+// The weights the next GEMV of the step reads first, for an L2 prefetch issued
+// by the current kernel once its own loads are in flight: the next GEMV's
+// warp w streams units [w * n_units / tw, (w + 1) * n_units / tw) in order, and
+// the first `frac` of every such range is prefetched (tw == 0: nothing).
+struct NextGemv {
+  GemvSeg seg[3];
+  int32_t nseg;
+  int32_t k;
+  int32_t n_units;  // row pairs (GeGLU: gate row u with up row u)
+  int32_t geglu;
+  int32_t tw;       // warps of the next GEMV's grid
+  float frac;
+};
+
 struct GemvParams {
+  NextGemv next;
   GemvSeg seg[3];
   int32_t nseg;
   int32_t k;        // columns
@@ -53,15 +68,28 @@ struct GemvParams {
   int32_t* am_idx;   // [kMaxRows][grid]
   int32_t* counter;  // one int, zero between launches
   int32_t* argmax_out;
+  // bulk-copy pipeline (set by the launcher)
+  int32_t kc;           // columns per streamed item
+  int32_t ns;           // stages per warp
+  int32_t stage_bytes;  // codes then scales of one item (2 rows)
+  int32_t* err;         // error word: bit 0 = a bounded wait gave up
+  uint64_t wait_ns;     // limit of one bounded wait
+  int32_t stall_test;   // 1: the first stage of the warp that owns unit 0 never completes (tests the timeout path)
 };
 
 // Largest number of activation rows one GEMV launch can stage for k columns.
 int gemv_max_rows(int k);
 size_t gemv_smem_bytes(int krm, int k);
 cudaError_t launch_gemv(const GemvParams& p, cudaStream_t st, bool pdl);
+// Descriptor of GEMV `p` as the next GEMV of a prefetch (tw = 0 if p does not
+// take the streamed path).
+NextGemv gemv_next_desc(const GemvParams& p, float frac);
+// Device address of the library's error word (bit 0: a bounded wait gave up).
+int32_t* device_error_word();
 
 // ------------------------------------------------------------ attention ----
 struct AttnParams {
+  NextGemv next;
   // queries: either the fused QKV epilogue (qkv != NULL) or ready fp16 q
   const float* qkv;      // [kr][qkv_stride] raw projections (q | k | v)
   int64_t qkv_stride;

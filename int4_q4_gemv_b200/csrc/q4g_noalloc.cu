@@ -62,6 +62,7 @@ extern "C" q4g_status q4g_flash_decode_ring_noalloc(const uint16_t* q, int32_t n
   if (head_dim != 256 && head_dim != 512) return bad(Q4G_EINVAL, "head_dim must be 256 or 512");
   if (n_q < 1 || n_kv < 1 || n_q % n_kv) return bad(Q4G_EINVAL, "n_q must be a positive multiple of n_kv");
   if (ring < 1 || window < 1 || window > ring) return bad(Q4G_EINVAL, "need 1 <= window <= ring");
+  if (ring > ((int64_t)1 << 30)) return bad(Q4G_ERANGE, "ring > 2^30");
   if (pos < 0) return bad(Q4G_ERANGE, "pos < 0");
   if (!aligned16(q) || !aligned16(k_ring) || !aligned16(v_ring) || !aligned16(out))
     return bad(Q4G_EINVAL, "misaligned pointer");

@@ -219,6 +219,26 @@ def test_capacity_invariance_and_graph_equivalence_bitwise():
     assert np.array_equal(outs[0], outs[2])
 
 
+def test_bounded_wait_gives_up_and_reports_timeout():
+    """Failure path without a fault: one pipeline stage of the step's first GEMV
+    expects bytes that never arrive; its bounded wait gives up after 20 ms, the
+    step completes, q4g_model_check reports Q4G_ETIMEOUT, and the next step on the
+    same context is clean and correct again."""
+    cfg = WRAP
+    p = Pair(cfg, seed=6, variant=0, capacity=64)
+    Q.q4g_model_set_option(p.gpu.handle, Q.Q4G_OPT_TEST_STALL, 1)
+    Q.q4g_decode_step(p.gpu.handle, p.gc.handle, 3, 0, 0, 0, sp())
+    with pytest.raises(Q.Q4GError) as e:
+        Q.q4g_model_check(p.gpu.handle, sp())
+    assert e.value.status == Q.Q4G_ETIMEOUT
+    Q.q4g_model_check(p.gpu.handle, sp())          # the word was cleared
+    # position 0 again, now cleanly, then one more step; both match the oracle
+    for pos, tok in ((0, 3), (1, 9)):
+        got, ga, ref, ra = p.step_token(tok, pos)
+        check_logits(got, ref, f"after timeout pos {pos}")
+    Q.q4g_model_check(p.gpu.handle, sp())
+
+
 def test_host_api_and_range_errors(tiny):
     cfg = WL.TINY
     g, c = tiny.gpu, tiny.gc
