@@ -98,6 +98,24 @@ q4g_status q4g_q4_0_unpack(const uint8_t* qs, const uint16_t* scales, int64_t ro
 q4g_status q4g_gemv(const uint8_t* qs, const uint16_t* scales, int64_t n, int64_t k,
                     const uint16_t* x_f16, int32_t nrhs, float* y, q4g_stream_t stream);
 
+/* Process-wide choice of the q4_0 GEMV kernel, for tuning and tests (not on
+ * the pages). All kernels compute the same operation within the same error
+ * bound; the default picks per shape:
+ *   Q4G_GEMV_AUTO          shape-based choice (default; Q4G_GEMV_KERNEL=cs|ws|reg
+ *                          in the environment overrides it at first use),
+ *   Q4G_GEMV_COLUMN_SPLIT  integer dot, x digits resident per chunk, one
+ *                          contiguous bulk-copy stream per CTA (k % 256 == 0,
+ *                          <= 2 activation rows, 16-byte aligned operands),
+ *   Q4G_GEMV_WARP_STREAM   per-warp bulk-copy rings (k % 256 == 0),
+ *   Q4G_GEMV_REGISTER      plain streaming loads (any k % 32 == 0).
+ * A kernel that cannot take a call falls back down this list. Affects launches
+ * made (and CUDA graphs captured) after the call. Q4G_EINVAL for other kinds. */
+#define Q4G_GEMV_AUTO 0
+#define Q4G_GEMV_COLUMN_SPLIT 1
+#define Q4G_GEMV_WARP_STREAM 2
+#define Q4G_GEMV_REGISTER 3
+q4g_status q4g_set_gemv_kernel(int32_t kind);
+
 /* Workspace for the split-KV flash-decode entry points below (bytes, >= 256). */
 size_t q4g_flash_decode_workspace_bytes(int32_t n_q_heads, int32_t head_dim);
 

@@ -490,6 +490,11 @@ extern "C" q4g_status q4g_q4_0_unpack(const uint8_t* qs, const uint16_t* scales,
   return Q4G_OK;
 }
 
+extern "C" q4g_status q4g_set_gemv_kernel(int32_t kind) {
+  if (!set_gemv_kernel_choice(kind)) return fail(Q4G_EINVAL, "GEMV kernel kind must be 0..3");
+  return Q4G_OK;
+}
+
 extern "C" q4g_status q4g_gemv(const uint8_t* qs, const uint16_t* scales, int64_t n, int64_t k,
                                const uint16_t* x_f16, int32_t nrhs, float* y, q4g_stream_t stream) {
   if (n < 0 || k <= 0 || k % 32 || n > INT32_MAX || k > (1 << 20))

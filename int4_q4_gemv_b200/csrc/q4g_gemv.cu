@@ -25,6 +25,9 @@
 
 #include <stdlib.h>
 
+#include <algorithm>
+#include <atomic>
+
 namespace q4g {
 
 namespace {
@@ -111,41 +114,37 @@ Q4G_DEV void put_x(__half* xs_h, int nb, int j, int col, __half v) {
   xs_h[((size_t)(j * 4 + (s >> 3)) * nb + blk) * 8 + (s & 7)] = v;
 }
 
-// Activations of the step into shared memory, in the order the nibble
-// unpacking consumes them, plus the per-block constant 72 * sum(x) that removes
-// the +64 of the unpacked codes and the -8 of the code offset.
+// The activations of the step, produced in groups of 4 consecutive columns:
 //   PRO_X16:   x = the fp16 input rows
 //   PRO_RESID: r_new = (r_in + rmsnorm(delta) * w_delta) * scale,
 //              x = fp16(rmsnorm(r_new) * w_x); block 0 stores r_new (and the dump)
-// Ends with __syncthreads().
-template <int KRM, int NT = kThreads, bool NAT = false>
-Q4G_DEV void stage_x(const GemvParams& p, uint4* xs, float* cblk, float* misc) {
-  const int k = p.k, nb = k >> 5, tid = threadIdx.x;
-  __half* xs_h = reinterpret_cast<__half*>(xs);
-  // NAT: x row j in natural column order at xs_h + j * k, no block constants
-  auto put = [&](int j, int col, __half v) {
-    if (NAT)
-      xs_h[(size_t)j * k + col] = v;
-    else
-      put_x(xs_h, nb, j, col, v);
-  };
+// emit(j, c4, h, valid) receives columns 4*c4 .. 4*c4+3 of row j. Every thread
+// calls emit the same number of times per row (valid = false past the end), so
+// emit may use warp shuffles; with NT % 8 == 0 the 8 groups of one 32-column
+// block sit in 8 consecutive lanes. Needs k <= 8192 for PRO_RESID.
+template <int KRM, int NT, class Emit>
+Q4G_DEV void produce_x(const GemvParams& p, float* misc, Emit&& emit) {
+  const int k = p.k, tid = threadIdx.x, n4 = k >> 2;
   for (int j = 0; j < KRM; ++j) {
     if (j >= p.kr) break;
     if (p.pro == PRO_X16) {
       const __half* xr = p.x + (size_t)j * p.x_stride;
-      if ((((uintptr_t)xr) & 15) == 0) {
-        for (int c8 = tid; c8 < (k >> 3); c8 += NT) {
-          const uint4 v = *reinterpret_cast<const uint4*>(xr + 8 * c8);
-          if (NAT) {
-            *reinterpret_cast<uint4*>(xs_h + (size_t)j * k + 8 * c8) = v;
-          } else {
-            const __half* h = reinterpret_cast<const __half*>(&v);
+      const bool vec = (((uintptr_t)xr) & 7) == 0;
+      const int iters = (n4 + NT - 1) / NT;
+      for (int i = 0; i < iters; ++i) {
+        const int c4 = tid + i * NT;
+        const bool valid = c4 < n4;
+        __half h[4];
+        if (valid && vec) {
+          const uint2 v = *reinterpret_cast<const uint2*>(xr + 4 * c4);
+          const __half* hv = reinterpret_cast<const __half*>(&v);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) put_x(xs_h, nb, j, 8 * c8 + e, h[e]);
-          }
+          for (int e = 0; e < 4; ++e) h[e] = hv[e];
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) h[e] = valid ? xr[4 * c4 + e] : __float2half_rn(0.f);
         }
-      } else {
-        for (int c = tid; c < k; c += NT) put(j, c, xr[c]);
+        emit(j, c4, h, valid);
       }
     } else {
       // k <= 8192: each thread keeps its float4s of r_new in registers
@@ -154,7 +153,6 @@ Q4G_DEV void stage_x(const GemvParams& p, uint4* xs, float* cblk, float* misc) {
       const float4* dl = p.delta ? reinterpret_cast<const float4*>(p.delta + (size_t)j * k) : nullptr;
       const float4* wd = reinterpret_cast<const float4*>(p.w_delta);
       const float4* wx = reinterpret_cast<const float4*>(p.w_x);
-      const int n4 = k >> 2;
       float4 rn[R4], dv[R4];
       float ss = 0.f;
 #pragma unroll
@@ -204,31 +202,104 @@ Q4G_DEV void stage_x(const GemvParams& p, uint4* xs, float* cblk, float* misc) {
 #pragma unroll
       for (int i = 0; i < R4; ++i) {
         const int c4 = tid + i * NT;
-        if (c4 < n4) {
+        const bool valid = c4 < n4;
+        __half h[4];
+        if (valid) {
           const float4 w = wx[c4];
-          put(j, 4 * c4 + 0, __float2half_rn(__fmul_rn(__fmul_rn(rn[i].x, inv_r), w.x)));
-          put(j, 4 * c4 + 1, __float2half_rn(__fmul_rn(__fmul_rn(rn[i].y, inv_r), w.y)));
-          put(j, 4 * c4 + 2, __float2half_rn(__fmul_rn(__fmul_rn(rn[i].z, inv_r), w.z)));
-          put(j, 4 * c4 + 3, __float2half_rn(__fmul_rn(__fmul_rn(rn[i].w, inv_r), w.w)));
+          h[0] = __float2half_rn(__fmul_rn(__fmul_rn(rn[i].x, inv_r), w.x));
+          h[1] = __float2half_rn(__fmul_rn(__fmul_rn(rn[i].y, inv_r), w.y));
+          h[2] = __float2half_rn(__fmul_rn(__fmul_rn(rn[i].z, inv_r), w.z));
+          h[3] = __float2half_rn(__fmul_rn(__fmul_rn(rn[i].w, inv_r), w.w));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) h[e] = __float2half_rn(0.f);
         }
+        emit(j, c4, h, valid);
       }
     }
+  }
+}
+
+// Activations into shared memory in the order the fp16 nibble unpacking
+// consumes them, plus the per-block constant 72 * sum(x) that removes the +64
+// of the unpacked codes and the -8 of the code offset. Ends with __syncthreads().
+template <int KRM, int NT = kThreads>
+Q4G_DEV void stage_x(const GemvParams& p, uint4* xs, float* cblk, float* misc) {
+  const int nb = p.k >> 5, tid = threadIdx.x;
+  __half* xs_h = reinterpret_cast<__half*>(xs);
+  produce_x<KRM, NT>(p, misc, [&](int j, int c4, const __half (&h)[4], bool valid) {
+    if (valid) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) put_x(xs_h, nb, j, 4 * c4 + e, h[e]);
+    }
+  });
+  __syncthreads();
+  for (int t = tid; t < p.kr * nb; t += NT) {
+    const int j = t / nb, blk = t - j * nb;
+    float sx = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const __half* h = xs_h + ((size_t)(j * 4 + q) * nb + blk) * 8;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) sx += __half2float(h[e]);
+    }
+    cblk[t] = 72.0f * sx;
   }
   __syncthreads();
-  if (!NAT) {
-    for (int t = tid; t < p.kr * nb; t += NT) {
-      const int j = t / nb, blk = t - j * nb;
-      float sx = 0.f;
+}
+
+// Activations as the digits of the integer dot product (block_dot_int):
+// thread (block blk, group sub) turns columns 4*sub..4*sub+3 of the block into
+// one 32-bit word per digit; the block's largest exponent and digit sums are
+// reduced over the block's 8 lanes. Ends with __syncthreads().
+template <int KRM, int NT>
+Q4G_DEV void stage_digits(const GemvParams& p, uint4* dg, int4* bc, float* misc) {
+  const int nb = p.k >> 5;
+  uint32_t* dw = reinterpret_cast<uint32_t*>(dg);
+  produce_x<KRM, NT>(p, misc, [&](int j, int c4, const __half (&h)[4], bool valid) {
+    const int blk = c4 >> 3, sub = c4 & 7;
+    int Ee[4], M[4], em = 1;
+    uint32_t neg = 0;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const __half* h = xs_h + ((size_t)(j * 4 + q) * nb + blk) * 8;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) sx += __half2float(h[e]);
-      }
-      cblk[t] = 72.0f * sx;
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t b = __half_as_ushort(h[e]);
+      const int E = (b >> 10) & 31;
+      Ee[e] = E ? E : 1;
+      M[e] = (int)(b & 1023) | (E ? 1024 : 0);
+      neg |= (b >> 15) << e;
+      em = max(em, Ee[e]);
     }
-    __syncthreads();
-  }
+    em = max(em, __shfl_xor_sync(0xffffffffu, em, 1));
+    em = max(em, __shfl_xor_sync(0xffffffffu, em, 2));
+    em = max(em, __shfl_xor_sync(0xffffffffu, em, 4));
+    uint32_t w0 = 0, w1 = 0, w2 = 0;
+    int s0 = 0, s1 = 0, s2 = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int sh = 12 + Ee[e] - em;  // <= 12
+      int X = sh >= 0 ? (M[e] << sh) : sh > -12 ? (M[e] + (1 << (-sh - 1))) >> -sh : 0;
+      if ((neg >> e) & 1) X = -X;
+      const int d0 = X & 255, d1 = (X >> 8) & 255, d2 = X >> 16;
+      w0 |= (uint32_t)d0 << (8 * e);
+      w1 |= (uint32_t)d1 << (8 * e);
+      w2 |= (uint32_t)(d2 & 255) << (8 * e);
+      s0 += d0, s1 += d1, s2 += d2;
+    }
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+      s0 += __shfl_xor_sync(0xffffffffu, s0, o);
+      s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+      s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+    }
+    if (valid) {
+      const int hh = sub >> 2, wd = sub & 3;
+      dw[((size_t)(j * 6 + 0 + hh) * nb + blk) * 4 + wd] = w0;
+      dw[((size_t)(j * 6 + 2 + hh) * nb + blk) * 4 + wd] = w1;
+      dw[((size_t)(j * 6 + 4 + hh) * nb + blk) * 4 + wd] = w2;
+      if (sub == 0) bc[j * nb + blk] = make_int4(-8 * s0, -8 * s1, -8 * s2, (em - 37 + 127) << 23);
+    }
+  });
+  __syncthreads();
 }
 
 template <int KRM>
@@ -492,33 +563,9 @@ Q4G_DEV void issue_item(const GemvParams& p, int u, int c, unsigned char* st, ui
 // and each S_t is a chain of 4-way byte dot products (dp4a) of the raw codes
 // with the digits, started at -8 * sum_i d_t,i. Every S_t is exact in int32.
 // Layout per x row j: dg[j][2t + h][blk] holds digit t of columns 16h..16h+15
-// of block blk (16 bytes), bc[j][blk] = (-8 D0, -8 D1, -8 D2, bits of 2^(Emax-37)).
+// of block blk (16 bytes), bc[j][blk] = (-8 D0, -8 D1, -8 D2, bits of 2^(Emax-37)),
+// written by stage_digits.
 // ---------------------------------------------------------------------------
-template <int NT>
-Q4G_DEV void stage_digits(const GemvParams& p, const __half* xn, uint4* dg, int4* bc) {
-  const int k = p.k, nb = k >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  unsigned char* db = reinterpret_cast<unsigned char*>(dg);
-  for (int t = warp; t < p.kr * nb; t += NT / 32) {
-    const int j = t / nb, blk = t - j * nb;
-    const uint32_t h = __half_as_ushort(xn[(size_t)j * k + blk * 32 + lane]);
-    const int E = (h >> 10) & 31, Ee = E ? E : 1;
-    const int M = (int)(h & 1023) | (E ? 1024 : 0);
-    const int emax = (int)__reduce_max_sync(0xffffffffu, (unsigned)Ee);
-    const int sh = 12 + Ee - emax;  // <= 12
-    int X = sh >= 0 ? (M << sh) : sh > -12 ? (M + (1 << (-sh - 1))) >> -sh : 0;
-    if (h & 0x8000) X = -X;
-    const int d0 = X & 255, d1 = (X >> 8) & 255, d2 = X >> 16;
-    const int hh = lane >> 4, col = lane & 15;
-    db[((size_t)(j * 6 + 0 + hh) * nb + blk) * 16 + col] = (unsigned char)d0;
-    db[((size_t)(j * 6 + 2 + hh) * nb + blk) * 16 + col] = (unsigned char)d1;
-    db[((size_t)(j * 6 + 4 + hh) * nb + blk) * 16 + col] = (unsigned char)d2;
-    const int s0 = __reduce_add_sync(0xffffffffu, d0);
-    const int s1 = __reduce_add_sync(0xffffffffu, d1);
-    const int s2 = __reduce_add_sync(0xffffffffu, d2);
-    if (lane == 0) bc[j * nb + blk] = make_int4(-8 * s0, -8 * s1, -8 * s2, (emax - 37 + 127) << 23);
-  }
-}
-
 Q4G_DEV float block_dot_int(const uint4 q, const uint4 (&g)[6], const int4 c) {
   const uint32_t w[4] = {q.x, q.y, q.z, q.w};
   int s0 = c.x, s1 = c.y, s2 = c.z;
@@ -542,7 +589,7 @@ enum : int { DOT_FMA_HALF = 0, DOT_FMA = 1, DOT_INT = 2 };
 
 __host__ __device__ inline size_t x_region_bytes(int dot, int krm, int k) {
   const size_t nb = (size_t)k / 32;
-  return dot == DOT_INT ? (size_t)krm * nb * (96 + 16 + 64) : (size_t)krm * nb * (64 + 4);
+  return dot == DOT_INT ? (size_t)krm * nb * (96 + 16) : (size_t)krm * nb * (64 + 4);
 }
 
 template <int KRM, int DOT>
@@ -554,7 +601,6 @@ __global__ void __launch_bounds__(kWarpThreads, 1) gemv_q4_tma_kernel(const Gemv
   uint4* xs = reinterpret_cast<uint4*>(ws_smem);                        // FMA: [KRM][4][nb]; INT: dg [KRM][6][nb]
   float* cblk = reinterpret_cast<float*>(xs + (size_t)KRM * 4 * nb);     // FMA: [KRM][nb]
   int4* bc = reinterpret_cast<int4*>(xs + (size_t)KRM * 6 * nb);         // INT: [KRM][nb]
-  __half* xn = reinterpret_cast<__half*>(bc + (size_t)KRM * nb);         // INT: [KRM][k]
   float* misc = reinterpret_cast<float*>(ws_smem + x_region_bytes(DOT, KRM, k));  // 64 floats
   float* bestv = misc + 64;                                              // [kWarps]
   int* besti = reinterpret_cast<int*>(bestv + kWarps);                   // [kWarps]
@@ -586,9 +632,7 @@ __global__ void __launch_bounds__(kWarpThreads, 1) gemv_q4_tma_kernel(const Gemv
 
   pdl_wait();
   if (DOT == DOT_INT) {
-    stage_x<KRM, kWarpThreads, true>(p, reinterpret_cast<uint4*>(xn), nullptr, misc);
-    stage_digits<kWarpThreads>(p, xn, xs, bc);
-    __syncthreads();
+    stage_digits<KRM, kWarpThreads>(p, xs, bc, misc);
   } else {
     stage_x<KRM, kWarpThreads>(p, xs, cblk, misc);
   }
@@ -848,6 +892,386 @@ bool plan_tma(GemvParams& p, int& dot) {
   return false;
 }
 
+// ---------------------------------------------------------------------------
+// Column-split integer GEMV (the default for k % 256 == 0, up to 2 activation
+// rows).
+//
+// Each CTA owns a contiguous, balanced range of units (R rows each, R = 8, 4
+// or 2; a GeGLU unit is R/2 gate rows and the same R/2 up rows) and streams it
+// in order through a ring of NS stages: one producer warp issues 2 (GeGLU: 4)
+// large 1-D bulk copies per stage (the unit's codes, then its scales), so every
+// SM reads one contiguous region, the access pattern that reaches the copy
+// bandwidth of HBM. The k columns are cut into NC chunks of 32 blocks (1024
+// columns); consumer warp (g, c) owns chunk c and takes the stages g, g + G,
+// ... (G = 16 / NC groups). Lane b of that warp holds the integer digits of
+// x for block 32c + b in registers for the whole kernel (block_dot_int) and
+// dots them with the R rows of every stage it takes. The R partial sums of a
+// warp go to shared memory with a transposing butterfly; the last of the NC
+// warps to finish a stage adds the chunk partials in chunk order
+// (deterministic), runs the epilogue and hands the stage back, so the producer
+// only waits and refills.
+// ---------------------------------------------------------------------------
+constexpr int kCsMaxConsumers = 16;
+constexpr int kCsThreads = (kCsMaxConsumers + 1) * 32;
+constexpr int kCsMaxStages = 16;
+
+__host__ __device__ inline size_t cs_red_floats(int ns, int nc, int rows, int krm) {
+  return (size_t)ns * nc * rows * krm;
+}
+__host__ __device__ inline size_t cs_fixed_bytes(int krm, int k, int ns, int nc, int rows) {
+  const size_t nb = (size_t)k / 32;
+  const size_t red = (cs_red_floats(ns, nc, rows, krm) * 4 + 15) & ~(size_t)15;
+  return (size_t)krm * nb * 112 + 64 * 4 + red + 128 + 2 * kCsMaxStages * 8;
+}
+
+// Sum v[0..R) over the 32 lanes: after the butterfly, lanes with (lane & (32/R
+// - 1)) == 0 hold the total of row cs_row<R>(lane).
+template <int R>
+Q4G_DEV float cs_reduce_rows(float (&v)[R], int lane) {
+#pragma unroll
+  for (int h = R / 2, o = 16; h >= 1; h >>= 1, o >>= 1) {
+    const bool upper = lane & o;
+#pragma unroll
+    for (int i = 0; i < h; ++i) {
+      const float send = upper ? v[i] : v[i + h];
+      const float keep = upper ? v[i + h] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  float t = v[0];
+#pragma unroll
+  for (int o = 16 / R; o >= 1; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+  return t;
+}
+template <int R>
+Q4G_DEV int cs_row(int lane) {
+  int r = 0;
+#pragma unroll
+  for (int h = R / 2, o = 16; h >= 1; h >>= 1, o >>= 1) r += (lane & o) ? h : 0;
+  return r;
+}
+
+// Wait for `phase` of `bar` until done, until another warp gave up (flag set),
+// or until limit_ns pass (then this warp sets the flag and the error word).
+Q4G_DEV bool cs_wait(uint64_t* bar, uint32_t phase, const GemvParams& p, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, phase)) return true;
+  const uint64_t t0 = global_ns();
+  for (int it = 0; it < kSpinLimit; ++it) {
+    if (*abort_flag) return false;
+    if (mbar_try_wait(bar, phase)) return true;
+    if (global_ns() - t0 > p.wait_ns) break;
+  }
+  *abort_flag = 1;
+  atomicOr(p.err, 1);
+  return false;
+}
+
+// Issue the bulk copies of unit u into stage `st` ([R rows of codes][R rows of scales]).
+template <int R>
+Q4G_DEV void cs_issue(const GemvParams& p, int u, unsigned char* st, uint64_t* bar, bool poison, uint64_t pol) {
+  const int kh = p.k >> 1, nb = p.k >> 5;
+  if (p.epi == EPI_GEGLU) {
+    const int r0 = (R / 2) * u;
+    const uint32_t qb = (uint32_t)(R / 2) * kh, sb = (uint32_t)(R / 2) * nb * 2;
+    mbar_arrive_expect_tx(bar, 2 * (qb + sb) + (poison ? 16u : 0u));
+    bulk_g2s_hint(st, p.seg[0].qs + (size_t)r0 * kh, qb, bar, pol);
+    bulk_g2s_hint(st + qb, p.seg[1].qs + (size_t)r0 * kh, qb, bar, pol);
+    bulk_g2s_hint(st + 2 * qb, p.seg[0].sc + (size_t)r0 * nb, sb, bar, pol);
+    bulk_g2s_hint(st + 2 * qb + sb, p.seg[1].sc + (size_t)r0 * nb, sb, bar, pol);
+  } else {
+    const GemvSeg* sg;
+    int r0;
+    seg_row(p, R * u, sg, r0);
+    const int n = min(R, sg->rows - r0);
+    const uint32_t qb = (uint32_t)n * kh, sb = (uint32_t)n * nb * 2;
+    mbar_arrive_expect_tx(bar, qb + sb + (poison ? 16u : 0u));
+    bulk_g2s_hint(st, sg->qs + (size_t)r0 * kh, qb, bar, pol);
+    bulk_g2s_hint(st + (size_t)R * kh, sg->sc + (size_t)r0 * nb, sb, bar, pol);
+  }
+}
+
+template <int KRM, int R>
+__global__ void __launch_bounds__(kCsThreads, 1) gemv_q4_cs_kernel(const GemvParams p) {
+  extern __shared__ __align__(16) unsigned char cs_smem[];
+  const int k = p.k, nb = k >> 5, kh = k >> 1, NS = p.ns, NC = p.nchunk, G = p.groups;
+  uint4* dg = reinterpret_cast<uint4*>(cs_smem);                          // [KRM][6][nb]
+  int4* bc = reinterpret_cast<int4*>(dg + (size_t)KRM * 6 * nb);          // [KRM][nb]
+  float* misc = reinterpret_cast<float*>(bc + (size_t)KRM * nb);          // 64 floats
+  float* red = misc + 64;                                                 // [NS][NC][R][KRM]
+  const size_t red_bytes = (cs_red_floats(NS, NC, R, KRM) * 4 + 15) & ~(size_t)15;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(
+      ((uintptr_t)(reinterpret_cast<unsigned char*>(red) + red_bytes) + 127) & ~(uintptr_t)127);
+  uint64_t* full = bars;                    // [kCsMaxStages]
+  uint64_t* empty = bars + kCsMaxStages;    // [kCsMaxStages]
+  unsigned char* stages = reinterpret_cast<unsigned char*>(bars + 2 * kCsMaxStages);
+  __shared__ int s_abort, s_ticket;
+  __shared__ int s_cnt[kCsMaxStages];       // consumer warps done with a stage
+  __shared__ float s_bestv[kCsMaxConsumers];
+  __shared__ int s_besti[kCsMaxConsumers];
+
+  // kCsThreads threads: consumer warps 0 .. NC*G-1, producer warp kCsMaxConsumers,
+  // the rest only help stage x
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n_cons = NC * G;
+  const bool producer = warp == kCsMaxConsumers;
+  const int u0 = (int)((long long)blockIdx.x * p.n_units / gridDim.x);
+  const int n_st = (int)((long long)(blockIdx.x + 1) * p.n_units / gridDim.x) - u0;
+  const size_t SB = (size_t)p.stage_bytes;
+  const uint64_t pol = policy_evict_first();
+  int issued = 0;
+
+  if (tid == 0) s_abort = 0;
+  if (tid < kCsMaxStages) s_cnt[tid] = 0;
+  if (tid < kCsMaxConsumers) s_bestv[tid] = -INFINITY, s_besti[tid] = 0x7fffffff;
+  if (producer && lane == 0) {
+    for (int s = 0; s < NS; ++s) mbar_init(&full[s], 1), mbar_init(&empty[s], 1);
+    fence_mbar_init();
+    for (; issued < NS && issued < n_st; ++issued)
+      cs_issue<R>(p, u0 + issued, stages + issued * SB, &full[issued],
+                  p.stall_test && u0 == 0 && issued == 0, pol);  // the CTA owning unit 0
+  }
+  pdl_wait();
+  stage_digits<KRM, kCsThreads>(p, dg, bc, misc);  // ends with __syncthreads
+  pdl_launch_dependents();
+  volatile int* abort_flag = &s_abort;
+
+  if (warp < n_cons) {
+    // ---------------- consumer: chunk c, stages g, g + G, ... ----------------
+    const int c = warp % NC, g = warp / NC;
+    const int blk = 32 * c + lane;
+    const bool has = blk < nb;
+    uint4 xg[KRM][6];
+    int4 cv[KRM];
+    float xsc[KRM];
+#pragma unroll
+    for (int j = 0; j < KRM; ++j) {
+      if (has && (KRM == 1 || j < p.kr)) {
+#pragma unroll
+        for (int q = 0; q < 6; ++q) xg[j][q] = dg[(size_t)(j * 6 + q) * nb + blk];
+        cv[j] = bc[j * nb + blk];
+      } else {
+#pragma unroll
+        for (int q = 0; q < 6; ++q) xg[j][q] = make_uint4(0, 0, 0, 0);
+        cv[j] = make_int4(0, 0, 0, 0);
+      }
+      xsc[j] = __int_as_float(cv[j].w);
+    }
+    float best_v = -INFINITY;
+    int best_i = 0x7fffffff;
+    int s = g % NS;
+    uint32_t ph = (uint32_t)((g / NS) & 1);
+    for (int t = g; t < n_st; t += G) {
+      if (!*abort_flag) cs_wait(&full[s], ph, p, abort_flag);
+      const unsigned char* st = stages + s * SB;
+      float v[KRM][R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        float a[KRM];
+#pragma unroll
+        for (int j = 0; j < KRM; ++j) a[j] = 0.f;
+        if (has) {
+          const uint4 qv = lds_u4(st + (size_t)r * kh + (size_t)blk * 16);
+          const float d = __half2float(__ushort_as_half(
+              *reinterpret_cast<const uint16_t*>(st + (size_t)R * kh + (size_t)r * nb * 2 + (size_t)blk * 2)));
+#pragma unroll
+          for (int j = 0; j < KRM; ++j)
+            if (KRM == 1 || j < p.kr) a[j] = d * xsc[j] * block_dot_int(qv, xg[j], cv[j]);
+        }
+#pragma unroll
+        for (int j = 0; j < KRM; ++j) v[j][r] = a[j];
+      }
+      float* rs = red + (size_t)s * NC * R * KRM;  // [NC][R][KRM] of this stage
+#pragma unroll
+      for (int j = 0; j < KRM; ++j) {
+        const float tot = cs_reduce_rows<R>(v[j], lane);
+        if ((lane & (32 / R - 1)) == 0) rs[((size_t)c * R + cs_row<R>(lane)) * KRM + j] = tot;
+      }
+      // the last of the NC warps of this stage adds the chunks in order, runs
+      // the epilogue and hands the stage back to the producer
+      __syncwarp();
+      int last = 0;
+      if (lane == 0) {
+        __threadfence_block();
+        last = atomicAdd(&s_cnt[s], 1) == NC - 1;
+      }
+      last = __shfl_sync(0xffffffffu, last, 0);
+      if (last) {
+        __threadfence_block();
+        const int u = u0 + t;
+        const int r = lane / KRM, j = lane % KRM;  // lanes l < R * KRM
+        float val = 0.f;
+        if (lane < R * KRM)
+          for (int cc = 0; cc < NC; ++cc) val += rs[((size_t)cc * R + r) * KRM + j];
+        if (p.epi == EPI_GEGLU) {
+          const float up = __shfl_sync(0xffffffffu, val, (lane + (R / 2) * KRM) & 31);
+          if (lane < (R / 2) * KRM && j < p.kr)
+            p.act[(size_t)j * p.act_stride + (size_t)(R / 2) * u + r] = __float2half_rn(gelu_tanh(val) * up);
+        } else if (lane < R * KRM && j < p.kr) {
+          const int row = R * u + r;
+          if (row < p.n_rows) {
+            if (p.epi == EPI_STORE) {
+              p.y[(size_t)j * p.y_stride + row] = val;
+            } else {
+              const float z = p.softcap * tanhf(val / p.softcap);
+              if (p.logits) p.logits[(size_t)j * p.logits_stride + row] = z;
+              if (z > best_v || (z == best_v && row < best_i)) best_v = z, best_i = row;
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) {
+          s_cnt[s] = 0;
+          mbar_arrive(&empty[s]);
+        }
+      }
+      s += G;
+      while (s >= NS) s -= NS, ph ^= 1u;
+    }
+    if (p.epi == EPI_HEAD) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float v2 = __shfl_xor_sync(0xffffffffu, best_v, o);
+        const int i2 = __shfl_xor_sync(0xffffffffu, best_i, o);
+        if (v2 > best_v || (v2 == best_v && i2 < best_i)) best_v = v2, best_i = i2;
+      }
+      if (lane == 0) s_bestv[warp] = best_v, s_besti[warp] = best_i;
+    }
+  } else if (producer) {
+    // ---------------- producer: refill each stage once it is handed back ----------------
+    if (lane == 0) {
+      for (int t = NS; t < n_st; ++t) {
+        const int s = t % NS;
+        if (!*abort_flag) cs_wait(&empty[s], (uint32_t)(((t - NS) / NS) & 1), p, abort_flag);
+        if (*abort_flag) break;
+        cs_issue<R>(p, u0 + t, stages + s * SB, &full[s], false, pol);
+        issued = t + 1;
+      }
+    }
+  }
+  if (p.epi == EPI_HEAD) {
+    __syncthreads();
+    if (tid == 0) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+      for (int w = 0; w < kCsMaxConsumers; ++w)
+        if (s_bestv[w] > bv || (s_bestv[w] == bv && s_besti[w] < bi)) bv = s_bestv[w], bi = s_besti[w];
+      p.am_val[blockIdx.x] = bv;
+      p.am_idx[blockIdx.x] = bi;
+      __threadfence();
+      s_ticket = atomicAdd(p.counter, 1);
+      if (s_ticket == (int)gridDim.x - 1) {
+        __threadfence();
+        float v = -INFINITY;
+        int ix = 0x7fffffff;
+        for (int b = 0; b < (int)gridDim.x; ++b) {
+          const float vb = __ldcg(p.am_val + b);
+          const int ib = __ldcg(p.am_idx + b);
+          if (vb > v || (vb == v && ib < ix)) v = vb, ix = ib;
+        }
+        if (p.argmax_out) p.argmax_out[0] = ix == 0x7fffffff ? 0 : ix;
+        *p.counter = 0;
+      }
+    }
+  }
+  // after a timeout, wait (bounded) for the copies still in flight
+  if (producer && lane == 0 && *abort_flag) {
+    for (int t = issued > NS ? issued - NS : 0; t < issued; ++t)
+      mbar_wait_bounded(&full[t % NS], (uint32_t)((t / NS) & 1), p.wait_ns);
+  }
+}
+
+// Plan of the column-split kernel: rows per stage R, chunks NC, groups G and
+// stages NS within the shared-memory budget.
+bool plan_cs(GemvParams& p, int& R, bool forced) {
+  const int k = p.k, nb = k >> 5;
+  if (k % 256 != 0 || p.kr > 2) return false;
+  // measured: the warp-streamed kernel is faster for long rows (k = 15360)
+  // and small matrices (3840 x 4096), where a stage carries less work
+  if (!forced && (k > 4096 || p.n_rows < 8192)) return false;
+  if (p.epi == EPI_HEAD && p.kr != 1) return false;
+  if (p.epi == EPI_GEGLU && (p.nseg != 2 || p.seg[0].rows != p.seg[1].rows || p.seg[0].rows % 4)) return false;
+  if (p.pro == PRO_RESID && k > 8192) return false;
+  for (int s = 0; s < p.nseg; ++s)
+    if (!aligned16(p.seg[s].qs) || !aligned16(p.seg[s].sc) || (s < p.nseg - 1 && p.seg[s].rows % 8))
+      return false;
+  if (p.pro == PRO_X16 && !aligned16(p.x)) return false;
+  const int NC = (nb + 31) / 32;
+  if (NC > kCsMaxConsumers) return false;
+  int G = kCsMaxConsumers / NC;
+  const int krm = p.kr <= 1 ? 1 : 2;
+  auto units = [&](int r) { return p.epi == EPI_GEGLU ? p.seg[0].rows / (r / 2) : (p.n_rows + r - 1) / r; };
+  R = k <= 4096 ? 8 : k <= 8192 ? 4 : 2;
+  if (p.epi == EPI_GEGLU && (p.seg[0].rows % (R / 2))) return false;
+  while (R > 2 && units(R) < 6 * device_sm_count()) R /= 2;
+  const size_t budget = 220 * 1024, stage = (size_t)R * ((size_t)k / 2 + (size_t)k / 16);
+  int ns = 0;
+  for (int n = kCsMaxStages; n >= 1; --n)
+    if (cs_fixed_bytes(krm, k, n, NC, R) + (size_t)n * stage <= budget) {
+      ns = n;
+      break;
+    }
+  G = std::min(G, ns - 2);  // at least 2 stages in flight while G are consumed
+  if (G < 1) return false;
+  p.ns = ns;
+  p.nchunk = NC;
+  p.groups = G;
+  p.stage_rows = R;
+  p.stage_bytes = (int)stage;
+  p.n_units = units(R);
+  return true;
+}
+
+template <int KRM, int R>
+cudaError_t launch_cs_r(const GemvParams& p, cudaStream_t st, bool pdl) {
+  static size_t configured = 0;
+  const size_t smem = cs_fixed_bytes(KRM, p.k, p.ns, p.nchunk, R) + (size_t)p.ns * p.stage_bytes;
+  cudaError_t e;
+  if (smem > configured) {
+    e = cudaFuncSetAttribute(gemv_q4_cs_kernel<KRM, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(gemv_q4_cs_kernel<KRM, R>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    configured = smem;
+  }
+  int grid = device_sm_count();
+  if (grid > p.n_units) grid = p.n_units;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kCsThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, gemv_q4_cs_kernel<KRM, R>, p);
+}
+
+template <int KRM>
+cudaError_t launch_cs_t(const GemvParams& p, int R, cudaStream_t st, bool pdl) {
+  if (R == 8) return launch_cs_r<KRM, 8>(p, st, pdl);
+  if (R == 4) return launch_cs_r<KRM, 4>(p, st, pdl);
+  return launch_cs_r<KRM, 2>(p, st, pdl);
+}
+
+// Kernel choice: Q4G_GEMV_KERNEL = "cs" (column-split) | "ws" (warp-streamed) |
+// "reg" (register path); default: cs where it plans, else ws, else reg.
+// -1 auto, 0 column-split, 1 warp-streamed, 2 register path; -2: not read yet
+std::atomic<int> g_kernel_choice{-2};
+
+int gemv_kernel_choice() {
+  int c = g_kernel_choice.load(std::memory_order_relaxed);
+  if (c == -2) {
+    const char* e = getenv("Q4G_GEMV_KERNEL");
+    c = !e ? -1 : e[0] == 'c' ? 0 : e[0] == 'w' ? 1 : 2;
+    int expected = -2;
+    if (!g_kernel_choice.compare_exchange_strong(expected, c)) c = expected;
+  }
+  return c;
+}
+
 template <int KRM>
 cudaError_t launch_t(const GemvParams& p, cudaStream_t st, bool pdl) {
   static int configured_smem = 0;
@@ -905,8 +1329,22 @@ int gemv_max_rows(int k) {
 NextGemv gemv_next_desc(const GemvParams& p_in, float frac) {
   NextGemv nx{};
   GemvParams p = p_in;
-  int dot = gemv_dot_kind();
-  if (getenv("Q4G_GEMV_REGISTER_PATH") || !plan_tma(p, dot)) return nx;
+  int dot = gemv_dot_kind(), R = 0;
+  const int choice = gemv_kernel_choice();
+  GemvParams px = p_in;
+  if (choice <= 0 && plan_cs(px, R, choice == 0)) {
+    // one stream per CTA: the first units of every CTA's range
+    for (int s = 0; s < 3; ++s) nx.seg[s] = px.seg[s];
+    nx.nseg = px.nseg;
+    nx.k = px.k;
+    nx.n_units = px.n_units;
+    nx.unit_rows = R;
+    nx.geglu = px.epi == EPI_GEGLU;
+    nx.tw = std::min(device_sm_count(), px.n_units);
+    nx.frac = frac;
+    return nx;
+  }
+  if (choice == 2 || !plan_tma(p, dot)) return nx;
   int grid = device_sm_count();
   const int min_units = (p.n_units + kWarps - 1) / kWarps;
   if (grid > min_units) grid = min_units;
@@ -914,6 +1352,7 @@ NextGemv gemv_next_desc(const GemvParams& p_in, float frac) {
   nx.nseg = p.nseg;
   nx.k = p.k;
   nx.n_units = p.n_units;
+  nx.unit_rows = 2;
   nx.geglu = p.epi == EPI_GEGLU;
   nx.tw = grid * kWarps;
   nx.frac = frac;
@@ -935,8 +1374,17 @@ int32_t* device_error_word() {
 
 cudaError_t launch_gemv(const GemvParams& p_in, cudaStream_t st, bool pdl) {
   GemvParams p = p_in;
+  const int choice = gemv_kernel_choice();
+  int R = 0;
+  if (choice <= 0 && plan_cs(p, R, choice == 0)) {
+    if (!p.err) p.err = device_error_word();
+    if (!p.err) return cudaErrorInvalidValue;
+    if (!p.wait_ns) p.wait_ns = 2000000000ull;
+    return p.kr <= 1 ? launch_cs_t<1>(p, R, st, pdl) : launch_cs_t<2>(p, R, st, pdl);
+  }
+  p = p_in;
   int dot = gemv_dot_kind();
-  if (!getenv("Q4G_GEMV_REGISTER_PATH") && plan_tma(p, dot)) {
+  if (choice != 2 && plan_tma(p, dot)) {
     if (!p.err) p.err = device_error_word();
     if (!p.err) return cudaErrorInvalidValue;
     if (!p.wait_ns) p.wait_ns = 2000000000ull;
@@ -949,6 +1397,12 @@ cudaError_t launch_gemv(const GemvParams& p_in, cudaStream_t st, bool pdl) {
   if (p.kr <= 2) return launch_t<2>(p, st, pdl);
   if (p.kr <= 4) return launch_t<4>(p, st, pdl);
   return launch_t<8>(p, st, pdl);
+}
+
+bool set_gemv_kernel_choice(int kind) {
+  if (kind < 0 || kind > 3) return false;
+  g_kernel_choice.store(kind - 1);
+  return true;
 }
 
 int device_sm_count() {

@@ -25,7 +25,8 @@ struct NextGemv {
   GemvSeg seg[3];
   int32_t nseg;
   int32_t k;
-  int32_t n_units;  // row pairs (GeGLU: gate row u with up row u)
+  int32_t n_units;    // units of unit_rows rows (GeGLU: unit_rows / 2 gate rows with the same up rows)
+  int32_t unit_rows;  // 2 or 8
   int32_t geglu;
   int32_t tw;       // warps of the next GEMV's grid
   float frac;
@@ -69,6 +70,9 @@ struct GemvParams {
   int32_t* counter;  // one int, zero between launches
   int32_t* argmax_out;
   // bulk-copy pipeline (set by the launcher)
+  int32_t nchunk;       // column-split kernel: 1024-column chunks,
+  int32_t groups;       //   consumer groups,
+  int32_t stage_rows;   //   rows per stage
   int32_t kc;           // columns per streamed item
   int32_t ns;           // stages per warp
   int32_t stage_bytes;  // codes then scales of one item (2 rows)
@@ -81,6 +85,8 @@ struct GemvParams {
 int gemv_max_rows(int k);
 size_t gemv_smem_bytes(int krm, int k);
 cudaError_t launch_gemv(const GemvParams& p, cudaStream_t st, bool pdl);
+// Q4G_GEMV_* kind; false if out of range
+bool set_gemv_kernel_choice(int kind);
 // Descriptor of GEMV `p` as the next GEMV of a prefetch (tw = 0 if p does not
 // take the streamed path).
 NextGemv gemv_next_desc(const GemvParams& p, float frac);

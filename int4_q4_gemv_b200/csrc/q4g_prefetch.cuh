@@ -16,13 +16,15 @@ Q4G_DEV void prefetch_next(const NextGemv& nx, long long part, long long nparts)
     const int ub = (int)(cw * nx.n_units / nx.tw), ue = (int)((cw + 1) * nx.n_units / nx.tw);
     const int cnt = (int)ceilf((float)(ue - ub) * nx.frac);
     if (cnt <= 0) continue;
+    const int R = nx.unit_rows;
     if (nx.geglu) {
+      const int h = R / 2;
       for (int s = 0; s < 2; ++s) {
-        l2_prefetch(nx.seg[s].qs + (size_t)ub * kh, (uint64_t)cnt * kh);
-        l2_prefetch(nx.seg[s].sc + (size_t)ub * nb, (uint64_t)cnt * nb * 2);
+        l2_prefetch(nx.seg[s].qs + (size_t)ub * h * kh, (uint64_t)cnt * h * kh);
+        l2_prefetch(nx.seg[s].sc + (size_t)ub * h * nb, (uint64_t)cnt * h * nb * 2);
       }
     } else {
-      const int r0 = 2 * ub, r1 = 2 * (ub + cnt);
+      const int r0 = R * ub, r1 = R * (ub + cnt);
       int base = 0;
       for (int s = 0; s < nx.nseg; ++s) {
         const int a = max(r0, base), b = min(r1, base + nx.seg[s].rows);

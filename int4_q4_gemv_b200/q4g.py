@@ -25,7 +25,7 @@ EXPORTS = [
     "q4g_cache_bytes", "q4g_cache_init", "q4g_cache_reset", "q4g_cache_destroy", "q4g_cache_layout",
     "q4g_decode_step", "q4g_decode_step_device_token", "q4g_decode_step_hidden",
     "q4g_decode_step_host", "q4g_verify_block", "q4g_model_profile_read",
-    "q4g_flash_decode_ring_noalloc",
+    "q4g_flash_decode_ring_noalloc", "q4g_set_gemv_kernel",
 ]
 Q4G_NOALLOC_SCRATCH_BYTES = 1 << 20
 
@@ -109,6 +109,7 @@ def lib() -> C.CDLL:
             "q4g_verify_block": (C.c_int, [vp, vp, vp, i32, i64, i32, vp, vp, vp]),
             "q4g_model_profile_read": (i32, [vp, C.POINTER(q4g_launch_record), i32, vp]),
             "q4g_flash_decode_ring_noalloc": (C.c_int, [vp, i32, i32, i32, vp, vp, i64, i64, i64, vp, vp]),
+            "q4g_set_gemv_kernel": (C.c_int, [i32]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -145,6 +146,13 @@ def q4g_q4_0_unpack(qs, scales, rows, k, w, on_device, stream):
 
 def q4g_gemv(qs, scales, n, k, x_f16, nrhs, y, stream):
     _call("q4g_gemv", qs, scales, n, k, x_f16, nrhs, y, stream)
+
+
+Q4G_GEMV_AUTO, Q4G_GEMV_COLUMN_SPLIT, Q4G_GEMV_WARP_STREAM, Q4G_GEMV_REGISTER = 0, 1, 2, 3
+
+
+def q4g_set_gemv_kernel(kind):
+    _call("q4g_set_gemv_kernel", kind)
 
 
 def q4g_flash_decode_workspace_bytes(n_q_heads, head_dim) -> int:
