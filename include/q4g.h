@@ -245,11 +245,15 @@ typedef enum {
   Q4G_OPT_PROFILE = 4,    /* [0] 1: launch eagerly and bracket every kernel with CUDA
                                  events on the launching stream (read with
                                  q4g_model_profile_read) */
-  Q4G_OPT_TEST_STALL = 5  /* [0] 1: failure-path test. In the next step, one pipeline
+  Q4G_OPT_TEST_STALL = 5, /* [0] 1: failure-path test. In the next step, one pipeline
                                  stage of the first GEMV expects 16 bytes that never
                                  arrive; its bounded wait (20 ms) gives up, the step
                                  finishes with unspecified results and
                                  q4g_model_check returns Q4G_ETIMEOUT. One-shot. */
+  Q4G_OPT_ATTN_CLUSTER = 6 /* [1] sliding layers: the 8 key chunks of a KV head run
+                                 as one thread-block cluster and merge their partial
+                                 softmax sums through distributed shared memory;
+                                 0: split-KV with a merge through global memory */
 } q4g_option;
 q4g_status q4g_model_set_option(q4g_model* m, q4g_option opt, intptr_t value);
 

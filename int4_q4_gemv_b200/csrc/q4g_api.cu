@@ -110,7 +110,7 @@ struct q4g_model {
   float* part_ml;
   float* part_acc;
   // options
-  bool use_graph = true, use_pdl = true;
+  bool use_graph = true, use_pdl = true, attn_cluster = true;
   float* dump = nullptr;
   // profile mode: events around every launch
   bool profile = false;
@@ -358,6 +358,7 @@ extern "C" q4g_status q4g_model_set_option(q4g_model* m, q4g_option opt, intptr_
     case Q4G_OPT_DUMP: m->dump = (float*)value; break;
     case Q4G_OPT_PROFILE: m->profile = value != 0; break;
     case Q4G_OPT_TEST_STALL: m->stall_next = value != 0; break;
+    case Q4G_OPT_ATTN_CLUSTER: m->attn_cluster = value != 0; break;
     default: return fail(Q4G_EINVAL, "unknown option %d", (int)opt);
   }
   free_graphs(m);
@@ -569,6 +570,15 @@ q4g_status flash_standalone(const uint16_t* q, int32_t n_q, int32_t n_kv, int32_
   p.part_acc = (float*)(w + 256 + ((sizeof(float) * 2 * (size_t)n_q * 2 * device_sm_count() + 255) & ~255ul));
   p.combine_in_kernel = ring ? 1 : 0;
   p.out = reinterpret_cast<__half*>(out);
+  if (ring) {
+    AttnParams pc = p;
+    pc.cluster = kAttnCluster;
+    pc.n_chunks = kAttnCluster;
+    if (ring_decode_rows(pc) > 0) {  // few rows per KV head: cluster kernel, no workspace use
+      CK(launch_attention(pc, st, false));
+      return Q4G_OK;
+    }
+  }
   if (p.n_kv * p.m_groups > 64) return fail(Q4G_EINVAL, "too many KV heads");
   CK(cudaMemsetAsync(p.counters, 0, 256, st));
   CK(launch_attention(p, st, false));
@@ -852,6 +862,12 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
       p.part_acc = m->part_acc;
       p.counters = m->counters + 8;
       p.combine_in_kernel = full ? 0 : 1;
+      if (!full && m->attn_cluster) {
+        // sliding layers: the chunks of one KV head form a cluster and merge in DSMEM
+        p.cluster = kAttnCluster;
+        p.n_chunks = kAttnCluster;
+        p.combine_in_kernel = 0;
+      }
       p.out = m->attn;
       const int64_t q_last = pos0 + kr - 1;
       const int64_t keys = full ? q_last + 1 : std::min<int64_t>(q_last + 1, (int64_t)cf.window + kr - 1);

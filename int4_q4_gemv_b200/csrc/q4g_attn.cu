@@ -62,16 +62,10 @@ Q4G_DEV void cp_async16(void* dst, const void* src, bool valid) {
                "r"(valid ? 16 : 0));
 }
 Q4G_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
 template <int N>
 Q4G_DEV void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-// a mod m in [0, m) for 32-bit a, m > 0; the common case (a >= -m) takes one add
-Q4G_DEV int wrap(int a, int m) {
-  if (a >= 0) return a < m ? a : a % m;
-  a += m;
-  return a >= 0 ? a : (a % m + m) % m;
 }
 
 template <int HD>
@@ -90,7 +84,9 @@ struct Smem {
   int ticket;
 };
 
-template <int HD>
+// CL > 0: the grid's y dimension is one cluster of CL CTAs (n_chunks == CL);
+// the chunk partials are merged through distributed shared memory.
+template <int HD, int CL>
 __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   Smem<HD>& sm = *reinterpret_cast<Smem<HD>*>(smem_raw);
@@ -132,10 +128,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
   const __half* vc = p.v_cache + (size_t)kv * p.cache_rows * HD;
   constexpr int CPR = HD / 8;  // 16-byte chunks per row
 
-  auto load_tile = [&](int t, bool kpart, bool patch_local) {
+  // mode 0: cache rows only (the block's own rows do not exist yet);
+  // 1: the block's own rows only, from shared memory; 2: both
+  auto load_tile = [&](int t, bool kpart, int mode) {
     const int buf = t & 1;
     const int a0 = a_begin + t * TK;
-    if (kpart && tid < TK) {
+    if (kpart && tid < TK && mode != 1) {
       const int a = a0 + tid;
       sm.kidx[buf][tid] = a < a_end ? key_row(a) : -1;
     }
@@ -147,12 +145,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
       const bool in = a < a_end;
       const int loc = in ? key_is_local(a) : -1;
       if (loc >= 0) {
-        if (patch_local) {
+        if (mode != 0) {
           const __half* l = kpart ? sm.kloc[loc] : sm.vloc[loc];
           *reinterpret_cast<uint4*>(&dst[key][part * 8]) =
               *reinterpret_cast<const uint4*>(l + part * 8);
         }
-      } else {
+      } else if (mode != 1) {
         const __half* s = in ? src + (size_t)key_row(a) * HD + part * 8 : src;
         cp_async16(&dst[key][part * 8], s, in);
       }
@@ -161,9 +159,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
 
   // first tile's cache rows go out before the prologue
   if (ntiles > 0) {
-    load_tile(0, true, false);
+    load_tile(0, true, 0);
     cp_async_commit();
-    load_tile(0, false, false);
+    load_tile(0, false, 0);
     cp_async_commit();
   }
   // the next GEMV's first weights towards L2, one slice per CTA
@@ -229,9 +227,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
       *reinterpret_cast<uint4*>(&sm.q[r][part * 8]) = *reinterpret_cast<const uint4*>(src);
     }
   }
-  // zero the unused query rows (their results are never written)
-  for (int c = tid; c < (MROWS - nrows) * LD; c += kThreads)
-    sm.q[nrows + c / LD][c % LD] = __float2half_rn(0.f);
+  // zero the unused query rows of the m16 tiles read below (their results are
+  // never written); rows are LD halves, a multiple of 8
+  {
+    const int zrows = ((nrows + 15) / 16) * 16 - nrows;
+    uint4* z = reinterpret_cast<uint4*>(&sm.q[nrows][0]);
+    for (int c = tid; c < zrows * LD / 8; c += kThreads) z[c] = make_uint4(0, 0, 0, 0);
+  }
   if (tid < MROWS) sm.m_run[tid] = -INFINITY, sm.l_run[tid] = 0.f;
   __syncthreads();
 
@@ -263,8 +265,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
   for (int t = 0; t < ntiles; ++t) {
     const int buf = t & 1;
     if (t == 0 && fused) {  // this block's own rows, now that they exist
-      load_tile(0, true, true);
-      load_tile(0, false, true);
+      load_tile(0, true, 1);
+      load_tile(0, false, 1);
     }
     cp_async_wait<1>();
     __syncthreads();
@@ -287,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
     }
     __syncthreads();  // K tile consumed
     if (t + 1 < ntiles) {
-      load_tile(t + 1, true, true);
+      load_tile(t + 1, true, 2);
     }
     cp_async_commit();
 
@@ -397,10 +399,55 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
       }
     }
     __syncthreads();  // V tile and P consumed
-    if (t + 1 < ntiles) load_tile(t + 1, false, true);
+    if (t + 1 < ntiles) load_tile(t + 1, false, 2);
     cp_async_commit();
   }
   cp_async_wait<0>();
+
+  if (CL > 0) {
+    // ---- merge the CL chunk partials of this KV head through DSMEM ----
+    __syncthreads();  // every warp is done with the K tile, reused below
+    float* pacc = reinterpret_cast<float*>(&sm.k[0][0]);  // [nrows][HD] unnormalised partial
+    for (int mt = 0; mt < mtiles; ++mt) {
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int lr = mt * 16 + g4 + hh * 8;
+        if (lr < nrows) {
+#pragma unroll
+          for (int nt = 0; nt < NT_PV; ++nt) {
+            const int d = warp * (HD / 8) + nt * 8 + t4 * 2;
+            *reinterpret_cast<float2*>(pacc + (size_t)lr * HD + d) =
+                make_float2(oacc[mt][nt][hh * 2], oacc[mt][nt][hh * 2 + 1]);
+          }
+        }
+      }
+    }
+    cluster_sync();  // all partials and (m, l) of the cluster are visible
+    constexpr int DPC = HD / (CL > 0 ? CL : 1);  // output dims merged by this CTA
+    const uint32_t rank = cluster_rank();
+    for (int w = tid; w < nrows * DPC; w += kThreads) {
+      const int lr = w / DPC, d = (int)rank * DPC + (w - lr * DPC);
+      float mc[CL > 0 ? CL : 1], mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < CL; ++c) {
+        mc[c] = ld_peer_f32(peer_addr(&sm.m_run[lr], c));
+        mx = fmaxf(mx, mc[c]);
+      }
+      float l = 0.f, o = 0.f;
+#pragma unroll
+      for (int c = 0; c < CL; ++c) {
+        if (mc[c] == -INFINITY) continue;
+        const float e = __expf(mc[c] - mx);
+        l = fmaf(ld_peer_f32(peer_addr(&sm.l_run[lr], c)), e, l);
+        o = fmaf(ld_peer_f32(peer_addr(pacc + (size_t)lr * HD + d, c)), e, o);
+      }
+      const int gr = row0 + lr;
+      const int orow = (gr / G) * p.n_q + kv * G + gr % G;
+      p.out[(size_t)orow * HD + d] = __float2half_rn(o / l);
+    }
+    cluster_sync();  // peers may still read this CTA's shared memory until here
+    return;
+  }
 
   // ---- partials ----
   const int nq_rows = p.kr * p.n_q;
@@ -539,30 +586,42 @@ __global__ void __launch_bounds__(kCombineThreads) attn_combine_kernel(const Att
   }
 }
 
-template <int HD>
+template <int HD, int CL>
 cudaError_t launch_attn_t(const AttnParams& p, cudaStream_t st, bool pdl) {
   static bool configured = false;
   const size_t smem = sizeof(Smem<HD>);
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(attn_kernel<HD, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(attn_kernel<HD>, cudaFuncAttributePreferredSharedMemoryCarveout,
+    e = cudaFuncSetAttribute(attn_kernel<HD, CL>, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     configured = true;
   }
+  if (CL > 0 && p.n_chunks != CL) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.n_kv, p.n_chunks, p.m_groups);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (CL > 0) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 1;
+    attr[na].val.clusterDim.y = CL;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, attn_kernel<HD>, p);
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, attn_kernel<HD, CL>, p);
 }
 
 template <int HD>
@@ -590,8 +649,15 @@ size_t attn_partial_floats(int kr, int n_q, int n_chunks, int hd) {
 }
 
 cudaError_t launch_attention(const AttnParams& p, cudaStream_t st, bool pdl) {
-  if (p.hd == 256) return launch_attn_t<256>(p, st, pdl);
-  if (p.hd == 512) return launch_attn_t<512>(p, st, pdl);
+  if (p.cluster == kAttnCluster && ring_decode_rows(p) > 0) return launch_attention_ring(p, st, pdl);
+  if (p.cluster == kAttnCluster) {
+    if (p.hd == 256) return launch_attn_t<256, kAttnCluster>(p, st, pdl);
+    if (p.hd == 512) return launch_attn_t<512, kAttnCluster>(p, st, pdl);
+    return cudaErrorInvalidValue;
+  }
+  if (p.cluster != 0) return cudaErrorInvalidValue;
+  if (p.hd == 256) return launch_attn_t<256, 0>(p, st, pdl);
+  if (p.hd == 512) return launch_attn_t<512, 0>(p, st, pdl);
   return cudaErrorInvalidValue;
 }
 

@@ -1,0 +1,415 @@
+// Flash-decode over the sliding ring for a few query rows per KV head, on CUDA
+// cores.
+//
+// Operation ("Gemma 4 12B" page, flash-decode paragraph: GQA decode, scale 1.0,
+// fp32 online softmax, the KV scan split across cooperating groups;
+// "Gemma-4-12B-CoreAI", v5 section: slot = position mod R, implied position
+// p = q - ((q - j) mod R), window test q - p < W).
+//
+// With 2 query rows per KV head (decode of the sliding layers) a key row is
+// used by 2 rows only, so the scan is a latency problem, not a throughput one:
+//   * the CL = 8 CTAs of one KV head form a thread-block cluster; CTA c scans
+//     keys [c * cs, (c + 1) * cs) by age, warp w a contiguous 1/8 of that;
+//   * lane l holds dims [l * HD/32, (l + 1) * HD/32) of a key: each warp loads
+//     its first 8 keys straight into registers (16 B per lane and key) before
+//     waiting on the previous kernel, and the next 8 while it works on these;
+//   * scores are fp32 dot products of the fp16 query (normed and rotated in the
+//     prologue) with the fp16 keys, reduced over the warp with a transposing
+//     butterfly; the online softmax and P.V stay in fp32;
+//   * warp partials merge in shared memory, CTA partials through distributed
+//     shared memory: CTA c of the cluster writes output dims [c * HD/CL, ...).
+// The block's own key/value rows (the new positions) come from shared memory;
+// chunk 0 also writes them to the ring.
+#include "q4g_common.cuh"
+#include "q4g_internal.h"
+
+namespace q4g {
+
+namespace {
+
+constexpr int kRingThreads = 256;
+constexpr int kRingWarps = kRingThreads / 32;
+
+template <int HD, int ROWS>
+struct RingSmem {
+  __half q[ROWS][HD];                  // queries after norm and RoPE (fp16, as stored)
+  __half kloc[kMaxRows][HD];           // the block's own K rows
+  __half vloc[kMaxRows][HD];           // the block's own V rows
+  float part[kRingWarps][ROWS][HD];    // warp partial sums of p * v
+  float pm[kRingWarps][ROWS], pl[kRingWarps][ROWS];
+  float cacc[ROWS][HD];                // CTA partial, relative to cm
+  float cm[ROWS], cl[ROWS];
+};
+
+// Sum v[0..N) over the 32 lanes (N a power of two <= 32) and give every lane
+// all N totals.
+template <int N>
+Q4G_DEV void warp_allreduce_vec(float (&v)[N], int lane) {
+#pragma unroll
+  for (int h = N / 2, o = 16; h >= 1; h >>= 1, o >>= 1) {
+    const bool upper = lane & o;
+#pragma unroll
+    for (int i = 0; i < h; ++i) {
+      const float send = upper ? v[i] : v[i + h];
+      const float keep = upper ? v[i + h] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  float t = v[0];
+#pragma unroll
+  for (int o = 16 / N; o >= 1; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+  // lane L holds total number sum_{steps} (L & o ? h : 0); broadcast them all
+#pragma unroll
+  for (int idx = 0; idx < N; ++idx) {
+    int src = 0;
+#pragma unroll
+    for (int h = N / 2, o = 16; h >= 1; h >>= 1, o >>= 1) src += (idx & h) ? o : 0;
+    v[idx] = __shfl_sync(0xffffffffu, t, src);
+  }
+}
+
+Q4G_DEV void unpack8(const uint4 u, float (&f)[8]) {
+  const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __half22float2(h[i]);
+    f[2 * i] = t.x, f[2 * i + 1] = t.y;
+  }
+}
+
+// One projection vector of the block by one warp: per-head RMSNorm (learned
+// gain, or scale-free), RoPE on the first rope_pairs rotate-half pairs, fp16.
+// All global loads are issued before the arithmetic that depends on them.
+template <int HD>
+Q4G_DEV void norm_rope_vec(const AttnParams& p, const float* src, const float* gain, bool do_norm,
+                           bool rotate, int j, __half* dst, int lane) {
+  constexpr int E = HD / 64;  // elements per lane per half
+  float lo[E], hi[E], glo[E], ghi[E];
+  float2 cs[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int i = lane * E + e;
+    lo[e] = src[i];
+    hi[e] = src[HD / 2 + i];
+    glo[e] = gain ? gain[i] : 1.0f;
+    ghi[e] = gain ? gain[HD / 2 + i] : 1.0f;
+    cs[e] = rotate && i < p.rope_pairs ? p.rope[(size_t)j * p.rope_pairs + i] : make_float2(1.f, 0.f);
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) ss = fmaf(lo[e], lo[e], fmaf(hi[e], hi[e], ss));
+  const float inv = do_norm ? rms_inv(warp_sum(ss), HD, p.eps) : 1.0f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int i = lane * E + e;
+    float a = __fmul_rn(lo[e], inv), b = __fmul_rn(hi[e], inv);
+    if (gain) a = __fmul_rn(a, glo[e]), b = __fmul_rn(b, ghi[e]);
+    if (rotate && i < p.rope_pairs) {
+      const float ra = a * cs[e].x - b * cs[e].y;
+      const float rb = b * cs[e].x + a * cs[e].y;
+      a = ra, b = rb;
+    }
+    dst[i] = __float2half_rn(a);
+    dst[HD / 2 + i] = __float2half_rn(b);
+  }
+}
+
+template <int HD, int ROWS, int CL>
+__global__ void __launch_bounds__(kRingThreads, 1) attn_ring_kernel(const AttnParams p) {
+  constexpr int DPL = HD / 32;   // dims per lane
+  constexpr int VPK = DPL / 8;   // 16-byte pieces per lane and key
+  constexpr int B = 8 / VPK;     // keys per batch
+  extern __shared__ __align__(16) unsigned char ring_smem[];
+  RingSmem<HD, ROWS>& sm = *reinterpret_cast<RingSmem<HD, ROWS>*>(ring_smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int kv = blockIdx.x;
+  const int chunk = (int)cluster_rank();
+  const int G = p.n_q / p.n_kv, nr = p.kr * G;  // nr <= ROWS (host)
+  const bool fused = p.qkv != nullptr;
+
+  // The position was written before the first kernel of the step and the cache
+  // rows read below by earlier steps: both may be read before griddepcontrol.wait.
+  const int64_t pos0 = p.pos_dev ? *p.pos_dev : p.pos0;
+  const int64_t q_last = pos0 + p.kr - 1;
+  const int R = (int)p.cache_rows, W = (int)p.window;
+  const int qlm = (int)(q_last % p.cache_rows);  // slot of the newest key
+  const int nscan = (int)min((int64_t)W + p.kr - 1, q_last + 1);
+  const int cs = (nscan + CL - 1) / CL;
+  const int a_begin = min(nscan, chunk * cs), a_end = min(nscan, a_begin + cs);
+  const int kpw = (a_end - a_begin + kRingWarps - 1) / kRingWarps;
+  const int wa0 = min(a_end, a_begin + warp * kpw), wa1 = min(a_end, wa0 + kpw);
+  const int first_cached = fused ? p.kr : 0;  // ages below are the block's own rows
+
+  const __half* kcache = p.k_cache + (size_t)kv * R * HD + lane * DPL;
+  const __half* vcache = p.v_cache + (size_t)kv * R * HD + lane * DPL;
+  auto load_batch = [&](int a0, uint4 (&kb)[B][VPK], uint4 (&vb)[B][VPK]) {
+#pragma unroll
+    for (int i = 0; i < B; ++i) {
+      const int a = a0 + i;
+      const bool in = a < wa1 && a >= first_cached;
+      const size_t off = in ? (size_t)wrap(qlm - a, R) * HD : 0;
+#pragma unroll
+      for (int v = 0; v < VPK; ++v) {
+        kb[i][v] = in ? ld_stream_u4(kcache + off + 8 * v) : make_uint4(0, 0, 0, 0);
+        vb[i][v] = in ? ld_stream_u4(vcache + off + 8 * v) : make_uint4(0, 0, 0, 0);
+      }
+    }
+  };
+  uint4 kb[B][VPK], vb[B][VPK];
+  load_batch(wa0, kb, vb);
+
+  pdl_wait();
+  // ---- prologue: queries and the block's own K/V rows ----
+  if (fused) {
+    const int nvec = nr + 2 * p.kr;
+    for (int vi = warp; vi < nvec; vi += kRingWarps) {
+      if (vi < nr) {
+        const int j = vi / G;
+        const float* src = p.qkv + (size_t)j * p.qkv_stride + (size_t)(kv * G + vi % G) * HD;
+        norm_rope_vec<HD>(p, src, p.w_q, true, true, j, sm.q[vi], lane);
+      } else if (vi < nr + p.kr) {
+        const int j = vi - nr;
+        const float* src = p.qkv + (size_t)j * p.qkv_stride + p.k_off + (size_t)kv * HD;
+        norm_rope_vec<HD>(p, src, p.w_k, true, true, j, sm.kloc[j], lane);
+      } else {
+        const int j = vi - nr - p.kr;
+        const float* src = p.qkv + (size_t)j * p.qkv_stride +
+                           (p.v_off >= 0 ? p.v_off + (size_t)kv * HD : p.k_off + (size_t)kv * HD);
+        norm_rope_vec<HD>(p, src, nullptr, p.v_norm != 0, false, j, sm.vloc[j], lane);
+      }
+    }
+  } else {
+    for (int c = tid; c < nr * HD / 8; c += kRingThreads) {
+      const int r = c / (HD / 8), part = c - r * (HD / 8);
+      const __half* src = p.q16 + ((size_t)(r / G) * p.n_q + kv * G + r % G) * HD + part * 8;
+      *reinterpret_cast<uint4*>(&sm.q[r][part * 8]) = *reinterpret_cast<const uint4*>(src);
+    }
+  }
+  __syncthreads();
+  if (fused && p.write_kv && chunk == 0) {
+    for (int c = tid; c < p.kr * HD / 8; c += kRingThreads) {
+      const int j = c / (HD / 8), part = c - j * (HD / 8);
+      const size_t row = (size_t)wrap(qlm - (p.kr - 1 - j), R);
+      *reinterpret_cast<uint4*>(p.k_cache + ((size_t)kv * R + row) * HD + part * 8) =
+          *reinterpret_cast<const uint4*>(&sm.kloc[j][part * 8]);
+      *reinterpret_cast<uint4*>(p.v_cache + ((size_t)kv * R + row) * HD + part * 8) =
+          *reinterpret_cast<const uint4*>(&sm.vloc[j][part * 8]);
+    }
+  }
+  pdl_launch_dependents();
+
+  // ---- scan: online softmax per query row over this warp's keys ----
+  float q[ROWS][DPL];
+#pragma unroll
+  for (int r = 0; r < ROWS; ++r) {
+    if (r < nr) {
+#pragma unroll
+      for (int v = 0; v < VPK; ++v) {
+        float f[8];
+        unpack8(*reinterpret_cast<const uint4*>(&sm.q[r][lane * DPL + 8 * v]), f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) q[r][8 * v + e] = f[e];
+      }
+    } else {
+#pragma unroll
+      for (int d = 0; d < DPL; ++d) q[r][d] = 0.f;
+    }
+  }
+  // key age a is live for row r (query j) iff d = (a - (kr - 1 - j)) mod R
+  // satisfies d < W and d <= q_j
+  int shift[ROWS];
+  int64_t qpos[ROWS];
+#pragma unroll
+  for (int r = 0; r < ROWS; ++r) {
+    const int j = r < nr ? r / G : 0;
+    shift[r] = p.kr - 1 - j;
+    qpos[r] = pos0 + j;
+  }
+  float m[ROWS], l[ROWS], acc[ROWS][DPL];
+#pragma unroll
+  for (int r = 0; r < ROWS; ++r) {
+    m[r] = -INFINITY, l[r] = 0.f;
+#pragma unroll
+    for (int d = 0; d < DPL; ++d) acc[r][d] = 0.f;
+  }
+  for (int a0 = wa0; a0 < wa1; a0 += B) {
+    if (fused && a0 < p.kr) {  // the block's own rows
+#pragma unroll
+      for (int i = 0; i < B; ++i) {
+        const int a = a0 + i;
+        if (a < p.kr && a < wa1) {
+          const int loc = p.kr - 1 - a;
+#pragma unroll
+          for (int v = 0; v < VPK; ++v) {
+            kb[i][v] = *reinterpret_cast<const uint4*>(&sm.kloc[loc][lane * DPL + 8 * v]);
+            vb[i][v] = *reinterpret_cast<const uint4*>(&sm.vloc[loc][lane * DPL + 8 * v]);
+          }
+        }
+      }
+    }
+    uint4 nk[B][VPK], nv[B][VPK];
+    if (a0 + B < wa1) load_batch(a0 + B, nk, nv);
+    // partial dot products: s[i * ROWS + r]
+    float s[B * ROWS];
+#pragma unroll
+    for (int i = 0; i < B; ++i) {
+      float kf[DPL];
+#pragma unroll
+      for (int v = 0; v < VPK; ++v) {
+        float f[8];
+        unpack8(kb[i][v], f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) kf[8 * v + e] = f[e];
+      }
+#pragma unroll
+      for (int r = 0; r < ROWS; ++r) {
+        float t = 0.f;
+#pragma unroll
+        for (int d = 0; d < DPL; ++d) t = fmaf(q[r][d], kf[d], t);
+        s[i * ROWS + r] = t;
+      }
+    }
+    warp_allreduce_vec<B * ROWS>(s, lane);
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r) {
+      if (r >= nr) continue;
+      float mx = m[r];
+#pragma unroll
+      for (int i = 0; i < B; ++i) {
+        const int a = a0 + i;
+        const int d = wrap(a - shift[r], R);
+        const bool live = a < wa1 && d < W && (int64_t)d <= qpos[r];
+        s[i * ROWS + r] = live ? s[i * ROWS + r] : -INFINITY;
+        mx = fmaxf(mx, s[i * ROWS + r]);
+      }
+      if (mx == -INFINITY) continue;  // nothing live yet for this row
+      const float scale = __expf(m[r] - mx);
+      l[r] *= scale;
+#pragma unroll
+      for (int dd = 0; dd < DPL; ++dd) acc[r][dd] *= scale;
+      m[r] = mx;
+#pragma unroll
+      for (int i = 0; i < B; ++i) {
+        const float sv = s[i * ROWS + r];
+        const float pv = sv == -INFINITY ? 0.f : __expf(sv - mx);
+        l[r] += pv;
+#pragma unroll
+        for (int v = 0; v < VPK; ++v) {
+          float f[8];
+          unpack8(vb[i][v], f);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[r][8 * v + e] = fmaf(pv, f[e], acc[r][8 * v + e]);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < B; ++i)
+#pragma unroll
+      for (int v = 0; v < VPK; ++v) kb[i][v] = nk[i][v], vb[i][v] = nv[i][v];
+  }
+
+  // ---- merge: warps in shared memory ----
+#pragma unroll
+  for (int r = 0; r < ROWS; ++r) {
+    if (r >= nr) continue;
+#pragma unroll
+    for (int d = 0; d < DPL; d += 4)
+      *reinterpret_cast<float4*>(&sm.part[warp][r][lane * DPL + d]) =
+          make_float4(acc[r][d], acc[r][d + 1], acc[r][d + 2], acc[r][d + 3]);
+    if (lane == 0) sm.pm[warp][r] = m[r], sm.pl[warp][r] = l[r];
+  }
+  __syncthreads();
+  for (int idx = tid; idx < nr * HD; idx += kRingThreads) {
+    const int r = idx / HD, d = idx - r * HD;
+    float mx = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kRingWarps; ++w) mx = fmaxf(mx, sm.pm[w][r]);
+    float o = 0.f, lsum = 0.f;
+    if (mx != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kRingWarps; ++w) {
+        const float mw = sm.pm[w][r];
+        if (mw == -INFINITY) continue;
+        const float e = __expf(mw - mx);
+        o = fmaf(sm.part[w][r][d], e, o);
+        lsum = fmaf(sm.pl[w][r], e, lsum);
+      }
+    }
+    sm.cacc[r][d] = o;
+    if (d == 0) sm.cm[r] = mx, sm.cl[r] = lsum;
+  }
+  // ---- merge: the CL CTAs of the cluster through distributed shared memory ----
+  cluster_sync();
+  constexpr int DPC = HD / CL;
+  for (int idx = tid; idx < nr * DPC; idx += kRingThreads) {
+    const int r = idx / DPC, d = chunk * DPC + (idx - r * DPC);
+    float mc[CL], mx = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < CL; ++c) {
+      mc[c] = ld_peer_f32(peer_addr(&sm.cm[r], c));
+      mx = fmaxf(mx, mc[c]);
+    }
+    float o = 0.f, lsum = 0.f;
+#pragma unroll
+    for (int c = 0; c < CL; ++c) {
+      if (mc[c] == -INFINITY) continue;
+      const float e = __expf(mc[c] - mx);
+      lsum = fmaf(ld_peer_f32(peer_addr(&sm.cl[r], c)), e, lsum);
+      o = fmaf(ld_peer_f32(peer_addr(&sm.cacc[r][d], c)), e, o);
+    }
+    const int j = r / G;
+    p.out[((size_t)j * p.n_q + kv * G + r % G) * HD + d] = __float2half_rn(o / lsum);
+  }
+  cluster_sync();  // peers may read this CTA's shared memory until here
+}
+
+template <int HD, int ROWS>
+cudaError_t launch_ring_t(const AttnParams& p, cudaStream_t st, bool pdl) {
+  static bool configured = false;
+  const size_t smem = sizeof(RingSmem<HD, ROWS>);
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(attn_ring_kernel<HD, ROWS, kAttnCluster>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.n_kv, kAttnCluster, 1);
+  cfg.blockDim = dim3(kRingThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  attr[na].id = cudaLaunchAttributeClusterDimension;
+  attr[na].val.clusterDim.x = 1;
+  attr[na].val.clusterDim.y = kAttnCluster;
+  attr[na].val.clusterDim.z = 1;
+  ++na;
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, attn_ring_kernel<HD, ROWS, kAttnCluster>, p);
+}
+
+}  // namespace
+
+int ring_decode_rows(const AttnParams& p) {
+  const int rows = p.kr * (p.n_q / p.n_kv);
+  if (!p.ring || p.hd != 256 || rows > 4) return 0;
+  return rows <= 1 ? 1 : rows <= 2 ? 2 : 4;
+}
+
+cudaError_t launch_attention_ring(const AttnParams& p, cudaStream_t st, bool pdl) {
+  switch (ring_decode_rows(p)) {
+    case 1: return launch_ring_t<256, 1>(p, st, pdl);
+    case 2: return launch_ring_t<256, 2>(p, st, pdl);
+    case 4: return launch_ring_t<256, 4>(p, st, pdl);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace q4g

@@ -186,6 +186,33 @@ Q4G_DEV bool mbar_wait_bounded(uint64_t* bar, uint32_t phase, uint64_t limit_ns)
   return false;
 }
 
+// a mod m in [0, m) for 32-bit a, m > 0; the common case (a >= -m) takes one add
+Q4G_DEV int wrap(int a, int m) {
+  if (a >= 0) return a < m ? a : a % m;
+  a += m;
+  return a >= 0 ? a : (a % m + m) % m;
+}
+
+// Thread-block clusters: rank, cluster-wide barrier (release/acquire) and loads
+// from a peer CTA's shared memory (distributed shared memory).
+Q4G_DEV uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+Q4G_DEV void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+Q4G_DEV uint32_t peer_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+Q4G_DEV float ld_peer_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
 // ---------------------------------------------------------------------------
 // Reductions.
 // ---------------------------------------------------------------------------

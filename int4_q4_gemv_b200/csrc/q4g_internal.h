@@ -125,12 +125,18 @@ struct AttnParams {
   float* part_acc;
   int32_t* counters;     // [n_kv] for the in-kernel combine (ring), zero between launches
   int32_t combine_in_kernel;
+  int32_t cluster;       // kAttnCluster: grid y is one cluster, merge through DSMEM (n_chunks == cluster)
   __half* out;           // [kr][n_q][hd]
 };
 
+constexpr int kAttnCluster = 8;  // CTAs per KV head when the merge runs in a cluster
 size_t attn_smem_bytes(int hd, int m_tiles_per_cta);
 size_t attn_partial_floats(int kr, int n_q, int n_chunks, int hd);
 cudaError_t launch_attention(const AttnParams& p, cudaStream_t st, bool pdl);
+// CUDA-core cluster kernel for ring layers with <= 4 query rows per KV head
+// (hd 256): 0 if it does not apply, else the row template it uses
+int ring_decode_rows(const AttnParams& p);
+cudaError_t launch_attention_ring(const AttnParams& p, cudaStream_t st, bool pdl);
 cudaError_t launch_attn_combine(const AttnParams& p, cudaStream_t st, bool pdl);
 
 // --------------------------------------------------------------- misc ----
