@@ -49,6 +49,8 @@ def parse_args():
     ap.add_argument("--profile-steps", type=int, default=4)
     ap.add_argument("--e2e-steps", type=int, default=32)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="fewer layers of the same shapes (profiling captures of a small case)")
     return ap.parse_args()
 
 
@@ -212,6 +214,8 @@ def main():
     args = parse_args()
     from datagen import workloads as WL
     cfg = dict(WL.B12)
+    if args.layers:
+        cfg["n_layers"] = args.layers
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -356,7 +360,7 @@ def main():
             "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": K,
             "warmup": W, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "q4_0 x f16 -> f32", "data": "synthetic",
-            "config": {"workload": f"12B-class q4_0 decoder (48 layers, h 3840, vocab 262144), "
+            "config": {"workload": f"12B-class q4_0 decoder ({cfg['n_layers']} layers, h 3840, vocab 262144), "
                                    f"context {C}, batch 1, greedy decode",
                        "context": C, "global_batch": world, "seq_len": C,
                        "parallelism": f"replicas{world}", "prefix": args.prefix,

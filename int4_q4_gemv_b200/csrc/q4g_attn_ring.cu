@@ -10,24 +10,28 @@
 // used by 2 rows only, so the scan is a latency problem, not a throughput one:
 //   * the CL = 8 CTAs of one KV head form a thread-block cluster; CTA c scans
 //     keys [c * cs, (c + 1) * cs) by age, warp w a contiguous 1/8 of that;
-//   * lane l holds dims [l * HD/32, (l + 1) * HD/32) of a key: each warp loads
-//     its first 8 keys straight into registers (16 B per lane and key) before
-//     waiting on the previous kernel, and the next 8 while it works on these;
-//   * scores are fp32 dot products of the fp16 query (normed and rotated in the
-//     prologue) with the fp16 keys, reduced over the warp with a transposing
-//     butterfly; the online softmax and P.V stay in fp32;
+//   * 16 warps per CTA; each warp loads its keys' K and V rows straight into
+//     registers (16 bytes per lane and row), the first group of keys before
+//     waiting on the previous kernel (the rows were written by earlier steps),
+//     the next group while it works on the current one;
+//   * lane l holds dims 8l .. 8l+7 (hd 256) of the query and of each key; per
+//     group of 4 keys the fp32 dot products are reduced over the warp with a
+//     transposing butterfly, followed by one online-softmax update and P.V,
+//     all in fp32;
 //   * warp partials merge in shared memory, CTA partials through distributed
 //     shared memory: CTA c of the cluster writes output dims [c * HD/CL, ...).
-// The block's own key/value rows (the new positions) come from shared memory;
+// The block's own key/value rows (the new positions) come from the prologue;
 // chunk 0 also writes them to the ring.
 #include "q4g_common.cuh"
 #include "q4g_internal.h"
+
+#include <algorithm>
 
 namespace q4g {
 
 namespace {
 
-constexpr int kRingThreads = 256;
+constexpr int kRingThreads = 512;
 constexpr int kRingWarps = kRingThreads / 32;
 
 template <int HD, int ROWS>
@@ -42,7 +46,8 @@ struct RingSmem {
 };
 
 // Sum v[0..N) over the 32 lanes (N a power of two <= 32) and give every lane
-// all N totals.
+// all N totals: a transposing butterfly (N - 1 + log2(32 / N) shuffles), then
+// N broadcasts.
 template <int N>
 Q4G_DEV void warp_allreduce_vec(float (&v)[N], int lane) {
 #pragma unroll
@@ -58,7 +63,7 @@ Q4G_DEV void warp_allreduce_vec(float (&v)[N], int lane) {
   float t = v[0];
 #pragma unroll
   for (int o = 16 / N; o >= 1; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-  // lane L holds total number sum_{steps} (L & o ? h : 0); broadcast them all
+  // lane L holds total number sum_{steps} (L & o ? h : 0)
 #pragma unroll
   for (int idx = 0; idx < N; ++idx) {
     int src = 0;
@@ -68,7 +73,7 @@ Q4G_DEV void warp_allreduce_vec(float (&v)[N], int lane) {
   }
 }
 
-Q4G_DEV void unpack8(const uint4 u, float (&f)[8]) {
+Q4G_DEV void unpack8(const uint4 u, float* f) {
   const __half2* h = reinterpret_cast<const __half2*>(&u);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -114,11 +119,12 @@ Q4G_DEV void norm_rope_vec(const AttnParams& p, const float* src, const float* g
   }
 }
 
+// Code size is kept small on purpose: every SM runs one CTA of this kernel per
+// layer, so its instructions are fetched cold; the loop over key groups is rolled.
 template <int HD, int ROWS, int CL>
 __global__ void __launch_bounds__(kRingThreads, 1) attn_ring_kernel(const AttnParams p) {
-  constexpr int DPL = HD / 32;   // dims per lane
-  constexpr int VPK = DPL / 8;   // 16-byte pieces per lane and key
-  constexpr int B = 8 / VPK;     // keys per batch
+  static_assert(HD == 256, "one 16-byte piece per lane and row");
+  constexpr int B = ROWS <= 2 ? 4 : 2;  // keys per group
   extern __shared__ __align__(16) unsigned char ring_smem[];
   RingSmem<HD, ROWS>& sm = *reinterpret_cast<RingSmem<HD, ROWS>*>(ring_smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -140,43 +146,36 @@ __global__ void __launch_bounds__(kRingThreads, 1) attn_ring_kernel(const AttnPa
   const int wa0 = min(a_end, a_begin + warp * kpw), wa1 = min(a_end, wa0 + kpw);
   const int first_cached = fused ? p.kr : 0;  // ages below are the block's own rows
 
-  const __half* kcache = p.k_cache + (size_t)kv * R * HD + lane * DPL;
-  const __half* vcache = p.v_cache + (size_t)kv * R * HD + lane * DPL;
-  auto load_batch = [&](int a0, uint4 (&kb)[B][VPK], uint4 (&vb)[B][VPK]) {
+  // lane l holds dims 8l .. 8l+7 of every row
+  const __half* kcache = p.k_cache + (size_t)kv * R * HD + lane * 8;
+  const __half* vcache = p.v_cache + (size_t)kv * R * HD + lane * 8;
+  auto load_group = [&](int a0, uint4 (&kb)[B], uint4 (&vb)[B]) {
 #pragma unroll
     for (int i = 0; i < B; ++i) {
       const int a = a0 + i;
       const bool in = a < wa1 && a >= first_cached;
       const size_t off = in ? (size_t)wrap(qlm - a, R) * HD : 0;
-#pragma unroll
-      for (int v = 0; v < VPK; ++v) {
-        kb[i][v] = in ? ld_stream_u4(kcache + off + 8 * v) : make_uint4(0, 0, 0, 0);
-        vb[i][v] = in ? ld_stream_u4(vcache + off + 8 * v) : make_uint4(0, 0, 0, 0);
-      }
+      kb[i] = in ? ld_stream_u4(kcache + off) : make_uint4(0, 0, 0, 0);
+      vb[i] = in ? ld_stream_u4(vcache + off) : make_uint4(0, 0, 0, 0);
     }
   };
-  uint4 kb[B][VPK], vb[B][VPK];
-  load_batch(wa0, kb, vb);
+  uint4 kb[B], vb[B];
+  load_group(wa0, kb, vb);
 
   pdl_wait();
   // ---- prologue: queries and the block's own K/V rows ----
   if (fused) {
     const int nvec = nr + 2 * p.kr;
     for (int vi = warp; vi < nvec; vi += kRingWarps) {
-      if (vi < nr) {
-        const int j = vi / G;
-        const float* src = p.qkv + (size_t)j * p.qkv_stride + (size_t)(kv * G + vi % G) * HD;
-        norm_rope_vec<HD>(p, src, p.w_q, true, true, j, sm.q[vi], lane);
-      } else if (vi < nr + p.kr) {
-        const int j = vi - nr;
-        const float* src = p.qkv + (size_t)j * p.qkv_stride + p.k_off + (size_t)kv * HD;
-        norm_rope_vec<HD>(p, src, p.w_k, true, true, j, sm.kloc[j], lane);
-      } else {
-        const int j = vi - nr - p.kr;
-        const float* src = p.qkv + (size_t)j * p.qkv_stride +
-                           (p.v_off >= 0 ? p.v_off + (size_t)kv * HD : p.k_off + (size_t)kv * HD);
-        norm_rope_vec<HD>(p, src, nullptr, p.v_norm != 0, false, j, sm.vloc[j], lane);
-      }
+      const int kind = vi < nr ? 0 : vi < nr + p.kr ? 1 : 2;
+      const int j = kind == 0 ? vi / G : kind == 1 ? vi - nr : vi - nr - p.kr;
+      const size_t col = kind == 0 ? (size_t)(kv * G + vi % G) * HD
+                         : kind == 1 || p.v_off < 0 ? p.k_off + (size_t)kv * HD
+                                                    : p.v_off + (size_t)kv * HD;
+      __half* dst = kind == 0 ? sm.q[vi] : kind == 1 ? sm.kloc[j] : sm.vloc[j];
+      norm_rope_vec<HD>(p, p.qkv + (size_t)j * p.qkv_stride + col,
+                        kind == 0 ? p.w_q : kind == 1 ? p.w_k : nullptr, kind != 2 || p.v_norm != 0,
+                        kind != 2, j, dst, lane);
     }
   } else {
     for (int c = tid; c < nr * HD / 8; c += kRingThreads) {
@@ -198,21 +197,15 @@ __global__ void __launch_bounds__(kRingThreads, 1) attn_ring_kernel(const AttnPa
   }
   pdl_launch_dependents();
 
-  // ---- scan: online softmax per query row over this warp's keys ----
-  float q[ROWS][DPL];
+  // ---- scan: per group of B keys, scores for every row, one online-softmax update ----
+  float q[ROWS][8];
 #pragma unroll
   for (int r = 0; r < ROWS; ++r) {
     if (r < nr) {
-#pragma unroll
-      for (int v = 0; v < VPK; ++v) {
-        float f[8];
-        unpack8(*reinterpret_cast<const uint4*>(&sm.q[r][lane * DPL + 8 * v]), f);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) q[r][8 * v + e] = f[e];
-      }
+      unpack8(*reinterpret_cast<const uint4*>(&sm.q[r][lane * 8]), q[r]);
     } else {
 #pragma unroll
-      for (int d = 0; d < DPL; ++d) q[r][d] = 0.f;
+      for (int e = 0; e < 8; ++e) q[r][e] = 0.f;
     }
   }
   // key age a is live for row r (query j) iff d = (a - (kr - 1 - j)) mod R
@@ -225,47 +218,37 @@ __global__ void __launch_bounds__(kRingThreads, 1) attn_ring_kernel(const AttnPa
     shift[r] = p.kr - 1 - j;
     qpos[r] = pos0 + j;
   }
-  float m[ROWS], l[ROWS], acc[ROWS][DPL];
+  float m[ROWS], l[ROWS], acc[ROWS][8];
 #pragma unroll
   for (int r = 0; r < ROWS; ++r) {
     m[r] = -INFINITY, l[r] = 0.f;
 #pragma unroll
-    for (int d = 0; d < DPL; ++d) acc[r][d] = 0.f;
+    for (int e = 0; e < 8; ++e) acc[r][e] = 0.f;
   }
+#pragma unroll 1
   for (int a0 = wa0; a0 < wa1; a0 += B) {
-    if (fused && a0 < p.kr) {  // the block's own rows
+    if (fused && a0 < first_cached) {  // the block's own rows, from the prologue
 #pragma unroll
       for (int i = 0; i < B; ++i) {
         const int a = a0 + i;
-        if (a < p.kr && a < wa1) {
-          const int loc = p.kr - 1 - a;
-#pragma unroll
-          for (int v = 0; v < VPK; ++v) {
-            kb[i][v] = *reinterpret_cast<const uint4*>(&sm.kloc[loc][lane * DPL + 8 * v]);
-            vb[i][v] = *reinterpret_cast<const uint4*>(&sm.vloc[loc][lane * DPL + 8 * v]);
-          }
+        if (a < first_cached && a < wa1) {
+          kb[i] = *reinterpret_cast<const uint4*>(&sm.kloc[p.kr - 1 - a][lane * 8]);
+          vb[i] = *reinterpret_cast<const uint4*>(&sm.vloc[p.kr - 1 - a][lane * 8]);
         }
       }
     }
-    uint4 nk[B][VPK], nv[B][VPK];
-    if (a0 + B < wa1) load_batch(a0 + B, nk, nv);
-    // partial dot products: s[i * ROWS + r]
+    uint4 nk[B], nv[B];
+    if (a0 + B < wa1) load_group(a0 + B, nk, nv);
     float s[B * ROWS];
 #pragma unroll
     for (int i = 0; i < B; ++i) {
-      float kf[DPL];
-#pragma unroll
-      for (int v = 0; v < VPK; ++v) {
-        float f[8];
-        unpack8(kb[i][v], f);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) kf[8 * v + e] = f[e];
-      }
+      float kf[8];
+      unpack8(kb[i], kf);
 #pragma unroll
       for (int r = 0; r < ROWS; ++r) {
         float t = 0.f;
 #pragma unroll
-        for (int d = 0; d < DPL; ++d) t = fmaf(q[r][d], kf[d], t);
+        for (int e = 0; e < 8; ++e) t = fmaf(q[r][e], kf[e], t);
         s[i * ROWS + r] = t;
       }
     }
@@ -276,9 +259,8 @@ __global__ void __launch_bounds__(kRingThreads, 1) attn_ring_kernel(const AttnPa
       float mx = m[r];
 #pragma unroll
       for (int i = 0; i < B; ++i) {
-        const int a = a0 + i;
-        const int d = wrap(a - shift[r], R);
-        const bool live = a < wa1 && d < W && (int64_t)d <= qpos[r];
+        const int d = wrap(a0 + i - shift[r], R);
+        const bool live = a0 + i < wa1 && d < W && (int64_t)d <= qpos[r];
         s[i * ROWS + r] = live ? s[i * ROWS + r] : -INFINITY;
         mx = fmaxf(mx, s[i * ROWS + r]);
       }
@@ -286,47 +268,40 @@ __global__ void __launch_bounds__(kRingThreads, 1) attn_ring_kernel(const AttnPa
       const float scale = __expf(m[r] - mx);
       l[r] *= scale;
 #pragma unroll
-      for (int dd = 0; dd < DPL; ++dd) acc[r][dd] *= scale;
+      for (int e = 0; e < 8; ++e) acc[r][e] *= scale;
       m[r] = mx;
 #pragma unroll
       for (int i = 0; i < B; ++i) {
         const float sv = s[i * ROWS + r];
         const float pv = sv == -INFINITY ? 0.f : __expf(sv - mx);
+        float vf[8];
+        unpack8(vb[i], vf);
         l[r] += pv;
 #pragma unroll
-        for (int v = 0; v < VPK; ++v) {
-          float f[8];
-          unpack8(vb[i][v], f);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[r][8 * v + e] = fmaf(pv, f[e], acc[r][8 * v + e]);
-        }
+        for (int e = 0; e < 8; ++e) acc[r][e] = fmaf(pv, vf[e], acc[r][e]);
       }
     }
 #pragma unroll
-    for (int i = 0; i < B; ++i)
-#pragma unroll
-      for (int v = 0; v < VPK; ++v) kb[i][v] = nk[i][v], vb[i][v] = nv[i][v];
+    for (int i = 0; i < B; ++i) kb[i] = nk[i], vb[i] = nv[i];
   }
 
   // ---- merge: warps in shared memory ----
 #pragma unroll
   for (int r = 0; r < ROWS; ++r) {
     if (r >= nr) continue;
-#pragma unroll
-    for (int d = 0; d < DPL; d += 4)
-      *reinterpret_cast<float4*>(&sm.part[warp][r][lane * DPL + d]) =
-          make_float4(acc[r][d], acc[r][d + 1], acc[r][d + 2], acc[r][d + 3]);
+    float* dst = &sm.part[warp][r][lane * 8];
+    *reinterpret_cast<float4*>(dst) = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+    *reinterpret_cast<float4*>(dst + 4) = make_float4(acc[r][4], acc[r][5], acc[r][6], acc[r][7]);
     if (lane == 0) sm.pm[warp][r] = m[r], sm.pl[warp][r] = l[r];
   }
   __syncthreads();
+#pragma unroll 1
   for (int idx = tid; idx < nr * HD; idx += kRingThreads) {
     const int r = idx / HD, d = idx - r * HD;
     float mx = -INFINITY;
-#pragma unroll
     for (int w = 0; w < kRingWarps; ++w) mx = fmaxf(mx, sm.pm[w][r]);
     float o = 0.f, lsum = 0.f;
     if (mx != -INFINITY) {
-#pragma unroll
       for (int w = 0; w < kRingWarps; ++w) {
         const float mw = sm.pm[w][r];
         if (mw == -INFINITY) continue;
@@ -341,6 +316,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) attn_ring_kernel(const AttnPa
   // ---- merge: the CL CTAs of the cluster through distributed shared memory ----
   cluster_sync();
   constexpr int DPC = HD / CL;
+#pragma unroll 1
   for (int idx = tid; idx < nr * DPC; idx += kRingThreads) {
     const int r = idx / DPC, d = chunk * DPC + (idx - r * DPC);
     float mc[CL], mx = -INFINITY;
