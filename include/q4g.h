@@ -250,16 +250,28 @@ typedef enum {
                                  arrive; its bounded wait (20 ms) gives up, the step
                                  finishes with unspecified results and
                                  q4g_model_check returns Q4G_ETIMEOUT. One-shot. */
-  Q4G_OPT_ATTN_CLUSTER = 6 /* [1] sliding layers: the 8 key chunks of a KV head run
+  Q4G_OPT_ATTN_CLUSTER = 6, /* [1] sliding layers: the 8 key chunks of a KV head run
                                  as one thread-block cluster and merge their partial
                                  softmax sums through distributed shared memory;
                                  0: split-KV with a merge through global memory */
+  Q4G_OPT_GEMV_CHAIN = 7,   /* [0] decode steps: O(l), gate|up(l), down(l) and QKV(l+1)
+                                 run as one persistent launch (one CTA per SM; a phase
+                                 starts when every CTA finished the previous one, a
+                                 bounded wait reported as Q4G_ETIMEOUT); 0: one launch
+                                 per GEMV */
+  Q4G_OPT_TRACE = 8         /* [0] value = device uint64_t* [n_layers][32]: the GEMV
+                                 chain of layer l writes %globaltimer stamps (ns) of
+                                 its CTA 0 to row l: 0 start, 1 dependency wait done,
+                                 per phase i at 2 + 4i: inputs ready, x digits built,
+                                 last stage of CTA 0 done, producer done issuing;
+                                 18 end. Unwritten slots keep their contents. */
 } q4g_option;
 q4g_status q4g_model_set_option(q4g_model* m, q4g_option opt, intptr_t value);
 
 /* One kernel launch recorded in profile mode. kind: 0 step init, 1 QKV GEMV,
  * 2 sliding attention, 3 full attention, 4 attention combine, 5 O GEMV,
- * 6 gate|up GEMV, 7 down GEMV, 8 head GEMV. bytes: algorithmic HBM bytes of the
+ * 6 gate|up GEMV, 7 down GEMV, 8 head GEMV, 9 GEMV chain (O, gate|up, down and
+ * the next layer's QKV in one launch). bytes: algorithmic HBM bytes of the
  * launch (q4_0 weights 0.5625 B/weight + activations; attention: the live K/V
  * rows, 2 * head_dim * 2 B per key and KV head). */
 typedef struct {

@@ -110,7 +110,8 @@ struct q4g_model {
   float* part_ml;
   float* part_acc;
   // options
-  bool use_graph = true, use_pdl = true, attn_cluster = true;
+  bool use_graph = true, use_pdl = true, attn_cluster = true, gemv_chain = false;
+  uint64_t* trace = nullptr;  // Q4G_OPT_TRACE
   float* dump = nullptr;
   // profile mode: events around every launch
   bool profile = false;
@@ -254,7 +255,7 @@ extern "C" q4g_status q4g_model_create(const q4g_config* cfg, const q4g_weights*
     part = b > part ? b : part;
   }
   const size_t part_ml = part / 128 + 1024;  // (m, l) per row and chunk: hd >= 256
-  m->n_counters = 64;
+  m->n_counters = 64 + kChainMaxPhases * c.n_layers;  // head, attention, chain phases
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -359,6 +360,8 @@ extern "C" q4g_status q4g_model_set_option(q4g_model* m, q4g_option opt, intptr_
     case Q4G_OPT_PROFILE: m->profile = value != 0; break;
     case Q4G_OPT_TEST_STALL: m->stall_next = value != 0; break;
     case Q4G_OPT_ATTN_CLUSTER: m->attn_cluster = value != 0; break;
+    case Q4G_OPT_GEMV_CHAIN: m->gemv_chain = value != 0; break;
+    case Q4G_OPT_TRACE: m->trace = (uint64_t*)value; break;
     default: return fail(Q4G_EINVAL, "unknown option %d", (int)opt);
   }
   free_graphs(m);
@@ -814,13 +817,14 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
     return pf > 0.f ? gemv_next_desc(q, std::min(1.0f, frac * pf)) : NextGemv{};
   };
 
+  bool qkv_done = false;  // QKV(l) already ran as the last phase of the previous chain
   for (int l = 0; l < L; ++l) {
     const q4g_layer_weights& W = m->layers[l];
     const bool full = m->full[l];
     const LayerShape& S = full ? m->gl : m->sl;
     const int ord = m->ordinal[l];
     const GemvParams gate_up = gate_up_params(l);
-    {
+    if (!qkv_done) {
       GemvParams p = qkv_params(l);
       p.next = next_of(o_params(l, 0), 1.0f);
       if (l == 0 && m->stall_next) {
@@ -881,6 +885,27 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
         e = pc.done(debug_sync(launch_attn_combine(p, st, pdl), "combine", l, st), 4, l,
                     (double)kr * cf.n_q_heads * p.n_chunks * (S.hd + 2) * 4.0);
         if (e != cudaSuccess) return e;
+      }
+    }
+    // O(l), gate|up(l), down(l) and QKV(l+1) as one persistent chain launch
+    qkv_done = false;
+    if (kr == 1 && m->gemv_chain) {
+      ChainParams ch{};
+      ch.ph[0] = o_params(l, 0);
+      ch.ph[1] = gate_up;
+      ch.ph[2] = down_params(l, 0);
+      ch.n_ph = 3;
+      if (l + 1 < L) ch.ph[3] = qkv_params(l + 1), ch.n_ph = 4;
+      ch.done = m->counters + 64 + kChainMaxPhases * l;
+      ch.trace = m->trace ? m->trace + (size_t)kChainTraceSlots * l : nullptr;
+      if (plan_chain(ch)) {
+        double bytes = 0;
+        for (int i = 0; i < ch.n_ph; ++i) bytes += gemv_bytes(ch.ph[i].n_rows, ch.ph[i].k, 1, 4);
+        Prof pr(m, st);
+        e = pr.done(debug_sync(launch_gemv_chain(ch, st, pdl), "gemv_chain", l, st), 9, l, bytes);
+        if (e != cudaSuccess) return e;
+        qkv_done = ch.n_ph == 4;
+        continue;
       }
     }
     {

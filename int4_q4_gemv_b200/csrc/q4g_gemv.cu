@@ -153,20 +153,27 @@ Q4G_DEV void produce_x(const GemvParams& p, float* misc, Emit&& emit) {
       const float4* dl = p.delta ? reinterpret_cast<const float4*>(p.delta + (size_t)j * k) : nullptr;
       const float4* wd = reinterpret_cast<const float4*>(p.w_delta);
       const float4* wx = reinterpret_cast<const float4*>(p.w_x);
-      float4 rn[R4], dv[R4];
-      float ss = 0.f;
+      // every global load of the prologue in one round (the gains do not
+      // depend on the reductions)
+      float4 rn[R4], dv[R4], wdv[R4], wxv[R4];
 #pragma unroll
       for (int i = 0; i < R4; ++i) {
         const int c4 = tid + i * NT;
         if (c4 < n4) {
           rn[i] = rin[c4];
-          if (dl) {
-            dv[i] = dl[c4];
-            ss = fmaf(dv[i].x, dv[i].x, ss);
-            ss = fmaf(dv[i].y, dv[i].y, ss);
-            ss = fmaf(dv[i].z, dv[i].z, ss);
-            ss = fmaf(dv[i].w, dv[i].w, ss);
-          }
+          wxv[i] = wx[c4];
+          if (dl) dv[i] = dl[c4], wdv[i] = wd[c4];
+        }
+      }
+      float ss = 0.f;
+#pragma unroll
+      for (int i = 0; i < R4; ++i) {
+        const int c4 = tid + i * NT;
+        if (c4 < n4 && dl) {
+          ss = fmaf(dv[i].x, dv[i].x, ss);
+          ss = fmaf(dv[i].y, dv[i].y, ss);
+          ss = fmaf(dv[i].z, dv[i].z, ss);
+          ss = fmaf(dv[i].w, dv[i].w, ss);
         }
       }
       if (dl) {
@@ -175,7 +182,7 @@ Q4G_DEV void produce_x(const GemvParams& p, float* misc, Emit&& emit) {
         for (int i = 0; i < R4; ++i) {
           const int c4 = tid + i * NT;
           if (c4 < n4) {
-            const float4 w = wd[c4];
+            const float4 w = wdv[i];
             rn[i].x = __fmul_rn(__fadd_rn(rn[i].x, __fmul_rn(__fmul_rn(dv[i].x, inv_d), w.x)), p.scale);
             rn[i].y = __fmul_rn(__fadd_rn(rn[i].y, __fmul_rn(__fmul_rn(dv[i].y, inv_d), w.y)), p.scale);
             rn[i].z = __fmul_rn(__fadd_rn(rn[i].z, __fmul_rn(__fmul_rn(dv[i].z, inv_d), w.z)), p.scale);
@@ -205,7 +212,7 @@ Q4G_DEV void produce_x(const GemvParams& p, float* misc, Emit&& emit) {
         const bool valid = c4 < n4;
         __half h[4];
         if (valid) {
-          const float4 w = wx[c4];
+          const float4 w = wxv[i];
           h[0] = __float2half_rn(__fmul_rn(__fmul_rn(rn[i].x, inv_r), w.x));
           h[1] = __float2half_rn(__fmul_rn(__fmul_rn(rn[i].y, inv_r), w.y));
           h[2] = __float2half_rn(__fmul_rn(__fmul_rn(rn[i].z, inv_r), w.z));
@@ -248,6 +255,37 @@ Q4G_DEV void stage_x(const GemvParams& p, uint4* xs, float* cblk, float* misc) {
   __syncthreads();
 }
 
+// Digits of 4 consecutive columns of one block (see block_dot_int): v_i =
+// rint(x_i * 2^(37 - Emax)) for low columns, rint(x_i * 2^(33 - Emax)) for high
+// ones. Exact: |x| * 2^(37 - Emax) < 2^23 and the scaling is a power of two.
+// Returns one packed word per digit (bytes = digits of the 4 columns) and adds
+// the (weighted) digit sums to sd.
+Q4G_DEV void digits4(const __half (&h)[4], int em, bool high, uint32_t (&wd)[3], int (&sd)[3]) {
+  const float sc = __int_as_float(((high ? 33 : 37) - em + 127) << 23);
+  int X[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) X[e] = __float2int_rn(__half2float(h[e]) * sc);
+  // byte t of every X: t = 0, 1 unsigned digits, t = 2 the signed top digit
+#pragma unroll
+  for (int t = 0; t < 3; ++t) {
+    const uint32_t sel = 0x0040u | (uint32_t)(t * 0x11);  // bytes (x.b_t, y.b_t)
+    const uint32_t lo = __byte_perm((uint32_t)X[0], (uint32_t)X[1], sel);
+    const uint32_t hi = __byte_perm((uint32_t)X[2], (uint32_t)X[3], sel);
+    wd[t] = __byte_perm(lo, hi, 0x5410);
+  }
+  const int m = high ? 16 : 1;
+  sd[0] += m * dp4a_uu(wd[0], 0x01010101u, 0);
+  sd[1] += m * dp4a_uu(wd[1], 0x01010101u, 0);
+  int s2;
+  asm("dp4a.s32.s32 %0, %1, %2, %3;" : "=r"(s2) : "r"(wd[2]), "r"(0x01010101u), "r"(0));
+  sd[2] += m * s2;
+}
+
+Q4G_DEV int half_exp(__half h) {
+  const int E = (__half_as_ushort(h) >> 10) & 31;
+  return E ? E : 1;
+}
+
 // Activations as the digits of the integer dot product (block_dot_int):
 // thread (block blk, group sub) turns columns 4*sub..4*sub+3 of the block into
 // one 32-bit word per digit; the block's largest exponent and digit sums are
@@ -258,33 +296,15 @@ Q4G_DEV void stage_digits(const GemvParams& p, uint4* dg, int4* bc, float* misc)
   uint32_t* dw = reinterpret_cast<uint32_t*>(dg);
   produce_x<KRM, NT>(p, misc, [&](int j, int c4, const __half (&h)[4], bool valid) {
     const int blk = c4 >> 3, sub = c4 & 7;
-    int Ee[4], M[4], em = 1;
-    uint32_t neg = 0;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const uint32_t b = __half_as_ushort(h[e]);
-      const int E = (b >> 10) & 31;
-      Ee[e] = E ? E : 1;
-      M[e] = (int)(b & 1023) | (E ? 1024 : 0);
-      neg |= (b >> 15) << e;
-      em = max(em, Ee[e]);
-    }
+    int em = max(max(half_exp(h[0]), half_exp(h[1])), max(half_exp(h[2]), half_exp(h[3])));
     em = max(em, __shfl_xor_sync(0xffffffffu, em, 1));
     em = max(em, __shfl_xor_sync(0xffffffffu, em, 2));
     em = max(em, __shfl_xor_sync(0xffffffffu, em, 4));
-    uint32_t w0 = 0, w1 = 0, w2 = 0;
-    int s0 = 0, s1 = 0, s2 = 0;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int sh = 12 + Ee[e] - em;  // <= 12
-      int X = sh >= 0 ? (M[e] << sh) : sh > -12 ? (M[e] + (1 << (-sh - 1))) >> -sh : 0;
-      if ((neg >> e) & 1) X = -X;
-      const int d0 = X & 255, d1 = (X >> 8) & 255, d2 = X >> 16;
-      w0 |= (uint32_t)d0 << (8 * e);
-      w1 |= (uint32_t)d1 << (8 * e);
-      w2 |= (uint32_t)(d2 & 255) << (8 * e);
-      s0 += d0, s1 += d1, s2 += d2;
-    }
+    uint32_t wdg[3];
+    int sd[3] = {0, 0, 0};
+    digits4(h, em, sub >= 4, wdg, sd);
+    const uint32_t w0 = wdg[0], w1 = wdg[1], w2 = wdg[2];
+    int s0 = sd[0], s1 = sd[1], s2 = sd[2];
 #pragma unroll
     for (int o = 1; o < 8; o <<= 1) {
       s0 += __shfl_xor_sync(0xffffffffu, s0, o);
@@ -557,21 +577,29 @@ Q4G_DEV void issue_item(const GemvParams& p, int u, int c, unsigned char* st, ui
 // x of one block (32 fp16 values) becomes signed 24-bit fixed point relative to
 // the block's largest exponent: X_i = round(x_i * 2^(37 - Emax)), exact for
 // every value within 2^12 of the block maximum (the rest carry an error below
-// 2^-24 of the block maximum), x_i ~= X_i * 2^(Emax - 37). X splits into bytes
-// X = d0 + 256 d1 + 65536 d2 (d0, d1 unsigned, d2 signed), so
-//   sum_i (c_i - 8) X_i = S0 + 256 S1 + 65536 S2,  S_t = sum_i (c_i - 8) d_t,i,
-// and each S_t is a chain of 4-way byte dot products (dp4a) of the raw codes
-// with the digits, started at -8 * sum_i d_t,i. Every S_t is exact in int32.
+// 2^-24 of the block maximum), x_i ~= X_i * 2^(Emax - 37).
+// The code byte b of a block holds column b in its low nibble and column b + 16
+// in its high nibble. Masking a code word with 0x0F0F0F0F gives four low codes
+// c; masking it with 0xF0F0F0F0 gives four high codes as 16 c. So the high
+// columns use Y_i = round(X_i / 16) (error <= 8 units of X, 2^-20 of the block
+// maximum) and 16 c Y_i stands for c X_i: every code word costs two masks.
+// The values (X for columns 0..15, Y for 16..31) split into bytes
+// v = d0 + 256 d1 + 65536 d2 (d0, d1 unsigned, d2 signed), so with m_i = 1 for
+// low and 16 for high columns
+//   sum_i (c_i - 8) m_i v_i = S0 + 256 S1 + 65536 S2,
+//   S_t = sum_i (m_i c_i) d_t,i - 8 sum_i m_i d_t,i,
+// and each S_t is a chain of 4-way byte dot products (dp4a) started at the
+// constant -8 sum_i m_i d_t,i. Every S_t is exact in int32.
 // Layout per x row j: dg[j][2t + h][blk] holds digit t of columns 16h..16h+15
-// of block blk (16 bytes), bc[j][blk] = (-8 D0, -8 D1, -8 D2, bits of 2^(Emax-37)),
-// written by stage_digits.
+// of block blk (16 bytes), bc[j][blk] = (-8 D0, -8 D1, -8 D2, bits of 2^(Emax-37))
+// with D_t = sum_i m_i d_t,i, written by stage_digits.
 // ---------------------------------------------------------------------------
 Q4G_DEV float block_dot_int(const uint4 q, const uint4 (&g)[6], const int4 c) {
   const uint32_t w[4] = {q.x, q.y, q.z, q.w};
   int s0 = c.x, s1 = c.y, s2 = c.z;
 #pragma unroll
   for (int t = 0; t < 4; ++t) {
-    const uint32_t lo = w[t] & 0x0F0F0F0Fu, hi = (w[t] >> 4) & 0x0F0F0F0Fu;
+    const uint32_t lo = w[t] & 0x0F0F0F0Fu, hi = w[t] & 0xF0F0F0F0u;  // hi: 16 x the high codes
     s0 = dp4a_uu(lo, (&g[0].x)[t], s0);
     s0 = dp4a_uu(hi, (&g[1].x)[t], s0);
     s1 = dp4a_uu(lo, (&g[2].x)[t], s1);
@@ -901,11 +929,12 @@ bool plan_tma(GemvParams& p, int& dot) {
 // in order through a ring of NS stages: one producer warp issues 2 (GeGLU: 4)
 // large 1-D bulk copies per stage (the unit's codes, then its scales), so every
 // SM reads one contiguous region, the access pattern that reaches the copy
-// bandwidth of HBM. The k columns are cut into NC chunks of 32 blocks (1024
-// columns); consumer warp (g, c) owns chunk c and takes the stages g, g + G,
-// ... (G = 16 / NC groups). Lane b of that warp holds the integer digits of
-// x for block 32c + b in registers for the whole kernel (block_dot_int) and
-// dots them with the R rows of every stage it takes. The R partial sums of a
+// bandwidth of HBM. The k columns are cut into NC chunks of 32 BPL blocks
+// (BPL = 2 for one activation row, else 1); consumer warp (g, c) owns chunk c
+// and takes the stages g, g + G, ... (G = 16 / NC groups). Lane l of that warp
+// holds the integer digits of x for blocks 32 BPL c + l + 32 b in registers
+// for the whole kernel (block_dot_int) and dots them with the R rows of every
+// stage it takes. The R partial sums of a
 // warp go to shared memory with a transposing butterfly; the last of the NC
 // warps to finish a stage adds the chunk partials in chunk order
 // (deterministic), runs the epilogue and hands the stage back, so the producer
@@ -966,6 +995,31 @@ Q4G_DEV bool cs_wait(uint64_t* bar, uint32_t phase, const GemvParams& p, volatil
   return false;
 }
 
+// Several consumer groups share one ring, so a group can reach slot s for
+// stage t while the slot's previous fill (stage t - NS, another group's) is
+// still in flight; the mbarrier parity of fill t equals that of fill t - 2 NS,
+// so a parity wait alone could pass early. The producer therefore publishes
+// the stage number it issued into each slot (after the expect-tx arrive), and
+// a consumer first waits until slot s carries stage t: from then on the slot's
+// pending phase is fill t's and the parity wait is exact.
+Q4G_DEV bool wait_issued(volatile int* seq, int t, const GemvParams& p, volatile int* abort_flag) {
+  if (*seq == t) return true;
+  const uint64_t t0 = global_ns();
+  for (int it = 0; it < kSpinLimit; ++it) {
+    if (*seq == t) return true;
+    if (*abort_flag) return false;
+    if (global_ns() - t0 > p.wait_ns) break;
+    __nanosleep(32);
+  }
+  *abort_flag = 1;
+  atomicOr(p.err, 1);
+  return false;
+}
+Q4G_DEV void publish_issued(volatile int* seq, int t) {
+  __threadfence_block();
+  *seq = t;
+}
+
 // Issue the bulk copies of unit u into stage `st` ([R rows of codes][R rows of scales]).
 template <int R>
 Q4G_DEV void cs_issue(const GemvParams& p, int u, unsigned char* st, uint64_t* bar, bool poison, uint64_t pol) {
@@ -990,7 +1044,7 @@ Q4G_DEV void cs_issue(const GemvParams& p, int u, unsigned char* st, uint64_t* b
   }
 }
 
-template <int KRM, int R>
+template <int KRM, int R, int BPL>
 __global__ void __launch_bounds__(kCsThreads, 1) gemv_q4_cs_kernel(const GemvParams p) {
   extern __shared__ __align__(16) unsigned char cs_smem[];
   const int k = p.k, nb = k >> 5, kh = k >> 1, NS = p.ns, NC = p.nchunk, G = p.groups;
@@ -1006,6 +1060,7 @@ __global__ void __launch_bounds__(kCsThreads, 1) gemv_q4_cs_kernel(const GemvPar
   unsigned char* stages = reinterpret_cast<unsigned char*>(bars + 2 * kCsMaxStages);
   __shared__ int s_abort, s_ticket;
   __shared__ int s_cnt[kCsMaxStages];       // consumer warps done with a stage
+  __shared__ int s_seq[kCsMaxStages];       // stage number last issued into each slot
   __shared__ float s_bestv[kCsMaxConsumers];
   __shared__ int s_besti[kCsMaxConsumers];
 
@@ -1021,7 +1076,7 @@ __global__ void __launch_bounds__(kCsThreads, 1) gemv_q4_cs_kernel(const GemvPar
   int issued = 0;
 
   if (tid == 0) s_abort = 0;
-  if (tid < kCsMaxStages) s_cnt[tid] = 0;
+  if (tid < kCsMaxStages) s_cnt[tid] = 0, s_seq[tid] = -1;
   if (tid < kCsMaxConsumers) s_bestv[tid] = -INFINITY, s_besti[tid] = 0x7fffffff;
   if (producer && lane == 0) {
     for (int s = 0; s < NS; ++s) mbar_init(&full[s], 1), mbar_init(&empty[s], 1);
@@ -1030,6 +1085,9 @@ __global__ void __launch_bounds__(kCsThreads, 1) gemv_q4_cs_kernel(const GemvPar
       cs_issue<R>(p, u0 + issued, stages + issued * SB, &full[issued],
                   p.stall_test && u0 == 0 && issued == 0, pol);  // the CTA owning unit 0
   }
+  __syncthreads();  // s_seq initialised before the producer publishes
+  if (producer && lane == 0)
+    for (int i = 0; i < issued; ++i) publish_issued(&s_seq[i], i);
   pdl_wait();
   stage_digits<KRM, kCsThreads>(p, dg, bc, misc);  // ends with __syncthreads
   pdl_launch_dependents();
@@ -1037,31 +1095,37 @@ __global__ void __launch_bounds__(kCsThreads, 1) gemv_q4_cs_kernel(const GemvPar
 
   if (warp < n_cons) {
     // ---------------- consumer: chunk c, stages g, g + G, ... ----------------
+    // lane l holds blocks 32 BPL c + l + 32 b, b < BPL, of every row
     const int c = warp % NC, g = warp / NC;
-    const int blk = 32 * c + lane;
-    const bool has = blk < nb;
-    uint4 xg[KRM][6];
-    int4 cv[KRM];
-    float xsc[KRM];
+    int blkb[BPL];
+    bool hasb[BPL];
+    uint4 xg[KRM][BPL][6];
+    int4 cv[KRM][BPL];
+    float xsc[KRM][BPL];
 #pragma unroll
-    for (int j = 0; j < KRM; ++j) {
-      if (has && (KRM == 1 || j < p.kr)) {
+    for (int b = 0; b < BPL; ++b) {
+      blkb[b] = 32 * BPL * c + lane + 32 * b;
+      hasb[b] = blkb[b] < nb;
 #pragma unroll
-        for (int q = 0; q < 6; ++q) xg[j][q] = dg[(size_t)(j * 6 + q) * nb + blk];
-        cv[j] = bc[j * nb + blk];
-      } else {
+      for (int j = 0; j < KRM; ++j) {
+        if (hasb[b] && (KRM == 1 || j < p.kr)) {
 #pragma unroll
-        for (int q = 0; q < 6; ++q) xg[j][q] = make_uint4(0, 0, 0, 0);
-        cv[j] = make_int4(0, 0, 0, 0);
+          for (int q = 0; q < 6; ++q) xg[j][b][q] = dg[(size_t)(j * 6 + q) * nb + blkb[b]];
+          cv[j][b] = bc[j * nb + blkb[b]];
+        } else {
+#pragma unroll
+          for (int q = 0; q < 6; ++q) xg[j][b][q] = make_uint4(0, 0, 0, 0);
+          cv[j][b] = make_int4(0, 0, 0, 0);
+        }
+        xsc[j][b] = __int_as_float(cv[j][b].w);
       }
-      xsc[j] = __int_as_float(cv[j].w);
     }
     float best_v = -INFINITY;
     int best_i = 0x7fffffff;
     int s = g % NS;
     uint32_t ph = (uint32_t)((g / NS) & 1);
     for (int t = g; t < n_st; t += G) {
-      if (!*abort_flag) cs_wait(&full[s], ph, p, abort_flag);
+      if (!*abort_flag && wait_issued(&s_seq[s], t, p, abort_flag)) cs_wait(&full[s], ph, p, abort_flag);
       const unsigned char* st = stages + s * SB;
       float v[KRM][R];
 #pragma unroll
@@ -1069,13 +1133,16 @@ __global__ void __launch_bounds__(kCsThreads, 1) gemv_q4_cs_kernel(const GemvPar
         float a[KRM];
 #pragma unroll
         for (int j = 0; j < KRM; ++j) a[j] = 0.f;
-        if (has) {
-          const uint4 qv = lds_u4(st + (size_t)r * kh + (size_t)blk * 16);
-          const float d = __half2float(__ushort_as_half(
-              *reinterpret_cast<const uint16_t*>(st + (size_t)R * kh + (size_t)r * nb * 2 + (size_t)blk * 2)));
 #pragma unroll
-          for (int j = 0; j < KRM; ++j)
-            if (KRM == 1 || j < p.kr) a[j] = d * xsc[j] * block_dot_int(qv, xg[j], cv[j]);
+        for (int b = 0; b < BPL; ++b) {
+          if (hasb[b]) {
+            const uint4 qv = lds_u4(st + (size_t)r * kh + (size_t)blkb[b] * 16);
+            const float d = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(
+                st + (size_t)R * kh + (size_t)r * nb * 2 + (size_t)blkb[b] * 2)));
+#pragma unroll
+            for (int j = 0; j < KRM; ++j)
+              if (KRM == 1 || j < p.kr) a[j] = fmaf(d * xsc[j][b], block_dot_int(qv, xg[j][b], cv[j][b]), a[j]);
+          }
         }
 #pragma unroll
         for (int j = 0; j < KRM; ++j) v[j][r] = a[j];
@@ -1144,6 +1211,7 @@ __global__ void __launch_bounds__(kCsThreads, 1) gemv_q4_cs_kernel(const GemvPar
         if (!*abort_flag) cs_wait(&empty[s], (uint32_t)(((t - NS) / NS) & 1), p, abort_flag);
         if (*abort_flag) break;
         cs_issue<R>(p, u0 + t, stages + s * SB, &full[s], false, pol);
+        publish_issued(&s_seq[s], t);
         issued = t + 1;
       }
     }
@@ -1182,7 +1250,7 @@ __global__ void __launch_bounds__(kCsThreads, 1) gemv_q4_cs_kernel(const GemvPar
 
 // Plan of the column-split kernel: rows per stage R, chunks NC, groups G and
 // stages NS within the shared-memory budget.
-bool plan_cs(GemvParams& p, int& R, bool forced) {
+bool plan_cs(GemvParams& p, int& R, int& BPL, bool forced) {
   const int k = p.k, nb = k >> 5;
   if (k % 256 != 0 || p.kr > 2) return false;
   // measured: the warp-streamed kernel is faster for long rows (k = 15360)
@@ -1195,7 +1263,11 @@ bool plan_cs(GemvParams& p, int& R, bool forced) {
     if (!aligned16(p.seg[s].qs) || !aligned16(p.seg[s].sc) || (s < p.nseg - 1 && p.seg[s].rows % 8))
       return false;
   if (p.pro == PRO_X16 && !aligned16(p.x)) return false;
-  const int NC = (nb + 31) / 32;
+  // two blocks per lane when the digits of one row fit the registers
+  // (Q4G_GEMV_BPL=1 forces one, a tuning switch)
+  static const int bpl_env = getenv("Q4G_GEMV_BPL") ? atoi(getenv("Q4G_GEMV_BPL")) : 0;
+  BPL = p.kr <= 1 && bpl_env != 1 ? 2 : 1;
+  const int NC = (nb + 32 * BPL - 1) / (32 * BPL);
   if (NC > kCsMaxConsumers) return false;
   int G = kCsMaxConsumers / NC;
   const int krm = p.kr <= 1 ? 1 : 2;
@@ -1221,15 +1293,15 @@ bool plan_cs(GemvParams& p, int& R, bool forced) {
   return true;
 }
 
-template <int KRM, int R>
+template <int KRM, int R, int BPL>
 cudaError_t launch_cs_r(const GemvParams& p, cudaStream_t st, bool pdl) {
   static size_t configured = 0;
   const size_t smem = cs_fixed_bytes(KRM, p.k, p.ns, p.nchunk, R) + (size_t)p.ns * p.stage_bytes;
   cudaError_t e;
   if (smem > configured) {
-    e = cudaFuncSetAttribute(gemv_q4_cs_kernel<KRM, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(gemv_q4_cs_kernel<KRM, R, BPL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(gemv_q4_cs_kernel<KRM, R>, cudaFuncAttributePreferredSharedMemoryCarveout,
+    e = cudaFuncSetAttribute(gemv_q4_cs_kernel<KRM, R, BPL>, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     configured = smem;
@@ -1246,14 +1318,372 @@ cudaError_t launch_cs_r(const GemvParams& p, cudaStream_t st, bool pdl) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, gemv_q4_cs_kernel<KRM, R>, p);
+  return cudaLaunchKernelEx(&cfg, gemv_q4_cs_kernel<KRM, R, BPL>, p);
 }
 
-template <int KRM>
+template <int KRM, int BPL>
 cudaError_t launch_cs_t(const GemvParams& p, int R, cudaStream_t st, bool pdl) {
-  if (R == 8) return launch_cs_r<KRM, 8>(p, st, pdl);
-  if (R == 4) return launch_cs_r<KRM, 4>(p, st, pdl);
-  return launch_cs_r<KRM, 2>(p, st, pdl);
+  if (R == 8) return launch_cs_r<KRM, 8, BPL>(p, st, pdl);
+  if (R == 4) return launch_cs_r<KRM, 4, BPL>(p, st, pdl);
+  return launch_cs_r<KRM, 2, BPL>(p, st, pdl);
+}
+
+// ---------------------------------------------------------------------------
+// Chain of q4_0 GEMVs in one persistent launch (one activation row).
+//
+// The GEMVs between two attention kernels of a decode step -- O(l),
+// gate|up(l), down(l) and QKV(l+1) -- depend on each other only through their
+// activations, never through their weights. One cooperative launch of one CTA
+// per SM runs them as phases:
+//   * the producer warp streams this CTA's unit range of every phase, phase
+//     after phase, through one ring of NS stage slots (one or two bulk copies
+//     per operand), never waiting for activations, so HBM keeps streaming
+//     while the consumers cross from one phase to the next;
+//   * before a phase the consumer warps wait until every CTA has finished the
+//     previous phase (a grid-wide counter, bounded wait), then build the
+//     integer digits of x for their own 32-column block straight into
+//     registers (RMSNorm reductions over the CTA use a named barrier that the
+//     producer never joins);
+//   * each stage is consumed as in the column-split kernel: warp (g, c) takes
+//     chunk c of the stages g, g + G, ...; the last of the NC warps of a stage
+//     adds the chunk partials in chunk order and runs the epilogue; the warp
+//     that completes the CTA's last stage of a phase publishes it grid-wide.
+// ---------------------------------------------------------------------------
+constexpr int kChainConsumers = 16;
+constexpr int kChainThreads = (kChainConsumers + 1) * 32;
+constexpr int kChainStages = 11;     // ring slots
+constexpr int kChainSlotBytes = 18432;  // largest stage: 8 rows x 4096 or 4 rows x 8192 columns
+
+Q4G_DEV void consumer_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kChainConsumers * 32) : "memory"); }
+
+Q4G_DEV int ld_acquire(const int32_t* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Integer digits (block_dot_int layout) of the 32 x values of block blk of
+// phase P's activation row, for one lane. PRO_RESID: the 512 consumer threads
+// first compute the normed row together (one round of loads, two reductions
+// over the consumer barrier in a fixed warp order) into the fp16 buffer xs;
+// every consumer warp calls this, warps without a block get zeros.
+constexpr int kChainMaxK = 8192;  // PRO_RESID rows
+
+Q4G_DEV void chain_digits(const GemvParams& P, int blk, bool has, float* s_norm, __half* xs, uint4 (&g)[6],
+                          int4& cv) {
+  const int k = P.k, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  constexpr int NT = kChainConsumers * 32;
+  __half xh[32];
+  if (P.pro == PRO_X16) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 v = has ? *reinterpret_cast<const uint4*>(P.x + (size_t)blk * 32 + 8 * q) : make_uint4(0, 0, 0, 0);
+      const __half* h = reinterpret_cast<const __half*>(&v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) xh[8 * q + e] = h[e];
+    }
+  } else {
+    constexpr int R4 = kChainMaxK / (4 * NT);
+    const int n4 = k >> 2;
+    const float4* rin = reinterpret_cast<const float4*>(P.r_in);
+    const float4* dl = reinterpret_cast<const float4*>(P.delta);
+    const float4* wd = reinterpret_cast<const float4*>(P.w_delta);
+    const float4* wx = reinterpret_cast<const float4*>(P.w_x);
+    float4 rn[R4], dv[R4], wdv[R4], wxv[R4];
+    const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < R4; ++i) {  // one round of loads
+      const int c4 = tid + i * NT;
+      const bool in = c4 < n4;
+      rn[i] = in ? rin[c4] : z4;
+      wxv[i] = in ? wx[c4] : z4;
+      dv[i] = in && dl ? dl[c4] : z4;
+      wdv[i] = in && dl ? wd[c4] : z4;
+    }
+    if (dl) {
+      float ss = 0.f;
+#pragma unroll
+      for (int i = 0; i < R4; ++i)
+        ss = fmaf(dv[i].x, dv[i].x, fmaf(dv[i].y, dv[i].y, fmaf(dv[i].z, dv[i].z, fmaf(dv[i].w, dv[i].w, ss))));
+      ss = warp_sum(ss);
+      if (lane == 0) s_norm[warp] = ss;
+      consumer_bar();
+      float tot = 0.f;
+#pragma unroll
+      for (int w = 0; w < kChainConsumers; ++w) tot += s_norm[w];
+      const float inv_d = rms_inv(tot, k, P.eps);
+#pragma unroll
+      for (int i = 0; i < R4; ++i) {
+        rn[i].x = __fmul_rn(__fadd_rn(rn[i].x, __fmul_rn(__fmul_rn(dv[i].x, inv_d), wdv[i].x)), P.scale);
+        rn[i].y = __fmul_rn(__fadd_rn(rn[i].y, __fmul_rn(__fmul_rn(dv[i].y, inv_d), wdv[i].y)), P.scale);
+        rn[i].z = __fmul_rn(__fadd_rn(rn[i].z, __fmul_rn(__fmul_rn(dv[i].z, inv_d), wdv[i].z)), P.scale);
+        rn[i].w = __fmul_rn(__fadd_rn(rn[i].w, __fmul_rn(__fmul_rn(dv[i].w, inv_d), wdv[i].w)), P.scale);
+      }
+    }
+    float ss2 = 0.f;
+#pragma unroll
+    for (int i = 0; i < R4; ++i) {
+      const int c4 = tid + i * NT;
+      ss2 = fmaf(rn[i].x, rn[i].x, fmaf(rn[i].y, rn[i].y, fmaf(rn[i].z, rn[i].z, fmaf(rn[i].w, rn[i].w, ss2))));
+      if (blockIdx.x == 0 && c4 < n4) {
+        reinterpret_cast<float4*>(P.r_out)[c4] = rn[i];
+        if (P.dump) reinterpret_cast<float4*>(P.dump)[c4] = rn[i];
+      }
+    }
+    ss2 = warp_sum(ss2);
+    if (lane == 0) s_norm[kChainConsumers + warp] = ss2;
+    consumer_bar();
+    float tot2 = 0.f;
+#pragma unroll
+    for (int w = 0; w < kChainConsumers; ++w) tot2 += s_norm[kChainConsumers + w];
+    const float inv_r = rms_inv(tot2, k, P.eps);
+#pragma unroll
+    for (int i = 0; i < R4; ++i) {
+      const int c4 = tid + i * NT;
+      if (c4 < n4) {
+        __half2* dst = reinterpret_cast<__half2*>(xs + 4 * c4);
+        dst[0] = __floats2half2_rn(__fmul_rn(__fmul_rn(rn[i].x, inv_r), wxv[i].x),
+                                   __fmul_rn(__fmul_rn(rn[i].y, inv_r), wxv[i].y));
+        dst[1] = __floats2half2_rn(__fmul_rn(__fmul_rn(rn[i].z, inv_r), wxv[i].z),
+                                   __fmul_rn(__fmul_rn(rn[i].w, inv_r), wxv[i].w));
+      }
+    }
+    consumer_bar();
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 v = has ? *reinterpret_cast<const uint4*>(xs + (size_t)blk * 32 + 8 * q) : make_uint4(0, 0, 0, 0);
+      const __half* h = reinterpret_cast<const __half*>(&v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) xh[8 * q + e] = h[e];
+    }
+  }
+  int em = 1;
+#pragma unroll
+  for (int e = 0; e < 32; ++e) em = max(em, half_exp(xh[e]));
+  int sd[3] = {0, 0, 0};
+  uint32_t words[3][8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const __half h4[4] = {xh[4 * q], xh[4 * q + 1], xh[4 * q + 2], xh[4 * q + 3]};
+    uint32_t wd[3];
+    digits4(h4, em, q >= 4, wd, sd);
+#pragma unroll
+    for (int t = 0; t < 3; ++t) words[t][q] = wd[t];
+  }
+#pragma unroll
+  for (int t = 0; t < 3; ++t) {
+    g[2 * t] = make_uint4(words[t][0], words[t][1], words[t][2], words[t][3]);
+    g[2 * t + 1] = make_uint4(words[t][4], words[t][5], words[t][6], words[t][7]);
+  }
+  cv = make_int4(-8 * sd[0], -8 * sd[1], -8 * sd[2], (em - 37 + 127) << 23);
+}
+
+struct ChainShared {
+  alignas(16) __half xs[kChainMaxK];            // the normed activation row (PRO_RESID), read as uint4
+  alignas(16) float red[kChainStages][kCsMaxConsumers][8];  // [slot][chunk][row]
+  uint64_t full[kChainStages], empty[kChainStages];
+  int cnt[kChainStages];                        // chunk warps done with a slot
+  int seq[kChainStages];                        // stage number last issued into each slot
+  int phase_done[kChainMaxPhases];              // stages of each phase finished in this CTA
+  float norm[2 * kChainConsumers];
+  int abort_flag;
+};
+
+template <int R>
+Q4G_DEV void chain_issue(const GemvParams& P, int u, unsigned char* st, uint64_t* bar, uint64_t pol) {
+  cs_issue<R>(P, u, st, bar, false, pol);
+}
+
+Q4G_DEV void chain_issue_r(const GemvParams& P, int u, unsigned char* st, uint64_t* bar, uint64_t pol) {
+  if (P.stage_rows == 8) chain_issue<8>(P, u, st, bar, pol);
+  else if (P.stage_rows == 4) chain_issue<4>(P, u, st, bar, pol);
+  else chain_issue<2>(P, u, st, bar, pol);
+}
+
+// One stage of phase P by consumer warp (chunk c): the R row partial sums go to
+// red[slot][c]; returns nothing, the caller runs the ticket.
+template <int R>
+Q4G_DEV void chain_stage(const GemvParams& P, const unsigned char* st, bool has, int blk, const uint4 (&xg)[6],
+                         const int4 cv, float* red_slot_c) {
+  const int kh = P.k >> 1, nb = P.k >> 5, lane = threadIdx.x & 31;
+  const float xsc = __int_as_float(cv.w);
+  float v[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    float a = 0.f;
+    if (has) {
+      const uint4 qv = lds_u4(st + (size_t)r * kh + (size_t)blk * 16);
+      const float d = __half2float(__ushort_as_half(
+          *reinterpret_cast<const uint16_t*>(st + (size_t)R * kh + (size_t)r * nb * 2 + (size_t)blk * 2)));
+      a = d * xsc * block_dot_int(qv, xg, cv);
+    }
+    v[r] = a;
+  }
+  const float tot = cs_reduce_rows<R>(v, lane);
+  if ((lane & (32 / R - 1)) == 0) red_slot_c[cs_row<R>(lane)] = tot;
+}
+
+__global__ void __launch_bounds__(kChainThreads, 1) gemv_q4_chain_kernel(const ChainParams c) {
+  extern __shared__ __align__(128) unsigned char chain_stages[];  // [kChainStages][kChainSlotBytes]
+  __shared__ __align__(16) ChainShared sh;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool producer = warp == kChainConsumers;
+  const int NS = kChainStages;
+  const uint64_t pol = policy_evict_first();
+
+  if (tid == 0) {
+    sh.abort_flag = 0;
+    for (int s = 0; s < NS; ++s) mbar_init(&sh.full[s], 1), mbar_init(&sh.empty[s], 1);
+    fence_mbar_init();
+  }
+  if (tid < NS) sh.cnt[tid] = 0, sh.seq[tid] = -1;
+  if (tid < kChainMaxPhases) sh.phase_done[tid] = 0;
+  __syncthreads();
+  volatile int* abort_flag = &sh.abort_flag;
+  const bool tr = c.trace && blockIdx.x == 0;
+  auto stamp = [&](int slot) {
+    if (tr) c.trace[slot] = global_ns();
+  };
+  // GemvParams-shaped view for the bounded waits (err word and limit)
+  GemvParams wp{};
+  wp.err = c.err;
+  wp.wait_ns = c.wait_ns;
+
+  if (producer) {
+    if (lane == 0) {
+      int t = 0;
+      for (int ph = 0; ph < c.n_ph; ++ph) {
+        const GemvParams& P = c.ph[ph];
+        const int u0 = (int)((long long)blockIdx.x * P.n_units / gridDim.x);
+        const int n_st = (int)((long long)(blockIdx.x + 1) * P.n_units / gridDim.x) - u0;
+        for (int i = 0; i < n_st; ++i, ++t) {
+          const int s = t % NS;
+          if (t >= NS && !*abort_flag) cs_wait(&sh.empty[s], (uint32_t)(((t - NS) / NS) & 1), wp, abort_flag);
+          if (*abort_flag) break;
+          chain_issue_r(P, u0 + i, chain_stages + (size_t)s * kChainSlotBytes, &sh.full[s], pol);
+          publish_issued(&sh.seq[s], t);
+        }
+        stamp(2 + 4 * ph + 3);
+        if (*abort_flag) break;
+      }
+      // after a timeout, wait (bounded) for the copies still in flight before exiting
+      if (*abort_flag)
+        for (int i = t > NS ? t - NS : 0; i < t; ++i)
+          mbar_wait_bounded(&sh.full[i % NS], (uint32_t)((i / NS) & 1), c.wait_ns);
+    }
+    return;
+  }
+
+  // ---------------- consumers ----------------
+  if (tid == 0) stamp(0);
+  pdl_wait();
+  if (tid == 0) stamp(1);
+  int t_base = 0;
+  for (int ph = 0; ph < c.n_ph; ++ph) {
+    const GemvParams& P = c.ph[ph];
+    const int NC = P.nchunk, G = P.groups, R = P.stage_rows, nb = P.k >> 5;
+    const int u0 = (int)((long long)blockIdx.x * P.n_units / gridDim.x);
+    const int n_st = (int)((long long)(blockIdx.x + 1) * P.n_units / gridDim.x) - u0;
+    if (ph == c.n_ph - 1) pdl_launch_dependents();
+    // every CTA finished the previous phase: its outputs are this phase's input
+    if (ph > 0) {
+      if (tid == 0 && !*abort_flag) {
+        const uint64_t t0 = global_ns();
+        for (int it = 0;; ++it) {
+          if (ld_acquire(&c.done[ph - 1]) >= (int)gridDim.x) break;
+          if (it >= kSpinLimit || global_ns() - t0 > c.wait_ns) {
+            *abort_flag = 1;
+            atomicOr(c.err, 1);
+            break;
+          }
+          __nanosleep(64);
+        }
+      }
+      consumer_bar();
+      __threadfence();
+    }
+    if (tid == 0) stamp(2 + 4 * ph);
+    const bool active = warp < NC * G;
+    const int cidx = warp % NC, g = warp / NC;
+    const int blk = 32 * cidx + lane;
+    const bool has = active && blk < nb;
+    uint4 xg[6];
+    int4 cv;
+    chain_digits(P, blk, has, sh.norm, sh.xs, xg, cv);
+    if (tid == 0) stamp(2 + 4 * ph + 1);
+    if (active) {
+      for (int i = g; i < n_st; i += G) {
+        const int t = t_base + i, s = t % NS;
+        if (!*abort_flag && wait_issued(&sh.seq[s], t, wp, abort_flag))
+          cs_wait(&sh.full[s], (uint32_t)((t / NS) & 1), wp, abort_flag);
+        const unsigned char* st = chain_stages + (size_t)s * kChainSlotBytes;
+        float* rs = &sh.red[s][0][0];
+        if (R == 8) chain_stage<8>(P, st, has, blk, xg, cv, rs + cidx * 8);
+        else if (R == 4) chain_stage<4>(P, st, has, blk, xg, cv, rs + cidx * 8);
+        else chain_stage<2>(P, st, has, blk, xg, cv, rs + cidx * 8);
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
+          __threadfence_block();
+          last = atomicAdd(&sh.cnt[s], 1) == NC - 1;
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (!last) continue;
+        __threadfence_block();
+        const int u = u0 + i;
+        float val = 0.f;
+        if (lane < R)
+          for (int cc = 0; cc < NC; ++cc) val += rs[cc * 8 + lane];
+        if (P.epi == EPI_GEGLU) {
+          const float up = __shfl_sync(0xffffffffu, val, (lane + R / 2) & 31);
+          if (lane < R / 2) P.act[(size_t)(R / 2) * u + lane] = __float2half_rn(gelu_tanh(val) * up);
+        } else if (lane < R && R * u + lane < P.n_rows) {
+          P.y[R * u + lane] = val;
+        }
+        __syncwarp();
+        if (lane == 0) {
+          sh.cnt[s] = 0;
+          mbar_arrive(&sh.empty[s]);
+          __threadfence();
+          if (atomicAdd(&sh.phase_done[ph], 1) == n_st - 1) {
+            __threadfence();
+            atomicAdd(&c.done[ph], 1);
+            stamp(2 + 4 * ph + 2);
+          }
+        }
+      }
+    }
+    if (n_st == 0 && tid == 0) atomicAdd(&c.done[ph], 1);
+    t_base += n_st;
+  }
+  if (tid == 0) stamp(18);
+}
+
+// Plan of one chain phase: rows per stage within a slot, chunks, groups.
+bool plan_chain_phase(GemvParams& p) {
+  const int k = p.k, nb = k >> 5;
+  if (k % 256 != 0 || p.kr != 1 || p.epi == EPI_HEAD) return false;
+  if (p.epi == EPI_GEGLU && (p.nseg != 2 || p.seg[0].rows != p.seg[1].rows || p.seg[0].rows % 4)) return false;
+  if (p.pro == PRO_RESID && k > 8192) return false;
+  for (int s = 0; s < p.nseg; ++s)
+    if (!aligned16(p.seg[s].qs) || !aligned16(p.seg[s].sc) || (s < p.nseg - 1 && p.seg[s].rows % 8))
+      return false;
+  if (p.pro == PRO_X16 && !aligned16(p.x)) return false;
+  const int NC = (nb + 31) / 32;
+  if (NC > kChainConsumers) return false;
+  const size_t row_bytes = (size_t)k / 2 + (size_t)k / 16;
+  auto units = [&](int r) { return p.epi == EPI_GEGLU ? p.seg[0].rows / (r / 2) : (p.n_rows + r - 1) / r; };
+  int R = 8;
+  while (R > 2 && (size_t)R * row_bytes > (size_t)kChainSlotBytes) R /= 2;
+  if ((size_t)R * row_bytes > (size_t)kChainSlotBytes) return false;
+  while (R > 2 && units(R) < device_sm_count()) R /= 2;  // small matrices: more, smaller stages
+  if (p.epi == EPI_GEGLU && p.seg[0].rows % (R / 2)) return false;
+  p.stage_rows = R;
+  p.nchunk = NC;
+  p.groups = std::min(kChainConsumers / NC, kChainStages - 2);
+  p.stage_bytes = (int)((size_t)R * row_bytes);
+  p.n_units = units(R);
+  return p.n_units >= 1;
 }
 
 // Kernel choice: Q4G_GEMV_KERNEL = "cs" (column-split) | "ws" (warp-streamed) |
@@ -1329,10 +1759,10 @@ int gemv_max_rows(int k) {
 NextGemv gemv_next_desc(const GemvParams& p_in, float frac) {
   NextGemv nx{};
   GemvParams p = p_in;
-  int dot = gemv_dot_kind(), R = 0;
+  int dot = gemv_dot_kind(), R = 0, BPL = 1;
   const int choice = gemv_kernel_choice();
   GemvParams px = p_in;
-  if (choice <= 0 && plan_cs(px, R, choice == 0)) {
+  if (choice <= 0 && plan_cs(px, R, BPL, choice == 0)) {
     // one stream per CTA: the first units of every CTA's range
     for (int s = 0; s < 3; ++s) nx.seg[s] = px.seg[s];
     nx.nseg = px.nseg;
@@ -1375,12 +1805,13 @@ int32_t* device_error_word() {
 cudaError_t launch_gemv(const GemvParams& p_in, cudaStream_t st, bool pdl) {
   GemvParams p = p_in;
   const int choice = gemv_kernel_choice();
-  int R = 0;
-  if (choice <= 0 && plan_cs(p, R, choice == 0)) {
+  int R = 0, BPL = 1;
+  if (choice <= 0 && plan_cs(p, R, BPL, choice == 0)) {
     if (!p.err) p.err = device_error_word();
     if (!p.err) return cudaErrorInvalidValue;
     if (!p.wait_ns) p.wait_ns = 2000000000ull;
-    return p.kr <= 1 ? launch_cs_t<1>(p, R, st, pdl) : launch_cs_t<2>(p, R, st, pdl);
+    if (p.kr > 1) return launch_cs_t<2, 1>(p, R, st, pdl);
+    return BPL == 2 ? launch_cs_t<1, 2>(p, R, st, pdl) : launch_cs_t<1, 1>(p, R, st, pdl);
   }
   p = p_in;
   int dot = gemv_dot_kind();
@@ -1403,6 +1834,51 @@ bool set_gemv_kernel_choice(int kind) {
   if (kind < 0 || kind > 3) return false;
   g_kernel_choice.store(kind - 1);
   return true;
+}
+
+bool plan_chain(ChainParams& c) {
+  if (c.n_ph < 1 || c.n_ph > kChainMaxPhases || gemv_kernel_choice() > 0) return false;
+  for (int i = 0; i < c.n_ph; ++i)
+    if (!plan_chain_phase(c.ph[i])) return false;
+  return true;
+}
+
+cudaError_t launch_gemv_chain(const ChainParams& c_in, cudaStream_t st, bool pdl) {
+  ChainParams c = c_in;
+  if (!c.err) c.err = device_error_word();
+  if (!c.err) return cudaErrorInvalidValue;
+  if (!c.wait_ns) c.wait_ns = 2000000000ull;
+  static bool configured = false;
+  const size_t smem = (size_t)kChainStages * kChainSlotBytes;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(gemv_q4_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(gemv_q4_chain_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  // one CTA per SM, and at least one unit of every phase per CTA
+  int grid = device_sm_count();
+  for (int i = 0; i < c.n_ph; ++i) grid = std::min(grid, c.ph[i].n_units);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kChainThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeCooperative;  // all CTAs resident: the phases wait on each other
+  attr[na].val.cooperative = 1;
+  ++na;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, gemv_q4_chain_kernel, c);
 }
 
 int device_sm_count() {

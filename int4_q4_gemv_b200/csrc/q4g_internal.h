@@ -87,6 +87,25 @@ size_t gemv_smem_bytes(int krm, int k);
 cudaError_t launch_gemv(const GemvParams& p, cudaStream_t st, bool pdl);
 // Q4G_GEMV_* kind; false if out of range
 bool set_gemv_kernel_choice(int kind);
+
+// Consecutive GEMVs of a decode step (one activation row) in one persistent,
+// cooperative launch; phase i + 1 starts once every CTA has finished phase i.
+constexpr int kChainMaxPhases = 4;
+struct ChainParams {
+  GemvParams ph[kChainMaxPhases];
+  int32_t n_ph;
+  int32_t* done;      // [n_ph] CTAs that finished each phase; zero before the launch
+  int32_t* err;       // bounded-wait error word (NULL: the library's)
+  uint64_t wait_ns;   // bounded-wait limit (0: 2 s)
+  uint64_t* trace;    // optional [kChainTraceSlots] %globaltimer stamps of CTA 0
+};
+// trace slots of one chain launch: 0 start, 1 after griddepcontrol.wait, then per
+// phase i at 2 + 4 i: inputs ready, digits built, last own stage done, producer
+// done issuing; 18 end
+constexpr int kChainTraceSlots = 32;
+// Plans every phase in place; false if a phase does not fit the chain kernel.
+bool plan_chain(ChainParams& c);
+cudaError_t launch_gemv_chain(const ChainParams& c, cudaStream_t st, bool pdl);
 // Descriptor of GEMV `p` as the next GEMV of a prefetch (tw = 0 if p does not
 // take the streamed path).
 NextGemv gemv_next_desc(const GemvParams& p, float frac);

@@ -15,8 +15,10 @@ LIB_PATH = os.path.join(_HERE, "libq4g.so")
 Q4G_OK, Q4G_EINVAL, Q4G_ERANGE, Q4G_ENOMEM, Q4G_ECUDA, Q4G_ETIMEOUT = range(6)
 Q4G_OPT_CUDA_GRAPH, Q4G_OPT_PDL, Q4G_OPT_DUMP, Q4G_OPT_PROFILE, Q4G_OPT_TEST_STALL = 1, 2, 3, 4, 5
 Q4G_OPT_ATTN_CLUSTER = 6
+Q4G_OPT_GEMV_CHAIN = 7
+Q4G_OPT_TRACE = 8
 KIND_NAMES = ["step_init", "qkv_gemv", "attn_sliding", "attn_full", "attn_combine", "o_gemv",
-              "gate_up_gemv", "down_gemv", "head_gemv"]
+              "gate_up_gemv", "down_gemv", "head_gemv", "chain_gemv"]
 
 EXPORTS = [
     "q4g_last_error", "q4g_status_string", "q4g_abi_version",

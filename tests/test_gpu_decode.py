@@ -144,15 +144,17 @@ def test_tiny_free_greedy_on_device_tokens():
     assert am.cpu().tolist() == seq_ref
 
 
-@pytest.mark.parametrize("cluster", [1, 0])
-def test_wrap_heavy_ring_and_layer_dumps(cluster):
+@pytest.mark.parametrize("cluster,chain", [(1, 1), (0, 0)])
+def test_wrap_heavy_ring_and_layer_dumps(cluster, chain):
     """300 positions through a ring of 64 slots (> 4 wraps), seeded gains and layer
     scalars; residual stream compared after every layer. Both merges of the
     sliding-layer attention chunks: in a thread-block cluster (8 CTAs per KV
-    head, most of them with no live key here) and through global memory."""
+    head, most of them with no live key here) and through global memory; and
+    the layer's GEMVs as one persistent chain launch or one launch each."""
     cfg = WRAP
     p = Pair(cfg, seed=5, variant=1, capacity=320)
     Q.q4g_model_set_option(p.gpu.handle, Q.Q4G_OPT_ATTN_CLUSTER, cluster)
+    Q.q4g_model_set_option(p.gpu.handle, Q.Q4G_OPT_GEMV_CHAIN, chain)
     L, H = cfg["n_layers"], cfg["hidden"]
     dump = torch.zeros((1, L + 1, H), dtype=torch.float32, device="cuda")
     Q.q4g_model_set_option(p.gpu.handle, Q.Q4G_OPT_DUMP, dump.data_ptr())
