@@ -101,19 +101,26 @@ q4g_status q4g_gemv(const uint8_t* qs, const uint16_t* scales, int64_t n, int64_
 /* Process-wide choice of the q4_0 GEMV kernel, for tuning and tests (not on
  * the pages). All kernels compute the same operation within the same error
  * bound; the default picks per shape:
- *   Q4G_GEMV_AUTO          shape-based choice (default; Q4G_GEMV_KERNEL=cs|ws|reg
- *                          in the environment overrides it at first use),
+ *   Q4G_GEMV_AUTO          the stage kernel where it can take the call, else a
+ *                          shape-based choice among the next three (default;
+ *                          Q4G_GEMV_KERNEL=cs|ws|reg|stage in the environment
+ *                          overrides it at first use),
  *   Q4G_GEMV_COLUMN_SPLIT  integer dot, x digits resident per chunk, one
  *                          contiguous bulk-copy stream per CTA (k % 256 == 0,
  *                          <= 2 activation rows, 16-byte aligned operands),
  *   Q4G_GEMV_WARP_STREAM   per-warp bulk-copy rings (k % 256 == 0),
- *   Q4G_GEMV_REGISTER      plain streaming loads (any k % 32 == 0).
- * A kernel that cannot take a call falls back down this list. Affects launches
+ *   Q4G_GEMV_REGISTER      plain streaming loads (any k % 32 == 0),
+ *   Q4G_GEMV_STAGE         integer dot, every warp of a CTA on each 16-36 KB
+ *                          stage of one contiguous bulk-copy stream, one warp
+ *                          reducing and refilling (k % 256 == 0, <= 2
+ *                          activation rows, 16-byte aligned operands).
+ * A kernel that cannot take a call falls back down this list (STAGE to AUTO). Affects launches
  * made (and CUDA graphs captured) after the call. Q4G_EINVAL for other kinds. */
 #define Q4G_GEMV_AUTO 0
 #define Q4G_GEMV_COLUMN_SPLIT 1
 #define Q4G_GEMV_WARP_STREAM 2
 #define Q4G_GEMV_REGISTER 3
+#define Q4G_GEMV_STAGE 4
 q4g_status q4g_set_gemv_kernel(int32_t kind);
 
 /* Workspace for the split-KV flash-decode entry points below (bytes, >= 256). */
@@ -264,7 +271,15 @@ typedef enum {
                                  its CTA 0 to row l: 0 start, 1 dependency wait done,
                                  per phase i at 2 + 4i: inputs ready, x digits built,
                                  last stage of CTA 0 done, producer done issuing;
-                                 18 end. Unwritten slots keep their contents. */
+                                 18 end. With GEMV_CHAIN 0 the buffer must hold 1024
+                                 entries instead: 256 each for gate|up, QKV, O and
+                                 down of layer 1 when they run on the column-split
+                                 kernel, per launch 0 entry, 1 dependency wait done,
+                                 2 x digits built, 3 and 4 (fused norm prologue)
+                                 first loads used and second norm reduced, 8 + t
+                                 stage t issued, 72 + t stage t ready, 136 + t
+                                 stage t reduced (t < 64).
+                                 Unwritten slots keep their contents. */
 } q4g_option;
 q4g_status q4g_model_set_option(q4g_model* m, q4g_option opt, intptr_t value);
 

@@ -495,7 +495,7 @@ extern "C" q4g_status q4g_q4_0_unpack(const uint8_t* qs, const uint16_t* scales,
 }
 
 extern "C" q4g_status q4g_set_gemv_kernel(int32_t kind) {
-  if (!set_gemv_kernel_choice(kind)) return fail(Q4G_EINVAL, "GEMV kernel kind must be 0..3");
+  if (!set_gemv_kernel_choice(kind)) return fail(Q4G_EINVAL, "GEMV kernel kind must be 0..4");
   return Q4G_OK;
 }
 
@@ -824,9 +824,12 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
     const LayerShape& S = full ? m->gl : m->sl;
     const int ord = m->ordinal[l];
     const GemvParams gate_up = gate_up_params(l);
+    // separate launches: the timeline of layer 1's QKV and gate|up (CTA 0)
+    uint64_t* const trace_sep = m->trace && !m->gemv_chain && l == 1 ? m->trace : nullptr;
     if (!qkv_done) {
       GemvParams p = qkv_params(l);
       p.next = next_of(o_params(l, 0), 1.0f);
+      p.trace = trace_sep ? trace_sep + kGemvTraceSlots : nullptr;
       if (l == 0 && m->stall_next) {
         p.stall_test = 1;
         p.wait_ns = 20000000ull;  // 20 ms
@@ -914,6 +917,7 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
       for (int r0 = 0; r0 < kr; r0 += maxr) {
         GemvParams p = o_params(l, r0);
         if (r0 + maxr >= kr) p.next = next_of(gate_up, 0.35f);
+        p.trace = trace_sep && r0 == 0 ? trace_sep + 2 * kGemvTraceSlots : nullptr;
         Prof pr(m, st);
         e = pr.done(debug_sync(launch_gemv(p, st, pdl), "o_proj", l, st), 5, l, gemv_bytes(H, kin, p.kr, 4));
         if (e != cudaSuccess) return e;
@@ -922,6 +926,7 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
     {
       GemvParams p = gate_up;
       p.next = next_of(down_params(l, 0), 0.6f);
+      p.trace = trace_sep;
       Prof pr(m, st);
       e = pr.done(debug_sync(launch_gemv(p, st, pdl), "gate_up", l, st), 6, l, gemv_bytes(2 * cf.ffn, H, kr, 1));
       if (e != cudaSuccess) return e;
@@ -931,6 +936,7 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
       for (int r0 = 0; r0 < kr; r0 += maxr) {
         GemvParams p = down_params(l, r0);
         if (r0 + maxr >= kr) p.next = l + 1 < L ? next_of(qkv_params(l + 1), 1.0f) : next_of(head_params(), 0.05f);
+        p.trace = trace_sep && r0 == 0 ? trace_sep + 3 * kGemvTraceSlots : nullptr;
         Prof pr(m, st);
         e = pr.done(debug_sync(launch_gemv(p, st, pdl), "down", l, st), 7, l, gemv_bytes(H, cf.ffn, p.kr, 4));
         if (e != cudaSuccess) return e;

@@ -32,6 +32,10 @@ namespace q4g {
 
 namespace {
 
+// x digits of the integer dot product per block and activation row: 4 uint4
+// (digit 0 / 1 of the low / high 16 columns), see block_dot_int.
+constexpr int kDigitQuads = 4;
+
 // Slot of column e (0..31) of a block in the x layout (inverse of xperm).
 Q4G_DEV int xslot(int e) {
   const int hi = e >> 4, e2 = e & 15, k = e2 >> 2, o = e2 & 3;
@@ -176,6 +180,7 @@ Q4G_DEV void produce_x(const GemvParams& p, float* misc, Emit&& emit) {
           ss = fmaf(dv[i].w, dv[i].w, ss);
         }
       }
+      if (p.trace && blockIdx.x == 0 && tid == 0) p.trace[3] = global_ns();
       if (dl) {
         const float inv_d = rms_inv(block_sum<NT>(ss, misc), k, p.eps);
 #pragma unroll
@@ -206,6 +211,7 @@ Q4G_DEV void produce_x(const GemvParams& p, float* misc, Emit&& emit) {
         }
       }
       const float inv_r = rms_inv(block_sum<NT>(ss2, misc + 32), k, p.eps);
+      if (p.trace && blockIdx.x == 0 && tid == 0) p.trace[4] = global_ns();
 #pragma unroll
       for (int i = 0; i < R4; ++i) {
         const int c4 = tid + i * NT;
@@ -255,30 +261,26 @@ Q4G_DEV void stage_x(const GemvParams& p, uint4* xs, float* cblk, float* misc) {
   __syncthreads();
 }
 
-// Digits of 4 consecutive columns of one block (see block_dot_int): v_i =
-// rint(x_i * 2^(37 - Emax)) for low columns, rint(x_i * 2^(33 - Emax)) for high
-// ones. Exact: |x| * 2^(37 - Emax) < 2^23 and the scaling is a power of two.
-// Returns one packed word per digit (bytes = digits of the 4 columns) and adds
-// the (weighted) digit sums to sd.
-Q4G_DEV void digits4(const __half (&h)[4], int em, bool high, uint32_t (&wd)[3], int (&sd)[3]) {
-  const float sc = __int_as_float(((high ? 33 : 37) - em + 127) << 23);
+// Digits of 4 consecutive columns of one block (see block_dot_int):
+// X_i = rint(x_i * 2^(29 - Emax)), |X_i| < 2^15 (the scaling is a power of two).
+// Returns one packed word per digit (byte e = digit of column e: byte 0 of X
+// unsigned, byte 1 signed) and adds the digit sums to sd.
+Q4G_DEV void digits4(const __half (&h)[4], int em, uint32_t (&wd)[2], int (&sd)[2]) {
+  const float sc = __int_as_float((29 - em + 127) << 23);
   int X[4];
 #pragma unroll
   for (int e = 0; e < 4; ++e) X[e] = __float2int_rn(__half2float(h[e]) * sc);
-  // byte t of every X: t = 0, 1 unsigned digits, t = 2 the signed top digit
 #pragma unroll
-  for (int t = 0; t < 3; ++t) {
+  for (int t = 0; t < 2; ++t) {
     const uint32_t sel = 0x0040u | (uint32_t)(t * 0x11);  // bytes (x.b_t, y.b_t)
     const uint32_t lo = __byte_perm((uint32_t)X[0], (uint32_t)X[1], sel);
     const uint32_t hi = __byte_perm((uint32_t)X[2], (uint32_t)X[3], sel);
     wd[t] = __byte_perm(lo, hi, 0x5410);
   }
-  const int m = high ? 16 : 1;
-  sd[0] += m * dp4a_uu(wd[0], 0x01010101u, 0);
-  sd[1] += m * dp4a_uu(wd[1], 0x01010101u, 0);
-  int s2;
-  asm("dp4a.s32.s32 %0, %1, %2, %3;" : "=r"(s2) : "r"(wd[2]), "r"(0x01010101u), "r"(0));
-  sd[2] += m * s2;
+  sd[0] += dp4a_uu(wd[0], 0x01010101u, 0);
+  int s1;
+  asm("dp4a.s32.s32 %0, %1, %2, %3;" : "=r"(s1) : "r"(wd[1]), "r"(0x01010101u), "r"(0));
+  sd[1] += s1;
 }
 
 Q4G_DEV int half_exp(__half h) {
@@ -300,23 +302,20 @@ Q4G_DEV void stage_digits(const GemvParams& p, uint4* dg, int4* bc, float* misc)
     em = max(em, __shfl_xor_sync(0xffffffffu, em, 1));
     em = max(em, __shfl_xor_sync(0xffffffffu, em, 2));
     em = max(em, __shfl_xor_sync(0xffffffffu, em, 4));
-    uint32_t wdg[3];
-    int sd[3] = {0, 0, 0};
-    digits4(h, em, sub >= 4, wdg, sd);
-    const uint32_t w0 = wdg[0], w1 = wdg[1], w2 = wdg[2];
-    int s0 = sd[0], s1 = sd[1], s2 = sd[2];
+    uint32_t wdg[2];
+    int sd[2] = {0, 0};
+    digits4(h, em, wdg, sd);
+    int s0 = sd[0], s1 = sd[1];
 #pragma unroll
     for (int o = 1; o < 8; o <<= 1) {
       s0 += __shfl_xor_sync(0xffffffffu, s0, o);
       s1 += __shfl_xor_sync(0xffffffffu, s1, o);
-      s2 += __shfl_xor_sync(0xffffffffu, s2, o);
     }
     if (valid) {
       const int hh = sub >> 2, wd = sub & 3;
-      dw[((size_t)(j * 6 + 0 + hh) * nb + blk) * 4 + wd] = w0;
-      dw[((size_t)(j * 6 + 2 + hh) * nb + blk) * 4 + wd] = w1;
-      dw[((size_t)(j * 6 + 4 + hh) * nb + blk) * 4 + wd] = w2;
-      if (sub == 0) bc[j * nb + blk] = make_int4(-8 * s0, -8 * s1, -8 * s2, (em - 37 + 127) << 23);
+      dw[((size_t)(j * kDigitQuads + 0 + hh) * nb + blk) * 4 + wd] = wdg[0];
+      dw[((size_t)(j * kDigitQuads + 2 + hh) * nb + blk) * 4 + wd] = wdg[1];
+      if (sub == 0) bc[j * nb + blk] = make_int4(-8 * s0, -8 * s1, 0, (em - 29 + 127) << 23);
     }
   });
   __syncthreads();
@@ -574,40 +573,34 @@ Q4G_DEV void issue_item(const GemvParams& p, int u, int c, unsigned char* st, ui
 // ---------------------------------------------------------------------------
 // Integer form of the block dot product.
 //
-// x of one block (32 fp16 values) becomes signed 24-bit fixed point relative to
-// the block's largest exponent: X_i = round(x_i * 2^(37 - Emax)), exact for
-// every value within 2^12 of the block maximum (the rest carry an error below
-// 2^-24 of the block maximum), x_i ~= X_i * 2^(Emax - 37).
+// x of one block (32 fp16 values) becomes signed 16-bit fixed point relative to
+// the block's largest exponent: X_i = round(x_i * 2^(29 - Emax)), |X_i| < 2^15,
+// exact for every value within 2^4 of the block maximum; the rest carry an
+// error of at most 2^-15 of the block maximum. x_i ~= X_i * 2^(Emax - 29).
 // The code byte b of a block holds column b in its low nibble and column b + 16
-// in its high nibble. Masking a code word with 0x0F0F0F0F gives four low codes
-// c; masking it with 0xF0F0F0F0 gives four high codes as 16 c. So the high
-// columns use Y_i = round(X_i / 16) (error <= 8 units of X, 2^-20 of the block
-// maximum) and 16 c Y_i stands for c X_i: every code word costs two masks.
-// The values (X for columns 0..15, Y for 16..31) split into bytes
-// v = d0 + 256 d1 + 65536 d2 (d0, d1 unsigned, d2 signed), so with m_i = 1 for
-// low and 16 for high columns
-//   sum_i (c_i - 8) m_i v_i = S0 + 256 S1 + 65536 S2,
-//   S_t = sum_i (m_i c_i) d_t,i - 8 sum_i m_i d_t,i,
-// and each S_t is a chain of 4-way byte dot products (dp4a) started at the
-// constant -8 sum_i m_i d_t,i. Every S_t is exact in int32.
+// in its high nibble, so a code word w gives the four low codes as
+// w & 0x0F0F0F0F and the four high codes as (w >> 4) & 0x0F0F0F0F.
+// X splits into bytes X = d0 + 256 d1 (d0 unsigned, d1 signed), and
+//   sum_i (c_i - 8) X_i = S0 + 256 S1,  S_t = sum_i c_i d_t,i - 8 sum_i d_t,i,
+// each S_t a chain of 4-way byte dot products (dp4a) started at the constant
+// -8 sum_i d_t,i. S0, S1 and S0 + 256 S1 (|.| <= 32 * 8 * 2^15 = 2^23) are exact
+// in int32 and the last one in fp32.
 // Layout per x row j: dg[j][2t + h][blk] holds digit t of columns 16h..16h+15
-// of block blk (16 bytes), bc[j][blk] = (-8 D0, -8 D1, -8 D2, bits of 2^(Emax-37))
-// with D_t = sum_i m_i d_t,i, written by stage_digits.
+// of block blk (16 bytes), bc[j][blk] = (-8 D0, -8 D1, 0, bits of 2^(Emax-29))
+// with D_t = sum_i d_t,i, written by stage_digits.
 // ---------------------------------------------------------------------------
-Q4G_DEV float block_dot_int(const uint4 q, const uint4 (&g)[6], const int4 c) {
+Q4G_DEV float block_dot_int(const uint4 q, const uint4 (&g)[kDigitQuads], const int4 c) {
   const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-  int s0 = c.x, s1 = c.y, s2 = c.z;
+  int s0 = c.x, s1 = c.y;
 #pragma unroll
   for (int t = 0; t < 4; ++t) {
-    const uint32_t lo = w[t] & 0x0F0F0F0Fu, hi = w[t] & 0xF0F0F0F0u;  // hi: 16 x the high codes
+    const uint32_t lo = w[t] & 0x0F0F0F0Fu, hi = (w[t] >> 4) & 0x0F0F0F0Fu;
     s0 = dp4a_uu(lo, (&g[0].x)[t], s0);
     s0 = dp4a_uu(hi, (&g[1].x)[t], s0);
-    s1 = dp4a_uu(lo, (&g[2].x)[t], s1);
-    s1 = dp4a_uu(hi, (&g[3].x)[t], s1);
-    s2 = dp4a_us(lo, (&g[4].x)[t], s2);
-    s2 = dp4a_us(hi, (&g[5].x)[t], s2);
+    s1 = dp4a_us(lo, (&g[2].x)[t], s1);
+    s1 = dp4a_us(hi, (&g[3].x)[t], s1);
   }
-  return fmaf((float)s2, 65536.0f, (float)(s1 * 256 + s0));
+  return (float)(s1 * 256 + s0);
 }
 
 // Shared memory of the warp-streamed kernel: the x region (layout per dot
@@ -617,7 +610,7 @@ enum : int { DOT_FMA_HALF = 0, DOT_FMA = 1, DOT_INT = 2 };
 
 __host__ __device__ inline size_t x_region_bytes(int dot, int krm, int k) {
   const size_t nb = (size_t)k / 32;
-  return dot == DOT_INT ? (size_t)krm * nb * (96 + 16) : (size_t)krm * nb * (64 + 4);
+  return dot == DOT_INT ? (size_t)krm * nb * (16 * kDigitQuads + 16) : (size_t)krm * nb * (64 + 4);
 }
 
 template <int KRM, int DOT>
@@ -626,9 +619,9 @@ __global__ void __launch_bounds__(kWarpThreads, 1) gemv_q4_tma_kernel(const Gemv
   const int k = p.k, nb = k >> 5, NS = p.ns;
   const int kc = p.kc, nbc = kc >> 5, qb = kc >> 1;
   // x region
-  uint4* xs = reinterpret_cast<uint4*>(ws_smem);                        // FMA: [KRM][4][nb]; INT: dg [KRM][6][nb]
+  uint4* xs = reinterpret_cast<uint4*>(ws_smem);                        // FMA: [KRM][4][nb]; INT: dg [KRM][kDigitQuads][nb]
   float* cblk = reinterpret_cast<float*>(xs + (size_t)KRM * 4 * nb);     // FMA: [KRM][nb]
-  int4* bc = reinterpret_cast<int4*>(xs + (size_t)KRM * 6 * nb);         // INT: [KRM][nb]
+  int4* bc = reinterpret_cast<int4*>(xs + (size_t)KRM * kDigitQuads * nb);  // INT: [KRM][nb]
   float* misc = reinterpret_cast<float*>(ws_smem + x_region_bytes(DOT, KRM, k));  // 64 floats
   float* bestv = misc + 64;                                              // [kWarps]
   int* besti = reinterpret_cast<int*>(bestv + kWarps);                   // [kWarps]
@@ -730,9 +723,9 @@ __global__ void __launch_bounds__(kWarpThreads, 1) gemv_q4_tma_kernel(const Gemv
                 acc[0][j] = fmaf(d0, a0 + a1, acc[0][j]);
                 acc[1][j] = fmaf(d1, b0 + b1, acc[1][j]);
               } else {
-                uint4 g[6];
+                uint4 g[kDigitQuads];
 #pragma unroll
-                for (int q = 0; q < 6; ++q) g[q] = lds_u4(xs + (size_t)(j * 6 + q) * nb + blk);
+                for (int q = 0; q < kDigitQuads; ++q) g[q] = lds_u4(xs + (size_t)(j * kDigitQuads + q) * nb + blk);
                 const int4 cv = bc[j * nb + blk];
                 const float xsc = __int_as_float(cv.w);
                 acc[0][j] = fmaf(d0 * xsc, block_dot_int(q0, g, cv), acc[0][j]);
@@ -950,7 +943,7 @@ __host__ __device__ inline size_t cs_red_floats(int ns, int nc, int rows, int kr
 __host__ __device__ inline size_t cs_fixed_bytes(int krm, int k, int ns, int nc, int rows) {
   const size_t nb = (size_t)k / 32;
   const size_t red = (cs_red_floats(ns, nc, rows, krm) * 4 + 15) & ~(size_t)15;
-  return (size_t)krm * nb * 112 + 64 * 4 + red + 128 + 2 * kCsMaxStages * 8;
+  return (size_t)krm * nb * (16 * kDigitQuads + 16) + 64 * 4 + red + 128 + 2 * kCsMaxStages * 8;
 }
 
 // Sum v[0..R) over the 32 lanes: after the butterfly, lanes with (lane & (32/R
@@ -1048,8 +1041,8 @@ template <int KRM, int R, int BPL>
 __global__ void __launch_bounds__(kCsThreads, 1) gemv_q4_cs_kernel(const GemvParams p) {
   extern __shared__ __align__(16) unsigned char cs_smem[];
   const int k = p.k, nb = k >> 5, kh = k >> 1, NS = p.ns, NC = p.nchunk, G = p.groups;
-  uint4* dg = reinterpret_cast<uint4*>(cs_smem);                          // [KRM][6][nb]
-  int4* bc = reinterpret_cast<int4*>(dg + (size_t)KRM * 6 * nb);          // [KRM][nb]
+  uint4* dg = reinterpret_cast<uint4*>(cs_smem);                          // [KRM][kDigitQuads][nb]
+  int4* bc = reinterpret_cast<int4*>(dg + (size_t)KRM * kDigitQuads * nb);  // [KRM][nb]
   float* misc = reinterpret_cast<float*>(bc + (size_t)KRM * nb);          // 64 floats
   float* red = misc + 64;                                                 // [NS][NC][R][KRM]
   const size_t red_bytes = (cs_red_floats(NS, NC, R, KRM) * 4 + 15) & ~(size_t)15;
@@ -1074,47 +1067,59 @@ __global__ void __launch_bounds__(kCsThreads, 1) gemv_q4_cs_kernel(const GemvPar
   const size_t SB = (size_t)p.stage_bytes;
   const uint64_t pol = policy_evict_first();
   int issued = 0;
+  uint64_t* const tr = blockIdx.x == 0 ? p.trace : nullptr;
+  auto stamp = [&](int i) {
+    if (tr) tr[i] = global_ns();
+  };
 
-  if (tid == 0) s_abort = 0;
+  if (tid == 0) stamp(0), s_abort = 0;
   if (tid < kCsMaxStages) s_cnt[tid] = 0, s_seq[tid] = -1;
   if (tid < kCsMaxConsumers) s_bestv[tid] = -INFINITY, s_besti[tid] = 0x7fffffff;
   if (producer && lane == 0) {
     for (int s = 0; s < NS; ++s) mbar_init(&full[s], 1), mbar_init(&empty[s], 1);
     fence_mbar_init();
-    for (; issued < NS && issued < n_st; ++issued)
+    const int pre = p.prefetch_stages > 0 ? min(NS, p.prefetch_stages) : NS;
+    for (; issued < pre && issued < n_st; ++issued) {
       cs_issue<R>(p, u0 + issued, stages + issued * SB, &full[issued],
                   p.stall_test && u0 == 0 && issued == 0, pol);  // the CTA owning unit 0
+      if (issued < 64) stamp(8 + issued);
+    }
   }
   __syncthreads();  // s_seq initialised before the producer publishes
   if (producer && lane == 0)
     for (int i = 0; i < issued; ++i) publish_issued(&s_seq[i], i);
   pdl_wait();
+  if (tid == 0) stamp(1);
   stage_digits<KRM, kCsThreads>(p, dg, bc, misc);  // ends with __syncthreads
+  if (tid == 0) stamp(2);
   pdl_launch_dependents();
   volatile int* abort_flag = &s_abort;
 
   if (warp < n_cons) {
     // ---------------- consumer: chunk c, stages g, g + G, ... ----------------
-    // lane l holds blocks 32 BPL c + l + 32 b, b < BPL, of every row
+    // lane l holds blocks 32 BPL c + l + 32 b, b < BPL, of every row. A lane
+    // past the end of the row reads block nb - 1 with zero digits and a zero
+    // x scale, so the loop below has no branch.
     const int c = warp % NC, g = warp / NC;
-    int blkb[BPL];
-    bool hasb[BPL];
-    uint4 xg[KRM][BPL][6];
+    int qoff[BPL], soff[BPL];
+    uint4 xg[KRM][BPL][kDigitQuads];
     int4 cv[KRM][BPL];
     float xsc[KRM][BPL];
 #pragma unroll
     for (int b = 0; b < BPL; ++b) {
-      blkb[b] = 32 * BPL * c + lane + 32 * b;
-      hasb[b] = blkb[b] < nb;
+      const int blk = 32 * BPL * c + lane + 32 * b;
+      const bool has = blk < nb;
+      qoff[b] = 16 * min(blk, nb - 1);
+      soff[b] = 2 * min(blk, nb - 1);
 #pragma unroll
       for (int j = 0; j < KRM; ++j) {
-        if (hasb[b] && (KRM == 1 || j < p.kr)) {
+        if (has && (KRM == 1 || j < p.kr)) {
 #pragma unroll
-          for (int q = 0; q < 6; ++q) xg[j][b][q] = dg[(size_t)(j * 6 + q) * nb + blkb[b]];
-          cv[j][b] = bc[j * nb + blkb[b]];
+          for (int q = 0; q < kDigitQuads; ++q) xg[j][b][q] = dg[(size_t)(j * kDigitQuads + q) * nb + blk];
+          cv[j][b] = bc[j * nb + blk];
         } else {
 #pragma unroll
-          for (int q = 0; q < 6; ++q) xg[j][b][q] = make_uint4(0, 0, 0, 0);
+          for (int q = 0; q < kDigitQuads; ++q) xg[j][b][q] = make_uint4(0, 0, 0, 0);
           cv[j][b] = make_int4(0, 0, 0, 0);
         }
         xsc[j][b] = __int_as_float(cv[j][b].w);
@@ -1126,7 +1131,9 @@ __global__ void __launch_bounds__(kCsThreads, 1) gemv_q4_cs_kernel(const GemvPar
     uint32_t ph = (uint32_t)((g / NS) & 1);
     for (int t = g; t < n_st; t += G) {
       if (!*abort_flag && wait_issued(&s_seq[s], t, p, abort_flag)) cs_wait(&full[s], ph, p, abort_flag);
+      if (c == 0 && lane == 0 && t < 64) stamp(72 + t);
       const unsigned char* st = stages + s * SB;
+      const unsigned char* ss = st + R * kh;
       float v[KRM][R];
 #pragma unroll
       for (int r = 0; r < R; ++r) {
@@ -1135,14 +1142,11 @@ __global__ void __launch_bounds__(kCsThreads, 1) gemv_q4_cs_kernel(const GemvPar
         for (int j = 0; j < KRM; ++j) a[j] = 0.f;
 #pragma unroll
         for (int b = 0; b < BPL; ++b) {
-          if (hasb[b]) {
-            const uint4 qv = lds_u4(st + (size_t)r * kh + (size_t)blkb[b] * 16);
-            const float d = __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(
-                st + (size_t)R * kh + (size_t)r * nb * 2 + (size_t)blkb[b] * 2)));
+          const uint4 qv = *reinterpret_cast<const uint4*>(st + r * kh + qoff[b]);
+          const float d = __half2float(*reinterpret_cast<const __half*>(ss + r * 2 * nb + soff[b]));
 #pragma unroll
-            for (int j = 0; j < KRM; ++j)
-              if (KRM == 1 || j < p.kr) a[j] = fmaf(d * xsc[j][b], block_dot_int(qv, xg[j][b], cv[j][b]), a[j]);
-          }
+          for (int j = 0; j < KRM; ++j)
+            if (KRM == 1 || j < p.kr) a[j] = fmaf(d * xsc[j][b], block_dot_int(qv, xg[j][b], cv[j][b]), a[j]);
         }
 #pragma unroll
         for (int j = 0; j < KRM; ++j) v[j][r] = a[j];
@@ -1189,6 +1193,7 @@ __global__ void __launch_bounds__(kCsThreads, 1) gemv_q4_cs_kernel(const GemvPar
         if (lane == 0) {
           s_cnt[s] = 0;
           mbar_arrive(&empty[s]);
+          if (t < 64) stamp(136 + t);
         }
       }
       s += G;
@@ -1206,12 +1211,13 @@ __global__ void __launch_bounds__(kCsThreads, 1) gemv_q4_cs_kernel(const GemvPar
   } else if (producer) {
     // ---------------- producer: refill each stage once it is handed back ----------------
     if (lane == 0) {
-      for (int t = NS; t < n_st; ++t) {
+      for (int t = issued; t < n_st; ++t) {
         const int s = t % NS;
-        if (!*abort_flag) cs_wait(&empty[s], (uint32_t)(((t - NS) / NS) & 1), p, abort_flag);
+        if (t >= NS && !*abort_flag) cs_wait(&empty[s], (uint32_t)(((t - NS) / NS) & 1), p, abort_flag);
         if (*abort_flag) break;
         cs_issue<R>(p, u0 + t, stages + s * SB, &full[s], false, pol);
         publish_issued(&s_seq[s], t);
+        if (t < 64) stamp(8 + t);
         issued = t + 1;
       }
     }
@@ -1272,7 +1278,12 @@ bool plan_cs(GemvParams& p, int& R, int& BPL, bool forced) {
   int G = kCsMaxConsumers / NC;
   const int krm = p.kr <= 1 ? 1 : 2;
   auto units = [&](int r) { return p.epi == EPI_GEGLU ? p.seg[0].rows / (r / 2) : (p.n_rows + r - 1) / r; };
+  // Q4G_CS_ROWS (2, 4, 8) and Q4G_CS_GROUPS cap the stage rows and the
+  // consumer groups: tuning switches
+  static const int rows_env = getenv("Q4G_CS_ROWS") ? atoi(getenv("Q4G_CS_ROWS")) : 0;
+  static const int groups_env = getenv("Q4G_CS_GROUPS") ? atoi(getenv("Q4G_CS_GROUPS")) : 0;
   R = k <= 4096 ? 8 : k <= 8192 ? 4 : 2;
+  if (rows_env == 2 || rows_env == 4 || rows_env == 8) R = std::min(R, rows_env);
   if (p.epi == EPI_GEGLU && (p.seg[0].rows % (R / 2))) return false;
   while (R > 2 && units(R) < 6 * device_sm_count()) R /= 2;
   const size_t budget = 220 * 1024, stage = (size_t)R * ((size_t)k / 2 + (size_t)k / 16);
@@ -1283,6 +1294,10 @@ bool plan_cs(GemvParams& p, int& R, int& BPL, bool forced) {
       break;
     }
   G = std::min(G, ns - 2);  // at least 2 stages in flight while G are consumed
+  if (groups_env > 0) G = std::min(G, groups_env);
+  // Q4G_CS_PREFETCH: stages issued before the dependency wait (0: all), a tuning switch
+  static const int prefetch_env = getenv("Q4G_CS_PREFETCH") ? atoi(getenv("Q4G_CS_PREFETCH")) : 0;
+  p.prefetch_stages = prefetch_env;
   if (G < 1) return false;
   p.ns = ns;
   p.nchunk = NC;
@@ -1329,6 +1344,309 @@ cudaError_t launch_cs_t(const GemvParams& p, int R, cudaStream_t st, bool pdl) {
 }
 
 // ---------------------------------------------------------------------------
+// Stage kernel: every compute warp works on every stage.
+//
+// One CTA per SM streams a contiguous range of R-row stages through a ring of
+// NS shared-memory slots (same stage layout as the column-split kernel). The R
+// rows of a stage form G groups of RG rows and the columns NC chunks of 32
+// blocks; compute warp (c, g) takes chunk c of group g, so the NC * G warps go
+// through the ring together, in order. A warp sums its RG rows over its lanes,
+// writes one partial per row and arrives on ready[s]. The reducer warp waits
+// for ready[s], adds the NC partials of each row in chunk order
+// (deterministic), runs the epilogue and refills slot s with the stage NS
+// ahead: one warp hands every slot back, so there is no empty barrier and no
+// per-slot bookkeeping between several consumer groups. Every wait is bounded
+// (error word and abort flag); after a timeout the reducer waits, bounded, for
+// the copies still in flight.
+// ---------------------------------------------------------------------------
+constexpr int kStageCompute = 16;
+constexpr int kStageThreads = (kStageCompute + 1) * 32;
+constexpr int kStageMaxSlots = 16;
+
+__host__ __device__ inline size_t stage_red_bytes(int ns, int nc, int rows, int krm) {
+  return ((size_t)ns * nc * rows * krm * 4 + 15) & ~(size_t)15;
+}
+__host__ __device__ inline size_t stage_fixed_bytes(int krm, int k, int ns, int nc, int rows) {
+  const size_t nb = (size_t)k / 32;
+  return (size_t)krm * nb * (16 * kDigitQuads + 16) + 64 * 4 + stage_red_bytes(ns, nc, rows, krm) + 128 +
+         2 * kStageMaxSlots * 8;
+}
+
+template <int KRM, int R, int RG>
+__global__ void __launch_bounds__(kStageThreads, 1) gemv_q4_stage_kernel(const GemvParams p) {
+  extern __shared__ __align__(16) unsigned char sk_smem[];
+  constexpr int G = R / RG;
+  const int k = p.k, nb = k >> 5, kh = k >> 1, NS = p.ns, NC = p.nchunk;
+  uint4* dg = reinterpret_cast<uint4*>(sk_smem);                          // [KRM][kDigitQuads][nb]
+  int4* bc = reinterpret_cast<int4*>(dg + (size_t)KRM * kDigitQuads * nb);  // [KRM][nb]
+  float* misc = reinterpret_cast<float*>(bc + (size_t)KRM * nb);          // 64 floats
+  float* red = misc + 64;                                                 // [NS][NC][R][KRM]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(
+      ((uintptr_t)(reinterpret_cast<unsigned char*>(red) + stage_red_bytes(NS, NC, R, KRM)) + 127) &
+      ~(uintptr_t)127);
+  uint64_t* full = bars;                    // [kStageMaxSlots]: the stage's bytes landed
+  uint64_t* ready = bars + kStageMaxSlots;  // [kStageMaxSlots]: every compute warp wrote its partials
+  unsigned char* stages = reinterpret_cast<unsigned char*>(bars + 2 * kStageMaxSlots);
+  __shared__ int s_abort, s_ticket;
+  __shared__ float s_bestv;
+  __shared__ int s_besti;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n_comp = NC * G;
+  const bool reducer = warp == kStageCompute;
+  const int u0 = (int)((long long)blockIdx.x * p.n_units / gridDim.x);
+  const int n_st = (int)((long long)(blockIdx.x + 1) * p.n_units / gridDim.x) - u0;
+  const size_t SB = (size_t)p.stage_bytes;
+  const uint64_t pol = policy_evict_first();
+  int issued = 0;
+  uint64_t* const tr = blockIdx.x == 0 ? p.trace : nullptr;
+  auto stamp = [&](int i) {
+    if (tr) tr[i] = global_ns();
+  };
+
+  if (tid == 0) stamp(0), s_abort = 0;
+  if (reducer && lane == 0) {
+    for (int s = 0; s < NS; ++s) mbar_init(&full[s], 1), mbar_init(&ready[s], n_comp);
+    fence_mbar_init();
+    const int pre = p.prefetch_stages > 0 ? min(NS, p.prefetch_stages) : NS;
+    for (; issued < pre && issued < n_st; ++issued) {
+      cs_issue<R>(p, u0 + issued, stages + issued * SB, &full[issued],
+                  p.stall_test && u0 == 0 && issued == 0, pol);  // the CTA owning unit 0
+      if (issued < 64) stamp(8 + issued);
+    }
+  }
+  __syncthreads();  // barriers initialised before any wait
+  pdl_wait();
+  if (tid == 0) stamp(1);
+  stage_digits<KRM, kStageThreads>(p, dg, bc, misc);  // ends with __syncthreads
+  if (tid == 0) stamp(2);
+  pdl_launch_dependents();
+  volatile int* abort_flag = &s_abort;
+
+  if (warp < n_comp) {
+    // ---------------- compute warp: chunk c of row group g ----------------
+    // lane l holds block 32 c + l of every row; a lane past the end of the row
+    // reads block nb - 1 with zero digits and a zero x scale (no branch)
+    const int c = warp % NC, g = warp / NC;
+    const int blk = 32 * c + lane;
+    const bool has = blk < nb;
+    const int qoff = 16 * min(blk, nb - 1), soff = 2 * min(blk, nb - 1);
+    uint4 xg[KRM][kDigitQuads];
+    int4 cv[KRM];
+    float xsc[KRM];
+#pragma unroll
+    for (int j = 0; j < KRM; ++j) {
+      if (has && (KRM == 1 || j < p.kr)) {
+#pragma unroll
+        for (int q = 0; q < kDigitQuads; ++q) xg[j][q] = dg[(size_t)(j * kDigitQuads + q) * nb + blk];
+        cv[j] = bc[j * nb + blk];
+      } else {
+#pragma unroll
+        for (int q = 0; q < kDigitQuads; ++q) xg[j][q] = make_uint4(0, 0, 0, 0);
+        cv[j] = make_int4(0, 0, 0, 0);
+      }
+      xsc[j] = __int_as_float(cv[j].w);
+    }
+    int s = 0;
+    uint32_t ph = 0;
+    for (int t = 0; t < n_st; ++t) {
+      if (!*abort_flag) cs_wait(&full[s], ph, p, abort_flag);
+      if (*abort_flag) break;
+      if (c == 0 && g == 0 && lane == 0 && t < 64) stamp(72 + t);
+      const unsigned char* st = stages + s * SB + (size_t)g * RG * kh + qoff;
+      const unsigned char* ss = stages + s * SB + (size_t)R * kh + (size_t)g * RG * 2 * nb + soff;
+      float v[KRM][RG];
+#pragma unroll
+      for (int r = 0; r < RG; ++r) {
+        const uint4 qv = *reinterpret_cast<const uint4*>(st + r * kh);
+        const float d = __half2float(*reinterpret_cast<const __half*>(ss + r * 2 * nb));
+#pragma unroll
+        for (int j = 0; j < KRM; ++j)
+          v[j][r] = (KRM == 1 || j < p.kr) ? d * xsc[j] * block_dot_int(qv, xg[j], cv[j]) : 0.f;
+      }
+      float* rs = red + (size_t)s * NC * R * KRM;  // [NC][R][KRM] of this slot
+#pragma unroll
+      for (int j = 0; j < KRM; ++j) {
+        const float tot = cs_reduce_rows<RG>(v[j], lane);
+        if ((lane & (32 / RG - 1)) == 0) rs[((size_t)c * R + g * RG + cs_row<RG>(lane)) * KRM + j] = tot;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ready[s]);  // release of the partials above
+      if (++s == NS) s = 0, ph ^= 1u;
+    }
+  } else if (reducer) {
+    // ---------------- reducer: partials -> epilogue, then refill the slot ----------------
+    if (lane == 0)  // the first stages not issued before the dependency wait
+      for (; issued < NS && issued < n_st; ++issued) {
+        cs_issue<R>(p, u0 + issued, stages + issued * SB, &full[issued], false, pol);
+        if (issued < 64) stamp(8 + issued);
+      }
+    float best_v = -INFINITY;
+    int best_i = 0x7fffffff;
+    const int r = lane / KRM, j = lane % KRM;  // lanes l < R * KRM
+    int s = 0;
+    uint32_t ph = 0;
+    for (int t = 0; t < n_st; ++t) {
+      if (!*abort_flag) cs_wait(&ready[s], ph, p, abort_flag);
+      if (*abort_flag) break;
+      const float* rs = red + (size_t)s * NC * R * KRM;
+      float val = 0.f;
+      if (lane < R * KRM)
+        for (int cc = 0; cc < NC; ++cc) val += rs[((size_t)cc * R + r) * KRM + j];
+      const int u = u0 + t;
+      if (p.epi == EPI_GEGLU) {
+        const float up = __shfl_sync(0xffffffffu, val, (lane + (R / 2) * KRM) & 31);
+        if (lane < (R / 2) * KRM && j < p.kr)
+          p.act[(size_t)j * p.act_stride + (size_t)(R / 2) * u + r] = __float2half_rn(gelu_tanh(val) * up);
+      } else if (lane < R * KRM && j < p.kr) {
+        const int row = R * u + r;
+        if (row < p.n_rows) {
+          if (p.epi == EPI_STORE) {
+            p.y[(size_t)j * p.y_stride + row] = val;
+          } else {
+            const float z = p.softcap * tanhf(val / p.softcap);
+            if (p.logits) p.logits[(size_t)j * p.logits_stride + row] = z;
+            if (z > best_v || (z == best_v && row < best_i)) best_v = z, best_i = row;
+          }
+        }
+      }
+      __syncwarp();  // every lane read slot s's partials before the refill can overwrite them
+      if (lane == 0) {
+        if (t < 64) stamp(136 + t);
+        if (t + NS < n_st) {
+          cs_issue<R>(p, u0 + t + NS, stages + s * SB, &full[s], false, pol);
+          if (t + NS < 64) stamp(8 + t + NS);
+          issued = t + NS + 1;
+        }
+      }
+      if (++s == NS) s = 0, ph ^= 1u;
+    }
+    if (p.epi == EPI_HEAD) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float v2 = __shfl_xor_sync(0xffffffffu, best_v, o);
+        const int i2 = __shfl_xor_sync(0xffffffffu, best_i, o);
+        if (v2 > best_v || (v2 == best_v && i2 < best_i)) best_v = v2, best_i = i2;
+      }
+      if (lane == 0) s_bestv = best_v, s_besti = best_i;
+    }
+  }
+  if (p.epi == EPI_HEAD) {
+    __syncthreads();
+    if (tid == 0) {
+      p.am_val[blockIdx.x] = s_bestv;
+      p.am_idx[blockIdx.x] = s_besti;
+      __threadfence();
+      s_ticket = atomicAdd(p.counter, 1);
+      if (s_ticket == (int)gridDim.x - 1) {
+        __threadfence();
+        float v = -INFINITY;
+        int ix = 0x7fffffff;
+        for (int b = 0; b < (int)gridDim.x; ++b) {
+          const float vb = __ldcg(p.am_val + b);
+          const int ib = __ldcg(p.am_idx + b);
+          if (vb > v || (vb == v && ib < ix)) v = vb, ix = ib;
+        }
+        if (p.argmax_out) p.argmax_out[0] = ix == 0x7fffffff ? 0 : ix;
+        *p.counter = 0;
+      }
+    }
+  }
+  // after a timeout, wait (bounded) for the copies still in flight
+  if (reducer && lane == 0 && *abort_flag) {
+    for (int t = issued > NS ? issued - NS : 0; t < issued; ++t)
+      mbar_wait_bounded(&full[t % NS], (uint32_t)((t / NS) & 1), p.wait_ns);
+  }
+}
+
+// Plan of the stage kernel: R rows per stage (about 16-36 KB), NC = 32-block
+// chunks, G row groups of RG rows, NS slots within the shared-memory budget.
+bool plan_stage(GemvParams& p, int& R, int& RG, bool forced) {
+  const int k = p.k, nb = k >> 5;
+  if (k % 256 != 0 || p.kr > 2) return false;
+  if (p.epi == EPI_HEAD && p.kr != 1) return false;
+  if (p.epi == EPI_GEGLU && (p.nseg != 2 || p.seg[0].rows != p.seg[1].rows || p.seg[0].rows % 8)) return false;
+  if (p.pro == PRO_RESID && k > 8192) return false;
+  for (int s = 0; s < p.nseg; ++s)
+    if (!aligned16(p.seg[s].qs) || !aligned16(p.seg[s].sc) || (s < p.nseg - 1 && p.seg[s].rows % 16))
+      return false;
+  if (p.pro == PRO_X16 && !aligned16(p.x)) return false;
+  (void)forced;
+  const int NC = (nb + 31) / 32;
+  if (NC > kStageCompute) return false;
+  const int krm = p.kr <= 1 ? 1 : 2;
+  const size_t row_bytes = (size_t)k / 2 + (size_t)k / 16;
+  // Q4G_STAGE_ROWS (2, 4, 8, 16) forces the stage rows: a tuning switch
+  static const int rows_env = getenv("Q4G_STAGE_ROWS") ? atoi(getenv("Q4G_STAGE_ROWS")) : 0;
+  R = 16;
+  while (R > 2 && (size_t)R * row_bytes > 36 * 1024) R /= 2;
+  if (rows_env == 2 || rows_env == 4 || rows_env == 8 || rows_env == 16) R = rows_env;
+  if (p.epi == EPI_GEGLU) R = std::max(R, 4);
+  auto units = [&](int r) { return p.epi == EPI_GEGLU ? p.seg[0].rows / (r / 2) : (p.n_rows + r - 1) / r; };
+  // keep every SM busy on small matrices
+  while (R > 4 && units(R) < 2 * device_sm_count()) R /= 2;
+  int G = std::min(kStageCompute / NC, R == 16 ? 4 : R / 2);
+  while (G > 1 && (G & (G - 1))) --G;  // power of two, divides R
+  RG = R / G;
+  if (R == 16 && RG != 4) return false;
+  if (RG != 2 && RG != 4) return false;
+  const size_t budget = 220 * 1024, stage = (size_t)R * row_bytes;
+  int ns = 0;
+  for (int n = kStageMaxSlots; n >= 2; --n)
+    if (stage_fixed_bytes(krm, k, n, NC, R) + (size_t)n * stage <= budget) {
+      ns = n;
+      break;
+    }
+  if (ns < 4) return false;
+  static const int prefetch_env = getenv("Q4G_CS_PREFETCH") ? atoi(getenv("Q4G_CS_PREFETCH")) : 0;
+  p.prefetch_stages = prefetch_env;
+  p.ns = ns;
+  p.nchunk = NC;
+  p.groups = G;
+  p.stage_rows = R;
+  p.stage_bytes = (int)stage;
+  p.n_units = units(R);
+  return true;
+}
+
+template <int KRM, int R, int RG>
+cudaError_t launch_stage_r(const GemvParams& p, cudaStream_t st, bool pdl) {
+  static size_t configured = 0;
+  const size_t smem = stage_fixed_bytes(KRM, p.k, p.ns, p.nchunk, R) + (size_t)p.ns * p.stage_bytes;
+  cudaError_t e;
+  if (smem > configured) {
+    e = cudaFuncSetAttribute(gemv_q4_stage_kernel<KRM, R, RG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(gemv_q4_stage_kernel<KRM, R, RG>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    configured = smem;
+  }
+  int grid = device_sm_count();
+  if (grid > p.n_units) grid = p.n_units;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kStageThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, gemv_q4_stage_kernel<KRM, R, RG>, p);
+}
+
+template <int KRM>
+cudaError_t launch_stage_t(const GemvParams& p, int R, int RG, cudaStream_t st, bool pdl) {
+  if (R == 16) return launch_stage_r<KRM, 16, 4>(p, st, pdl);
+  if (R == 8) return RG == 4 ? launch_stage_r<KRM, 8, 4>(p, st, pdl) : launch_stage_r<KRM, 8, 2>(p, st, pdl);
+  if (R == 4) return RG == 4 ? launch_stage_r<KRM, 4, 4>(p, st, pdl) : launch_stage_r<KRM, 4, 2>(p, st, pdl);
+  return launch_stage_r<KRM, 2, 2>(p, st, pdl);
+}
+
+// ---------------------------------------------------------------------------
 // Chain of q4_0 GEMVs in one persistent launch (one activation row).
 //
 // The GEMVs between two attention kernels of a decode step -- O(l),
@@ -1369,8 +1687,8 @@ Q4G_DEV int ld_acquire(const int32_t* p) {
 // every consumer warp calls this, warps without a block get zeros.
 constexpr int kChainMaxK = 8192;  // PRO_RESID rows
 
-Q4G_DEV void chain_digits(const GemvParams& P, int blk, bool has, float* s_norm, __half* xs, uint4 (&g)[6],
-                          int4& cv) {
+Q4G_DEV void chain_digits(const GemvParams& P, int blk, bool has, float* s_norm, __half* xs,
+                          uint4 (&g)[kDigitQuads], int4& cv) {
   const int k = P.k, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   constexpr int NT = kChainConsumers * 32;
   __half xh[32];
@@ -1460,22 +1778,23 @@ Q4G_DEV void chain_digits(const GemvParams& P, int blk, bool has, float* s_norm,
   int em = 1;
 #pragma unroll
   for (int e = 0; e < 32; ++e) em = max(em, half_exp(xh[e]));
-  int sd[3] = {0, 0, 0};
-  uint32_t words[3][8];
+  int sd[2] = {0, 0};
+  uint32_t words[2][8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
     const __half h4[4] = {xh[4 * q], xh[4 * q + 1], xh[4 * q + 2], xh[4 * q + 3]};
-    uint32_t wd[3];
-    digits4(h4, em, q >= 4, wd, sd);
+    uint32_t wd[2];
+    digits4(h4, em, wd, sd);
 #pragma unroll
-    for (int t = 0; t < 3; ++t) words[t][q] = wd[t];
+    for (int t = 0; t < 2; ++t) words[t][q] = wd[t];
   }
 #pragma unroll
-  for (int t = 0; t < 3; ++t) {
+  for (int t = 0; t < 2; ++t) {
     g[2 * t] = make_uint4(words[t][0], words[t][1], words[t][2], words[t][3]);
     g[2 * t + 1] = make_uint4(words[t][4], words[t][5], words[t][6], words[t][7]);
   }
-  cv = make_int4(-8 * sd[0], -8 * sd[1], -8 * sd[2], (em - 37 + 127) << 23);
+  // a lane without a block has zero digits and a zero x scale
+  cv = has ? make_int4(-8 * sd[0], -8 * sd[1], 0, (em - 29 + 127) << 23) : make_int4(0, 0, 0, 0);
 }
 
 struct ChainShared {
@@ -1503,21 +1822,19 @@ Q4G_DEV void chain_issue_r(const GemvParams& P, int u, unsigned char* st, uint64
 // One stage of phase P by consumer warp (chunk c): the R row partial sums go to
 // red[slot][c]; returns nothing, the caller runs the ticket.
 template <int R>
-Q4G_DEV void chain_stage(const GemvParams& P, const unsigned char* st, bool has, int blk, const uint4 (&xg)[6],
+Q4G_DEV void chain_stage(const GemvParams& P, const unsigned char* st, int blk, const uint4 (&xg)[kDigitQuads],
                          const int4 cv, float* red_slot_c) {
   const int kh = P.k >> 1, nb = P.k >> 5, lane = threadIdx.x & 31;
-  const float xsc = __int_as_float(cv.w);
+  const float xsc = __int_as_float(cv.w);  // 0 for a lane without a block
+  const int bq = min(blk, nb - 1);
+  const unsigned char* sq = st + 16 * bq;
+  const unsigned char* ss = st + R * kh + 2 * bq;
   float v[R];
 #pragma unroll
   for (int r = 0; r < R; ++r) {
-    float a = 0.f;
-    if (has) {
-      const uint4 qv = lds_u4(st + (size_t)r * kh + (size_t)blk * 16);
-      const float d = __half2float(__ushort_as_half(
-          *reinterpret_cast<const uint16_t*>(st + (size_t)R * kh + (size_t)r * nb * 2 + (size_t)blk * 2)));
-      a = d * xsc * block_dot_int(qv, xg, cv);
-    }
-    v[r] = a;
+    const uint4 qv = *reinterpret_cast<const uint4*>(sq + r * kh);
+    const float d = __half2float(*reinterpret_cast<const __half*>(ss + r * 2 * nb));
+    v[r] = d * xsc * block_dot_int(qv, xg, cv);
   }
   const float tot = cs_reduce_rows<R>(v, lane);
   if ((lane & (32 / R - 1)) == 0) red_slot_c[cs_row<R>(lane)] = tot;
@@ -1599,15 +1916,14 @@ __global__ void __launch_bounds__(kChainThreads, 1) gemv_q4_chain_kernel(const C
           __nanosleep(64);
         }
       }
-      consumer_bar();
-      __threadfence();
+      consumer_bar();  // orders every consumer thread after thread 0's acquire
     }
     if (tid == 0) stamp(2 + 4 * ph);
     const bool active = warp < NC * G;
     const int cidx = warp % NC, g = warp / NC;
     const int blk = 32 * cidx + lane;
     const bool has = active && blk < nb;
-    uint4 xg[6];
+    uint4 xg[kDigitQuads];
     int4 cv;
     chain_digits(P, blk, has, sh.norm, sh.xs, xg, cv);
     if (tid == 0) stamp(2 + 4 * ph + 1);
@@ -1618,9 +1934,9 @@ __global__ void __launch_bounds__(kChainThreads, 1) gemv_q4_chain_kernel(const C
           cs_wait(&sh.full[s], (uint32_t)((t / NS) & 1), wp, abort_flag);
         const unsigned char* st = chain_stages + (size_t)s * kChainSlotBytes;
         float* rs = &sh.red[s][0][0];
-        if (R == 8) chain_stage<8>(P, st, has, blk, xg, cv, rs + cidx * 8);
-        else if (R == 4) chain_stage<4>(P, st, has, blk, xg, cv, rs + cidx * 8);
-        else chain_stage<2>(P, st, has, blk, xg, cv, rs + cidx * 8);
+        if (R == 8) chain_stage<8>(P, st, blk, xg, cv, rs + cidx * 8);
+        else if (R == 4) chain_stage<4>(P, st, blk, xg, cv, rs + cidx * 8);
+        else chain_stage<2>(P, st, blk, xg, cv, rs + cidx * 8);
         __syncwarp();
         int last = 0;
         if (lane == 0) {
@@ -1644,7 +1960,9 @@ __global__ void __launch_bounds__(kChainThreads, 1) gemv_q4_chain_kernel(const C
         if (lane == 0) {
           sh.cnt[s] = 0;
           mbar_arrive(&sh.empty[s]);
-          __threadfence();
+          // CTA-scope release of this stage's outputs; the warp that completes
+          // the phase acquires them all and publishes them with one GPU-scope fence
+          __threadfence_block();
           if (atomicAdd(&sh.phase_done[ph], 1) == n_st - 1) {
             __threadfence();
             atomicAdd(&c.done[ph], 1);
@@ -1695,7 +2013,7 @@ int gemv_kernel_choice() {
   int c = g_kernel_choice.load(std::memory_order_relaxed);
   if (c == -2) {
     const char* e = getenv("Q4G_GEMV_KERNEL");
-    c = !e ? -1 : e[0] == 'c' ? 0 : e[0] == 'w' ? 1 : 2;
+    c = !e ? -1 : e[0] == 'c' ? 0 : e[0] == 'w' ? 1 : e[0] == 's' ? 3 : 2;
     int expected = -2;
     if (!g_kernel_choice.compare_exchange_strong(expected, c)) c = expected;
   }
@@ -1762,6 +2080,19 @@ NextGemv gemv_next_desc(const GemvParams& p_in, float frac) {
   int dot = gemv_dot_kind(), R = 0, BPL = 1;
   const int choice = gemv_kernel_choice();
   GemvParams px = p_in;
+  int RG = 2;
+  if ((choice == 3 || choice == -1) && plan_stage(px, R, RG, choice == 3)) {
+    for (int s = 0; s < 3; ++s) nx.seg[s] = px.seg[s];
+    nx.nseg = px.nseg;
+    nx.k = px.k;
+    nx.n_units = px.n_units;
+    nx.unit_rows = R;
+    nx.geglu = px.epi == EPI_GEGLU;
+    nx.tw = std::min(device_sm_count(), px.n_units);
+    nx.frac = frac;
+    return nx;
+  }
+  px = p_in;
   if (choice <= 0 && plan_cs(px, R, BPL, choice == 0)) {
     // one stream per CTA: the first units of every CTA's range
     for (int s = 0; s < 3; ++s) nx.seg[s] = px.seg[s];
@@ -1805,7 +2136,14 @@ int32_t* device_error_word() {
 cudaError_t launch_gemv(const GemvParams& p_in, cudaStream_t st, bool pdl) {
   GemvParams p = p_in;
   const int choice = gemv_kernel_choice();
-  int R = 0, BPL = 1;
+  int R = 0, BPL = 1, RG = 2;
+  if ((choice == 3 || choice == -1) && plan_stage(p, R, RG, choice == 3)) {
+    if (!p.err) p.err = device_error_word();
+    if (!p.err) return cudaErrorInvalidValue;
+    if (!p.wait_ns) p.wait_ns = 2000000000ull;
+    return p.kr > 1 ? launch_stage_t<2>(p, R, RG, st, pdl) : launch_stage_t<1>(p, R, RG, st, pdl);
+  }
+  p = p_in;
   if (choice <= 0 && plan_cs(p, R, BPL, choice == 0)) {
     if (!p.err) p.err = device_error_word();
     if (!p.err) return cudaErrorInvalidValue;
@@ -1831,7 +2169,7 @@ cudaError_t launch_gemv(const GemvParams& p_in, cudaStream_t st, bool pdl) {
 }
 
 bool set_gemv_kernel_choice(int kind) {
-  if (kind < 0 || kind > 3) return false;
+  if (kind < 0 || kind > 4) return false;
   g_kernel_choice.store(kind - 1);
   return true;
 }

@@ -76,8 +76,13 @@ struct GemvParams {
   int32_t kc;           // columns per streamed item
   int32_t ns;           // stages per warp
   int32_t stage_bytes;  // codes then scales of one item (2 rows)
+  int32_t prefetch_stages;  // column-split kernel: stages issued before the dependency wait (0: all)
   int32_t* err;         // error word: bit 0 = a bounded wait gave up
   uint64_t wait_ns;     // limit of one bounded wait
+  // optional timeline of CTA 0 (globaltimer ns): [0] entry, [1] after the
+  // dependency wait, [2] after the x prologue, [8 + t] stage t issued,
+  // [72 + t] stage t ready for its consumers, [136 + t] stage t reduced (t < 64)
+  uint64_t* trace;
   int32_t stall_test;   // 1: the first stage of the warp that owns unit 0 never completes (tests the timeout path)
 };
 
@@ -103,6 +108,7 @@ struct ChainParams {
 // phase i at 2 + 4 i: inputs ready, digits built, last own stage done, producer
 // done issuing; 18 end
 constexpr int kChainTraceSlots = 32;
+constexpr int kGemvTraceSlots = 256;  // one GEMV launch's timeline (GemvParams::trace)
 // Plans every phase in place; false if a phase does not fit the chain kernel.
 bool plan_chain(ChainParams& c);
 cudaError_t launch_gemv_chain(const ChainParams& c, cudaStream_t st, bool pdl);

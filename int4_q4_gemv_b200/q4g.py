@@ -151,7 +151,7 @@ def q4g_gemv(qs, scales, n, k, x_f16, nrhs, y, stream):
     _call("q4g_gemv", qs, scales, n, k, x_f16, nrhs, y, stream)
 
 
-Q4G_GEMV_AUTO, Q4G_GEMV_COLUMN_SPLIT, Q4G_GEMV_WARP_STREAM, Q4G_GEMV_REGISTER = 0, 1, 2, 3
+Q4G_GEMV_AUTO, Q4G_GEMV_COLUMN_SPLIT, Q4G_GEMV_WARP_STREAM, Q4G_GEMV_REGISTER, Q4G_GEMV_STAGE = 0, 1, 2, 3, 4
 
 
 def q4g_set_gemv_kernel(kind):

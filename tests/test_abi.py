@@ -69,11 +69,12 @@ def test_host_validation_without_gpu(lib):
 
 
 def test_gemv_kernel_choice_validation(lib):
-    for bad in (-1, 4, 99):
+    for bad in (-1, 5, 99):
         with pytest.raises(Q.Q4GError) as e:
             Q.q4g_set_gemv_kernel(bad)
         assert e.value.status == Q.Q4G_EINVAL
-    for kind in (Q.Q4G_GEMV_COLUMN_SPLIT, Q.Q4G_GEMV_WARP_STREAM, Q.Q4G_GEMV_REGISTER, Q.Q4G_GEMV_AUTO):
+    for kind in (Q.Q4G_GEMV_COLUMN_SPLIT, Q.Q4G_GEMV_WARP_STREAM, Q.Q4G_GEMV_REGISTER, Q.Q4G_GEMV_STAGE,
+                 Q.Q4G_GEMV_AUTO):
         Q.q4g_set_gemv_kernel(kind)                       # no CUDA call
     cfg = dict(WL.TINY, hidden=8192 + 256)               # the fused residual prologue caps the hidden size
     c = Q.q4g_config(*[cfg[n] for n, _ in Q.q4g_config._fields_])

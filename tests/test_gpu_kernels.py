@@ -2,10 +2,14 @@
 
 Tolerances:
   * q4_0 pack: bit-exact (integer codes and fp16 scales).
-  * GEMV: |y - y_ref| <= 2e-4 * sum_blocks |d| * sum_block |x| + 1e-6. Derivation: per
-    block the kernel accumulates 32 products (64 + c) x (each <= 79 |x|) in fp32, so
-    the rounding error is below 32 * 2^-24 * 79 * sum|x| ~ 1.5e-4 sum|x| before the
-    scale d; the reference is fp64 on the same fp16 x and dequantised weights.
+  * GEMV: |y - y_ref| <= 2e-4 * sum_b |d_b| sum_b |x| + 2^-15 * sum_b |d_b| max_b |x| sum_b |c - 8|
+    + 1e-6 (sums over the 32 columns of block b). First term, the fp32 arithmetic: per
+    block the fp16 path accumulates 32 products (64 + c) x (each <= 79 |x|) in fp32, a
+    rounding error below 32 * 2^-24 * 79 * sum|x| ~ 1.5e-4 sum|x| before the scale d.
+    Second term, the integer path: x enters it as 16-bit fixed point relative to the
+    block's largest exponent, each value off by at most 2^-15 of the block maximum and
+    weighted by |c - 8|; the block sums themselves are exact integers. The reference is
+    fp64 on the same fp16 x and dequantised weights.
   * attention: fp16 output, |o - o_ref| <= 2e-3 * (1 + |o_ref|): half an fp16 ulp
     (2^-11 relative) plus the fp16 hi/lo probability split (~2^-22).
 """
@@ -87,9 +91,12 @@ def test_pack_rejects_non_finite():
 def _gemv_bound(qs, sc, x16):
     d = np.abs(O.f16_value(sc))                                  # [n][nb]
     xa = np.abs(x16.view(np.float16).astype(np.float64))         # [r][k]
-    nb = sc.shape[1]
+    n, nb = sc.shape
     xb = xa.reshape(xa.shape[0], nb, 32).sum(axis=2)             # [r][nb]
-    return 2e-4 * (xb @ d.T) + 1e-6                              # [r][n]
+    xm = xa.reshape(xa.shape[0], nb, 32).max(axis=2)             # [r][nb]
+    q = qs.reshape(n, nb, 16).astype(np.int64)                   # byte b: column b (low), b + 16 (high)
+    cabs = np.abs((q & 15) - 8).sum(axis=2) + np.abs((q >> 4) - 8).sum(axis=2)  # [n][nb]
+    return 2e-4 * (xb @ d.T) + 2.0 ** -15 * (xm @ (d * cabs).T) + 1e-6   # [r][n]
 
 
 def _run_gemv(qs_t, sc_t, n, k, x16):
@@ -184,7 +191,8 @@ def test_flash_decode_linear_vs_oracle(n_q, length):
     assert np.all(np.abs(got - ref) <= 2e-3 * (1 + np.abs(ref)))
 
 
-@pytest.mark.parametrize("kind", [Q.Q4G_GEMV_COLUMN_SPLIT, Q.Q4G_GEMV_WARP_STREAM, Q.Q4G_GEMV_REGISTER])
+@pytest.mark.parametrize("kind", [Q.Q4G_GEMV_COLUMN_SPLIT, Q.Q4G_GEMV_WARP_STREAM, Q.Q4G_GEMV_REGISTER,
+                                  Q.Q4G_GEMV_STAGE])
 @pytest.mark.parametrize("n,k,nrhs", [(3840, 15360, 1), (8192, 3840, 1), (1000, 1024, 2), (3840, 4096, 4),
                                       (260, 3840, 2), (77, 256, 1)])
 def test_gemv_every_kernel_meets_the_oracle_bound(kind, n, k, nrhs):
