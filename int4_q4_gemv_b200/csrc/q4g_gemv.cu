@@ -135,6 +135,27 @@ Q4G_DEV void produce_x(const GemvParams& p, float* misc, Emit&& emit) {
       const __half* xr = p.x + (size_t)j * p.x_stride;
       const bool vec = (((uintptr_t)xr) & 7) == 0;
       const int iters = (n4 + NT - 1) / NT;
+      constexpr int kHoist = (15360 / 4 + NT - 1) / NT;  // rounds whose loads are issued together
+      if (vec && iters <= kHoist) {
+        // every load first (one round trip), then the rounds; iters is the same
+        // for the whole CTA, so a round is skipped by whole warps
+        uint2 v[kHoist];
+#pragma unroll
+        for (int i = 0; i < kHoist; ++i) {
+          const int c4 = tid + i * NT;
+          v[i] = c4 < n4 ? *reinterpret_cast<const uint2*>(xr + 4 * c4) : make_uint2(0u, 0u);
+        }
+#pragma unroll
+        for (int i = 0; i < kHoist; ++i) {
+          if (i < iters) {
+            const int c4 = tid + i * NT;
+            const __half* hv = reinterpret_cast<const __half*>(&v[i]);
+            const __half h[4] = {hv[0], hv[1], hv[2], hv[3]};
+            emit(j, c4, h, c4 < n4);
+          }
+        }
+        continue;
+      }
       for (int i = 0; i < iters; ++i) {
         const int c4 = tid + i * NT;
         const bool valid = c4 < n4;
@@ -214,6 +235,7 @@ Q4G_DEV void produce_x(const GemvParams& p, float* misc, Emit&& emit) {
       if (p.trace && blockIdx.x == 0 && tid == 0) p.trace[4] = global_ns();
 #pragma unroll
       for (int i = 0; i < R4; ++i) {
+        if (i * NT >= n4) break;  // no thread of the CTA has columns left
         const int c4 = tid + i * NT;
         const bool valid = c4 < n4;
         __half h[4];
@@ -267,9 +289,12 @@ Q4G_DEV void stage_x(const GemvParams& p, uint4* xs, float* cblk, float* misc) {
 // unsigned, byte 1 signed) and adds the digit sums to sd.
 Q4G_DEV void digits4(const __half (&h)[4], int em, uint32_t (&wd)[2], int (&sd)[2]) {
   const float sc = __int_as_float((29 - em + 127) << 23);
+  // round to nearest even through the fp32 adder: x * sc is exact and
+  // |x * sc| < 2^15, so x * sc + 1.5 * 2^23 rounds once at unit spacing and its
+  // bit pattern minus that of 1.5 * 2^23 is the integer
   int X[4];
 #pragma unroll
-  for (int e = 0; e < 4; ++e) X[e] = __float2int_rn(__half2float(h[e]) * sc);
+  for (int e = 0; e < 4; ++e) X[e] = __float_as_int(fmaf(__half2float(h[e]), sc, 12582912.0f)) - 0x4B400000;
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     const uint32_t sel = 0x0040u | (uint32_t)(t * 0x11);  // bytes (x.b_t, y.b_t)
@@ -316,6 +341,56 @@ Q4G_DEV void stage_digits(const GemvParams& p, uint4* dg, int4* bc, float* misc)
       dw[((size_t)(j * kDigitQuads + 0 + hh) * nb + blk) * 4 + wd] = wdg[0];
       dw[((size_t)(j * kDigitQuads + 2 + hh) * nb + blk) * 4 + wd] = wdg[1];
       if (sub == 0) bc[j * nb + blk] = make_int4(-8 * s0, -8 * s1, 0, (em - 29 + 127) << 23);
+    }
+  });
+  __syncthreads();
+}
+
+// Digits of one whole 32-column block in one lane (see block_dot_int): xv[q]
+// holds columns 8q .. 8q+7 as fp16. The largest exponent field comes from the
+// largest magnitude (fp16 bit patterns of |x| order like the values; zero and
+// subnormals count as exponent 1).
+Q4G_DEV void lane_block_digits(const uint4 (&xv)[4], uint4 (&g)[kDigitQuads], int4& cv) {
+  uint32_t mx = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    mx = __vmaxu2(mx, xv[q].x & 0x7FFF7FFFu);
+    mx = __vmaxu2(mx, xv[q].y & 0x7FFF7FFFu);
+    mx = __vmaxu2(mx, xv[q].z & 0x7FFF7FFFu);
+    mx = __vmaxu2(mx, xv[q].w & 0x7FFF7FFFu);
+  }
+  const uint32_t mh = max(mx & 0xFFFFu, mx >> 16);
+  const int em = max((int)((mh >> 10) & 31u), 1);
+  int sd[2] = {0, 0};
+  uint32_t words[2][8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const uint32_t w0 = (&xv[q >> 1].x)[2 * (q & 1)], w1 = (&xv[q >> 1].x)[2 * (q & 1) + 1];
+    const __half h4[4] = {__ushort_as_half((unsigned short)(w0 & 0xFFFFu)), __ushort_as_half((unsigned short)(w0 >> 16)),
+                          __ushort_as_half((unsigned short)(w1 & 0xFFFFu)), __ushort_as_half((unsigned short)(w1 >> 16))};
+    uint32_t wd[2];
+    digits4(h4, em, wd, sd);
+    words[0][q] = wd[0];
+    words[1][q] = wd[1];
+  }
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    g[2 * t] = make_uint4(words[t][0], words[t][1], words[t][2], words[t][3]);
+    g[2 * t + 1] = make_uint4(words[t][4], words[t][5], words[t][6], words[t][7]);
+  }
+  cv = make_int4(-8 * sd[0], -8 * sd[1], 0, (em - 29 + 127) << 23);
+}
+
+// The activation rows as fp16 in shared memory ([KRM][k]), from the fused
+// residual/RMSNorm prologue. Ends with __syncthreads().
+template <int KRM, int NT>
+Q4G_DEV void stage_x_half(const GemvParams& p, __half* xh, float* misc) {
+  const int k = p.k;
+  produce_x<KRM, NT>(p, misc, [&](int j, int c4, const __half (&h)[4], bool valid) {
+    if (valid) {
+      __half2* d = reinterpret_cast<__half2*>(xh + (size_t)j * k + 4 * c4);
+      d[0] = __halves2half2(h[0], h[1]);
+      d[1] = __halves2half2(h[2], h[3]);
     }
   });
   __syncthreads();
@@ -1366,10 +1441,12 @@ constexpr int kStageMaxSlots = 16;
 __host__ __device__ inline size_t stage_red_bytes(int ns, int nc, int rows, int krm) {
   return ((size_t)ns * nc * rows * krm * 4 + 15) & ~(size_t)15;
 }
-__host__ __device__ inline size_t stage_fixed_bytes(int krm, int k, int ns, int nc, int rows) {
-  const size_t nb = (size_t)k / 32;
-  return (size_t)krm * nb * (16 * kDigitQuads + 16) + 64 * 4 + stage_red_bytes(ns, nc, rows, krm) + 128 +
-         2 * kStageMaxSlots * 8;
+// x region: the normed fp16 rows (PRO_RESID only; PRO_X16 lanes read x itself)
+__host__ __device__ inline size_t stage_x_bytes(int krm, int k, int pro) {
+  return pro == PRO_RESID ? (size_t)krm * k * 2 : 0;
+}
+__host__ __device__ inline size_t stage_fixed_bytes(int krm, int k, int pro, int ns, int nc, int rows) {
+  return stage_x_bytes(krm, k, pro) + 64 * 4 + stage_red_bytes(ns, nc, rows, krm) + 128 + 2 * kStageMaxSlots * 8;
 }
 
 template <int KRM, int R, int RG>
@@ -1377,9 +1454,8 @@ __global__ void __launch_bounds__(kStageThreads, 1) gemv_q4_stage_kernel(const G
   extern __shared__ __align__(16) unsigned char sk_smem[];
   constexpr int G = R / RG;
   const int k = p.k, nb = k >> 5, kh = k >> 1, NS = p.ns, NC = p.nchunk;
-  uint4* dg = reinterpret_cast<uint4*>(sk_smem);                          // [KRM][kDigitQuads][nb]
-  int4* bc = reinterpret_cast<int4*>(dg + (size_t)KRM * kDigitQuads * nb);  // [KRM][nb]
-  float* misc = reinterpret_cast<float*>(bc + (size_t)KRM * nb);          // 64 floats
+  __half* xh = reinterpret_cast<__half*>(sk_smem);                        // PRO_RESID: [KRM][k]
+  float* misc = reinterpret_cast<float*>(sk_smem + stage_x_bytes(KRM, k, p.pro));  // 64 floats
   float* red = misc + 64;                                                 // [NS][NC][R][KRM]
   uint64_t* bars = reinterpret_cast<uint64_t*>(
       ((uintptr_t)(reinterpret_cast<unsigned char*>(red) + stage_red_bytes(NS, NC, R, KRM)) + 127) &
@@ -1418,35 +1494,40 @@ __global__ void __launch_bounds__(kStageThreads, 1) gemv_q4_stage_kernel(const G
   __syncthreads();  // barriers initialised before any wait
   pdl_wait();
   if (tid == 0) stamp(1);
-  stage_digits<KRM, kStageThreads>(p, dg, bc, misc);  // ends with __syncthreads
-  if (tid == 0) stamp(2);
-  pdl_launch_dependents();
+  if (p.pro == PRO_RESID) stage_x_half<KRM, kStageThreads>(p, xh, misc);  // ends with __syncthreads
   volatile int* abort_flag = &s_abort;
 
-  if (warp < n_comp) {
-    // ---------------- compute warp: chunk c of row group g ----------------
-    // lane l holds block 32 c + l of every row; a lane past the end of the row
-    // reads block nb - 1 with zero digits and a zero x scale (no branch)
-    const int c = warp % NC, g = warp / NC;
-    const int blk = 32 * c + lane;
-    const bool has = blk < nb;
-    const int qoff = 16 * min(blk, nb - 1), soff = 2 * min(blk, nb - 1);
-    uint4 xg[KRM][kDigitQuads];
-    int4 cv[KRM];
-    float xsc[KRM];
+  // compute warp (c, g): chunk c of row group g. Lane l holds block 32 c + l of
+  // every row and builds that block's x digits itself; a lane past the end of
+  // the row reads block nb - 1 with zero digits and a zero x scale (no branch).
+  const int c = warp % NC, g = warp / NC;
+  const int blk = 32 * c + lane;
+  const bool has = warp < n_comp && blk < nb;
+  uint4 xg[KRM][kDigitQuads];
+  int4 cv[KRM];
+  float xsc[KRM];
 #pragma unroll
-    for (int j = 0; j < KRM; ++j) {
-      if (has && (KRM == 1 || j < p.kr)) {
+  for (int j = 0; j < KRM; ++j) {
+    if (has && (KRM == 1 || j < p.kr)) {
+      const __half* xb = p.pro == PRO_RESID ? xh + (size_t)j * k + 32 * blk : p.x + (size_t)j * p.x_stride + 32 * blk;
+      uint4 xv[4];
 #pragma unroll
-        for (int q = 0; q < kDigitQuads; ++q) xg[j][q] = dg[(size_t)(j * kDigitQuads + q) * nb + blk];
-        cv[j] = bc[j * nb + blk];
-      } else {
+      for (int q = 0; q < 4; ++q) xv[q] = *reinterpret_cast<const uint4*>(xb + 8 * q);
+      lane_block_digits(xv, xg[j], cv[j]);
+    } else {
 #pragma unroll
-        for (int q = 0; q < kDigitQuads; ++q) xg[j][q] = make_uint4(0, 0, 0, 0);
-        cv[j] = make_int4(0, 0, 0, 0);
-      }
-      xsc[j] = __int_as_float(cv[j].w);
+      for (int q = 0; q < kDigitQuads; ++q) xg[j][q] = make_uint4(0, 0, 0, 0);
+      cv[j] = make_int4(0, 0, 0, 0);
     }
+    xsc[j] = __int_as_float(cv[j].w);
+  }
+  // x read from global: its loads go first, the weight stream resumes after
+  if (p.pro != PRO_RESID) __syncthreads();
+  if (tid == 0) stamp(2);
+  pdl_launch_dependents();
+
+  if (warp < n_comp) {
+    const int qoff = 16 * min(blk, nb - 1), soff = 2 * min(blk, nb - 1);
     int s = 0;
     uint32_t ph = 0;
     for (int t = 0; t < n_st; ++t) {
@@ -1476,11 +1557,14 @@ __global__ void __launch_bounds__(kStageThreads, 1) gemv_q4_stage_kernel(const G
     }
   } else if (reducer) {
     // ---------------- reducer: partials -> epilogue, then refill the slot ----------------
-    if (lane == 0)  // the first stages not issued before the dependency wait
+    if (lane == 0) {  // the first stages not issued before the dependency wait
       for (; issued < NS && issued < n_st; ++issued) {
         cs_issue<R>(p, u0 + issued, stages + issued * SB, &full[issued], false, pol);
         if (issued < 64) stamp(8 + issued);
       }
+      // all own loads issued: start the next GEMV's weights towards L2
+      if (issued == n_st) prefetch_next(p.next, blockIdx.x, gridDim.x);
+    }
     float best_v = -INFINITY;
     int best_i = 0x7fffffff;
     const int r = lane / KRM, j = lane % KRM;  // lanes l < R * KRM
@@ -1517,6 +1601,7 @@ __global__ void __launch_bounds__(kStageThreads, 1) gemv_q4_stage_kernel(const G
           cs_issue<R>(p, u0 + t + NS, stages + s * SB, &full[s], false, pol);
           if (t + NS < 64) stamp(8 + t + NS);
           issued = t + NS + 1;
+          if (issued == n_st) prefetch_next(p.next, blockIdx.x, gridDim.x);
         }
       }
       if (++s == NS) s = 0, ph ^= 1u;
@@ -1570,7 +1655,7 @@ bool plan_stage(GemvParams& p, int& R, int& RG, bool forced) {
   for (int s = 0; s < p.nseg; ++s)
     if (!aligned16(p.seg[s].qs) || !aligned16(p.seg[s].sc) || (s < p.nseg - 1 && p.seg[s].rows % 16))
       return false;
-  if (p.pro == PRO_X16 && !aligned16(p.x)) return false;
+  if (p.pro == PRO_X16 && (!aligned16(p.x) || (p.kr > 1 && p.x_stride % 8))) return false;
   (void)forced;
   const int NC = (nb + 31) / 32;
   if (NC > kStageCompute) return false;
@@ -1593,12 +1678,15 @@ bool plan_stage(GemvParams& p, int& R, int& RG, bool forced) {
   const size_t budget = 220 * 1024, stage = (size_t)R * row_bytes;
   int ns = 0;
   for (int n = kStageMaxSlots; n >= 2; --n)
-    if (stage_fixed_bytes(krm, k, n, NC, R) + (size_t)n * stage <= budget) {
+    if (stage_fixed_bytes(krm, k, p.pro, n, NC, R) + (size_t)n * stage <= budget) {
       ns = n;
       break;
     }
   if (ns < 4) return false;
-  static const int prefetch_env = getenv("Q4G_CS_PREFETCH") ? atoi(getenv("Q4G_CS_PREFETCH")) : 0;
+  // stages issued before the dependency wait: measured best at 2 (more delays
+  // the prologue's own loads behind the weight stream); Q4G_CS_PREFETCH
+  // overrides it (0: all), a tuning switch
+  static const int prefetch_env = getenv("Q4G_CS_PREFETCH") ? atoi(getenv("Q4G_CS_PREFETCH")) : 2;
   p.prefetch_stages = prefetch_env;
   p.ns = ns;
   p.nchunk = NC;
@@ -1612,7 +1700,7 @@ bool plan_stage(GemvParams& p, int& R, int& RG, bool forced) {
 template <int KRM, int R, int RG>
 cudaError_t launch_stage_r(const GemvParams& p, cudaStream_t st, bool pdl) {
   static size_t configured = 0;
-  const size_t smem = stage_fixed_bytes(KRM, p.k, p.ns, p.nchunk, R) + (size_t)p.ns * p.stage_bytes;
+  const size_t smem = stage_fixed_bytes(KRM, p.k, p.pro, p.ns, p.nchunk, R) + (size_t)p.ns * p.stage_bytes;
   cudaError_t e;
   if (smem > configured) {
     e = cudaFuncSetAttribute(gemv_q4_stage_kernel<KRM, R, RG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
