@@ -51,6 +51,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=None,
                     help="fewer layers of the same shapes (profiling captures of a small case)")
+    ap.add_argument("--gemv-chain", type=int, choices=[0, 1], default=None,
+                    help="run O, gate|up, down and the next QKV of a layer as one persistent launch "
+                         "(default: the library's default)")
     return ap.parse_args()
 
 
@@ -248,6 +251,8 @@ def main():
     assert K >= 1 and W >= 3 and K + W < C, "need steps >= 1, warmup >= 3 and steps + warmup < context"
     t_setup = time.perf_counter()
     model = S.SynthDecoder(cfg, seed=args.seed)
+    if args.gemv_chain is not None:
+        Q.q4g_model_set_option(model.handle, Q.Q4G_OPT_GEMV_CHAIN, args.gemv_chain)
     cache = model.new_cache(C)
     stream = torch.cuda.current_stream()
     sp = stream.cuda_stream

@@ -255,7 +255,8 @@ extern "C" q4g_status q4g_model_create(const q4g_config* cfg, const q4g_weights*
     part = b > part ? b : part;
   }
   const size_t part_ml = part / 128 + 1024;  // (m, l) per row and chunk: hd >= 256
-  m->n_counters = 64 + kChainMaxPhases * c.n_layers;  // head, attention, chain phases
+  // head, attention, chain phases, then the two-cluster ring attention merge
+  m->n_counters = 64 + kChainMaxPhases * c.n_layers + kRingSplitCounters;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -871,6 +872,11 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
       p.combine_in_kernel = full ? 0 : 1;
       if (!full && m->attn_cluster) {
         // sliding layers: the chunks of one KV head form a cluster and merge in DSMEM
+        p.trace = trace_sep ? trace_sep + 4 * kGemvTraceSlots : nullptr;
+        if (S.nkv * kAttnCluster <= kRingSplitCounters) {
+          p.ring_split = 2;
+          p.counters = m->counters + 64 + kChainMaxPhases * L;
+        }
         p.cluster = kAttnCluster;
         p.n_chunks = kAttnCluster;
         p.combine_in_kernel = 0;

@@ -10,10 +10,10 @@
 // used by 2 rows only, so the scan is a latency problem, not a throughput one:
 //   * the CL = 8 CTAs of one KV head form a thread-block cluster; CTA c scans
 //     keys [c * cs, (c + 1) * cs) by age, warp w a contiguous 1/8 of that;
-//   * 16 warps per CTA; each warp loads its keys' K and V rows straight into
-//     registers (16 bytes per lane and row), the first group of keys before
-//     waiting on the previous kernel (the rows were written by earlier steps),
-//     the next group while it works on the current one;
+//   * 16 warps per CTA; each warp copies the K and V rows of all its keys
+//     (at most kRingKeysPerWarp) into its own shared-memory buffer with 16-byte
+//     asynchronous copies before waiting on the previous kernel (the rows were
+//     written by earlier steps), so the scan reads shared memory only;
 //   * lane l holds dims 8l .. 8l+7 (hd 256) of the query and of each key; per
 //     group of 4 keys the fp32 dot products are reduced over the warp with a
 //     transposing butterfly, followed by one online-softmax update and P.V,
@@ -25,7 +25,10 @@
 #include "q4g_common.cuh"
 #include "q4g_internal.h"
 
+#include <stdlib.h>
+
 #include <algorithm>
+#include <cstddef>
 
 namespace q4g {
 
@@ -33,17 +36,33 @@ namespace {
 
 constexpr int kRingThreads = 512;
 constexpr int kRingWarps = kRingThreads / 32;
+constexpr int kRingKeysPerWarp = 10;  // 1024-key window, 8 CTAs, 16 warps, up to 4 query rows
 
 template <int HD, int ROWS>
 struct RingSmem {
-  __half q[ROWS][HD];                  // queries after norm and RoPE (fp16, as stored)
-  __half kloc[kMaxRows][HD];           // the block's own K rows
-  __half vloc[kMaxRows][HD];           // the block's own V rows
-  float part[kRingWarps][ROWS][HD];    // warp partial sums of p * v
+  alignas(16) __half q[ROWS][HD];      // queries after norm and RoPE (fp16, as stored)
+  alignas(16) __half kloc[kMaxRows][HD];  // the block's own K rows
+  alignas(16) __half vloc[kMaxRows][HD];  // the block's own V rows
   float pm[kRingWarps][ROWS], pl[kRingWarps][ROWS];
   float cacc[ROWS][HD];                // CTA partial, relative to cm
   float cm[ROWS], cl[ROWS];
+  union alignas(16) {  // read and written 16 bytes at a time
+    __half kv[kRingWarps][kRingKeysPerWarp][2][HD];  // scan: each warp's K and V rows
+    float part[kRingWarps][ROWS][HD];                // merge: warp partial sums of p * v
+  };
 };
+using RingSmem1 = RingSmem<256, 1>;
+using RingSmem2 = RingSmem<256, 2>;
+using RingSmem4 = RingSmem<256, 4>;
+static_assert(offsetof(RingSmem1, kv) % 16 == 0 && offsetof(RingSmem2, kv) % 16 == 0 &&
+                  offsetof(RingSmem4, kv) % 16 == 0 && offsetof(RingSmem1, kloc) % 16 == 0,
+              "16-byte accesses need 16-byte aligned buffers");
+static_assert(sizeof(RingSmem<256, 4>) <= 227 * 1024, "shared memory of one CTA");
+
+Q4G_DEV void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
+               : "memory");
+}
 
 // Sum v[0..N) over the 32 lanes (N a power of two <= 32) and give every lane
 // all N totals: a transposing butterfly (N - 1 + log2(32 / N) shuffles), then
@@ -121,7 +140,7 @@ Q4G_DEV void norm_rope_vec(const AttnParams& p, const float* src, const float* g
 
 // Code size is kept small on purpose: every SM runs one CTA of this kernel per
 // layer, so its instructions are fetched cold; the loop over key groups is rolled.
-template <int HD, int ROWS, int CL>
+template <int HD, int ROWS, int CL, int S>
 __global__ void __launch_bounds__(kRingThreads, 1) attn_ring_kernel(const AttnParams p) {
   static_assert(HD == 256, "one 16-byte piece per lane and row");
   constexpr int B = ROWS <= 2 ? 4 : 2;  // keys per group
@@ -130,8 +149,15 @@ __global__ void __launch_bounds__(kRingThreads, 1) attn_ring_kernel(const AttnPa
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int kv = blockIdx.x;
   const int chunk = (int)cluster_rank();
+  const int half = (int)blockIdx.y / CL;  // cluster index: S clusters per KV head split the keys
+  const int gchunk = half * CL + chunk;
   const int G = p.n_q / p.n_kv, nr = p.kr * G;  // nr <= ROWS (host)
   const bool fused = p.qkv != nullptr;
+  uint64_t* const tr = kv == 0 && gchunk == 0 && tid == 0 ? p.trace : nullptr;
+  auto stamp = [&](int i) {
+    if (tr) tr[i] = global_ns();
+  };
+  stamp(0);
 
   // The position was written before the first kernel of the step and the cache
   // rows read below by earlier steps: both may be read before griddepcontrol.wait.
@@ -140,29 +166,26 @@ __global__ void __launch_bounds__(kRingThreads, 1) attn_ring_kernel(const AttnPa
   const int R = (int)p.cache_rows, W = (int)p.window;
   const int qlm = (int)(q_last % p.cache_rows);  // slot of the newest key
   const int nscan = (int)min((int64_t)W + p.kr - 1, q_last + 1);
-  const int cs = (nscan + CL - 1) / CL;
-  const int a_begin = min(nscan, chunk * cs), a_end = min(nscan, a_begin + cs);
+  const int cs = (nscan + CL * S - 1) / (CL * S);
+  const int a_begin = min(nscan, gchunk * cs), a_end = min(nscan, a_begin + cs);
   const int kpw = (a_end - a_begin + kRingWarps - 1) / kRingWarps;
   const int wa0 = min(a_end, a_begin + warp * kpw), wa1 = min(a_end, wa0 + kpw);
   const int first_cached = fused ? p.kr : 0;  // ages below are the block's own rows
 
-  // lane l holds dims 8l .. 8l+7 of every row
+  // lane l holds dims 8l .. 8l+7 of every row; every cached key of the warp
+  // (wa1 - wa0 <= kRingKeysPerWarp, checked on the host) goes to shared memory
   const __half* kcache = p.k_cache + (size_t)kv * R * HD + lane * 8;
   const __half* vcache = p.v_cache + (size_t)kv * R * HD + lane * 8;
-  auto load_group = [&](int a0, uint4 (&kb)[B], uint4 (&vb)[B]) {
-#pragma unroll
-    for (int i = 0; i < B; ++i) {
-      const int a = a0 + i;
-      const bool in = a < wa1 && a >= first_cached;
-      const size_t off = in ? (size_t)wrap(qlm - a, R) * HD : 0;
-      kb[i] = in ? ld_stream_u4(kcache + off) : make_uint4(0, 0, 0, 0);
-      vb[i] = in ? ld_stream_u4(vcache + off) : make_uint4(0, 0, 0, 0);
-    }
-  };
-  uint4 kb[B], vb[B];
-  load_group(wa0, kb, vb);
+#pragma unroll 1
+  for (int a = max(wa0, first_cached); a < wa1; ++a) {
+    const size_t off = (size_t)wrap(qlm - a, R) * HD;
+    cp_async16(&sm.kv[warp][a - wa0][0][lane * 8], kcache + off);
+    cp_async16(&sm.kv[warp][a - wa0][1][lane * 8], vcache + off);
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
 
   pdl_wait();
+  stamp(1);
   // ---- prologue: queries and the block's own K/V rows ----
   if (fused) {
     const int nvec = nr + 2 * p.kr;
@@ -185,7 +208,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) attn_ring_kernel(const AttnPa
     }
   }
   __syncthreads();
-  if (fused && p.write_kv && chunk == 0) {
+  if (fused && p.write_kv && gchunk == 0) {
     for (int c = tid; c < p.kr * HD / 8; c += kRingThreads) {
       const int j = c / (HD / 8), part = c - j * (HD / 8);
       const size_t row = (size_t)wrap(qlm - (p.kr - 1 - j), R);
@@ -196,6 +219,9 @@ __global__ void __launch_bounds__(kRingThreads, 1) attn_ring_kernel(const AttnPa
     }
   }
   pdl_launch_dependents();
+  stamp(2);
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncwarp();  // every lane's copies landed: the warp reads all of them
 
   // ---- scan: per group of B keys, scores for every row, one online-softmax update ----
   float q[ROWS][8];
@@ -227,18 +253,20 @@ __global__ void __launch_bounds__(kRingThreads, 1) attn_ring_kernel(const AttnPa
   }
 #pragma unroll 1
   for (int a0 = wa0; a0 < wa1; a0 += B) {
-    if (fused && a0 < first_cached) {  // the block's own rows, from the prologue
+    uint4 kb[B], vb[B];
 #pragma unroll
-      for (int i = 0; i < B; ++i) {
-        const int a = a0 + i;
-        if (a < first_cached && a < wa1) {
-          kb[i] = *reinterpret_cast<const uint4*>(&sm.kloc[p.kr - 1 - a][lane * 8]);
-          vb[i] = *reinterpret_cast<const uint4*>(&sm.vloc[p.kr - 1 - a][lane * 8]);
-        }
+    for (int i = 0; i < B; ++i) {
+      const int a = a0 + i;
+      if (a >= wa1) {
+        kb[i] = vb[i] = make_uint4(0, 0, 0, 0);
+      } else if (a < first_cached) {  // the block's own rows, from the prologue
+        kb[i] = *reinterpret_cast<const uint4*>(&sm.kloc[p.kr - 1 - a][lane * 8]);
+        vb[i] = *reinterpret_cast<const uint4*>(&sm.vloc[p.kr - 1 - a][lane * 8]);
+      } else {
+        kb[i] = *reinterpret_cast<const uint4*>(&sm.kv[warp][a - wa0][0][lane * 8]);
+        vb[i] = *reinterpret_cast<const uint4*>(&sm.kv[warp][a - wa0][1][lane * 8]);
       }
     }
-    uint4 nk[B], nv[B];
-    if (a0 + B < wa1) load_group(a0 + B, nk, nv);
     float s[B * ROWS];
 #pragma unroll
     for (int i = 0; i < B; ++i) {
@@ -281,11 +309,11 @@ __global__ void __launch_bounds__(kRingThreads, 1) attn_ring_kernel(const AttnPa
         for (int e = 0; e < 8; ++e) acc[r][e] = fmaf(pv, vf[e], acc[r][e]);
       }
     }
-#pragma unroll
-    for (int i = 0; i < B; ++i) kb[i] = nk[i], vb[i] = nv[i];
   }
 
   // ---- merge: warps in shared memory ----
+  stamp(3);
+  __syncthreads();  // the partials reuse the key buffers
 #pragma unroll
   for (int r = 0; r < ROWS; ++r) {
     if (r >= nr) continue;
@@ -314,8 +342,15 @@ __global__ void __launch_bounds__(kRingThreads, 1) attn_ring_kernel(const AttnPa
     if (d == 0) sm.cm[r] = mx, sm.cl[r] = lsum;
   }
   // ---- merge: the CL CTAs of the cluster through distributed shared memory ----
+  stamp(4);
   cluster_sync();
+  stamp(5);
   constexpr int DPC = HD / CL;
+  static_assert(ROWS * DPC <= kRingThreads, "one output element per thread");
+  // this thread's output element (r, d): its merged sum, weight and maximum
+  float o_t = 0.f, l_t = 0.f, m_t = -INFINITY;
+  const bool has_t = tid < nr * DPC;
+  const int r_t = tid / DPC, d_t = chunk * DPC + (tid - r_t * DPC);
 #pragma unroll 1
   for (int idx = tid; idx < nr * DPC; idx += kRingThreads) {
     const int r = idx / DPC, d = chunk * DPC + (idx - r * DPC);
@@ -333,28 +368,73 @@ __global__ void __launch_bounds__(kRingThreads, 1) attn_ring_kernel(const AttnPa
       lsum = fmaf(ld_peer_f32(peer_addr(&sm.cl[r], c)), e, lsum);
       o = fmaf(ld_peer_f32(peer_addr(&sm.cacc[r][d], c)), e, o);
     }
-    const int j = r / G;
-    p.out[((size_t)j * p.n_q + kv * G + r % G) * HD + d] = __float2half_rn(o / lsum);
+    if (S == 1) {
+      const int j = r / G;
+      p.out[((size_t)j * p.n_q + kv * G + r % G) * HD + d] = __float2half_rn(o / lsum);
+    }
+    o_t = o, l_t = lsum, m_t = mx;
   }
+  stamp(6);
   cluster_sync();  // peers may read this CTA's shared memory until here
+  stamp(7);
+  if (S == 1) return;
+  // ---- merge of the S clusters of this KV head: the last CTA of each
+  // (head, output slice) group to finish combines the S partials ----
+  __shared__ int s_ticket;
+  float* xo = p.part_acc + (size_t)kv * S * ROWS * HD;  // [S][ROWS][HD]
+  float* xml = p.part_ml + (size_t)kv * S * ROWS * 2;   // [S][ROWS][2]
+  if (has_t) {
+    xo[((size_t)half * ROWS + r_t) * HD + d_t] = o_t;
+    if (d_t == chunk * DPC) xml[(half * ROWS + r_t) * 2] = m_t, xml[(half * ROWS + r_t) * 2 + 1] = l_t;
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_ticket = atomicAdd(&p.counters[kv * CL + chunk], 1);
+  __syncthreads();
+  if (s_ticket != S - 1) return;
+  __threadfence();
+  if (has_t) {
+    // in cluster order whichever CTA merges, so the result does not depend on timing
+    float mh[S], mm = -INFINITY;
+#pragma unroll
+    for (int h = 0; h < S; ++h) {
+      mh[h] = h == half ? m_t : __ldcg(xml + (h * ROWS + r_t) * 2);
+      mm = fmaxf(mm, mh[h]);
+    }
+    float o = 0.f, l = 0.f;
+#pragma unroll
+    for (int h = 0; h < S; ++h) {
+      const float e = mh[h] == -INFINITY ? 0.f : __expf(mh[h] - mm);
+      const float oh = h == half ? o_t : __ldcg(xo + ((size_t)h * ROWS + r_t) * HD + d_t);
+      const float lh = h == half ? l_t : __ldcg(xml + (h * ROWS + r_t) * 2 + 1);
+      o = fmaf(oh, e, o);
+      l = fmaf(lh, e, l);
+    }
+    const int j = r_t / G;
+    p.out[((size_t)j * p.n_q + kv * G + r_t % G) * HD + d_t] = __float2half_rn(o / l);
+  }
+  if (tid == 0) p.counters[kv * CL + chunk] = 0;  // ready for the next layer
 }
 
-template <int HD, int ROWS>
-cudaError_t launch_ring_t(const AttnParams& p, cudaStream_t st, bool pdl) {
+template <int HD, int ROWS, int CL, int S>
+cudaError_t configure_ring() {
   static bool configured = false;
-  const size_t smem = sizeof(RingSmem<HD, ROWS>);
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attn_ring_kernel<HD, ROWS, kAttnCluster>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  if (configured) return cudaSuccess;
+  auto kern = attn_ring_kernel<HD, ROWS, CL, S>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)sizeof(RingSmem<HD, ROWS>));
+  if (e == cudaSuccess && CL > 8) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess) configured = true;
+  return e;
+}
+
+template <int HD, int ROWS, int CL, int S>
+cudaLaunchConfig_t ring_config(const AttnParams& p, cudaStream_t st, bool pdl, cudaLaunchAttribute (&attr)[2]) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.n_kv, kAttnCluster, 1);
+  cfg.gridDim = dim3(p.n_kv, CL * S, 1);
   cfg.blockDim = dim3(kRingThreads);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = sizeof(RingSmem<HD, ROWS>);
   cfg.stream = st;
-  cudaLaunchAttribute attr[2];
   int na = 0;
   if (pdl) {
     attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -363,12 +443,46 @@ cudaError_t launch_ring_t(const AttnParams& p, cudaStream_t st, bool pdl) {
   }
   attr[na].id = cudaLaunchAttributeClusterDimension;
   attr[na].val.clusterDim.x = 1;
-  attr[na].val.clusterDim.y = kAttnCluster;
+  attr[na].val.clusterDim.y = CL;
   attr[na].val.clusterDim.z = 1;
   ++na;
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, attn_ring_kernel<HD, ROWS, kAttnCluster>, p);
+  return cfg;
+}
+
+template <int HD, int ROWS, int CL, int S>
+cudaError_t launch_ring_t(const AttnParams& p, cudaStream_t st, bool pdl) {
+  cudaError_t e = configure_ring<HD, ROWS, CL, S>();
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[2];
+  const cudaLaunchConfig_t cfg = ring_config<HD, ROWS, CL, S>(p, st, pdl, attr);
+  return cudaLaunchKernelEx(&cfg, attn_ring_kernel<HD, ROWS, CL, S>, p);
+}
+
+// CTAs per KV head: 16 (a non-portable cluster, twice the SMs on the scan) when
+// eight such clusters fit on the device at once, else 8; Q4G_ATTN_CLUSTER=8|16
+// forces it (a tuning switch).
+int ring_cluster_size() {
+  static int cl = 0;
+  if (cl) return cl;
+  const char* env = getenv("Q4G_ATTN_CLUSTER");
+  int pick = env ? atoi(env) : 0;
+  if (pick != 8 && pick != 16) {
+    pick = 8;
+    AttnParams p{};
+    p.n_kv = 8;
+    int n = 0;
+    cudaLaunchAttribute attr[2];
+    if (configure_ring<256, 2, 16, 1>() == cudaSuccess) {
+      const cudaLaunchConfig_t cfg = ring_config<256, 2, 16, 1>(p, 0, false, attr);
+      if (cudaOccupancyMaxActiveClusters(&n, attn_ring_kernel<256, 2, 16, 1>, &cfg) == cudaSuccess && n >= 8)
+        pick = 16;
+    }
+    cudaGetLastError();  // a refused query leaves no error behind
+  }
+  cl = pick;
+  return cl;
 }
 
 }  // namespace
@@ -376,14 +490,48 @@ cudaError_t launch_ring_t(const AttnParams& p, cudaStream_t st, bool pdl) {
 int ring_decode_rows(const AttnParams& p) {
   const int rows = p.kr * (p.n_q / p.n_kv);
   if (!p.ring || p.hd != 256 || rows > 4) return 0;
+  // keys per warp: the scan covers window + kr - 1 ages in kAttnCluster CTAs
+  const int64_t nscan = p.window + p.kr - 1, per_cta = (nscan + kAttnCluster - 1) / kAttnCluster;
+  if ((per_cta + kRingWarps - 1) / kRingWarps > kRingKeysPerWarp) return 0;
   return rows <= 1 ? 1 : rows <= 2 ? 2 : 4;
 }
 
+// Four clusters of 4 CTAs per KV head fit at once for this many KV heads
+// (cluster placement is per GPC, so the SM count alone does not tell).
+bool ring_split_fits(int n_kv) {
+  static int max_clusters = -1;
+  if (max_clusters < 0) {
+    max_clusters = 0;
+    AttnParams p{};
+    p.n_kv = 8;
+    cudaLaunchAttribute attr[2];
+    if (configure_ring<256, 2, 4, 4>() == cudaSuccess) {
+      const cudaLaunchConfig_t cfg = ring_config<256, 2, 4, 4>(p, 0, false, attr);
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, attn_ring_kernel<256, 2, 4, 4>, &cfg) == cudaSuccess) max_clusters = n;
+    }
+    cudaGetLastError();
+  }
+  return n_kv * 4 <= max_clusters;
+}
+
 cudaError_t launch_attention_ring(const AttnParams& p, cudaStream_t st, bool pdl) {
+  // 16 CTAs per KV head (four clusters of 4, merged through the caller's
+  // counters and scratch) when they all fit at once: one SM reads about
+  // 50 GB/s, so the scan wants as many SMs as it can get; else one cluster of
+  // 16 or 8
+  const bool split = p.ring_split == 2 && ring_split_fits(p.n_kv);
+  const bool wide = !split && ring_cluster_size() == 16;
   switch (ring_decode_rows(p)) {
-    case 1: return launch_ring_t<256, 1>(p, st, pdl);
-    case 2: return launch_ring_t<256, 2>(p, st, pdl);
-    case 4: return launch_ring_t<256, 4>(p, st, pdl);
+    case 1:
+      return split ? launch_ring_t<256, 1, 4, 4>(p, st, pdl)
+             : wide ? launch_ring_t<256, 1, 16, 1>(p, st, pdl) : launch_ring_t<256, 1, 8, 1>(p, st, pdl);
+    case 2:
+      return split ? launch_ring_t<256, 2, 4, 4>(p, st, pdl)
+             : wide ? launch_ring_t<256, 2, 16, 1>(p, st, pdl) : launch_ring_t<256, 2, 8, 1>(p, st, pdl);
+    case 4:
+      return split ? launch_ring_t<256, 4, 4, 4>(p, st, pdl)
+             : wide ? launch_ring_t<256, 4, 16, 1>(p, st, pdl) : launch_ring_t<256, 4, 8, 1>(p, st, pdl);
     default: return cudaErrorInvalidValue;
   }
 }

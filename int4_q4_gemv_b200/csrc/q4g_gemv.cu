@@ -1606,6 +1606,7 @@ __global__ void __launch_bounds__(kStageThreads, 1) gemv_q4_stage_kernel(const G
       }
       if (++s == NS) s = 0, ph ^= 1u;
     }
+    if (lane == 0) stamp(5);
     if (p.epi == EPI_HEAD) {
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
@@ -1757,8 +1758,9 @@ cudaError_t launch_stage_t(const GemvParams& p, int R, int RG, cudaStream_t st, 
 // ---------------------------------------------------------------------------
 constexpr int kChainConsumers = 16;
 constexpr int kChainThreads = (kChainConsumers + 1) * 32;
-constexpr int kChainStages = 11;     // ring slots
-constexpr int kChainSlotBytes = 18432;  // largest stage: 8 rows x 4096 or 4 rows x 8192 columns
+constexpr int kChainStages = 5;         // ring slots
+constexpr int kChainSlotBytes = 36864;  // largest stage: 16 rows x 4096 or 8 rows x 8192 columns
+constexpr int kChainMaxRows = 16;       // rows per stage
 
 Q4G_DEV void consumer_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kChainConsumers * 32) : "memory"); }
 
@@ -1779,15 +1781,11 @@ Q4G_DEV void chain_digits(const GemvParams& P, int blk, bool has, float* s_norm,
                           uint4 (&g)[kDigitQuads], int4& cv) {
   const int k = P.k, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   constexpr int NT = kChainConsumers * 32;
-  __half xh[32];
+  uint4 xv[4];
   if (P.pro == PRO_X16) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint4 v = has ? *reinterpret_cast<const uint4*>(P.x + (size_t)blk * 32 + 8 * q) : make_uint4(0, 0, 0, 0);
-      const __half* h = reinterpret_cast<const __half*>(&v);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) xh[8 * q + e] = h[e];
-    }
+    for (int q = 0; q < 4; ++q)
+      xv[q] = has ? *reinterpret_cast<const uint4*>(P.x + (size_t)blk * 32 + 8 * q) : make_uint4(0, 0, 0, 0);
   } else {
     constexpr int R4 = kChainMaxK / (4 * NT);
     const int n4 = k >> 2;
@@ -1856,93 +1854,58 @@ Q4G_DEV void chain_digits(const GemvParams& P, int blk, bool has, float* s_norm,
     }
     consumer_bar();
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint4 v = has ? *reinterpret_cast<const uint4*>(xs + (size_t)blk * 32 + 8 * q) : make_uint4(0, 0, 0, 0);
-      const __half* h = reinterpret_cast<const __half*>(&v);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) xh[8 * q + e] = h[e];
-    }
+    for (int q = 0; q < 4; ++q)
+      xv[q] = has ? *reinterpret_cast<const uint4*>(xs + (size_t)blk * 32 + 8 * q) : make_uint4(0, 0, 0, 0);
   }
-  int em = 1;
-#pragma unroll
-  for (int e = 0; e < 32; ++e) em = max(em, half_exp(xh[e]));
-  int sd[2] = {0, 0};
-  uint32_t words[2][8];
-#pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    const __half h4[4] = {xh[4 * q], xh[4 * q + 1], xh[4 * q + 2], xh[4 * q + 3]};
-    uint32_t wd[2];
-    digits4(h4, em, wd, sd);
-#pragma unroll
-    for (int t = 0; t < 2; ++t) words[t][q] = wd[t];
-  }
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    g[2 * t] = make_uint4(words[t][0], words[t][1], words[t][2], words[t][3]);
-    g[2 * t + 1] = make_uint4(words[t][4], words[t][5], words[t][6], words[t][7]);
-  }
-  // a lane without a block has zero digits and a zero x scale
-  cv = has ? make_int4(-8 * sd[0], -8 * sd[1], 0, (em - 29 + 127) << 23) : make_int4(0, 0, 0, 0);
+  lane_block_digits(xv, g, cv);
+  if (!has) cv = make_int4(0, 0, 0, 0);  // a lane without a block: zero digits and x scale
 }
 
 struct ChainShared {
-  alignas(16) __half xs[kChainMaxK];            // the normed activation row (PRO_RESID), read as uint4
-  alignas(16) float red[kChainStages][kCsMaxConsumers][8];  // [slot][chunk][row]
-  uint64_t full[kChainStages], empty[kChainStages];
-  int cnt[kChainStages];                        // chunk warps done with a slot
-  int seq[kChainStages];                        // stage number last issued into each slot
-  int phase_done[kChainMaxPhases];              // stages of each phase finished in this CTA
+  alignas(16) __half xs[kChainMaxK];                    // the normed activation row (PRO_RESID), read as uint4
+  alignas(16) float red[kChainStages][kCsMaxConsumers][kChainMaxRows];  // [slot][chunk][row]
+  uint64_t full[kChainStages];   // the stage's bytes landed
+  uint64_t ready[kChainStages];  // every compute warp wrote its partials of the stage
   float norm[2 * kChainConsumers];
   int abort_flag;
 };
 
-template <int R>
-Q4G_DEV void chain_issue(const GemvParams& P, int u, unsigned char* st, uint64_t* bar, uint64_t pol) {
-  cs_issue<R>(P, u, st, bar, false, pol);
-}
-
 Q4G_DEV void chain_issue_r(const GemvParams& P, int u, unsigned char* st, uint64_t* bar, uint64_t pol) {
-  if (P.stage_rows == 8) chain_issue<8>(P, u, st, bar, pol);
-  else if (P.stage_rows == 4) chain_issue<4>(P, u, st, bar, pol);
-  else chain_issue<2>(P, u, st, bar, pol);
+  if (P.stage_rows == 16) cs_issue<16>(P, u, st, bar, false, pol);
+  else if (P.stage_rows == 8) cs_issue<8>(P, u, st, bar, false, pol);
+  else cs_issue<4>(P, u, st, bar, false, pol);
 }
 
-// One stage of phase P by consumer warp (chunk c): the R row partial sums go to
-// red[slot][c]; returns nothing, the caller runs the ticket.
-template <int R>
-Q4G_DEV void chain_stage(const GemvParams& P, const unsigned char* st, int blk, const uint4 (&xg)[kDigitQuads],
-                         const int4 cv, float* red_slot_c) {
-  const int kh = P.k >> 1, nb = P.k >> 5, lane = threadIdx.x & 31;
-  const float xsc = __int_as_float(cv.w);  // 0 for a lane without a block
-  const int bq = min(blk, nb - 1);
-  const unsigned char* sq = st + 16 * bq;
-  const unsigned char* ss = st + R * kh + 2 * bq;
-  float v[R];
-#pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const uint4 qv = *reinterpret_cast<const uint4*>(sq + r * kh);
-    const float d = __half2float(*reinterpret_cast<const __half*>(ss + r * 2 * nb));
-    v[r] = d * xsc * block_dot_int(qv, xg, cv);
-  }
-  const float tot = cs_reduce_rows<R>(v, lane);
-  if ((lane & (32 / R - 1)) == 0) red_slot_c[cs_row<R>(lane)] = tot;
+// Units of phase P owned by this CTA.
+Q4G_DEV void chain_range(const GemvParams& P, int& u0, int& n_st) {
+  u0 = (int)((long long)blockIdx.x * P.n_units / gridDim.x);
+  n_st = (int)((long long)(blockIdx.x + 1) * P.n_units / gridDim.x) - u0;
 }
 
+// The GEMVs of one decode layer (O, gate|up, down, next QKV) in one persistent
+// launch, one CTA per SM, built like the stage kernel: one ring of
+// kChainStages slots runs through all phases in order, compute warp (c, g)
+// takes chunk c of row group g (4 rows) of every stage, and the reducer warp
+// adds the partials, runs the phase's epilogue and refills the slot with the
+// next stage of the whole sequence, which may belong to a later phase: the
+// weights keep streaming while the compute warps wait for the previous phase
+// to finish everywhere (a per-phase counter every CTA bumps once its last
+// stage of the phase is reduced) and build the next x digits. Every wait is
+// bounded; the launch is cooperative, so all CTAs are resident.
 __global__ void __launch_bounds__(kChainThreads, 1) gemv_q4_chain_kernel(const ChainParams c) {
   extern __shared__ __align__(128) unsigned char chain_stages[];  // [kChainStages][kChainSlotBytes]
   __shared__ __align__(16) ChainShared sh;
+  constexpr int RG = 4;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool producer = warp == kChainConsumers;
+  const bool reducer = warp == kChainConsumers;
   const int NS = kChainStages;
   const uint64_t pol = policy_evict_first();
 
   if (tid == 0) {
     sh.abort_flag = 0;
-    for (int s = 0; s < NS; ++s) mbar_init(&sh.full[s], 1), mbar_init(&sh.empty[s], 1);
+    for (int s = 0; s < NS; ++s) mbar_init(&sh.full[s], 1), mbar_init(&sh.ready[s], kChainConsumers);
     fence_mbar_init();
   }
-  if (tid < NS) sh.cnt[tid] = 0, sh.seq[tid] = -1;
-  if (tid < kChainMaxPhases) sh.phase_done[tid] = 0;
   __syncthreads();
   volatile int* abort_flag = &sh.abort_flag;
   const bool tr = c.trace && blockIdx.x == 0;
@@ -1953,42 +1916,77 @@ __global__ void __launch_bounds__(kChainThreads, 1) gemv_q4_chain_kernel(const C
   GemvParams wp{};
   wp.err = c.err;
   wp.wait_ns = c.wait_ns;
+  // the whole stage sequence of this CTA: phase ph holds global stages
+  // [base[ph], base[ph] + cnt[ph])
+  int base[kChainMaxPhases + 1], u0s[kChainMaxPhases];
+  base[0] = 0;
+  for (int ph = 0; ph < c.n_ph; ++ph) {
+    int n;
+    chain_range(c.ph[ph], u0s[ph], n);
+    base[ph + 1] = base[ph] + n;
+  }
+  const int total = base[c.n_ph];
+  auto issue = [&](int T) {  // global stage T into slot T % NS
+    int ph = 0;
+    while (T >= base[ph + 1]) ++ph;
+    chain_issue_r(c.ph[ph], u0s[ph] + T - base[ph], chain_stages + (size_t)(T % NS) * kChainSlotBytes,
+                  &sh.full[T % NS], pol);
+    if (T == base[ph + 1] - 1) stamp(2 + 4 * ph + 3);
+  };
 
-  if (producer) {
-    if (lane == 0) {
-      int t = 0;
-      for (int ph = 0; ph < c.n_ph; ++ph) {
-        const GemvParams& P = c.ph[ph];
-        const int u0 = (int)((long long)blockIdx.x * P.n_units / gridDim.x);
-        const int n_st = (int)((long long)(blockIdx.x + 1) * P.n_units / gridDim.x) - u0;
-        for (int i = 0; i < n_st; ++i, ++t) {
-          const int s = t % NS;
-          if (t >= NS && !*abort_flag) cs_wait(&sh.empty[s], (uint32_t)(((t - NS) / NS) & 1), wp, abort_flag);
-          if (*abort_flag) break;
-          chain_issue_r(P, u0 + i, chain_stages + (size_t)s * kChainSlotBytes, &sh.full[s], pol);
-          publish_issued(&sh.seq[s], t);
-        }
-        stamp(2 + 4 * ph + 3);
+  if (reducer) {
+    // ---------------- reducer: partials -> epilogue, refill, phase counters ----------------
+    int issued = 0;
+    if (lane == 0)
+      for (; issued < NS && issued < total; ++issued) issue(issued);
+    int T = 0;
+    for (int ph = 0; ph < c.n_ph && !*abort_flag; ++ph) {
+      const GemvParams& P = c.ph[ph];
+      const int R = P.stage_rows, NC = P.nchunk;
+      for (int i = 0; i < base[ph + 1] - base[ph]; ++i, ++T) {
+        const int s = T % NS;
+        if (!*abort_flag) cs_wait(&sh.ready[s], (uint32_t)((T / NS) & 1), wp, abort_flag);
         if (*abort_flag) break;
+        float val = 0.f;
+        if (lane < R)
+          for (int cc = 0; cc < NC; ++cc) val += sh.red[s][cc][lane];
+        const int u = u0s[ph] + i;
+        if (P.epi == EPI_GEGLU) {
+          const float up = __shfl_sync(0xffffffffu, val, (lane + R / 2) & 31);
+          if (lane < R / 2) P.act[(size_t)(R / 2) * u + lane] = __float2half_rn(gelu_tanh(val) * up);
+        } else if (lane < R && R * u + lane < P.n_rows) {
+          P.y[R * u + lane] = val;
+        }
+        __syncwarp();  // every lane read slot s's partials before the refill
+        if (lane == 0) {
+          if (T + NS < total) issue(T + NS), issued = T + NS + 1;
+          if (i == base[ph + 1] - base[ph] - 1) {
+            // this CTA's outputs of the phase, visible GPU-wide before the count
+            __threadfence();
+            atomicAdd(&c.done[ph], 1);
+            stamp(2 + 4 * ph + 2);
+          }
+        }
       }
-      // after a timeout, wait (bounded) for the copies still in flight before exiting
-      if (*abort_flag)
-        for (int i = t > NS ? t - NS : 0; i < t; ++i)
-          mbar_wait_bounded(&sh.full[i % NS], (uint32_t)((i / NS) & 1), c.wait_ns);
+      if (base[ph + 1] == base[ph] && lane == 0) {
+        __threadfence();
+        atomicAdd(&c.done[ph], 1);
+      }
     }
+    // after a timeout, wait (bounded) for the copies still in flight
+    if (lane == 0 && *abort_flag)
+      for (int i = issued > NS ? issued - NS : 0; i < issued; ++i)
+        mbar_wait_bounded(&sh.full[i % NS], (uint32_t)((i / NS) & 1), c.wait_ns);
     return;
   }
 
-  // ---------------- consumers ----------------
+  // ---------------- compute warps ----------------
   if (tid == 0) stamp(0);
   pdl_wait();
   if (tid == 0) stamp(1);
-  int t_base = 0;
   for (int ph = 0; ph < c.n_ph; ++ph) {
     const GemvParams& P = c.ph[ph];
-    const int NC = P.nchunk, G = P.groups, R = P.stage_rows, nb = P.k >> 5;
-    const int u0 = (int)((long long)blockIdx.x * P.n_units / gridDim.x);
-    const int n_st = (int)((long long)(blockIdx.x + 1) * P.n_units / gridDim.x) - u0;
+    const int NC = P.nchunk, G = P.groups, R = P.stage_rows, nb = P.k >> 5, kh = P.k >> 1;
     if (ph == c.n_ph - 1) pdl_launch_dependents();
     // every CTA finished the previous phase: its outputs are this phase's input
     if (ph > 0) {
@@ -2004,7 +2002,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) gemv_q4_chain_kernel(const C
           __nanosleep(64);
         }
       }
-      consumer_bar();  // orders every consumer thread after thread 0's acquire
+      consumer_bar();  // orders every compute thread after thread 0's acquire
     }
     if (tid == 0) stamp(2 + 4 * ph);
     const bool active = warp < NC * G;
@@ -2014,53 +2012,31 @@ __global__ void __launch_bounds__(kChainThreads, 1) gemv_q4_chain_kernel(const C
     uint4 xg[kDigitQuads];
     int4 cv;
     chain_digits(P, blk, has, sh.norm, sh.xs, xg, cv);
+    const float xsc = __int_as_float(cv.w);  // 0 for a lane without a block
     if (tid == 0) stamp(2 + 4 * ph + 1);
-    if (active) {
-      for (int i = g; i < n_st; i += G) {
-        const int t = t_base + i, s = t % NS;
-        if (!*abort_flag && wait_issued(&sh.seq[s], t, wp, abort_flag))
-          cs_wait(&sh.full[s], (uint32_t)((t / NS) & 1), wp, abort_flag);
+    const int bq = min(blk, nb - 1);
+    // after a timeout the loops run on without waiting or computing: every
+    // compute warp reaches every consumer barrier of the later phases
+    for (int T = base[ph]; T < base[ph + 1]; ++T) {
+      const int s = T % NS;
+      if (!*abort_flag) cs_wait(&sh.full[s], (uint32_t)((T / NS) & 1), wp, abort_flag);
+      if (active && !*abort_flag) {
         const unsigned char* st = chain_stages + (size_t)s * kChainSlotBytes;
-        float* rs = &sh.red[s][0][0];
-        if (R == 8) chain_stage<8>(P, st, blk, xg, cv, rs + cidx * 8);
-        else if (R == 4) chain_stage<4>(P, st, blk, xg, cv, rs + cidx * 8);
-        else chain_stage<2>(P, st, blk, xg, cv, rs + cidx * 8);
-        __syncwarp();
-        int last = 0;
-        if (lane == 0) {
-          __threadfence_block();
-          last = atomicAdd(&sh.cnt[s], 1) == NC - 1;
+        const unsigned char* sq = st + (size_t)g * RG * kh + 16 * bq;
+        const unsigned char* ss = st + (size_t)R * kh + (size_t)g * RG * 2 * nb + 2 * bq;
+        float v[RG];
+#pragma unroll
+        for (int r = 0; r < RG; ++r) {
+          const uint4 qv = *reinterpret_cast<const uint4*>(sq + r * kh);
+          const float d = __half2float(*reinterpret_cast<const __half*>(ss + r * 2 * nb));
+          v[r] = d * xsc * block_dot_int(qv, xg, cv);
         }
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (!last) continue;
-        __threadfence_block();
-        const int u = u0 + i;
-        float val = 0.f;
-        if (lane < R)
-          for (int cc = 0; cc < NC; ++cc) val += rs[cc * 8 + lane];
-        if (P.epi == EPI_GEGLU) {
-          const float up = __shfl_sync(0xffffffffu, val, (lane + R / 2) & 31);
-          if (lane < R / 2) P.act[(size_t)(R / 2) * u + lane] = __float2half_rn(gelu_tanh(val) * up);
-        } else if (lane < R && R * u + lane < P.n_rows) {
-          P.y[R * u + lane] = val;
-        }
-        __syncwarp();
-        if (lane == 0) {
-          sh.cnt[s] = 0;
-          mbar_arrive(&sh.empty[s]);
-          // CTA-scope release of this stage's outputs; the warp that completes
-          // the phase acquires them all and publishes them with one GPU-scope fence
-          __threadfence_block();
-          if (atomicAdd(&sh.phase_done[ph], 1) == n_st - 1) {
-            __threadfence();
-            atomicAdd(&c.done[ph], 1);
-            stamp(2 + 4 * ph + 2);
-          }
-        }
+        const float tot = cs_reduce_rows<RG>(v, lane);
+        if ((lane & (32 / RG - 1)) == 0) sh.red[s][cidx][g * RG + cs_row<RG>(lane)] = tot;
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.ready[s]);  // release of the partials above
     }
-    if (n_st == 0 && tid == 0) atomicAdd(&c.done[ph], 1);
-    t_base += n_st;
   }
   if (tid == 0) stamp(18);
 }
@@ -2069,24 +2045,28 @@ __global__ void __launch_bounds__(kChainThreads, 1) gemv_q4_chain_kernel(const C
 bool plan_chain_phase(GemvParams& p) {
   const int k = p.k, nb = k >> 5;
   if (k % 256 != 0 || p.kr != 1 || p.epi == EPI_HEAD) return false;
-  if (p.epi == EPI_GEGLU && (p.nseg != 2 || p.seg[0].rows != p.seg[1].rows || p.seg[0].rows % 4)) return false;
-  if (p.pro == PRO_RESID && k > 8192) return false;
+  if (p.epi == EPI_GEGLU && (p.nseg != 2 || p.seg[0].rows != p.seg[1].rows)) return false;
+  if (p.pro == PRO_RESID && k > kChainMaxK) return false;
   for (int s = 0; s < p.nseg; ++s)
-    if (!aligned16(p.seg[s].qs) || !aligned16(p.seg[s].sc) || (s < p.nseg - 1 && p.seg[s].rows % 8))
-      return false;
+    if (!aligned16(p.seg[s].qs) || !aligned16(p.seg[s].sc)) return false;
   if (p.pro == PRO_X16 && !aligned16(p.x)) return false;
   const int NC = (nb + 31) / 32;
   if (NC > kChainConsumers) return false;
   const size_t row_bytes = (size_t)k / 2 + (size_t)k / 16;
   auto units = [&](int r) { return p.epi == EPI_GEGLU ? p.seg[0].rows / (r / 2) : (p.n_rows + r - 1) / r; };
-  int R = 8;
-  while (R > 2 && (size_t)R * row_bytes > (size_t)kChainSlotBytes) R /= 2;
-  if ((size_t)R * row_bytes > (size_t)kChainSlotBytes) return false;
-  while (R > 2 && units(R) < device_sm_count()) R /= 2;  // small matrices: more, smaller stages
+  // rows per stage: a multiple of the 4-row groups, within a slot and within
+  // the 16 compute warps
+  auto fits = [&](int r) { return (size_t)r * row_bytes <= (size_t)kChainSlotBytes && NC * (r / 4) <= kChainConsumers; };
+  int R = kChainMaxRows;
+  while (R > 4 && !fits(R)) R /= 2;
+  if (!fits(R)) return false;
+  while (R > 4 && units(R) < device_sm_count()) R /= 2;  // small matrices: more, smaller stages
   if (p.epi == EPI_GEGLU && p.seg[0].rows % (R / 2)) return false;
+  for (int s = 0; s + 1 < p.nseg; ++s)
+    if (p.seg[s].rows % R) return false;  // no stage straddles two segments
   p.stage_rows = R;
   p.nchunk = NC;
-  p.groups = std::min(kChainConsumers / NC, kChainStages - 2);
+  p.groups = R / 4;
   p.stage_bytes = (int)((size_t)R * row_bytes);
   p.n_units = units(R);
   return p.n_units >= 1;

@@ -151,10 +151,14 @@ struct AttnParams {
   int32_t* counters;     // [n_kv] for the in-kernel combine (ring), zero between launches
   int32_t combine_in_kernel;
   int32_t cluster;       // kAttnCluster: grid y is one cluster, merge through DSMEM (n_chunks == cluster)
+  uint64_t* trace;       // optional timeline of the first CTA (ring cluster kernel), %globaltimer ns
+  int32_t ring_split;    // ring cluster kernel: 2 = several clusters per KV head, merged through
+                         // part_ml / part_acc and counters[n_kv * 4] (zero, left zero)
   __half* out;           // [kr][n_q][hd]
 };
 
 constexpr int kAttnCluster = 8;  // CTAs per KV head when the merge runs in a cluster
+constexpr int kRingSplitCounters = 64;  // model counters of the two-cluster ring merge (n_kv * kAttnCluster)
 size_t attn_smem_bytes(int hd, int m_tiles_per_cta);
 size_t attn_partial_floats(int kr, int n_q, int n_chunks, int hd);
 cudaError_t launch_attention(const AttnParams& p, cudaStream_t st, bool pdl);
