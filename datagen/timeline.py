@@ -3,9 +3,11 @@
 Runs a few decode steps of the synthetic 12B-class decoder (fewer layers by
 default) with the library's trace option and prints, for layer 1 on a common
 time base (ns of %globaltimer from the QKV launch's entry), when CTA 0 of each
-launch entered, when its dependency wait ended, when its x prologue finished,
+launch entered, when its dependency wait ended, when the fused norm's inputs had arrived and
+both norms were reduced (fused-norm launches), when its x prologue finished,
 when its first stage was ready and when its last stage was reduced; for the
-sliding-window attention launch the phases of its first CTA.
+sliding-window attention launch the phases of its first CTA, and the spread of
+the times at which gate|up's CTAs finished.
 
     python -m datagen.timeline [--layers 6] [--context 4096] [--steps 3]
 """
@@ -36,7 +38,7 @@ def main() -> None:
     c = g.new_cache(a.context)
     S.fill_history(c)
     sp = S.stream_ptr()
-    tr = torch.zeros(5 * GEMV_SLOTS, dtype=torch.int64, device="cuda")
+    tr = torch.zeros(6 * GEMV_SLOTS, dtype=torch.int64, device="cuda")
     am = torch.zeros(a.steps + 8, dtype=torch.int32, device="cuda")
     pos0 = a.context - a.steps - 8
     for i in range(6):  # warm-up: graphs captured, caches in steady state
@@ -58,8 +60,16 @@ def main() -> None:
         out["attention"] = {n: us(v) for n, v in zip(names, t[4 * GEMV_SLOTS:4 * GEMV_SLOTS + 8])}
         for name, base in (("qkv", 1), ("o", 2), ("gate_up", 0), ("down", 3)):
             r = t[base * GEMV_SLOTS:(base + 1) * GEMV_SLOTS]
-            out[name] = {"entry": us(r[0]), "dependency_wait": us(r[1]), "x_digits": us(r[2]),
-                         "first_stage_ready": us(r[72]), "last_stage_reduced": us(r[5])}
+            out[name] = {"entry": us(r[0]), "dependency_wait": us(r[1]), "norm_inputs": us(r[3]),
+                         "norms": us(r[4]), "x_digits": us(r[2]), "first_stage_ready": us(r[72]),
+                         "last_stage_reduced": us(r[5])}
+        ends = t[5 * GEMV_SLOTS:6 * GEMV_SLOTS]
+        ends = ends[ends > 0]
+        if len(ends):
+            e = np.sort((ends - t0) / 1e3)
+            out["gate_up_cta_ends"] = {"ctas": int(len(e)), "first": round(float(e[0]), 2),
+                                        "median": round(float(np.median(e)), 2), "p90": round(float(e[int(0.9 * (len(e) - 1))]), 2),
+                                        "last": round(float(e[-1]), 2)}
         if a.json:
             print(json.dumps(out))
             continue
@@ -68,6 +78,8 @@ def main() -> None:
         print("  attention " + " ".join(f"{k} {v}" for k, v in att.items()))
         for name in ("qkv", "o", "gate_up", "down"):
             print(f"  {name:9s} " + " ".join(f"{k} {v}" for k, v in out[name].items()))
+        if "gate_up_cta_ends" in out:
+            print("  gate_up CTA ends " + " ".join(f"{k} {v}" for k, v in out["gate_up_cta_ends"].items()))
     Q.q4g_model_set_option(g.handle, Q.Q4G_OPT_TRACE, 0)
 
 

@@ -272,13 +272,15 @@ typedef enum {
                                  per phase i at 2 + 4i: inputs ready, x digits built,
                                  last stage of CTA 0 done, producer done issuing;
                                  18 end. With GEMV_CHAIN 0 the buffer must hold 1280
-                                 entries instead: 256 each for gate|up, QKV, O and
+                                 entries instead (1536 with the per-CTA ends): 256 each for gate|up, QKV, O and
                                  down of layer 1 when they run on the column-split
                                  or stage kernel, then 256 for layer 1's sliding
                                  attention when it runs on the cluster kernel (0
                                  entry, 1 dependency wait, 2 queries ready, 3 scan
                                  done, 4 warps merged, 5 cluster synced, 6 output
-                                 written, 7 exit); per GEMV launch 0 entry, 1 dependency wait done,
+                                 written, 7 exit), then from entry 1280 when each
+                                 CTA of layer 1's gate|up finished its last stage
+                                 (stage kernel); per GEMV launch 0 entry, 1 dependency wait done,
                                  2 x digits built, 3 and 4 (fused norm prologue)
                                  first loads used and second norm reduced, 5 last
                                  stage reduced (stage kernel), 8 + t

@@ -933,6 +933,7 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
       GemvParams p = gate_up;
       p.next = next_of(down_params(l, 0), 0.6f);
       p.trace = trace_sep;
+      p.trace_ends = trace_sep ? trace_sep + 5 * kGemvTraceSlots : nullptr;
       Prof pr(m, st);
       e = pr.done(debug_sync(launch_gemv(p, st, pdl), "gate_up", l, st), 6, l, gemv_bytes(2 * cf.ffn, H, kr, 1));
       if (e != cudaSuccess) return e;

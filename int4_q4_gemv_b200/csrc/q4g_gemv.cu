@@ -1607,6 +1607,7 @@ __global__ void __launch_bounds__(kStageThreads, 1) gemv_q4_stage_kernel(const G
       if (++s == NS) s = 0, ph ^= 1u;
     }
     if (lane == 0) stamp(5);
+    if (lane == 0 && p.trace_ends) p.trace_ends[blockIdx.x] = global_ns();
     if (p.epi == EPI_HEAD) {
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {

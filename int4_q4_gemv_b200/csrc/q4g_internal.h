@@ -83,6 +83,7 @@ struct GemvParams {
   // dependency wait, [2] after the x prologue, [8 + t] stage t issued,
   // [72 + t] stage t ready for its consumers, [136 + t] stage t reduced (t < 64)
   uint64_t* trace;
+  uint64_t* trace_ends;  // optional [grid]: when each CTA's reducer finished (stage kernel)
   int32_t stall_test;   // 1: the first stage of the warp that owns unit 0 never completes (tests the timeout path)
 };
 
