@@ -262,3 +262,41 @@ def test_host_api_and_range_errors(tiny):
             Q.q4g_verify_block(g.handle, c.handle, ids.data_ptr(), K, pos0, acc, 0, 0, sp())
         assert e.value.status == Q.Q4G_ERANGE
     Q.q4g_model_check(g.handle, sp())
+
+
+def test_trace_timeline_is_ordered():
+    """The trace option (observability, no effect on results): with separate
+    launches, layer 1's GEMV launches stamp entry <= dependency wait <= x ready
+    <= first stage ready <= last stage reduced on the device clock, the ring
+    attention launch stamps its phases in order, gate|up stamps the end of every
+    CTA, and the step's logits equal those of an untraced step."""
+    cfg = WL.TINY
+    g = S.SynthDecoder(cfg, seed=3, variant=0)
+    c = g.new_cache(512)
+    tr = torch.zeros(1536, dtype=torch.int64, device="cuda")
+    lg = torch.empty((2, cfg["vocab"]), dtype=torch.float32, device="cuda")
+    ids = DG.uniform_int(3, DG.STREAM_PREFIX_IDS, 12, cfg["vocab"])
+    for pos in range(10):
+        Q.q4g_decode_step(g.handle, c.handle, int(ids[pos]), pos, 0, 0, sp())
+    torch.cuda.synchronize()
+    # the same step with and without the trace
+    c2 = g.new_cache(512)
+    for pos in range(10):
+        Q.q4g_decode_step(g.handle, c2.handle, int(ids[pos]), pos, 0, 0, sp())
+    Q.q4g_decode_step(g.handle, c2.handle, int(ids[10]), 10, lg[0].data_ptr(), 0, sp())
+    Q.q4g_model_set_option(g.handle, Q.Q4G_OPT_TRACE, tr.data_ptr())
+    Q.q4g_decode_step(g.handle, c.handle, int(ids[10]), 10, lg[1].data_ptr(), 0, sp())
+    torch.cuda.synchronize()
+    Q.q4g_model_set_option(g.handle, Q.Q4G_OPT_TRACE, 0)
+    t = tr.cpu().numpy().astype(np.int64)
+    assert np.array_equal(lg[0].cpu().numpy(), lg[1].cpu().numpy())
+    for base in (0, 256, 512, 768):  # gate|up, QKV, O, down
+        r = t[base:base + 256]
+        seq = [r[0], r[1], r[2], r[72], r[5]]
+        assert all(v > 0 for v in seq), (base, seq)
+        assert all(a <= b for a, b in zip(seq, seq[1:])), (base, seq)
+    att = t[1024:1032]
+    assert all(v > 0 for v in att) and all(a <= b for a, b in zip(att, att[1:])), att
+    ends = t[1280:1536]
+    n = int((ends > 0).sum())
+    assert n >= 1 and np.all(ends[:n] >= t[0]), n  # every CTA of gate|up, from CTA 0 up
