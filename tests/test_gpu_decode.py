@@ -300,3 +300,48 @@ def test_trace_timeline_is_ordered():
     ends = t[1280:1536]
     n = int((ends > 0).sum())
     assert n >= 1 and np.all(ends[:n] >= t[0]), n  # every CTA of gate|up, from CTA 0 up
+
+
+def test_long_context_decode_vs_oracle_32k():
+    """The 32K-context decode config on one period of the 12B shapes (5 sliding
+    layers, 1 full layer, the 262,144-row head): both sides fill every ring slot and
+    every global row from the same seeded history, then run the last two positions
+    of the context and compare logits and argmax."""
+    cfg = dict(WL.B12, n_layers=WL.B12["full_every"])
+    C = 32768
+    p = Pair(cfg, seed=4, variant=1, capacity=C)
+    S.fill_history(p.gc)
+    O.fill_history(p.oc)
+    ids = DG.uniform_int(4, DG.STREAM_PREFIX_IDS, 2, cfg["vocab"])
+    for i, pos in enumerate((C - 2, C - 1)):
+        g, ga, r, ra = p.step_token(int(ids[i]), pos)
+        check_logits(g, r, f"32K decode at {pos}")
+
+
+def test_long_context_verify_vs_oracle_two_pass_128k():
+    """The 128K verify config (K = 4, accepted_count drawn from 0..4) on one period of
+    the 12B shapes over the same seeded history: the single-pass verify against the
+    oracle's two-pass protocol, two blocks ending at the context's last positions."""
+    cfg = dict(WL.B12, n_layers=WL.B12["full_every"])
+    C, K = 131072, 4
+    p = Pair(cfg, seed=5, variant=1, capacity=C)
+    S.fill_history(p.gc)
+    O.fill_history(p.oc)
+    V = cfg["vocab"]
+    ids = DG.uniform_int(5, DG.STREAM_DRAFT_IDS, 2 * K, V).reshape(2, K).astype(np.int32)
+    acc = DG.uniform_int(5, DG.STREAM_ACCEPTED, 2, K + 1)
+    ids_d = torch.from_numpy(ids).cuda()
+    logits = torch.empty((K, V), dtype=torch.float32, device="cuda")
+    am = torch.empty(K, dtype=torch.int32, device="cuda")
+    pos = C - 2 * K
+    for b in range(2):
+        n = int(acc[b])
+        Q.q4g_verify_block(p.gpu.handle, p.gc.handle, ids_d[b].data_ptr(), K, pos, K,
+                           logits.data_ptr(), am.data_ptr(), sp())
+        r = O.verify_block(p.orc, p.oc, pos, ids=ids[b], accepted=0, mode=0)
+        O.verify_block(p.orc, p.oc, pos, ids=ids[b], accepted=n, mode=0, want_logits=False)
+        torch.cuda.synchronize()
+        got = logits.cpu().numpy().astype(np.float64)
+        for i in range(K):
+            check_logits(got[i], r["logits"][i], f"128K block {b} row {i}")
+        pos += n
