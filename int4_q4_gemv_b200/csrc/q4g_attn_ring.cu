@@ -7,9 +7,12 @@
 // p = q - ((q - j) mod R), window test q - p < W).
 //
 // With 2 query rows per KV head (decode of the sliding layers) a key row is
-// used by 2 rows only, so the scan is a latency problem, not a throughput one:
-//   * the CL = 8 CTAs of one KV head form a thread-block cluster; CTA c scans
-//     keys [c * cs, (c + 1) * cs) by age, warp w a contiguous 1/8 of that;
+// used by 2 rows only, so the scan is a latency problem, not a throughput one.
+// One SM reads about 50 GB/s, so the keys of one KV head are spread over as
+// many SMs as fit: S clusters of CL CTAs (4 x 4 when they all fit at once,
+// else one cluster of 16 or 8):
+//   * CTA c of cluster h scans keys [g * cs, (g + 1) * cs) by age, g = h * CL + c,
+//     warp w a contiguous 1/16 of that;
 //   * 16 warps per CTA; each warp copies the K and V rows of all its keys
 //     (at most kRingKeysPerWarp) into its own shared-memory buffer with 16-byte
 //     asynchronous copies before waiting on the previous kernel (the rows were
@@ -19,9 +22,12 @@
 //     transposing butterfly, followed by one online-softmax update and P.V,
 //     all in fp32;
 //   * warp partials merge in shared memory, CTA partials through distributed
-//     shared memory: CTA c of the cluster writes output dims [c * HD/CL, ...).
+//     shared memory: CTA c of a cluster owns output dims [c * HD/CL, ...);
+//   * with S > 1 the CTAs owning the same dims in the S clusters write their
+//     partials to global scratch, and the last to finish (a ticket) merges the S
+//     partials in cluster order, so the result does not depend on timing.
 // The block's own key/value rows (the new positions) come from the prologue;
-// chunk 0 also writes them to the ring.
+// global chunk 0 also writes them to the ring.
 #include "q4g_common.cuh"
 #include "q4g_internal.h"
 
