@@ -35,6 +35,23 @@ if ROOT not in sys.path:
 METRIC = "decode tokens/s at batch 1 and achieved HBM GB/s as % of B200 peak, per context"
 
 
+def max_over_ranks(v: float, world: int, device) -> float:
+    """The maximum of v over all ranks (one all-reduce that every rank takes)."""
+    if world <= 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_rate(units_per_rank: int, world: int, seconds: float) -> float:
+    """Whole-job throughput of `world` independent replicas that each process
+    units_per_rank units, timed by the slowest rank's seconds (weak scaling)."""
+    return world * units_per_rank / seconds
+
+
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -297,14 +314,11 @@ def main():
     ev1.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
-    ms = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, "cuda")
     if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
     ms_per_step = ms / K
-    tok_s = world * K / (ms / 1e3)
+    tok_s = replica_rate(K, world, ms / 1e3)
     positions = range(prefix + W, C)
     bytes_per_tok = weight_bytes(cfg) + statistics.mean(kv_bytes(cfg, q) for q in positions)
     peak, peak_kind = measured_peaks()
@@ -351,12 +365,8 @@ def main():
     for p in range(C - E, C):
         Q.q4g_decode_step_host(model.handle, cache.handle, tok, p, 0, am_host.data_ptr(), sp)
         tok = int(am_host[0])
-    e2e_s = time.perf_counter() - t0
-    if world > 1:
-        t = torch.tensor([e2e_s], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_s = float(t.item())
-    e2e_tok_s = world * E / e2e_s
+    e2e_s = max_over_ranks(time.perf_counter() - t0, world, "cuda")
+    e2e_tok_s = replica_rate(E, world, e2e_s)
 
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
