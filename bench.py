@@ -100,7 +100,8 @@ def weight_bytes(cfg) -> float:
 
 
 def kv_bytes(cfg, q) -> float:
-    """Live K/V bytes read at query position q (SURVEY 8(d) per-unit figures)."""
+    """Live K/V bytes read at query position q: per sliding layer K and V of
+    min(q + 1, W) positions, per full layer K and V of q + 1 positions (fp16)."""
     from datagen import workloads as WL
     n_sl = sum(1 for l in range(cfg["n_layers"]) if not WL.layer_is_full(cfg, l))
     n_gl = cfg["n_layers"] - n_sl
