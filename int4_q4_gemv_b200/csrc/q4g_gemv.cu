@@ -4,7 +4,26 @@
 // "gemma-4-E4B-CoreAI", Provenance: the q4_0 grid): y[j][r] = sum_c w(r,c) x[j][c]
 // with w(r,c) = (code - 8) * d(r, c/32), x fp16, fp32 accumulation.
 //
-// Work decomposition (one launch, persistent over 16-row units):
+// Kernels (one operation, chosen per call; see launch_gemv):
+//   * stage kernel (default): one CTA per SM streams a contiguous range of
+//     16-36 KB row stages through a bulk-copy ring; every compute warp works on
+//     every stage (a column chunk of a row group), with the integer block dot
+//     (16-bit block fixed-point x, dp4a over the raw nibble codes); a reducer
+//     warp adds the chunk partials in a fixed order, runs the epilogue and
+//     refills the slot;
+//   * column-split kernel: the same dot, consumer groups on alternate stages;
+//   * warp-streamed kernel: each warp streams its own row pairs through its own
+//     ring, fp16 nibble unpacking with mixed-precision FMAs (also the fallback
+//     for more than two activation rows);
+//   * register kernel (below): plain streaming loads, any k % 32 == 0;
+//   * chain kernel: O, gate|up, down and the next QKV of a layer in one
+//     cooperative launch built like the stage kernel.
+// The fused prologues (RMSNorm, residual, layer scalar) and epilogues (store,
+// GeGLU, softcap + logits + argmax) are shared by all of them. The first weight
+// loads of every kernel are issued before griddepcontrol.wait, so with
+// programmatic dependent launch they overlap the previous kernel's tail.
+//
+// Register kernel, work decomposition (one launch, persistent over 16-row units):
 //   * a CTA (8 warps) owns a contiguous, balanced range of 16-row units;
 //   * warp w owns columns blocks [w*NB/8, (w+1)*NB/8) of every unit (NB = k/32);
 //   * a warp step covers 4 rows x 8 consecutive blocks: lane (r4 = lane/8,
@@ -16,9 +35,7 @@
 //     produces, and per block the constant 72 * sum(x) removes the +64 offset
 //     of the unpacked values and the -8 of the code (see block_dot);
 //   * partial row sums are reduced with shuffles across the 8 lanes of a row
-//     and in a fixed order across warps through shared memory (deterministic);
-//   * the first weight loads are issued before griddepcontrol.wait, so with
-//     programmatic dependent launch they overlap the previous kernel's tail.
+//     and in a fixed order across warps through shared memory (deterministic).
 #include "q4g_common.cuh"
 #include "q4g_internal.h"
 #include "q4g_prefetch.cuh"
