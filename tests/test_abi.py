@@ -81,3 +81,17 @@ def test_gemv_kernel_choice_validation(lib):
     with pytest.raises(Q.Q4GError) as e:
         Q.q4g_model_create(c, Q.q4g_weights())
     assert e.value.status == Q.Q4G_EINVAL
+
+
+def test_binding_constants_match_the_header():
+    """Every status, option and GEMV-kernel constant the binding defines has the value
+    the header gives it (enum members and #defines parsed from include/q4g.h)."""
+    text = open(HEADER).read()
+    values = {m.group(1): int(m.group(2)) for m in re.finditer(r"\b(Q4G_[A-Z_]+)\s*=\s*(\d+)", text)}
+    values.update({m.group(1): int(m.group(2))
+                   for m in re.finditer(r"^#define\s+(Q4G_[A-Z_]+)\s+(\d+)\s*$", text, flags=re.M)})
+    names = [n for n in dir(Q) if re.fullmatch(r"Q4G_(OK|E[A-Z]+|OPT_[A-Z_]+|GEMV_[A-Z_]+)", n)]
+    assert len(names) >= 19  # statuses, options, GEMV kernel kinds
+    for n in names:
+        assert n in values, f"{n} is not in the header"
+        assert getattr(Q, n) == values[n], f"{n}: binding {getattr(Q, n)} != header {values[n]}"
