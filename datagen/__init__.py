@@ -119,6 +119,14 @@ def history_stream(kind: str, ordinal: int, kv: int) -> int:
     return stream_attn((0x1000 if kind == "ring" else 0x2000) + 2 * ordinal + kv)
 
 
+def history_sigma(kv: int, hd: int) -> float:
+    """Standard deviation of the synthetic K/V history: the per-element scale the
+    decoder itself writes. K rows are RoPE(rmsnorm(k) * gain) with gains of
+    hd^(-1/4) (variants 0 and 1), whose elements have RMS hd^(-1/4); V rows are a
+    scale-free RMSNorm, RMS 1."""
+    return float(qk_gain_base(hd)) if kv == 0 else 1.0
+
+
 def qk_gain_base(hd: int) -> np.float32:
     """hd^(-1/4) as the fp32 constant of the C header (unit-variance q.k scores)."""
     return np.float32({256: 0.25, 512: 0.21022410381342863, 64: 0.35355339059327373,
@@ -126,7 +134,11 @@ def qk_gain_base(hd: int) -> np.float32:
 
 
 def qk_gain(seed: int, stream: int, hd: int, variant: int) -> np.ndarray:
+    """q_norm / k_norm gains: variant 0 the base, 1 the base times the seeded
+    gain, 2 unit gains."""
+    if variant == 2:
+        return np.ones(hd, dtype=np.float32)
     b = qk_gain_base(hd)
-    if not variant:
+    if variant != 1:
         return np.full(hd, b, dtype=np.float32)
     return (b * gain(seed, stream, hd)).astype(np.float32)

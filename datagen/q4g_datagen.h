@@ -105,11 +105,13 @@ DG_FN float dg_qk_gain_base(int hd) {
        : hd == 32 ? 0.42044820762685725f : 1.0f;
 }
 
-/* q_norm / k_norm gain element i: base, or base * (1 + N(0, 0.1)) in the seeded
- * variant (one fp32 multiply). */
+/* q_norm / k_norm gain element i: base (variant 0), base * (1 + N(0, 0.1)) in the
+ * seeded variant 1 (one fp32 multiply), or 1 in variant 2 (unit gains: the
+ * softmax logits q.k are of order head_dim, a sharp softmax). */
 DG_FN float dg_qk_gain(uint64_t key, uint64_t i, int hd, int variant) {
+  if (variant == 2) return 1.0f;
   float b = dg_qk_gain_base(hd);
-  if (!variant) return b;
+  if (variant != 1) return b;
 #ifdef __CUDA_ARCH__
   return __fmul_rn(b, dg_gain(key, i));
 #else

@@ -118,23 +118,24 @@ class SynthDecoder:
                                ("norm_pre_ffn", H, DG.T_NORM_PRE_FFN),
                                ("norm_post_ffn", H, DG.T_NORM_POST_FFN)]:
                 g = torch.ones(n, dtype=torch.float32, device=device)
-                if variant:
+                if variant == 1:
                     fill_gain(g, seed, s(t))
                 self._keep.append(g)
                 setattr(Lw, name, g.data_ptr())
             for name, t in [("norm_q", DG.T_NORM_Q), ("norm_k", DG.T_NORM_K)]:
-                g = torch.full((hd,), float(DG.qk_gain_base(hd)), dtype=torch.float32, device=device)
-                if variant:
+                base = 1.0 if variant == 2 else float(DG.qk_gain_base(hd))  # variant 2: unit gains
+                g = torch.full((hd,), base, dtype=torch.float32, device=device)
+                if variant == 1:
                     gv = torch.empty(hd, dtype=torch.float32, device=device)
                     fill_gain(gv, seed, s(t))
                     g = g * gv                    # one fp32 multiply, as the recipe defines
                 self._keep.append(g)
                 setattr(Lw, name, g.data_ptr())
-            Lw.layer_scalar = 1.0 if not variant else float(
+            Lw.layer_scalar = 1.0 if variant != 1 else float(
                 DG.uniform_float(seed, s(DG.T_LAYER_SCALAR), 1, 0.5, 1.5)[0])
         eq, es = packed_tensor(c["vocab"], H, seed, DG.STREAM_EMBED, device)
         nf = torch.ones(H, dtype=torch.float32, device=device)
-        if variant:
+        if variant == 1:
             fill_gain(nf, seed, DG.STREAM_FINAL_NORM)
         self._keep += [eq, es, nf]
         self.embed_qs, self.embed_sc = eq, es
@@ -205,11 +206,14 @@ class SynthCache:
 
 
 def fill_history(cache: SynthCache, seed: int = 99):
-    """Seeded N(0, 1) fp16 K/V in every ring slot and every global row."""
+    """Seeded fp16 K/V history in every ring slot and every global row, at the scale
+    the decoder writes (datagen.history_sigma: K ~ N(0, hd^(-1/2)), V ~ N(0, 1))."""
     v = cache.view
     for i in range(v.n_sliding):
         for kv in (0, 1):
-            fill_normal_f16(cache.ring(i, kv), seed, DG.history_stream("ring", i, kv), 1.0)
+            fill_normal_f16(cache.ring(i, kv), seed, DG.history_stream("ring", i, kv),
+                            DG.history_sigma(kv, v.sl_head_dim))
     for i in range(v.n_full):
         for kv in (0, 1):
-            fill_normal_f16(cache.global_(i, kv), seed, DG.history_stream("global", i, kv), 1.0)
+            fill_normal_f16(cache.global_(i, kv), seed, DG.history_stream("global", i, kv),
+                            DG.history_sigma(kv, v.gl_head_dim))

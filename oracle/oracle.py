@@ -268,17 +268,20 @@ def fill_normal_f16(out: np.ndarray, seed: int, stream: int, sigma: float = 1.0,
 
 
 def fill_history(cache: Cache, seed: int = 99):
-    """Seeded N(0, 1) fp16 K/V in every ring slot and every global row (the
-    same streams as the GPU harness: datagen.history_stream)."""
+    """Seeded fp16 K/V in every ring slot and every global row at the scale the
+    decoder writes (datagen.history_sigma), from the same streams as the GPU
+    harness (datagen.history_stream)."""
     cfg = cache.model.cfg
     n_sl = sum(1 for l in range(cfg["n_layers"]) if not _is_full(cfg, l))
     n_gl = cfg["n_layers"] - n_sl
     for i in range(n_sl):
         for kv in (0, 1):
-            fill_normal_f16(cache.ring(i, kv), seed, DG.history_stream("ring", i, kv))
+            fill_normal_f16(cache.ring(i, kv), seed, DG.history_stream("ring", i, kv),
+                            DG.history_sigma(kv, cfg["sl_head_dim"]))
     for i in range(n_gl):
         for kv in (0, 1):
-            fill_normal_f16(cache.global_(i, kv), seed, DG.history_stream("global", i, kv))
+            fill_normal_f16(cache.global_(i, kv), seed, DG.history_stream("global", i, kv),
+                            DG.history_sigma(kv, cfg["gl_head_dim"]))
 
 
 def _is_full(cfg, l):

@@ -343,7 +343,7 @@ static int make_qmat(qmat* m, uint64_t seed, uint64_t stream, int64_t rows, int6
 static double* make_gain(uint64_t seed, uint64_t stream, int64_t n, int variant) {
   double* g = (double*)malloc(sizeof(double) * (size_t)n);
   uint64_t key = dg_key(seed, stream);
-  for (int64_t i = 0; i < n; ++i) g[i] = variant ? (double)dg_gain(key, (uint64_t)i) : 1.0;
+  for (int64_t i = 0; i < n; ++i) g[i] = variant == 1 ? (double)dg_gain(key, (uint64_t)i) : 1.0;
   return g;
 }
 
@@ -388,7 +388,7 @@ or_model* or_model_create(const or_config* cfg, uint64_t seed, int variant, int 
     L->n_po = make_gain(seed, DG_STREAM_LAYER(l, DG_T_NORM_POST_FFN), H, variant);
     L->n_q = make_qk_gain(seed, DG_STREAM_LAYER(l, DG_T_NORM_Q), hd, variant);
     L->n_k = make_qk_gain(seed, DG_STREAM_LAYER(l, DG_T_NORM_K), hd, variant);
-    L->lscalar = variant ? (double)dg_uniform_float(dg_key(seed, DG_STREAM_LAYER(l, DG_T_LAYER_SCALAR)),
+    L->lscalar = variant == 1 ? (double)dg_uniform_float(dg_key(seed, DG_STREAM_LAYER(l, DG_T_LAYER_SCALAR)),
                                                     0, 0.5f, 1.5f)
                          : 1.0;
   }

@@ -83,9 +83,10 @@ typedef struct or_model or_model;
 typedef struct or_cache or_cache;
 
 /* Weights generated from the seeded recipe: linear weights N(0, 0.02) packed
- * to q4_0; residual-stream norm gains 1 (variant 0) or 1 + N(0, 0.1)
+ * to q4_0; residual-stream norm gains 1 (variants 0 and 2) or 1 + N(0, 0.1)
  * (variant 1); q_norm / k_norm gains hd^(-1/4), times 1 + N(0, 0.1) in
- * variant 1; layer scalars 1 (variant 0) or U(0.5, 1.5) (variant 1).
+ * variant 1, and 1 in variant 2 (unit gains); layer scalars 1 (variants 0
+ * and 2) or U(0.5, 1.5) (variant 1).
  * nthreads <= 0: all. */
 or_model* or_model_create(const or_config* cfg, uint64_t seed, int variant, int nthreads);
 void or_model_destroy(or_model* m);

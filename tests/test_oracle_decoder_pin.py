@@ -12,6 +12,7 @@ pinned) q4_0 unpack.
 from __future__ import annotations
 
 import numpy as np
+import pytest
 import torch
 import torch.nn.functional as F
 
@@ -45,7 +46,7 @@ class TorchDecoder:
             return None if got is None else torch.from_numpy(O.q4_0_unpack(*got))
 
         def gain(stream, n):
-            if variant == 0:
+            if variant != 1:
                 return torch.ones(n, dtype=torch.float64)
             return torch.from_numpy(DG.gain(seed, stream, n).astype(np.float64))
 
@@ -54,7 +55,7 @@ class TorchDecoder:
             full = WL.layer_is_full(cfg, l)
             hd = cfg["gl_head_dim"] if full else cfg["sl_head_dim"]
             s = lambda t: DG.stream_layer(l, t)
-            scal = 1.0 if variant == 0 else float(DG.uniform_float(seed, s(DG.T_LAYER_SCALAR), 1, 0.5, 1.5)[0])
+            scal = 1.0 if variant != 1 else float(DG.uniform_float(seed, s(DG.T_LAYER_SCALAR), 1, 0.5, 1.5)[0])
             self.layers.append(dict(
                 full=full, hd=hd, wq=mat(l, 0), wk=mat(l, 1), wv=mat(l, 2), wo=mat(l, 3),
                 wg=mat(l, 4), wu=mat(l, 5), wd=mat(l, 6),
@@ -103,9 +104,12 @@ class TorchDecoder:
         return torch.tanh((self.embed @ z) / c["softcap"]) * c["softcap"]
 
 
-def test_oracle_decoder_matches_torch_composition():
+@pytest.mark.parametrize("variant", [1, 2])
+def test_oracle_decoder_matches_torch_composition(variant):
+    """Variant 1: seeded gains and layer scalars; variant 2: unit q/k gains (a sharp
+    softmax, logits of order head_dim)."""
     cfg = dict(WL.MICRO)
-    seed, variant, steps = 4, 1, 40          # 40 steps > 2 ring wraps at R = 16
+    seed, steps = 4, 40                      # 40 steps > 2 ring wraps at R = 16
     om = O.Model(cfg, seed=seed, variant=variant)
     cache = O.Cache(om, 64)
     ref = TorchDecoder(om, cfg, seed, variant)
