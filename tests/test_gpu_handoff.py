@@ -1,0 +1,263 @@
+"""Whole-depth decode parity through a cache hand-off, and the cache rows the CUDA
+path writes.
+
+The GPU runs a seeded prefix through q4g_decode_step; its cache is copied byte for
+byte (through the q4g_cache_layout offsets) into the oracle's cache; then both
+sides run the same next positions (teacher-forced with the oracle's greedy tokens)
+and are compared:
+  * logits and the residual stream after every layer: max |err| <= 2e-2 * RMS(ref),
+    identical argmax (a differing argmax only where the oracle's top-1 gap is
+    below 1e-3 * RMS, reported);
+  * the cache after the step: every ring slot except pos mod R and every global
+    row except pos is bytewise unchanged on the GPU (slot placement is exact);
+    the written rows match the oracle's rows: within one fp16 ulp in layer 0, whose
+    input both sides compute from the same embedding row, and within 2e-2 * RMS of
+    the row in deeper layers, whose inputs carry the residual stream's difference.
+
+The 12B-class decoder runs at its full 48 layers: the 4K decode config with a
+GPU-written prefix, the 32K decode config and the 128K verify config (K = 4,
+seeded accepted counts, against the oracle's two-pass protocol) over seeded
+synthetic history, which both sides fill identically (the 32K and 131K serial
+prefixes do not fit a test's time on the CPU oracle side).
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import datagen as DG
+from datagen import synth as S
+from datagen import workloads as WL
+from int4_q4_gemv_b200 import build as B
+from int4_q4_gemv_b200 import q4g as Q
+from oracle import oracle as O
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-2
+TIE = 1e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    B.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+
+
+def sp():
+    return S.stream_ptr()
+
+
+def check_vec(got, ref, where):
+    rms = float(np.sqrt(np.mean(np.asarray(ref, dtype=np.float64) ** 2)))
+    err = float(np.max(np.abs(np.asarray(got, dtype=np.float64) - ref)))
+    assert err <= TOL * rms, f"{where}: max err {err} > {TOL} * rms {rms}"
+    return err / rms
+
+
+def check_logits(got, ref, where):
+    rel = check_vec(got, ref, where)
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    a_ref, a_got = int(np.argmax(ref.astype(np.float32))), int(np.argmax(got))
+    if a_ref != a_got:
+        gap = float(ref[a_ref] - ref[a_got])
+        assert gap <= TIE * rms, f"{where}: argmax {a_got} != {a_ref} with gap {gap}"
+        print(f"near tie at {where}: gap {gap:.3g}")
+    return rel
+
+
+def f16_order(bits: np.ndarray) -> np.ndarray:
+    """fp16 bit patterns mapped to integers whose differences count ulps."""
+    b = bits.astype(np.int64)
+    return np.where(b & 0x8000, -(b & 0x7FFF), b)
+
+
+def handoff(gpu_cache: S.SynthCache, or_cache: O.Cache):
+    """Copy every ring layer and global layer of the GPU cache into the oracle's."""
+    v = gpu_cache.view
+    for i in range(v.n_sliding):
+        for kv in (0, 1):
+            or_cache.ring(i, kv)[...] = gpu_cache.ring(i, kv).cpu().numpy().view(np.uint16)
+    for i in range(v.n_full):
+        for kv in (0, 1):
+            or_cache.global_(i, kv)[...] = gpu_cache.global_(i, kv).cpu().numpy().view(np.uint16)
+
+
+def check_cache_rows(cfg, gpu_cache, before, or_cache, pos):
+    """Placement: only the rows of `pos` changed on the GPU. Values: against the
+    oracle's rows of `pos` after its own step."""
+    v = gpu_cache.view
+    R = v.ring
+    sl = gl = 0
+    for l in range(cfg["n_layers"]):
+        full = WL.layer_is_full(cfg, l)
+        for kv in (0, 1):
+            if full:
+                after = gpu_cache.global_(gl, kv)
+                prev = before["global"][gl][kv]
+                row, ref = pos, or_cache.global_(gl, kv)
+            else:
+                after = gpu_cache.ring(sl, kv)
+                prev = before["ring"][sl][kv]
+                row, ref = pos % R, or_cache.ring(sl, kv)
+            changed = (after.view(torch.int16) != prev.view(torch.int16)).any(dim=-1)  # [n_kv][rows], bitwise
+            changed[:, row] = False
+            assert not bool(changed.any()), f"layer {l} kv {kv}: rows other than {row} changed"
+            got = after[:, row].cpu().numpy().view(np.uint16)
+            want = np.ascontiguousarray(ref[:, row])
+            if l == 0:
+                ulps = np.abs(f16_order(got) - f16_order(want))
+                assert int(ulps.max()) <= 1, f"layer 0 kv {kv}: {int(ulps.max())} ulps"
+            else:
+                check_vec(O.f16_value(got), O.f16_value(want), f"cache row layer {l} kv {kv}")
+        if full:
+            gl += 1
+        else:
+            sl += 1
+
+
+def snapshot(gpu_cache):
+    v = gpu_cache.view
+    return {"ring": [[gpu_cache.ring(i, kv).clone() for kv in (0, 1)] for i in range(v.n_sliding)],
+            "global": [[gpu_cache.global_(i, kv).clone() for kv in (0, 1)] for i in range(v.n_full)]}
+
+
+def run_pair_steps(cfg, g, gc, om, oc, pos0, tok0, steps, check_rows=True):
+    """`steps` decode steps on both sides from the same cache contents, teacher-forced
+    with the oracle's argmax; per-layer residual dumps and logits compared."""
+    L, H, V = cfg["n_layers"], cfg["hidden"], cfg["vocab"]
+    dump = torch.zeros((1, L + 1, H), dtype=torch.float32, device="cuda")
+    logits = torch.empty(V, dtype=torch.float32, device="cuda")
+    am = torch.empty(1, dtype=torch.int32, device="cuda")
+    Q.q4g_model_set_option(g.handle, Q.Q4G_OPT_DUMP, dump.data_ptr())
+    tok, worst = tok0, 0.0
+    for pos in range(pos0, pos0 + steps):
+        before = snapshot(gc) if check_rows else None
+        Q.q4g_decode_step(g.handle, gc.handle, int(tok), pos, logits.data_ptr(), am.data_ptr(), sp())
+        r = O.decode_step(om, oc, pos, token=int(tok), want_dump=True)
+        torch.cuda.synchronize()
+        worst = max(worst, check_logits(logits.cpu().numpy().astype(np.float64), r["logits"][0], f"pos {pos}"))
+        d = dump[0].cpu().numpy().astype(np.float64)
+        for l in range(L + 1):
+            worst = max(worst, check_vec(d[l], r["dump"][0, l], f"pos {pos} residual after layer {l - 1}"))
+        if check_rows:
+            check_cache_rows(cfg, gc, before, oc, pos)
+        tok = int(r["argmax"][0])
+    Q.q4g_model_set_option(g.handle, Q.Q4G_OPT_DUMP, 0)
+    Q.q4g_model_check(g.handle, sp())
+    print(f"worst max|err|/rms over {steps} steps: {worst:.3g}")
+    return tok
+
+
+def test_tiny_handoff_and_cache_rows():
+    """Tiny decoder: 300 GPU-run positions (the ring of 512 holds 256 live keys), hand-off,
+    then 4 steps compared with per-layer dumps and the written cache rows."""
+    cfg = WL.TINY
+    g = S.SynthDecoder(cfg, seed=7, variant=1)
+    gc = g.new_cache(512)
+    ids = DG.uniform_int(7, DG.STREAM_PREFIX_IDS, 301, cfg["vocab"])
+    for pos in range(300):
+        Q.q4g_decode_step(g.handle, gc.handle, int(ids[pos]), pos, 0, 0, sp())
+    torch.cuda.synchronize()
+    om = O.Model(cfg, seed=7, variant=1)
+    oc = O.Cache(om, 512)
+    handoff(gc, oc)
+    run_pair_steps(cfg, g, gc, om, oc, 300, int(ids[300]), 4)
+
+
+def test_tiny_unit_qk_gains_single_step():
+    """Unit q/k norm gains (recipe variant 2): the attention logits q.k are of order
+    head_dim, so the softmax is sharp. One step from a handed-off cache, every layer
+    compared."""
+    cfg = WL.TINY
+    g = S.SynthDecoder(cfg, seed=8, variant=2)
+    gc = g.new_cache(512)
+    ids = DG.uniform_int(8, DG.STREAM_PREFIX_IDS, 281, cfg["vocab"])
+    for pos in range(280):
+        Q.q4g_decode_step(g.handle, gc.handle, int(ids[pos]), pos, 0, 0, sp())
+    torch.cuda.synchronize()
+    om = O.Model(cfg, seed=8, variant=2)
+    oc = O.Cache(om, 512)
+    handoff(gc, oc)
+    run_pair_steps(cfg, g, gc, om, oc, 280, int(ids[280]), 1)
+
+
+# ------------------------------------------------------- 12B-class, 48 layers ----
+
+@pytest.fixture(scope="module")
+def b12_v0():
+    """The benchmarked decoder: 12B-class shapes, 48 layers, recipe variant 0, seed 0."""
+    cfg = WL.B12
+    g = S.SynthDecoder(cfg, seed=0, variant=0)
+    om = O.Model(cfg, seed=0, variant=0)
+    yield cfg, g, om
+    g.close()
+    om.close()
+
+
+def test_b12_4k_gpu_prefix_handoff(b12_v0):
+    """Config 3 at its full depth: the GPU runs a seeded random-id prefix of 4093 tokens
+    through the 48 layers (context 4096), the cache is handed to the oracle, and the
+    last 3 positions of the context are compared step by step."""
+    cfg, g, om = b12_v0
+    C = 4096
+    gc = g.new_cache(C)
+    prefix = C - 3
+    ids = DG.uniform_int(0, DG.STREAM_PREFIX_IDS, prefix + 1, cfg["vocab"])
+    for pos in range(prefix):
+        Q.q4g_decode_step(g.handle, gc.handle, int(ids[pos]), pos, 0, 0, sp())
+    torch.cuda.synchronize()
+    Q.q4g_model_check(g.handle, sp())
+    oc = O.Cache(om, C)
+    handoff(gc, oc)
+    run_pair_steps(cfg, g, gc, om, oc, prefix, int(ids[prefix]), 3)
+    gc.close()
+
+
+def test_b12_32k_full_depth(b12_v0):
+    """Config 4 at its full depth: both sides hold the same seeded 32K history in every
+    ring slot and global row; the last 2 positions of the context are compared."""
+    cfg, g, om = b12_v0
+    C = 32768
+    gc = g.new_cache(C)
+    S.fill_history(gc, seed=41)
+    oc = O.Cache(om, C)
+    O.fill_history(oc, seed=41)
+    tok = int(DG.uniform_int(41, DG.STREAM_PREFIX_IDS, 1, cfg["vocab"])[0])
+    run_pair_steps(cfg, g, gc, om, oc, C - 2, tok, 2)
+    gc.close()
+
+
+def test_b12_128k_verify_full_depth(b12_v0):
+    """Config 5 at its full depth: two verify blocks of K = 4 rows over the same seeded
+    128K history, the single pass (accepted_count = K) against the oracle's two-pass
+    protocol with a seeded accepted count n in 0..4, the next block at pos0 + n."""
+    cfg, g, om = b12_v0
+    C, K = 131072, 4
+    V = cfg["vocab"]
+    gc = g.new_cache(C)
+    S.fill_history(gc, seed=42)
+    oc = O.Cache(om, C)
+    O.fill_history(oc, seed=42)
+    ids = DG.uniform_int(42, DG.STREAM_DRAFT_IDS, 2 * K, V).reshape(2, K).astype(np.int32)
+    acc = DG.uniform_int(42, DG.STREAM_ACCEPTED, 2, K + 1)
+    ids_d = torch.from_numpy(ids).cuda()
+    logits = torch.empty((K, V), dtype=torch.float32, device="cuda")
+    am = torch.empty(K, dtype=torch.int32, device="cuda")
+    pos = C - 2 * K
+    for b in range(2):
+        n = int(acc[b])
+        Q.q4g_verify_block(g.handle, gc.handle, ids_d[b].data_ptr(), K, pos, K,
+                           logits.data_ptr(), am.data_ptr(), sp())
+        r = O.verify_block(om, oc, pos, ids=ids[b], accepted=0, mode=0)
+        torch.cuda.synchronize()
+        got = logits.cpu().numpy().astype(np.float64)
+        for i in range(K):
+            check_logits(got[i], r["logits"][i], f"128K block {b} row {i}")
+        assert am.cpu().numpy().tolist() == [int(np.argmax(got[i].astype(np.float32))) for i in range(K)]
+        if b == 0:   # commit n rows on the oracle side: the second pass of the protocol
+            O.verify_block(om, oc, pos, ids=ids[b], accepted=n, mode=0, want_logits=False)
+        pos += n
+    Q.q4g_model_check(g.handle, sp())
+    gc.close()
