@@ -10,6 +10,15 @@ K timed greedy decode steps end at position C - 1. A step is one full decode ste
 (embedding, 48 layers, head, softcap, argmax). The weights (6.7 GB) exceed L2, so no
 flush is needed between steps.
 
+Besides the headline context the line carries:
+  * per_context: 32K decode over seeded synthetic history and the 128K verify config
+    (K = 4 draft rows, seeded accepted counts) in blocks/s, each with its HBM fraction;
+  * roofline: the dominant kernel (the persistent step kernel: the whole step after
+    its init launch) timed with CUDA events around its launches;
+  * microbench: the four q4_0 GEMV shapes (seeds 1-4) and flash-decode alone (hd 256
+    ring, hd 512 linear at 4K..128K), each rotated over copies larger than L2;
+  * cpu_baseline: the oracle on the host cores, all threads and one thread.
+
     python bench.py [--gpus N] [--steps K] [--warmup W] [--context C] [--impl reference]
 
 Prints one JSON line. Under torchrun each rank decodes its own sequence on its own
@@ -71,6 +80,10 @@ def parse_args():
     ap.add_argument("--gemv-chain", type=int, choices=[0, 1], default=None,
                     help="run O, gate|up, down and the next QKV of a layer as one persistent launch "
                          "(default: the library's default)")
+    ap.add_argument("--step-kernel", type=int, choices=[0, 1], default=None,
+                    help="decode steps as one persistent launch (default: the library's default, 1)")
+    ap.add_argument("--quick", action="store_true",
+                    help="the headline context only (no other contexts, no microbenchmarks)")
     return ap.parse_args()
 
 
@@ -172,39 +185,67 @@ class ClockSampler:
 
 # ------------------------------------------------------------ reference ----
 
-def oracle_sample(cfg, seed, max_seconds=120.0, min_steps=1, max_steps=4, context=4096, warmup=0):
+def cpu_model_name() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def oracle_sample(cfg, seed, max_seconds=120.0, min_steps=1, max_steps=4, context=4096, warmup=0,
+                  threads=0, model=None):
     """The oracle on a bounded sample of the decode step: a 12B-shaped model with one
     period of the layer pattern (5 sliding + 1 full layer) and the full tied head, one
     decode step at `context` - 1 over seeded synthetic history (after `warmup` untimed
-    steps of the same kind); the per-token time of the 48-layer step is
-    8 x (sample step - head) + head."""
+    steps of the same kind); the per-token time of the 48-layer step is extrapolated as
+    8 x (sample step - head) + head. threads = 0: every host core."""
     import numpy as np
     from oracle import oracle as O
     sample_cfg = dict(cfg, n_layers=cfg["full_every"])
     t0 = time.perf_counter()
-    m = O.Model(sample_cfg, seed=seed)
+    m = model if model is not None else O.Model(sample_cfg, seed=seed)
     build_s = time.perf_counter() - t0
-    c = O.Cache(m, context)
-    O.fill_history(c, seed=99)
-    qs, sc = m.tensor(-1, 100)
-    x16 = np.random.default_rng(0).standard_normal(cfg["hidden"]).astype(np.float16).view(np.uint16)
-    th = time.perf_counter()
-    O.gemv(qs, sc, x16)
-    t_head = time.perf_counter() - th
-    for i in range(warmup):
-        O.decode_step(m, c, context - 1, token=3 + i, want_logits=False)
-    times = []
-    budget_t = time.perf_counter()
-    for i in range(max_steps):
-        ts = time.perf_counter()
-        O.decode_step(m, c, context - 1, token=7 + i, want_logits=False)
-        times.append(time.perf_counter() - ts)
-        if i + 1 >= min_steps and time.perf_counter() - budget_t > max_seconds:
-            break
+    all_threads = O.num_threads()
+    if threads:
+        O.set_threads(threads)
+    try:
+        c = O.Cache(m, context)
+        O.fill_history(c, seed=99)
+        qs, sc = m.tensor(-1, 100)
+        x16 = np.random.default_rng(0).standard_normal(cfg["hidden"]).astype(np.float16).view(np.uint16)
+        th = time.perf_counter()
+        O.gemv(qs, sc, x16)
+        t_head = time.perf_counter() - th
+        for i in range(warmup):
+            O.decode_step(m, c, context - 1, token=3 + i, want_logits=False)
+        times = []
+        budget_t = time.perf_counter()
+        for i in range(max_steps):
+            ts = time.perf_counter()
+            O.decode_step(m, c, context - 1, token=7 + i, want_logits=False)
+            times.append(time.perf_counter() - ts)
+            if i + 1 >= min_steps and time.perf_counter() - budget_t > max_seconds:
+                break
+        cores = O.num_threads()
+    finally:
+        O.set_threads(all_threads)
     t_step = statistics.median(times)
     per_token = (cfg["n_layers"] // cfg["full_every"]) * (t_step - t_head) + t_head
     return dict(tok_s=1.0 / per_token, per_token_s=per_token, steps=len(times), t_head=t_head,
-                t_sample=t_step, cores=O.num_threads(), build_s=build_s, warmup=warmup)
+                t_sample=t_step, cores=cores, build_s=build_s, warmup=warmup, model=m)
+
+
+def sample_text(r, cfg, context):
+    return (f"{r['steps']} oracle decode step(s) (after {r['warmup']} untimed) of a 12B-shaped "
+            f"{cfg['full_every']}-layer sample (5 sliding + 1 full + the 262144-row head) at position "
+            f"{context - 1} over seeded history, {r['t_sample']:.2f} s each on {r['cores']} thread(s); "
+            f"tokens/s extrapolated to the 48-layer step as 8 x (sample - head) + head; "
+            f"CPU: {cpu_model_name()}")
 
 
 def run_reference(args, cfg):
@@ -212,26 +253,186 @@ def run_reference(args, cfg):
     if rank != 0:
         return None
     t0 = time.perf_counter()
-    # warm-up steps of the same sample (at most 3: one oracle step takes ~20 s)
+    # each step is one bounded sample step (about 3-20 s): at most 4 of them, so the run
+    # ends within a few minutes whatever --steps says
     r = oracle_sample(cfg, args.seed, max_seconds=120.0, min_steps=1, max_steps=max(1, min(args.steps, 4)),
                       context=args.context, warmup=min(max(args.warmup, 0), 3))
-    sample = (f"{r['steps']} oracle decode step(s), after {r['warmup']} untimed, of a 12B-shaped "
-              f"{cfg['full_every']}-layer sample "
-              f"(5 sliding + 1 full + 262144-row head) at position {args.context - 1} over seeded "
-              f"history, scaled to 48 layers")
+    sample = sample_text(r, cfg, args.context)
     line = {
         "impl": "reference", "metric": METRIC, "value": r["tok_s"], "unit": "tokens/s",
-        "n_gpus": args.gpus, "steps": r["steps"], "warmup": r["warmup"], "ms_per_step": r["per_token_s"] * 1e3,
+        "n_gpus": args.gpus, "steps": r["steps"], "warmup": r["warmup"],
+        "ms_per_step": r["t_sample"] * 1e3, "ms_per_token_extrapolated": r["per_token_s"] * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
         "config": {"workload": f"12B-class q4_0 decoder, context {args.context}, batch 1",
                    "context": args.context},
         "cpu_baseline": {"value": r["tok_s"], "unit": "tokens/s", "cores": r["cores"], "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "extrapolated": True, "cpu": cpu_model_name()},
         "e2e": {"value": r["tok_s"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "wall_s": time.perf_counter() - t0,
     }
     return line
+
+
+# ------------------------------------------------------------ GPU parts ----
+
+def decode_loop(Q, model, cache, am, p0, n, sp):
+    """n greedy steps from p0: each step's token is the previous step's argmax on the device."""
+    for p in range(p0, p0 + n):
+        Q.q4g_decode_step_device_token(model.handle, cache.handle, am[p - 1:].data_ptr(), p, 0,
+                                       am[p:].data_ptr(), sp)
+
+
+def measure_context(Q, S, model, cfg, C, K, W, sp, stream):
+    """K timed decode steps ending at position C - 1 over seeded synthetic history."""
+    import torch
+    cache = model.new_cache(C)
+    S.fill_history(cache, seed=99)
+    am = torch.zeros(C + 1, dtype=torch.int32, device="cuda")
+    p0 = C - (W + K)
+    am[p0 - 1] = 11
+    decode_loop(Q, model, cache, am, p0, W, sp)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    decode_loop(Q, model, cache, am, p0 + W, K, sp)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / K
+    bpt = weight_bytes(cfg) + statistics.mean(kv_bytes(cfg, q) for q in range(p0 + W, C))
+    Q.q4g_model_check(model.handle, sp)
+    cache.close()
+    del cache
+    return ms, bpt
+
+
+def measure_verify(Q, S, DG, model, cfg, C, Kv, blocks, warm, seed, sp, stream):
+    """Verify blocks of Kv draft rows (seeded ids, seeded accepted counts n ~ U{0..Kv},
+    the next block at pos0 + n) over seeded synthetic history at context C."""
+    import numpy as np
+    import torch
+    V = cfg["vocab"]
+    nb = blocks + warm
+    ids = torch.from_numpy(DG.uniform_int(seed, DG.STREAM_DRAFT_IDS, nb * Kv, V).astype(np.int32)).cuda()
+    acc = DG.uniform_int(seed, DG.STREAM_ACCEPTED, nb, Kv + 1)
+    cache = model.new_cache(C)
+    S.fill_history(cache, seed=98)
+    am = torch.zeros(nb * Kv, dtype=torch.int32, device="cuda")
+    pos = C - Kv * nb
+    starts = []
+    for b in range(nb):
+        starts.append(pos)
+        pos += int(acc[b])
+    for b in range(warm):
+        Q.q4g_verify_block(model.handle, cache.handle, ids[b * Kv:].data_ptr(), Kv, starts[b], Kv, 0,
+                           am[b * Kv:].data_ptr(), sp)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for b in range(warm, nb):
+        Q.q4g_verify_block(model.handle, cache.handle, ids[b * Kv:].data_ptr(), Kv, starts[b], Kv, 0,
+                           am[b * Kv:].data_ptr(), sp)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    Q.q4g_model_check(model.handle, sp)
+    ms = e0.elapsed_time(e1) / blocks
+    bpb = weight_bytes(cfg) + statistics.mean(kv_bytes(cfg, starts[b] + Kv - 1) for b in range(warm, nb))
+    accepted = int(sum(int(acc[b]) for b in range(warm, nb)))
+    cache.close()
+    del cache
+    return ms, bpb, accepted
+
+
+def time_rotating(fn, n_items, reps, stream):
+    """Mean time of fn(i) over reps passes of i = 0..n_items-1 (CUDA events)."""
+    import torch
+    for i in range(min(n_items, 3)):
+        fn(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        for i in range(n_items):
+            fn(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / (reps * n_items)
+
+
+def microbench(Q, S, DG, WL, peak, sp, stream):
+    """The kernel microbenchmarks of the decode step's pieces, through the standalone
+    C-ABI entry points, each rotated over copies larger than L2 (126 MB)."""
+    import math
+    import torch
+    l2 = 126e6
+    out = {"gemv": [], "flash_decode": []}
+    for name, n, k, seed0 in WL.GEMV_SHAPES:
+        wbytes = n * k * 0.5625
+        per_seed = max(1, math.ceil(4 * l2 / wbytes / 4))
+        mats = []
+        for sd in (1, 2, 3, 4):
+            qs, sc = S.packed_tensor(n, k, sd, DG.stream_bench_w(sd))
+            mats.append((qs, sc))
+            for _ in range(per_seed - 1):
+                mats.append((qs.clone(), sc.clone()))
+        x = torch.empty(k, dtype=torch.float16, device="cuda")
+        S.fill_normal_f16(x, seed0, DG.stream_bench_x(seed0), 1.0)
+        y = torch.empty(n, dtype=torch.float32, device="cuda")
+        ms = time_rotating(lambda i: Q.q4g_gemv(mats[i][0].data_ptr(), mats[i][1].data_ptr(), n, k, x.data_ptr(), 1,
+                                                y.data_ptr(), sp), len(mats), 4, stream)
+        b = wbytes + k * 2 + n * 4
+        out["gemv"].append({"shape": name, "rows": n, "cols": k, "seeds": [1, 2, 3, 4], "copies": len(mats),
+                            "us": ms * 1e3, "gbs": b / (ms / 1e3) / 1e9, "frac": b / (ms / 1e3) / 1e9 / peak})
+        del mats
+        torch.cuda.empty_cache()
+    # flash-decode alone: 16 query heads over an hd 256 ring (8 KV heads, W 1024, R 2048, full window)
+    nq, hd, nkv, W, R = 16, 256, 8, 1024, 2048
+    kvb = nkv * R * hd * 2
+    copies = max(2, math.ceil(4 * l2 / (2 * kvb)))
+    ks = [torch.empty(nkv * R * hd, dtype=torch.float16, device="cuda") for _ in range(copies)]
+    vs = [torch.empty_like(ks[0]) for _ in range(copies)]
+    for i in range(copies):
+        S.fill_normal_f16(ks[i], 1, DG.stream_attn(10 + 2 * i), 0.25)
+        S.fill_normal_f16(vs[i], 1, DG.stream_attn(11 + 2 * i), 1.0)
+    q = torch.empty(nq * hd, dtype=torch.float16, device="cuda")
+    S.fill_normal_f16(q, 1, DG.stream_attn(1), 1.0)
+    o = torch.empty(nq * hd, dtype=torch.float16, device="cuda")
+    wsb = Q.q4g_flash_decode_workspace_bytes(nq, hd)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    ms = time_rotating(lambda i: Q.q4g_flash_decode_ring(q.data_ptr(), nq, nkv, hd, ks[i].data_ptr(), vs[i].data_ptr(),
+                                                         R, W, 5000, o.data_ptr(), ws.data_ptr(), wsb, sp),
+                       copies, 4, stream)
+    b = nkv * W * hd * 2 * 2
+    out["flash_decode"].append({"kind": "ring hd256", "n_q": nq, "n_kv": nkv, "window": W, "ring": R,
+                                "copies": copies, "us": ms * 1e3, "gbs": b / (ms / 1e3) / 1e9,
+                                "frac": b / (ms / 1e3) / 1e9 / peak})
+    del ks, vs
+    torch.cuda.empty_cache()
+    # hd 512, one KV head, linear cache of length L
+    hd = 512
+    wsb = Q.q4g_flash_decode_workspace_bytes(nq, hd)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    q = torch.empty(nq * hd, dtype=torch.float16, device="cuda")
+    S.fill_normal_f16(q, 2, DG.stream_attn(2), 1.0)
+    o = torch.empty(nq * hd, dtype=torch.float16, device="cuda")
+    for L in WL.ATTN_GLOBAL_LENGTHS:
+        per = L * hd * 2
+        copies = max(2, math.ceil(4 * l2 / (2 * per)))
+        ks = [torch.empty(L * hd, dtype=torch.float16, device="cuda") for _ in range(copies)]
+        vs = [torch.empty_like(ks[0]) for _ in range(copies)]
+        for i in range(copies):
+            S.fill_normal_f16(ks[i], 2, DG.stream_attn(100 + 2 * i), 0.21)
+            S.fill_normal_f16(vs[i], 2, DG.stream_attn(101 + 2 * i), 1.0)
+        ms = time_rotating(lambda i: Q.q4g_flash_decode_linear(q.data_ptr(), nq, 1, hd, ks[i].data_ptr(),
+                                                               vs[i].data_ptr(), L, o.data_ptr(), ws.data_ptr(),
+                                                               wsb, sp), copies, 4, stream)
+        b = 2 * per
+        out["flash_decode"].append({"kind": "linear hd512", "n_q": nq, "n_kv": 1, "length": L, "copies": copies,
+                                    "us": ms * 1e3, "gbs": b / (ms / 1e3) / 1e9,
+                                    "frac": b / (ms / 1e3) / 1e9 / peak})
+        del ks, vs
+        torch.cuda.empty_cache()
+    return out
 
 
 # ----------------------------------------------------------------- main ----
@@ -276,6 +477,8 @@ def main():
     model = S.SynthDecoder(cfg, seed=args.seed)
     if args.gemv_chain is not None:
         Q.q4g_model_set_option(model.handle, Q.Q4G_OPT_GEMV_CHAIN, args.gemv_chain)
+    if args.step_kernel is not None:
+        Q.q4g_model_set_option(model.handle, Q.Q4G_OPT_STEP_KERNEL, args.step_kernel)
     cache = model.new_cache(C)
     stream = torch.cuda.current_stream()
     sp = stream.cuda_stream
@@ -292,12 +495,7 @@ def main():
     torch.cuda.synchronize()
     setup_s = time.perf_counter() - t_setup
 
-    def steps(p0, n):
-        for p in range(p0, p0 + n):
-            Q.q4g_decode_step_device_token(model.handle, cache.handle, am[p - 1:].data_ptr(), p, 0,
-                                           am[p:].data_ptr(), sp)
-
-    steps(prefix, W)
+    decode_loop(Q, model, cache, am, prefix, W, sp)
     torch.cuda.synchronize()
     props = torch.cuda.get_device_properties(local)
     gpu_id = str(getattr(props, "uuid", local))
@@ -311,10 +509,11 @@ def main():
     time.sleep(0.3)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
-    steps(prefix + W, K)
+    decode_loop(Q, model, cache, am, prefix + W, K, sp)
     ev1.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
+    Q.q4g_model_check(model.handle, sp)
     ms = max_over_ranks(ev0.elapsed_time(ev1), world, "cuda")
     if world > 1:
         dist.barrier()
@@ -325,10 +524,10 @@ def main():
     peak, peak_kind = measured_peaks()
     gbs = bytes_per_tok / (ms_per_step / 1e3) / 1e9
 
-    # ---- per-kernel breakdown (profile mode: eager launches bracketed by events) ----
+    # ---- per-kernel breakdown (profile mode: the launches of a step bracketed by events) ----
     Q.q4g_model_set_option(model.handle, Q.Q4G_OPT_PROFILE, 1)
     P = args.profile_steps
-    steps(C - P, P)
+    decode_loop(Q, model, cache, am, C - P, P, sp)
     recs = Q.q4g_model_profile_read(model.handle, sp)
     Q.q4g_model_set_option(model.handle, Q.Q4G_OPT_PROFILE, 0)
     kinds = {}
@@ -337,22 +536,31 @@ def main():
         k["launches"] += 1
         k["ms"] += kms
         k["bytes"] += kbytes
-    gemv = [v for n, v in kinds.items() if n.endswith("_gemv")]
-    g_ms = sum(v["ms"] for v in gemv)
-    g_bytes = sum(v["bytes"] for v in gemv)
-    g_launch = sum(v["launches"] for v in gemv)
     prof_step_ms = sum(v["ms"] for v in kinds.values()) / max(P, 1)
     launches_step = sum(v["launches"] for v in kinds.values()) / max(P, 1)
     breakdown = {n: {"launches_per_step": v["launches"] / P, "ms_per_step": v["ms"] / P,
                      "gbs": v["bytes"] / (v["ms"] / 1e3) / 1e9 if v["ms"] else None}
                  for n, v in sorted(kinds.items())}
-    achieved = g_bytes / (g_ms / 1e3) / 1e9 if g_ms else None
+    kv_prof = statistics.mean(kv_bytes(cfg, q) for q in range(C - P, C))
+    if "step_kernel" in kinds:
+        # the whole step after its init launch is one persistent kernel: its algorithmic
+        # bytes are the weights plus the live K/V rows of the step
+        sk = kinds["step_kernel"]
+        k_ms = sk["ms"] / sk["launches"]
+        k_bytes = weight_bytes(cfg) + kv_prof
+        kernel_name = "persistent decode-step kernel (all 48 layers and the head in one launch)"
+    else:
+        gemv = [v for n, v in kinds.items() if n.endswith("_gemv")]
+        k_ms = sum(v["ms"] for v in gemv) / max(P, 1)
+        k_bytes = sum(v["bytes"] for v in gemv) / max(P, 1)
+        kernel_name = "q4_0 GEMV (every GEMV launch of a step)"
+    achieved = k_bytes / (k_ms / 1e3) / 1e9 if k_ms else None
     traffic = None
-    tp = os.path.join(ROOT, "profiles", "gemv_q4_traffic.json")
-    if os.path.exists(tp):
+    tp = os.path.join(ROOT, "profiles", "step_kernel_traffic.json")
+    if os.path.exists(tp) and "step_kernel" in kinds:
         with open(tp) as f:
             tr = json.load(f)
-        src = open(os.path.join(ROOT, "int4_q4_gemv_b200", "csrc", "q4g_gemv.cu"), "rb").read()
+        src = open(os.path.join(ROOT, "int4_q4_gemv_b200", "csrc", "q4g_step.cu"), "rb").read()
         if tr.get("source_sha256") == hashlib.sha256(src).hexdigest():
             traffic = tr.get("bytes_per_launch")
 
@@ -368,14 +576,43 @@ def main():
         tok = int(am_host[0])
     e2e_s = max_over_ranks(time.perf_counter() - t0, world, "cuda")
     e2e_tok_s = replica_rate(E, world, e2e_s)
+    cache.close()
+    del cache
+    torch.cuda.empty_cache()
+
+    # ---- the other contexts and the microbenchmarks (rank 0 of a single-GPU run) ----
+    per_context = {str(C): {"kind": "decode", "tokens_per_s": tok_s / world, "ms_per_step": ms_per_step,
+                            "bytes_per_token": bytes_per_tok, "gbs": gbs, "frac": gbs / peak,
+                            "history": args.prefix}}
+    micro = None
+    if world == 1 and not args.quick:
+        for C2 in (32768,):
+            if C2 == C:
+                continue
+            K2 = min(K, 50)
+            ms2, bpt2 = measure_context(Q, S, model, cfg, C2, K2, max(W, 3), sp, stream)
+            per_context[str(C2)] = {"kind": "decode", "tokens_per_s": 1e3 / ms2, "ms_per_step": ms2,
+                                    "bytes_per_token": bpt2, "gbs": bpt2 / (ms2 / 1e3) / 1e9,
+                                    "frac": bpt2 / (ms2 / 1e3) / 1e9 / peak, "steps": K2,
+                                    "history": "synthetic"}
+        Kv, nb = 4, 16
+        msv, bpb, accepted = measure_verify(Q, S, DG, model, cfg, 131072, Kv, nb, 2, args.seed, sp, stream)
+        per_context["131072_verify_k4"] = {
+            "kind": "verify", "k": Kv, "blocks": nb, "blocks_per_s": 1e3 / msv, "ms_per_block": msv,
+            "accepted_tokens_per_s": accepted / (nb * msv / 1e3), "rows_per_s": Kv * 1e3 / msv,
+            "bytes_per_block": bpb, "gbs": bpb / (msv / 1e3) / 1e9, "frac": bpb / (msv / 1e3) / 1e9 / peak,
+            "accepted_count": "seeded U{0..4}", "history": "synthetic"}
+        micro = microbench(Q, S, DG, WL, peak, sp, stream)
 
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         r = oracle_sample(cfg, args.seed, max_seconds=20.0, min_steps=1, max_steps=2, context=C)
         cpu = {"value": r["tok_s"], "unit": "tokens/s", "cores": r["cores"], "kind": "oracle",
-               "sample": f"{r['steps']} oracle decode step(s) of a 12B-shaped 6-layer sample "
-                         f"(5 sliding + 1 full + the 262144-row head) at position {C - 1} over seeded "
-                         f"history, scaled to 48 layers"}
+               "sample": sample_text(r, cfg, C), "extrapolated": True, "cpu": cpu_model_name()}
+        r1 = oracle_sample(cfg, args.seed, max_seconds=1.0, min_steps=1, max_steps=1, context=C, threads=1,
+                           model=r["model"])
+        cpu["single_thread"] = {"value": r1["tok_s"], "unit": "tokens/s", "cores": 1,
+                                "sample": sample_text(r1, cfg, C)}
 
     if rank == 0:
         line = {
@@ -389,12 +626,15 @@ def main():
                        "l2": "inputs larger than L2 (6.7 GB of weights read per step)"},
             "hbm": {"bytes_per_token": bytes_per_tok, "gbs_per_gpu": gbs, "peak_gbs": peak,
                     "frac": gbs / peak, "peak_kind": peak_kind},
-            "roofline": {"bound": "hbm", "kernel": "q4_0 GEMV (every GEMV launch of a step, chains included)",
+            "per_context": per_context,
+            "roofline": {"bound": "hbm", "kernel": kernel_name,
                          "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": (achieved / peak) if achieved else None, "traffic": traffic,
-                         "launches_per_step": g_launch / max(P, 1),
+                         "bytes_per_launch": k_bytes, "ms_per_launch": k_ms,
+                         "timing": "CUDA events around the kernel's launches (profile pass, eager launches)",
                          "peak_kind": f"{peak_kind} (burst copy)"},
             "kernels": breakdown, "profiled_step_ms": prof_step_ms,
+            "microbench": micro,
             "e2e": {"value": e2e_tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 4,
                     "d2h_bytes_per_step": 4, "api": "q4g_decode_step_host"},
             "cpu_baseline": cpu, "gpu_launches": int(round(launches_step * K)),

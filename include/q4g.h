@@ -266,7 +266,7 @@ typedef enum {
                                  starts when every CTA finished the previous one, a
                                  bounded wait reported as Q4G_ETIMEOUT); 0: one launch
                                  per GEMV */
-  Q4G_OPT_TRACE = 8         /* [0] value = device uint64_t* [n_layers][32]: the GEMV
+  Q4G_OPT_TRACE = 8,        /* [0] value = device uint64_t* [n_layers][32]: the GEMV
                                  chain of layer l writes %globaltimer stamps (ns) of
                                  its CTA 0 to row l: 0 start, 1 dependency wait done,
                                  per phase i at 2 + 4i: inputs ready, x digits built,
@@ -286,16 +286,40 @@ typedef enum {
                                  stage reduced (stage kernel), 8 + t
                                  stage t issued, 72 + t stage t ready, 136 + t
                                  stage t reduced (t < 64).
+                                 With the step kernel (Q4G_OPT_STEP_KERNEL) the
+                                 buffer holds 4 * (6 * n_layers + 1) + 2 entries
+                                 instead: per phase p (6 per layer: QKV, attention,
+                                 attention merge, O, gate|up, down; then the head)
+                                 at 4p, CTA 0's 0 phase start (every CTA finished
+                                 phase p - 1), 1 inputs ready (norm / queries /
+                                 x digits), 2 compute done, 3 outputs published
+                                 (GEMV phases); then the kernel's entry and exit.
                                  Unwritten slots keep their contents. */
+  Q4G_OPT_STEP_KERNEL = 9,  /* [0] decode steps (one row) run as one persistent,
+                                 cooperative launch of one CTA per SM: every
+                                 layer's QKV, attention, attention merge, O,
+                                 gate|up and down, then the head, as phases that
+                                 start once every CTA finished the previous one
+                                 (a bounded wait, reported as Q4G_ETIMEOUT), while
+                                 each CTA's producer warp streams the weights and
+                                 K/V rows of the coming phases through one ring of
+                                 shared-memory stages. Used when the shapes fit
+                                 (hidden <= 4096, head dims 256 / 512); 0: one
+                                 launch per GEMV / attention kernel. Verify blocks
+                                 (K > 1 rows) always use the per-kernel path. */
+  Q4G_OPT_STEP_POLL_NS = 10 /* [64] step kernel: nanoseconds each CTA sleeps between two
+                                 polls of a phase counter (0..100000) */
 } q4g_option;
 q4g_status q4g_model_set_option(q4g_model* m, q4g_option opt, intptr_t value);
 
 /* One kernel launch recorded in profile mode. kind: 0 step init, 1 QKV GEMV,
  * 2 sliding attention, 3 full attention, 4 attention combine, 5 O GEMV,
  * 6 gate|up GEMV, 7 down GEMV, 8 head GEMV, 9 GEMV chain (O, gate|up, down and
- * the next layer's QKV in one launch). bytes: algorithmic HBM bytes of the
- * launch (q4_0 weights 0.5625 B/weight + activations; attention: the live K/V
- * rows, 2 * head_dim * 2 B per key and KV head). */
+ * the next layer's QKV in one launch), 10 the persistent step kernel (the whole
+ * step after step init). bytes: algorithmic HBM bytes of the launch (q4_0
+ * weights 0.5625 B/weight + activations; attention: the live K/V rows,
+ * 2 * head_dim * 2 B per key and KV head; the step kernel: its GEMVs' bytes,
+ * the K/V rows are not included). */
 typedef struct {
   int32_t kind;
   int32_t layer;

@@ -109,8 +109,20 @@ struct q4g_model {
   double* inv_freq_gl;
   float* part_ml;
   float* part_acc;
+  // persistent step kernel: per-layer descriptors (device) and its partials / counters
+  StepLayer* step_layers = nullptr;
+  float* sk_part_ml = nullptr;
+  float* sk_part_acc = nullptr;
+  int32_t* sk_done = nullptr;
+  // its activations as tagged words (value | tag << 32) and the step number in the tags
+  uint64_t *sk_r[2] = {nullptr, nullptr}, *sk_qkv = nullptr, *sk_attn = nullptr, *sk_o = nullptr;
+  uint64_t *sk_act = nullptr, *sk_d = nullptr;
+  uint32_t* sk_epoch = nullptr;
+  uint32_t epoch = 0;
+  bool step_ok = false;  // the shapes fit the step kernel
+  uint32_t poll_ns = 64;  // step kernel: back-off between polls of a phase counter
   // options
-  bool use_graph = true, use_pdl = true, attn_cluster = true, gemv_chain = false;
+  bool use_graph = true, use_pdl = true, attn_cluster = true, gemv_chain = false, use_step = false;
   uint64_t* trace = nullptr;  // Q4G_OPT_TRACE
   float* dump = nullptr;
   // profile mode: events around every launch
@@ -255,8 +267,19 @@ extern "C" q4g_status q4g_model_create(const q4g_config* cfg, const q4g_weights*
     part = b > part ? b : part;
   }
   const size_t part_ml = part / 128 + 1024;  // (m, l) per row and chunk: hd >= 256
-  // head, attention, chain phases, then the two-cluster ring attention merge
-  m->n_counters = 64 + kChainMaxPhases * c.n_layers + kRingSplitCounters;
+  // head, attention, chain phases, the two-cluster ring attention merge, then the
+  // phase counters of the persistent step kernel
+  const int sk_counters = step_kernel_counters(c.n_layers, c.sl_kv_heads);
+  m->n_counters = 64 + kChainMaxPhases * c.n_layers + kRingSplitCounters + sk_counters;
+  StepKernelParams skp{};
+  skp.n_q = c.n_q_heads, skp.sl_nkv = c.sl_kv_heads, skp.gl_nkv = c.gl_kv_heads;
+  skp.sl_hd = c.sl_head_dim, skp.gl_hd = c.gl_head_dim, skp.hidden = c.hidden, skp.ffn = c.ffn;
+  skp.n_layers = c.n_layers, skp.rope_pairs_sl = c.sl_head_dim / 2, skp.rope_pairs_gl = c.rope_pairs_full;
+  {
+    char why[128];
+    m->step_ok = step_kernel_supported(skp, why, sizeof why);
+  }
+  const size_t sk_acc = step_kernel_partial_floats(skp, m->sm_count), sk_ml = step_kernel_ml_floats(skp, m->sm_count);
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -281,6 +304,12 @@ extern "C" q4g_status q4g_model_create(const q4g_config* cfg, const q4g_weights*
   const size_t o_ifg = take(sizeof(double) * (m->gl.rope_pairs > 0 ? m->gl.rope_pairs : 1));
   const size_t o_pml = take(sizeof(float) * 2 * part_ml);
   const size_t o_pacc = take(sizeof(float) * part);
+  const size_t o_skml = take(sizeof(float) * sk_ml);
+  const size_t o_skacc = take(sizeof(float) * sk_acc);
+  const size_t o_layers = take(sizeof(StepLayer) * c.n_layers);
+  const size_t o_tr0 = take(8 * (size_t)H), o_tr1 = take(8 * (size_t)H), o_tqkv = take(8 * (size_t)qkv_max);
+  const size_t o_tattn = take(8 * (size_t)attn_max / 2), o_to = take(8 * (size_t)H);
+  const size_t o_tact = take(8 * (size_t)c.ffn / 2), o_td = take(8 * (size_t)H), o_epoch = take(sizeof(uint32_t));
   m->scratch_bytes = off;
   cudaError_t e = cudaMalloc(&m->scratch, off);
   if (e != cudaSuccess) {
@@ -307,7 +336,45 @@ extern "C" q4g_status q4g_model_create(const q4g_config* cfg, const q4g_weights*
   m->inv_freq_gl = (double*)(b + o_ifg);
   m->part_ml = (float*)(b + o_pml);
   m->part_acc = (float*)(b + o_pacc);
+  m->sk_part_ml = (float*)(b + o_skml);
+  m->sk_part_acc = (float*)(b + o_skacc);
+  m->sk_done = m->counters + (m->n_counters - sk_counters);
+  m->step_layers = (StepLayer*)(b + o_layers);
+  m->sk_r[0] = (uint64_t*)(b + o_tr0), m->sk_r[1] = (uint64_t*)(b + o_tr1), m->sk_qkv = (uint64_t*)(b + o_tqkv);
+  m->sk_attn = (uint64_t*)(b + o_tattn), m->sk_o = (uint64_t*)(b + o_to), m->sk_act = (uint64_t*)(b + o_tact);
+  m->sk_d = (uint64_t*)(b + o_td), m->sk_epoch = (uint32_t*)(b + o_epoch);
+  // the step kernel streams every tensor with bulk copies and reads the gains as
+  // float4: 16-byte aligned operands only (else the per-kernel path serves)
+  auto a16 = [](const void* ptr) { return aligned(ptr, 16); };
+  for (int l = 0; l < c.n_layers && m->step_ok; ++l) {
+    const q4g_layer_weights& W = m->layers[l];
+    const q4g_qtensor* ts[7] = {&W.wq, &W.wk, &W.wv, &W.wo, &W.wgate, &W.wup, &W.wdown};
+    for (int t = 0; t < 7; ++t)
+      if (!(t == 2 && m->full[l]) && (!a16(ts[t]->qs) || !a16(ts[t]->scales))) m->step_ok = false;
+    if (!a16(W.norm_in) || !a16(W.norm_post_attn) || !a16(W.norm_pre_ffn) || !a16(W.norm_post_ffn))
+      m->step_ok = false;
+  }
+  if (!a16(m->embed.qs) || !a16(m->embed.scales) || !a16(m->norm_final)) m->step_ok = false;
   e = cudaMemset(m->scratch, 0, off);
+  {  // per-layer descriptors of the persistent step kernel
+    std::vector<StepLayer> sl(c.n_layers);
+    for (int l = 0; l < c.n_layers; ++l) {
+      const q4g_layer_weights& W = m->layers[l];
+      const q4g_qtensor* ts[7] = {&W.wq, &W.wk, &W.wv, &W.wo, &W.wgate, &W.wup, &W.wdown};
+      for (int t = 0; t < 7; ++t) {
+        const bool absent = t == 2 && m->full[l];
+        sl[l].q[t] = absent ? nullptr : ts[t]->qs;
+        sl[l].s[t] = absent ? nullptr : ts[t]->scales;
+      }
+      sl[l].norm_in = W.norm_in, sl[l].norm_post_attn = W.norm_post_attn, sl[l].norm_pre_ffn = W.norm_pre_ffn;
+      sl[l].norm_post_ffn = W.norm_post_ffn, sl[l].norm_q = W.norm_q, sl[l].norm_k = W.norm_k;
+      sl[l].layer_scalar = W.layer_scalar;
+      sl[l].full = m->full[l];
+      sl[l].ordinal = m->ordinal[l];
+    }
+    if (e == cudaSuccess)
+      e = cudaMemcpy(m->step_layers, sl.data(), sizeof(StepLayer) * sl.size(), cudaMemcpyHostToDevice);
+  }
   // RoPE inverse frequencies theta^(-2i/hd), in fp64 ("Gemma 4 12B" architecture:
   // dual RoPE; the full layers' frequencies are those of head dim 512, first pairs only)
   std::vector<double> fs(m->sl.rope_pairs), fg(m->gl.rope_pairs > 0 ? m->gl.rope_pairs : 1, 0.0);
@@ -363,6 +430,8 @@ extern "C" q4g_status q4g_model_set_option(q4g_model* m, q4g_option opt, intptr_
     case Q4G_OPT_ATTN_CLUSTER: m->attn_cluster = value != 0; break;
     case Q4G_OPT_GEMV_CHAIN: m->gemv_chain = value != 0; break;
     case Q4G_OPT_TRACE: m->trace = (uint64_t*)value; break;
+    case Q4G_OPT_STEP_KERNEL: m->use_step = value != 0; break;
+    case Q4G_OPT_STEP_POLL_NS: m->poll_ns = (uint32_t)std::max<intptr_t>(0, std::min<intptr_t>(value, 100000)); break;
     default: return fail(Q4G_EINVAL, "unknown option %d", (int)opt);
   }
   free_graphs(m);
@@ -531,8 +600,9 @@ extern "C" q4g_status q4g_gemv(const uint8_t* qs, const uint16_t* scales, int64_
 
 extern "C" size_t q4g_flash_decode_workspace_bytes(int32_t n_q_heads, int32_t head_dim) {
   if (n_q_heads < 1 || head_dim < 1) return 256;
+  // the largest plan: at most 2 chunks per SM
   const int chunks = 2 * device_sm_count();
-  return 256 + ((sizeof(float) * 2 * (size_t)n_q_heads * chunks + 255) & ~255ul) +
+  return kFlashCounterBytes + ((sizeof(float) * 2 * (size_t)n_q_heads * chunks + 255) & ~255ul) +
          sizeof(float) * (size_t)n_q_heads * chunks * head_dim;
 }
 
@@ -558,20 +628,9 @@ q4g_status flash_standalone(const uint16_t* q, int32_t n_q, int32_t n_kv, int32_
   p.n_q = n_q;
   p.n_kv = n_kv;
   p.hd = hd;
-  const int G = n_q / n_kv;
-  p.m_groups = m_groups_for(1, G);
-  const int slots = (hd == 256 ? 2 : 1) * device_sm_count();
-  int nch = slots / (n_kv * p.m_groups);
-  if (ring) {
-    const int want = (int)((window + 63) / 64);
-    nch = want < nch ? want : nch;
-  }
-  if (nch > 2 * device_sm_count()) nch = 2 * device_sm_count();
-  p.n_chunks = nch < 1 ? 1 : nch;
-  char* w = (char*)ws;
-  p.counters = (int32_t*)w;
-  p.part_ml = (float*)(w + 256);
-  p.part_acc = (float*)(w + 256 + ((sizeof(float) * 2 * (size_t)n_q * 2 * device_sm_count() + 255) & ~255ul));
+  const FlashPlan plan = flash_plan(n_q, n_kv, hd, ring, window);
+  if (plan.bytes > ws_bytes) return fail(Q4G_EINVAL, "workspace too small");
+  flash_bind(p, plan, ws);
   p.combine_in_kernel = ring ? 1 : 0;
   p.out = reinterpret_cast<__half*>(out);
   if (ring) {
@@ -960,6 +1019,49 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
   return cudaSuccess;
 }
 
+// One decode step (one row) as the persistent step kernel.
+cudaError_t enqueue_step_kernel(q4g_model* m, const q4g_cache* c, float* logits, int32_t* argmax, cudaStream_t st) {
+  const q4g_config& cf = m->cfg;
+  StepKernelParams p{};
+  p.layers = m->step_layers;
+  p.n_layers = cf.n_layers, p.hidden = cf.hidden, p.n_q = cf.n_q_heads, p.ffn = cf.ffn, p.vocab = cf.vocab;
+  p.sl_nkv = cf.sl_kv_heads, p.sl_hd = cf.sl_head_dim, p.gl_nkv = cf.gl_kv_heads, p.gl_hd = cf.gl_head_dim;
+  p.window = cf.window, p.ring = cf.ring, p.capacity = c->capacity;
+  p.rope_pairs_sl = m->sl.rope_pairs, p.rope_pairs_gl = m->gl.rope_pairs, p.v_norm_sliding = cf.v_norm_sliding;
+  p.eps = cf.rms_eps, p.softcap = cf.softcap;
+  p.cache = c->buf;
+  p.ring_k_off = c->view.ring_k_offset, p.ring_v_off = c->view.ring_v_offset, p.ring_layer_bytes = c->view.ring_layer_bytes;
+  p.glob_k_off = c->view.global_k_offset, p.glob_v_off = c->view.global_v_offset;
+  p.glob_layer_bytes = c->view.global_layer_bytes;
+  p.emb_q = m->embed.qs, p.emb_s = m->embed.scales, p.norm_final = m->norm_final;
+  p.r0 = m->sk_r[0], p.r1 = m->sk_r[1], p.qkv = m->sk_qkv, p.attn = m->sk_attn, p.o = m->sk_o;
+  p.act = m->sk_act, p.d = m->sk_d, p.epoch = m->sk_epoch;
+  p.part_ml = m->sk_part_ml, p.part_acc = m->sk_part_acc;
+  p.rope_sl = m->rope_sl, p.rope_gl = m->rope_gl, p.pos_dev = m->pos_dev;
+  p.logits = logits, p.argmax_out = argmax ? argmax : m->argmax_buf;
+  p.am_val = m->am_val, p.am_idx = m->am_idx;
+  p.done = m->sk_done;
+  p.tickets = m->sk_done + step_kernel_phases(cf.n_layers) + 1;
+  p.dump = m->dump;
+  p.trace = m->trace;
+  p.poll_ns = m->poll_ns;
+  if (m->stall_next) {
+    p.stall_test = 1;
+    p.wait_ns = 20000000ull;  // 20 ms
+  }
+  Prof pr(m, st);
+  double bytes = 0;
+  for (int l = 0; l < cf.n_layers; ++l) {
+    const LayerShape& S = m->full[l] ? m->gl : m->sl;
+    bytes += gemv_bytes(S.qkv_cols, cf.hidden, 1, 4) + gemv_bytes(cf.hidden, (int64_t)cf.n_q_heads * S.hd, 1, 4) +
+             gemv_bytes(2 * (int64_t)cf.ffn, cf.hidden, 1, 1) + gemv_bytes(cf.hidden, cf.ffn, 1, 4);
+  }
+  bytes += gemv_bytes(cf.vocab, cf.hidden, 1, logits ? 4 : 0);
+  return pr.done(debug_sync(launch_step_kernel(p, st), "step_kernel", -1, st), 10, -1, bytes);
+}
+
+bool use_step_kernel(const q4g_model* m, int kr) { return kr == 1 && m->use_step && m->step_ok; }
+
 q4g_status run_step(q4g_model* m, q4g_cache* c, int kr, int64_t pos0, const int32_t* ids_dev,
                     const int32_t* ids_host, const float* hidden, float* logits, int32_t* argmax,
                     cudaStream_t st) {
@@ -991,12 +1093,20 @@ q4g_status run_step(q4g_model* m, q4g_cache* c, int kr, int64_t pos0, const int3
   sp.pos_dev = m->pos_dev;
   sp.counters = m->counters;
   sp.n_counters = m->n_counters;
+  if (use_step_kernel(m, kr)) {  // the layer-0 input as tagged words, and this step's number
+    sp.r_tagged = m->sk_r[0];
+    sp.epoch_dev = m->sk_epoch;
+    sp.epoch = ++m->epoch;  // never 0: the zeroed buffers carry tag 0
+    if (m->epoch >= (1u << 25) - 1) m->epoch = 0;  // epoch * 128 stays within 32 bits
+  }
   {
     Prof pr(m, st);
     CK(pr.done(launch_step_init(sp, st), 0, -1, (double)kr * cf.hidden * (4 + 0.5625)));
   }
+  const bool step_kernel = use_step_kernel(m, kr);
   if (!m->use_graph || m->profile || m->stall_next) {
-    cudaError_t e = enqueue_body(m, c, kr, pos0, logits, argmax, st);
+    cudaError_t e = step_kernel ? enqueue_step_kernel(m, c, logits, argmax, st)
+                                : enqueue_body(m, c, kr, pos0, logits, argmax, st);
     m->stall_next = false;
     CK(e);
     return Q4G_OK;
@@ -1009,7 +1119,8 @@ q4g_status run_step(q4g_model* m, q4g_cache* c, int kr, int64_t pos0, const int3
     if (m->graphs.size() >= 16) free_graphs(m);
     cudaGraph_t graph = nullptr;
     CK(cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal));
-    cudaError_t e = enqueue_body(m, c, kr, pos0, logits, argmax, m->cap_stream);
+    cudaError_t e = step_kernel ? enqueue_step_kernel(m, c, logits, argmax, m->cap_stream)
+                                : enqueue_body(m, c, kr, pos0, logits, argmax, m->cap_stream);
     cudaError_t e2 = cudaStreamEndCapture(m->cap_stream, &graph);
     if (e != cudaSuccess) {
       if (graph) cudaGraphDestroy(graph);

@@ -644,6 +644,33 @@ size_t attn_smem_bytes(int hd, int) {
   return hd == 256 ? sizeof(Smem<256>) : sizeof(Smem<512>);
 }
 
+FlashPlan flash_plan(int n_q, int n_kv, int hd, bool ring, int64_t window) {
+  FlashPlan f{};
+  const int G = n_q / n_kv;
+  f.m_groups = (G + 31) / 32;
+  const int sms = device_sm_count();
+  int nch = ((hd == 256 ? 2 : 1) * sms) / (n_kv * f.m_groups);
+  if (ring) {
+    const int64_t want = (window + 63) / 64;
+    if (want < nch) nch = (int)want;
+  }
+  if (nch > 2 * sms) nch = 2 * sms;
+  f.n_chunks = nch < 1 ? 1 : nch;
+  f.ml_offset = kFlashCounterBytes;
+  f.acc_offset = f.ml_offset + ((sizeof(float) * 2 * (size_t)n_q * f.n_chunks + 255) & ~(size_t)255);
+  f.bytes = f.acc_offset + sizeof(float) * (size_t)n_q * f.n_chunks * hd;
+  return f;
+}
+
+void flash_bind(AttnParams& p, const FlashPlan& f, void* scratch) {
+  char* w = static_cast<char*>(scratch);
+  p.m_groups = f.m_groups;
+  p.n_chunks = f.n_chunks;
+  p.counters = reinterpret_cast<int32_t*>(w);
+  p.part_ml = reinterpret_cast<float*>(w + f.ml_offset);
+  p.part_acc = reinterpret_cast<float*>(w + f.acc_offset);
+}
+
 size_t attn_partial_floats(int kr, int n_q, int n_chunks, int hd) {
   return (size_t)kr * n_q * n_chunks * (size_t)hd;
 }

@@ -37,6 +37,7 @@
 //   * partial row sums are reduced with shuffles across the 8 lanes of a row
 //     and in a fixed order across warps through shared memory (deterministic).
 #include "q4g_common.cuh"
+#include "q4g_dot.cuh"
 #include "q4g_internal.h"
 #include "q4g_prefetch.cuh"
 
@@ -49,9 +50,6 @@ namespace q4g {
 
 namespace {
 
-// x digits of the integer dot product per block and activation row: 4 uint4
-// (digit 0 / 1 of the low / high 16 columns), see block_dot_int.
-constexpr int kDigitQuads = 4;
 
 // Slot of column e (0..31) of a block in the x layout (inverse of xperm).
 Q4G_DEV int xslot(int e) {
@@ -300,35 +298,7 @@ Q4G_DEV void stage_x(const GemvParams& p, uint4* xs, float* cblk, float* misc) {
   __syncthreads();
 }
 
-// Digits of 4 consecutive columns of one block (see block_dot_int):
-// X_i = rint(x_i * 2^(29 - Emax)), |X_i| < 2^15 (the scaling is a power of two).
-// Returns one packed word per digit (byte e = digit of column e: byte 0 of X
-// unsigned, byte 1 signed) and adds the digit sums to sd.
-Q4G_DEV void digits4(const __half (&h)[4], int em, uint32_t (&wd)[2], int (&sd)[2]) {
-  const float sc = __int_as_float((29 - em + 127) << 23);
-  // round to nearest even through the fp32 adder: x * sc is exact and
-  // |x * sc| < 2^15, so x * sc + 1.5 * 2^23 rounds once at unit spacing and its
-  // bit pattern minus that of 1.5 * 2^23 is the integer
-  int X[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) X[e] = __float_as_int(fmaf(__half2float(h[e]), sc, 12582912.0f)) - 0x4B400000;
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const uint32_t sel = 0x0040u | (uint32_t)(t * 0x11);  // bytes (x.b_t, y.b_t)
-    const uint32_t lo = __byte_perm((uint32_t)X[0], (uint32_t)X[1], sel);
-    const uint32_t hi = __byte_perm((uint32_t)X[2], (uint32_t)X[3], sel);
-    wd[t] = __byte_perm(lo, hi, 0x5410);
-  }
-  sd[0] += dp4a_uu(wd[0], 0x01010101u, 0);
-  int s1;
-  asm("dp4a.s32.s32 %0, %1, %2, %3;" : "=r"(s1) : "r"(wd[1]), "r"(0x01010101u), "r"(0));
-  sd[1] += s1;
-}
 
-Q4G_DEV int half_exp(__half h) {
-  const int E = (__half_as_ushort(h) >> 10) & 31;
-  return E ? E : 1;
-}
 
 // Activations as the digits of the integer dot product (block_dot_int):
 // thread (block blk, group sub) turns columns 4*sub..4*sub+3 of the block into
@@ -363,40 +333,6 @@ Q4G_DEV void stage_digits(const GemvParams& p, uint4* dg, int4* bc, float* misc)
   __syncthreads();
 }
 
-// Digits of one whole 32-column block in one lane (see block_dot_int): xv[q]
-// holds columns 8q .. 8q+7 as fp16. The largest exponent field comes from the
-// largest magnitude (fp16 bit patterns of |x| order like the values; zero and
-// subnormals count as exponent 1).
-Q4G_DEV void lane_block_digits(const uint4 (&xv)[4], uint4 (&g)[kDigitQuads], int4& cv) {
-  uint32_t mx = 0;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    mx = __vmaxu2(mx, xv[q].x & 0x7FFF7FFFu);
-    mx = __vmaxu2(mx, xv[q].y & 0x7FFF7FFFu);
-    mx = __vmaxu2(mx, xv[q].z & 0x7FFF7FFFu);
-    mx = __vmaxu2(mx, xv[q].w & 0x7FFF7FFFu);
-  }
-  const uint32_t mh = max(mx & 0xFFFFu, mx >> 16);
-  const int em = max((int)((mh >> 10) & 31u), 1);
-  int sd[2] = {0, 0};
-  uint32_t words[2][8];
-#pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    const uint32_t w0 = (&xv[q >> 1].x)[2 * (q & 1)], w1 = (&xv[q >> 1].x)[2 * (q & 1) + 1];
-    const __half h4[4] = {__ushort_as_half((unsigned short)(w0 & 0xFFFFu)), __ushort_as_half((unsigned short)(w0 >> 16)),
-                          __ushort_as_half((unsigned short)(w1 & 0xFFFFu)), __ushort_as_half((unsigned short)(w1 >> 16))};
-    uint32_t wd[2];
-    digits4(h4, em, wd, sd);
-    words[0][q] = wd[0];
-    words[1][q] = wd[1];
-  }
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    g[2 * t] = make_uint4(words[t][0], words[t][1], words[t][2], words[t][3]);
-    g[2 * t + 1] = make_uint4(words[t][4], words[t][5], words[t][6], words[t][7]);
-  }
-  cv = make_int4(-8 * sd[0], -8 * sd[1], 0, (em - 29 + 127) << 23);
-}
 
 // The activation rows as fp16 in shared memory ([KRM][k]), from the fused
 // residual/RMSNorm prologue. Ends with __syncthreads().
@@ -662,38 +598,6 @@ Q4G_DEV void issue_item(const GemvParams& p, int u, int c, unsigned char* st, ui
   }
 }
 
-// ---------------------------------------------------------------------------
-// Integer form of the block dot product.
-//
-// x of one block (32 fp16 values) becomes signed 16-bit fixed point relative to
-// the block's largest exponent: X_i = round(x_i * 2^(29 - Emax)), |X_i| < 2^15,
-// exact for every value within 2^4 of the block maximum; the rest carry an
-// error of at most 2^-15 of the block maximum. x_i ~= X_i * 2^(Emax - 29).
-// The code byte b of a block holds column b in its low nibble and column b + 16
-// in its high nibble, so a code word w gives the four low codes as
-// w & 0x0F0F0F0F and the four high codes as (w >> 4) & 0x0F0F0F0F.
-// X splits into bytes X = d0 + 256 d1 (d0 unsigned, d1 signed), and
-//   sum_i (c_i - 8) X_i = S0 + 256 S1,  S_t = sum_i c_i d_t,i - 8 sum_i d_t,i,
-// each S_t a chain of 4-way byte dot products (dp4a) started at the constant
-// -8 sum_i d_t,i. S0, S1 and S0 + 256 S1 (|.| <= 32 * 8 * 2^15 = 2^23) are exact
-// in int32 and the last one in fp32.
-// Layout per x row j: dg[j][2t + h][blk] holds digit t of columns 16h..16h+15
-// of block blk (16 bytes), bc[j][blk] = (-8 D0, -8 D1, 0, bits of 2^(Emax-29))
-// with D_t = sum_i d_t,i, written by stage_digits.
-// ---------------------------------------------------------------------------
-Q4G_DEV float block_dot_int(const uint4 q, const uint4 (&g)[kDigitQuads], const int4 c) {
-  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-  int s0 = c.x, s1 = c.y;
-#pragma unroll
-  for (int t = 0; t < 4; ++t) {
-    const uint32_t lo = w[t] & 0x0F0F0F0Fu, hi = (w[t] >> 4) & 0x0F0F0F0Fu;
-    s0 = dp4a_uu(lo, (&g[0].x)[t], s0);
-    s0 = dp4a_uu(hi, (&g[1].x)[t], s0);
-    s1 = dp4a_us(lo, (&g[2].x)[t], s1);
-    s1 = dp4a_us(hi, (&g[3].x)[t], s1);
-  }
-  return (float)(s1 * 256 + s0);
-}
 
 // Shared memory of the warp-streamed kernel: the x region (layout per dot
 // kind), then 64 floats of reduction scratch, per-warp argmax candidates, the
@@ -1038,32 +942,6 @@ __host__ __device__ inline size_t cs_fixed_bytes(int krm, int k, int ns, int nc,
   return (size_t)krm * nb * (16 * kDigitQuads + 16) + 64 * 4 + red + 128 + 2 * kCsMaxStages * 8;
 }
 
-// Sum v[0..R) over the 32 lanes: after the butterfly, lanes with (lane & (32/R
-// - 1)) == 0 hold the total of row cs_row<R>(lane).
-template <int R>
-Q4G_DEV float cs_reduce_rows(float (&v)[R], int lane) {
-#pragma unroll
-  for (int h = R / 2, o = 16; h >= 1; h >>= 1, o >>= 1) {
-    const bool upper = lane & o;
-#pragma unroll
-    for (int i = 0; i < h; ++i) {
-      const float send = upper ? v[i] : v[i + h];
-      const float keep = upper ? v[i + h] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-    }
-  }
-  float t = v[0];
-#pragma unroll
-  for (int o = 16 / R; o >= 1; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-  return t;
-}
-template <int R>
-Q4G_DEV int cs_row(int lane) {
-  int r = 0;
-#pragma unroll
-  for (int h = R / 2, o = 16; h >= 1; h >>= 1, o >>= 1) r += (lane & o) ? h : 0;
-  return r;
-}
 
 // Wait for `phase` of `bar` until done, until another warp gave up (flag set),
 // or until limit_ns pass (then this warp sets the flag and the error word).
@@ -2306,12 +2184,15 @@ cudaError_t launch_gemv_chain(const ChainParams& c_in, cudaStream_t st, bool pdl
 }
 
 int device_sm_count() {
-  static int n = 0;
+  // per device, looked up once with that device current
+  constexpr int kMaxDev = 64;
+  static std::atomic<int> counts[kMaxDev];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return 1;
+  int n = counts[dev].load(std::memory_order_relaxed);
   if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 1;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 1;
+    counts[dev].store(n, std::memory_order_relaxed);
   }
   return n;
 }

@@ -17,7 +17,6 @@
 namespace {
 
 constexpr size_t kScratchBytes = Q4G_NOALLOC_SCRATCH_BYTES;
-constexpr size_t kCounterBytes = 256;
 
 // Shared by every call on a device; each call clears the counters it needs.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
@@ -79,37 +78,23 @@ extern "C" q4g_status q4g_flash_decode_ring_noalloc(const uint16_t* q, int32_t n
   p.n_q = n_q;
   p.n_kv = n_kv;
   p.hd = head_dim;
-  const int G = n_q / n_kv;
-  p.m_groups = (G + 31) / 32;
-  const int sms = q4g::device_sm_count();
-  int nch = ((head_dim == 256 ? 2 : 1) * sms) / (n_kv * p.m_groups);
-  const int want = (int)((window + 63) / 64);
-  if (want < nch) nch = want;
-  if (nch > 2 * sms) nch = 2 * sms;
-  p.n_chunks = nch < 1 ? 1 : nch;
-  if (n_kv * p.m_groups * (int)sizeof(int32_t) > (int)kCounterBytes)
+  const q4g::FlashPlan plan = q4g::flash_plan(n_q, n_kv, head_dim, true, window);
+  if (n_kv * plan.m_groups * (int)sizeof(int32_t) > (int)q4g::kFlashCounterBytes)
     return bad(Q4G_EINVAL, "too many KV heads for the fixed scratch");
-
-  // scratch: [counters 256 B][(m, l) per row and chunk][acc per row, chunk, dim]
-  const size_t ml_bytes = ((sizeof(float) * 2 * (size_t)n_q * p.n_chunks) + 255) & ~(size_t)255;
-  const size_t acc_bytes = sizeof(float) * (size_t)n_q * p.n_chunks * head_dim;
-  if (kCounterBytes + ml_bytes + acc_bytes > kScratchBytes)
+  if (plan.bytes > kScratchBytes)
     return bad(Q4G_ERANGE, "split-KV scratch for these sizes exceeds Q4G_NOALLOC_SCRATCH_BYTES "
                            "(n_q * chunks * head_dim * 4 bytes plus (m, l) and counters)");
 
   void* base = nullptr;
   cudaError_t e = scratch_address(&base);
   if (e != cudaSuccess) return bad(Q4G_ECUDA, cudaGetErrorString(e));
-  char* w = static_cast<char*>(base);
-  p.counters = reinterpret_cast<int32_t*>(w);
-  p.part_ml = reinterpret_cast<float*>(w + kCounterBytes);
-  p.part_acc = reinterpret_cast<float*>(w + kCounterBytes + ml_bytes);
+  q4g::flash_bind(p, plan, base);
   p.combine_in_kernel = 1;
   p.out = reinterpret_cast<__half*>(out);
 
   cudaStream_t st = (cudaStream_t)stream;
   // the completion counters must start at zero; the partials are overwritten
-  if ((e = cudaMemsetAsync(p.counters, 0, kCounterBytes, st)) != cudaSuccess)
+  if ((e = cudaMemsetAsync(p.counters, 0, q4g::kFlashCounterBytes, st)) != cudaSuccess)
     return bad(Q4G_ECUDA, cudaGetErrorString(e));
   if ((e = q4g::launch_attention(p, st, false)) != cudaSuccess) return bad(Q4G_ECUDA, cudaGetErrorString(e));
   return Q4G_OK;

@@ -17,8 +17,10 @@ Q4G_OPT_CUDA_GRAPH, Q4G_OPT_PDL, Q4G_OPT_DUMP, Q4G_OPT_PROFILE, Q4G_OPT_TEST_STA
 Q4G_OPT_ATTN_CLUSTER = 6
 Q4G_OPT_GEMV_CHAIN = 7
 Q4G_OPT_TRACE = 8
+Q4G_OPT_STEP_KERNEL = 9
+Q4G_OPT_STEP_POLL_NS = 10
 KIND_NAMES = ["step_init", "qkv_gemv", "attn_sliding", "attn_full", "attn_combine", "o_gemv",
-              "gate_up_gemv", "down_gemv", "head_gemv", "chain_gemv"]
+              "gate_up_gemv", "down_gemv", "head_gemv", "chain_gemv", "step_kernel"]
 
 EXPORTS = [
     "q4g_last_error", "q4g_status_string", "q4g_abi_version",

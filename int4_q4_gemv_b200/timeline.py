@@ -1,4 +1,5 @@
-"""Timeline of one decode layer on the device clock (observability harness).
+"""Timeline of one decode layer of the per-kernel path (one launch per GEMV and
+attention kernel) on the device clock (observability harness).
 
 Runs a few decode steps of the synthetic 12B-class decoder (fewer layers by
 default) with the library's trace option and prints, for layer 1 on a common
@@ -9,7 +10,7 @@ when its first stage was ready and when its last stage was reduced; for the
 sliding-window attention launch the phases of its first CTA, and the spread of
 the times at which gate|up's CTAs finished.
 
-    python -m datagen.timeline [--layers 6] [--context 4096] [--steps 3]
+    python -m int4_q4_gemv_b200.timeline [--layers 6] [--context 4096] [--steps 3]
 """
 from __future__ import annotations
 
@@ -35,6 +36,7 @@ def main() -> None:
     a = ap.parse_args()
     cfg = dict(WL.B12, n_layers=a.layers)
     g = S.SynthDecoder(cfg, seed=0)
+    Q.q4g_model_set_option(g.handle, Q.Q4G_OPT_STEP_KERNEL, 0)  # the per-kernel path's trace layout
     c = g.new_cache(a.context)
     S.fill_history(c)
     sp = S.stream_ptr()
