@@ -82,6 +82,8 @@ def parse_args():
                          "(default: the library's default)")
     ap.add_argument("--step-kernel", type=int, choices=[0, 1], default=None,
                     help="decode steps as one persistent launch (default: the library's default, 1)")
+    ap.add_argument("--grid-sync", type=int, choices=[0, 1], default=None,
+                    help="step kernel: grid counts between phases (default: the library's)")
     ap.add_argument("--quick", action="store_true",
                     help="the headline context only (no other contexts, no microbenchmarks)")
     return ap.parse_args()
@@ -479,6 +481,8 @@ def main():
         Q.q4g_model_set_option(model.handle, Q.Q4G_OPT_GEMV_CHAIN, args.gemv_chain)
     if args.step_kernel is not None:
         Q.q4g_model_set_option(model.handle, Q.Q4G_OPT_STEP_KERNEL, args.step_kernel)
+    if args.grid_sync is not None:
+        Q.q4g_model_set_option(model.handle, Q.Q4G_OPT_STEP_GRID_SYNC, args.grid_sync)
     cache = model.new_cache(C)
     stream = torch.cuda.current_stream()
     sp = stream.cuda_stream

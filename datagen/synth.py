@@ -136,14 +136,25 @@ class SynthDecoder:
                 setattr(Lw, name, g.data_ptr())
             Lw.layer_scalar = 1.0 if variant != 1 else float(
                 DG.uniform_float(seed, s(DG.T_LAYER_SCALAR), 1, 0.5, 1.5)[0])
-        eq, es = packed_tensor(c["vocab"], H, seed, DG.STREAM_EMBED, device)
         nf = torch.ones(H, dtype=torch.float32, device=device)
         if variant == 1:
             fill_gain(nf, seed, DG.STREAM_FINAL_NORM)
-        self._keep += [eq, es, nf]
+        self.embed_f16 = None
+        if c.get("head_fp16"):  # the same N(0, 0.02) draws, kept at fp16
+            e16 = torch.empty((c["vocab"], H), dtype=torch.float16, device=device)
+            fill_normal_f16(e16, seed, DG.STREAM_EMBED, 0.02)
+            eq = es = None
+            self.embed_f16 = e16
+            self._keep += [e16, nf]
+            emb = Q.q4g_qtensor(0, 0)
+        else:
+            eq, es = packed_tensor(c["vocab"], H, seed, DG.STREAM_EMBED, device)
+            self._keep += [eq, es, nf]
+            emb = Q.q4g_qtensor(eq.data_ptr(), es.data_ptr())
         self.embed_qs, self.embed_sc = eq, es
         self._layers = layers
-        self._w = Q.q4g_weights(layers, Q.q4g_qtensor(eq.data_ptr(), es.data_ptr()), nf.data_ptr())
+        self._w = Q.q4g_weights(layers, emb, nf.data_ptr(),
+                                self.embed_f16.data_ptr() if self.embed_f16 is not None else 0)
         self._cfg_struct = config_struct(c)
         torch.cuda.synchronize()
         self.handle = Q.q4g_model_create(self._cfg_struct, self._w)

@@ -24,12 +24,15 @@ def decoder(n_layers, hidden, n_q_heads, ffn, vocab, sl_kv_heads, window, ring,
         gl_kv_heads=gl_kv_heads, gl_head_dim=gl_head_dim, full_every=full_every,
         full_offset=full_offset, rope_pairs_full=rope_pairs_full,
         rope_theta_sl=1.0e4, rope_theta_gl=1.0e6, rms_eps=_f32(1e-6), softcap=30.0,
-        embed_scale=_f32(math.sqrt(hidden)), v_norm_sliding=1)
+        embed_scale=_f32(math.sqrt(hidden)), v_norm_sliding=1, head_fp16=0)
 
 
 # Tiny 6-layer decoder (layers 0-4 sliding, layer 5 full): parity config.
 TINY = decoder(n_layers=6, hidden=1024, n_q_heads=8, ffn=4096, vocab=4096,
                sl_kv_heads=2, window=256, ring=512)
+
+# TINY with the fp16 tied embedding / head.
+TINY_F16 = dict(TINY, head_fp16=1)
 
 # 12B-class decoder: 48 layers, full attention at 5, 11, ..., 47.
 B12 = decoder(n_layers=48, hidden=3840, n_q_heads=16, ffn=15360, vocab=262144,
@@ -47,6 +50,8 @@ GEMV_SHAPES = [
     ("qkv_3840x8192", 8192, 3840, 3),
     ("vocab_head_3840x262144", 262144, 3840, 4),
 ]
+# the fp16 tied head's GEMV (2 bytes per weight)
+GEMV_F16_SHAPES = [("vocab_head_f16_3840x262144", 262144, 3840, 5)]
 
 # Flash-decode microbench: hd512 single-KV-head cache lengths.
 ATTN_GLOBAL_LENGTHS = [4096, 8192, 16384, 32768, 65536, 131072]

@@ -40,7 +40,7 @@
 extern "C" {
 #endif
 
-#define Q4G_ABI_VERSION 1
+#define Q4G_ABI_VERSION 2
 
 /* A CUDA stream (cudaStream_t / CUstream). NULL selects the legacy default stream. */
 typedef struct CUstream_st* q4g_stream_t;
@@ -97,6 +97,14 @@ q4g_status q4g_q4_0_unpack(const uint8_t* qs, const uint16_t* scales, int64_t ro
  * aligned, x 16-byte aligned. No scratch memory. */
 q4g_status q4g_gemv(const uint8_t* qs, const uint16_t* scales, int64_t n, int64_t k,
                     const uint16_t* x_f16, int32_t nrhs, float* y, q4g_stream_t stream);
+
+/* fp16 matrix-vector product (the fp16 tied head's GEMV without its epilogue):
+ * y[j][r] = sum_c w16[r][c] * x[j][c] for j < nrhs, IEEE binary16 w16 [n][k]
+ * and x [nrhs][k], products exact in fp32, fp32 accumulation, fp32 y [nrhs][n].
+ * Requires k % 256 == 0, k <= 8192, 1 <= nrhs <= 8, w16 and x 16-byte aligned.
+ * No scratch memory. Q4G_EINVAL on a bad size or pointer. */
+q4g_status q4g_gemv_f16(const uint16_t* w16, int64_t n, int64_t k, const uint16_t* x_f16, int32_t nrhs,
+                        float* y, q4g_stream_t stream);
 
 /* Process-wide choice of the q4_0 GEMV kernel, for tuning and tests (not on
  * the pages). All kernels compute the same operation within the same error
@@ -202,6 +210,11 @@ typedef struct {
   float softcap;           /* final logit softcap c: c * tanh(z / c) [30] */
   float embed_scale;       /* embedding multiplier [sqrt(h)] */
   int32_t v_norm_sliding;  /* 1: scale-free RMSNorm on sliding-layer V as on full layers */
+  int32_t head_fp16;       /* 0: the tied embedding / head is q4_0 (q4g_weights.embed);
+                              1: it is fp16 (q4g_weights.embed_f16, [vocab][h] IEEE
+                              binary16, the "fp16 vocab path" of "Gemma-4-12B-CoreAI",
+                              tiered-v3/ section): the head GEMV reads 2 B per weight
+                              and the embedding row is the fp16 row times embed_scale */
 } q4g_config;
 
 /* One q4_0 tensor in the layout above (device pointers, borrowed). */
@@ -224,8 +237,10 @@ typedef struct {
 
 typedef struct {
   const q4g_layer_weights* layers; /* host array [n_layers], copied by q4g_model_create */
-  q4g_qtensor embed;               /* tied embedding and LM head [vocab][h] */
+  q4g_qtensor embed;               /* tied embedding and LM head [vocab][h] (head_fp16 = 0) */
   const float* norm_final;         /* [h] */
+  const uint16_t* embed_f16;       /* tied embedding and LM head [vocab][h] fp16, 16-byte
+                                      aligned (head_fp16 = 1; NULL otherwise) */
 } q4g_weights;
 
 typedef struct q4g_model q4g_model;
@@ -307,8 +322,15 @@ typedef enum {
                                  (hidden <= 4096, head dims 256 / 512); 0: one
                                  launch per GEMV / attention kernel. Verify blocks
                                  (K > 1 rows) always use the per-kernel path. */
-  Q4G_OPT_STEP_POLL_NS = 10 /* [64] step kernel: nanoseconds each CTA sleeps between two
-                                 polls of a phase counter (0..100000) */
+  Q4G_OPT_STEP_POLL_NS = 10, /* [64] step kernel: nanoseconds a thread first sleeps between
+                                 two polls of a phase counter or of tagged activation
+                                 words (0..100000; tagged words back off by doubling) */
+  Q4G_OPT_STEP_GRID_SYNC = 11 /* [1] step kernel: 1: every phase starts once every CTA
+                                 has counted itself done with the previous phase; 0: a
+                                 phase starts as soon as its own inputs (tagged words:
+                                 value and the step and layer that wrote it) have
+                                 arrived, with one grid-wide count per full-attention
+                                 layer only */
 } q4g_option;
 q4g_status q4g_model_set_option(q4g_model* m, q4g_option opt, intptr_t value);
 

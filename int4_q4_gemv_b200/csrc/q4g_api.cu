@@ -83,6 +83,7 @@ struct q4g_model {
   std::vector<int> ordinal;  // sliding or full ordinal of each layer
   std::vector<char> full;
   q4g_qtensor embed;
+  const uint16_t* embed_f16;  // the fp16 tied table (head_fp16), else NULL
   const float* norm_final;
   int n_sl = 0, n_gl = 0;
   LayerShape sl{}, gl{};
@@ -121,6 +122,7 @@ struct q4g_model {
   uint32_t epoch = 0;
   bool step_ok = false;  // the shapes fit the step kernel
   uint32_t poll_ns = 64;  // step kernel: back-off between polls of a phase counter
+  int32_t step_grid_sync = 1;  // step kernel: grid counts between phases (0: tagged reads only)
   // options
   bool use_graph = true, use_pdl = true, attn_cluster = true, gemv_chain = false, use_step = false;
   uint64_t* trace = nullptr;  // Q4G_OPT_TRACE
@@ -186,6 +188,7 @@ q4g_status validate_config(const q4g_config* c) {
     return fail(Q4G_EINVAL, "bad rope theta / eps / softcap / embed_scale");
   if (c->full_every < 0 || (c->full_every > 0 && (c->full_offset < 0 || c->full_offset >= c->full_every)))
     return fail(Q4G_EINVAL, "bad full_every / full_offset");
+  if (c->head_fp16 != 0 && c->head_fp16 != 1) return fail(Q4G_EINVAL, "head_fp16 must be 0 or 1");
   return Q4G_OK;
 }
 
@@ -208,12 +211,17 @@ extern "C" q4g_status q4g_model_create(const q4g_config* cfg, const q4g_weights*
   q4g_status st = validate_config(cfg);
   if (st) return st;
   if (!w || !w->layers || !w->norm_final) return fail(Q4G_EINVAL, "weights are NULL");
-  if ((st = check_q(w->embed, "embed"))) return st;
+  if (cfg->head_fp16) {
+    if (!w->embed_f16 || !aligned(w->embed_f16, 16)) return fail(Q4G_EINVAL, "embed_f16: NULL or not 16-byte aligned");
+  } else if ((st = check_q(w->embed, "embed"))) {
+    return st;
+  }
   const q4g_config& c = *cfg;
   q4g_model* m = new (std::nothrow) q4g_model();
   if (!m) return fail(Q4G_ENOMEM, "model handle");
   m->cfg = c;
   m->embed = w->embed;
+  m->embed_f16 = c.head_fp16 ? w->embed_f16 : nullptr;
   m->norm_final = w->norm_final;
   for (int l = 0; l < c.n_layers; ++l) {
     const q4g_layer_weights& L = w->layers[l];
@@ -355,6 +363,7 @@ extern "C" q4g_status q4g_model_create(const q4g_config* cfg, const q4g_weights*
       m->step_ok = false;
   }
   if (!a16(m->embed.qs) || !a16(m->embed.scales) || !a16(m->norm_final)) m->step_ok = false;
+  if (m->embed_f16) m->step_ok = false;  // the step kernel streams the q4_0 head only
   e = cudaMemset(m->scratch, 0, off);
   {  // per-layer descriptors of the persistent step kernel
     std::vector<StepLayer> sl(c.n_layers);
@@ -432,6 +441,7 @@ extern "C" q4g_status q4g_model_set_option(q4g_model* m, q4g_option opt, intptr_
     case Q4G_OPT_TRACE: m->trace = (uint64_t*)value; break;
     case Q4G_OPT_STEP_KERNEL: m->use_step = value != 0; break;
     case Q4G_OPT_STEP_POLL_NS: m->poll_ns = (uint32_t)std::max<intptr_t>(0, std::min<intptr_t>(value, 100000)); break;
+    case Q4G_OPT_STEP_GRID_SYNC: m->step_grid_sync = value != 0; break;
     default: return fail(Q4G_EINVAL, "unknown option %d", (int)opt);
   }
   free_graphs(m);
@@ -595,6 +605,29 @@ extern "C" q4g_status q4g_gemv(const uint8_t* qs, const uint16_t* scales, int64_
     p.y_stride = n;
     CK(launch_gemv(p, (cudaStream_t)stream, false));
   }
+  return Q4G_OK;
+}
+
+extern "C" q4g_status q4g_gemv_f16(const uint16_t* w16, int64_t n, int64_t k, const uint16_t* x_f16, int32_t nrhs,
+                                   float* y, q4g_stream_t stream) {
+  if (n < 0 || n > INT32_MAX || k <= 0 || k % 256 || k > 8192)
+    return fail(Q4G_EINVAL, "need n >= 0 and k a positive multiple of 256, at most 8192");
+  if (nrhs < 1 || nrhs > kMaxRows) return fail(Q4G_EINVAL, "nrhs must be 1..8");
+  if (n == 0) return Q4G_OK;
+  if (!w16 || !x_f16 || !y) return fail(Q4G_EINVAL, "NULL pointer");
+  if (!aligned(w16, 16) || !aligned(x_f16, 16) || !aligned(y, 4)) return fail(Q4G_EINVAL, "misaligned pointer");
+  GemvParams p{};
+  p.w16 = w16;
+  p.k = (int)k;
+  p.n_rows = (int)n;
+  p.kr = nrhs;
+  p.pro = PRO_X16;
+  p.epi = EPI_STORE;
+  p.x = reinterpret_cast<const __half*>(x_f16);
+  p.x_stride = k;
+  p.y = y;
+  p.y_stride = n;
+  CK(launch_gemv_f16(p, (cudaStream_t)stream, false));
   return Q4G_OK;
 }
 
@@ -1001,7 +1034,8 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
       const int maxr = gemv_max_rows(cf.ffn);
       for (int r0 = 0; r0 < kr; r0 += maxr) {
         GemvParams p = down_params(l, r0);
-        if (r0 + maxr >= kr) p.next = l + 1 < L ? next_of(qkv_params(l + 1), 1.0f) : next_of(head_params(), 0.05f);
+        if (r0 + maxr >= kr && (l + 1 < L || !m->embed_f16))
+          p.next = l + 1 < L ? next_of(qkv_params(l + 1), 1.0f) : next_of(head_params(), 0.05f);
         p.trace = trace_sep && r0 == 0 ? trace_sep + 3 * kGemvTraceSlots : nullptr;
         Prof pr(m, st);
         e = pr.done(debug_sync(launch_gemv(p, st, pdl), "down", l, st), 7, l, gemv_bytes(H, cf.ffn, p.kr, 4));
@@ -1012,8 +1046,14 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
   {
     GemvParams p = head_params();
     Prof pr(m, st);
-    e = pr.done(debug_sync(launch_gemv(p, st, pdl), "head", L, st), 8, L,
-                gemv_bytes(cf.vocab, H, kr, logits ? 4 : 0));
+    if (m->embed_f16) {  // (f3) fp16 tied head: 2 bytes per weight
+      p.w16 = m->embed_f16;
+      e = pr.done(debug_sync(launch_gemv_f16(p, st, pdl), "head_f16", L, st), 8, L,
+                  (double)cf.vocab * H * 2 + (logits ? 4.0 * kr * cf.vocab : 0.0));
+    } else {
+      e = pr.done(debug_sync(launch_gemv(p, st, pdl), "head", L, st), 8, L,
+                  gemv_bytes(cf.vocab, H, kr, logits ? 4 : 0));
+    }
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -1045,6 +1085,7 @@ cudaError_t enqueue_step_kernel(q4g_model* m, const q4g_cache* c, float* logits,
   p.dump = m->dump;
   p.trace = m->trace;
   p.poll_ns = m->poll_ns;
+  p.grid_sync = m->step_grid_sync;
   if (m->stall_next) {
     p.stall_test = 1;
     p.wait_ns = 20000000ull;  // 20 ms
@@ -1078,6 +1119,7 @@ q4g_status run_step(q4g_model* m, q4g_cache* c, int kr, int64_t pos0, const int3
   sp.hidden = hidden;
   sp.emb_qs = m->embed.qs;
   sp.emb_sc = m->embed.scales;
+  sp.emb_f16 = m->embed_f16;
   sp.hidden_size = cf.hidden;
   sp.vocab = cf.vocab;
   sp.embed_scale = cf.embed_scale;

@@ -1426,8 +1426,10 @@ __global__ void __launch_bounds__(kStageThreads, 1) gemv_q4_stage_kernel(const G
     int s = 0;
     uint32_t ph = 0;
     for (int t = 0; t < n_st; ++t) {
-      if (!*abort_flag) cs_wait(&full[s], ph, p, abort_flag);
-      if (*abort_flag) break;
+      // warp-uniform decisions: lanes that waited for different lengths of time must
+      // all enter the block below (it holds warp collectives) or all leave
+      if (!__any_sync(0xffffffffu, *abort_flag != 0)) cs_wait(&full[s], ph, p, abort_flag);
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
       if (c == 0 && g == 0 && lane == 0 && t < 64) stamp(72 + t);
       const unsigned char* st = stages + s * SB + (size_t)g * RG * kh + qoff;
       const unsigned char* ss = stages + s * SB + (size_t)R * kh + (size_t)g * RG * 2 * nb + soff;
@@ -1466,8 +1468,8 @@ __global__ void __launch_bounds__(kStageThreads, 1) gemv_q4_stage_kernel(const G
     int s = 0;
     uint32_t ph = 0;
     for (int t = 0; t < n_st; ++t) {
-      if (!*abort_flag) cs_wait(&ready[s], ph, p, abort_flag);
-      if (*abort_flag) break;
+      if (!__any_sync(0xffffffffu, *abort_flag != 0)) cs_wait(&ready[s], ph, p, abort_flag);
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
       const float* rs = red + (size_t)s * NC * R * KRM;
       float val = 0.f;
       if (lane < R * KRM)
@@ -2130,6 +2132,163 @@ cudaError_t launch_gemv(const GemvParams& p_in, cudaStream_t st, bool pdl) {
   if (p.kr <= 2) return launch_t<2>(p, st, pdl);
   if (p.kr <= 4) return launch_t<4>(p, st, pdl);
   return launch_t<8>(p, st, pdl);
+}
+
+// ---------------------------------------------------------------------------
+// GEMV with fp16 weights: the tied head in its fp16 variant ("Gemma-4-12B-CoreAI",
+// tiered-v3/ section: the vocabulary path kept at fp16). The activation rows (the
+// fused residual/final-norm prologue, or given fp16 rows) are staged once per CTA in
+// shared memory; every warp of the grid takes rows r = warp, warp + all warps, ...;
+// a lane loads its 16-byte pieces of the row (8 weights each) with streaming loads,
+// all of them before the first use, and multiplies them with the matching x pieces
+// (fp16 products, exact in fp32, accumulated in fp32); the row total comes from a
+// warp reduction. Epilogue: softcap, logits and the argmax (per warp, per CTA, then
+// the last CTA of the grid; lowest index on ties), or a plain store.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int kF16Warps = 16;
+constexpr int kF16Threads = kF16Warps * 32;
+constexpr int kF16Batch = 16;  // 16-byte pieces per lane loaded before use
+
+template <int KRM>
+__global__ void __launch_bounds__(kF16Threads, 1) gemv_f16_kernel(const GemvParams p) {
+  extern __shared__ __align__(16) unsigned char f16_smem[];
+  const int k = p.k, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  __half* xh = reinterpret_cast<__half*>(f16_smem);                            // [KRM][k]
+  float* misc = reinterpret_cast<float*>(f16_smem + (size_t)KRM * k * 2);      // 64 floats
+  float* cand_v = misc + 64;                                                   // [kF16Warps][KRM]
+  int* cand_i = reinterpret_cast<int*>(cand_v + kF16Warps * KRM);              // [kF16Warps][KRM]
+  __shared__ int s_ticket;
+  pdl_wait();
+  if (p.pro == PRO_RESID) {
+    stage_x_half<KRM, kF16Threads>(p, xh, misc);  // ends with __syncthreads
+  } else {
+    for (int c = tid; c < p.kr * (k / 8); c += kF16Threads) {
+      const int j = c / (k / 8), q = c - j * (k / 8);
+      *reinterpret_cast<uint4*>(xh + (size_t)j * k + 8 * q) =
+          *reinterpret_cast<const uint4*>(p.x + (size_t)j * p.x_stride + 8 * q);
+    }
+    __syncthreads();
+  }
+  pdl_launch_dependents();
+  const int pieces = k / 8, per_lane = (pieces + 31) / 32;
+  float best_v[KRM];
+  int best_i[KRM];
+#pragma unroll
+  for (int j = 0; j < KRM; ++j) best_v[j] = -INFINITY, best_i[j] = 0x7fffffff;
+  const int gw = blockIdx.x * kF16Warps + warp, nw = gridDim.x * kF16Warps;
+  for (int r = gw; r < p.n_rows; r += nw) {
+    const uint4* wrow = reinterpret_cast<const uint4*>(p.w16 + (size_t)r * k);
+    float acc[KRM];
+#pragma unroll
+    for (int j = 0; j < KRM; ++j) acc[j] = 0.f;
+    for (int i0 = 0; i0 < per_lane; i0 += kF16Batch) {  // k <= 4096: one batch
+      uint4 wv[kF16Batch];
+#pragma unroll
+      for (int i = 0; i < kF16Batch; ++i) {
+        const int c = lane + 32 * (i0 + i);
+        if (i0 + i < per_lane && c < pieces) wv[i] = ld_stream_u4(wrow + c);
+      }
+#pragma unroll
+      for (int i = 0; i < kF16Batch; ++i) {
+        const int c = lane + 32 * (i0 + i);
+        if (i0 + i < per_lane && c < pieces) {
+#pragma unroll
+          for (int j = 0; j < KRM; ++j) {
+            if (KRM == 1 || j < p.kr) {
+              const uint4 xv = lds_u4(xh + (size_t)j * k + 8 * c);
+              acc[j] = fma2_h_f32(wv[i].x, xv.x, acc[j]);
+              acc[j] = fma2_h_f32(wv[i].y, xv.y, acc[j]);
+              acc[j] = fma2_h_f32(wv[i].z, xv.z, acc[j]);
+              acc[j] = fma2_h_f32(wv[i].w, xv.w, acc[j]);
+            }
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < KRM; ++j) {
+      const float v = warp_sum(acc[j]);
+      if (lane == 0 && (KRM == 1 || j < p.kr)) {
+        if (p.epi == EPI_STORE) {
+          p.y[(size_t)j * p.y_stride + r] = v;
+        } else {
+          const float z = p.softcap * tanhf(v / p.softcap);
+          if (p.logits) p.logits[(size_t)j * p.logits_stride + r] = z;
+          if (z > best_v[j] || (z == best_v[j] && r < best_i[j])) best_v[j] = z, best_i[j] = r;
+        }
+      }
+    }
+  }
+  if (p.epi != EPI_HEAD) return;
+  // argmax: lane 0 of each warp holds its candidates; CTA, then grid (last CTA)
+  if (lane == 0)
+#pragma unroll
+    for (int j = 0; j < KRM; ++j) cand_v[warp * KRM + j] = best_v[j], cand_i[warp * KRM + j] = best_i[j];
+  __syncthreads();
+  if (tid < KRM && tid < p.kr) {
+    float v = -INFINITY;
+    int i = 0x7fffffff;
+    for (int w = 0; w < kF16Warps; ++w) {
+      const float v2 = cand_v[w * KRM + tid];
+      const int i2 = cand_i[w * KRM + tid];
+      if (v2 > v || (v2 == v && i2 < i)) v = v2, i = i2;
+    }
+    p.am_val[tid * gridDim.x + blockIdx.x] = v;
+    p.am_idx[tid * gridDim.x + blockIdx.x] = i;
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_ticket = atomicAdd(p.counter, 1);
+  __syncthreads();
+  if (s_ticket == (int)gridDim.x - 1 && tid < p.kr) {
+    __threadfence();
+    float v = -INFINITY;
+    int i = 0x7fffffff;
+    for (int b = 0; b < (int)gridDim.x; ++b) {
+      const float v2 = __ldcg(p.am_val + tid * gridDim.x + b);
+      const int i2 = __ldcg(p.am_idx + tid * gridDim.x + b);
+      if (v2 > v || (v2 == v && i2 < i)) v = v2, i = i2;
+    }
+    if (p.argmax_out) p.argmax_out[tid] = i == 0x7fffffff ? 0 : i;
+  }
+  if (s_ticket == (int)gridDim.x - 1 && tid == 0) *p.counter = 0;
+}
+
+template <int KRM>
+cudaError_t launch_f16_t(const GemvParams& p, cudaStream_t st, bool pdl) {
+  const size_t smem = (size_t)KRM * p.k * 2 + 64 * 4 + (size_t)kF16Warps * KRM * 8;
+  constexpr int kMaxDev = 64;  // the attribute is per device: raised once on each
+  static std::atomic<size_t> configured[kMaxDev];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  if (smem > configured[dev].load(std::memory_order_relaxed)) {
+    cudaError_t e = cudaFuncSetAttribute(gemv_f16_kernel<KRM>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured[dev].store(smem, std::memory_order_relaxed);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(device_sm_count());
+  cfg.blockDim = dim3(kF16Threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, gemv_f16_kernel<KRM>, p);
+}
+
+}  // namespace
+
+cudaError_t launch_gemv_f16(const GemvParams& p, cudaStream_t st, bool pdl) {
+  if (p.k % 256 || p.k > 8192 || p.kr < 1 || p.kr > kMaxRows) return cudaErrorInvalidValue;
+  if (p.kr <= 1) return launch_f16_t<1>(p, st, pdl);
+  if (p.kr <= 2) return launch_f16_t<2>(p, st, pdl);
+  if (p.kr <= 4) return launch_f16_t<4>(p, st, pdl);
+  return launch_f16_t<8>(p, st, pdl);
 }
 
 bool set_gemv_kernel_choice(int kind) {

@@ -35,6 +35,7 @@ struct NextGemv {
 struct GemvParams {
   NextGemv next;
   GemvSeg seg[3];
+  const uint16_t* w16;  // fp16 weights [n_rows][k] (launch_gemv_f16 only)
   int32_t nseg;
   int32_t k;        // columns
   int32_t n_rows;   // output rows (STORE / HEAD); the last unit may be partial
@@ -86,6 +87,11 @@ struct GemvParams {
   uint64_t* trace_ends;  // optional [grid]: when each CTA's reducer finished (stage kernel)
   int32_t stall_test;   // 1: the first stage of the warp that owns unit 0 never completes (tests the timeout path)
 };
+
+// GEMV with fp16 weights p.w16 (the fp16 tied head): PRO_RESID or PRO_X16 prologue,
+// EPI_HEAD or EPI_STORE epilogue, up to kMaxRows activation rows, k % 256 == 0 and
+// k <= 8192, w16 and x 16-byte aligned.
+cudaError_t launch_gemv_f16(const GemvParams& p, cudaStream_t st, bool pdl);
 
 // Largest number of activation rows one GEMV launch can stage for k columns.
 int gemv_max_rows(int k);
@@ -244,6 +250,7 @@ struct StepKernelParams {
   uint64_t* trace;     // optional [step_kernel_trace_slots(n_layers)] %globaltimer stamps of CTA 0
   int32_t stall_test;  // 1: CTA 0's first stage expects 16 bytes that never arrive
   uint32_t poll_ns;    // back-off between two polls of a counter or of tagged words
+  int32_t grid_sync;   // 1: every phase also waits for all CTAs to finish the previous one
 };
 // phases per step: 6 per layer (QKV, attention, merge, O, gate|up, down) + head
 int step_kernel_phases(int n_layers);
@@ -272,6 +279,7 @@ struct StepParams {
   const float* hidden;      // [kr][h] replaces the embedding
   const uint8_t* emb_qs;
   const uint16_t* emb_sc;
+  const uint16_t* emb_f16;  // fp16 tied table (if non-NULL, instead of the q4_0 one)
   int32_t hidden_size, vocab;
   float embed_scale;
   float* r_out;             // [kr][h]

@@ -74,10 +74,14 @@ __global__ void step_init_kernel(const StepParams p) {
       int tok = p.ids_dev ? p.ids_dev[j] : p.ids_host[j];
       tok = tok < 0 ? 0 : (tok >= p.vocab ? p.vocab - 1 : tok);
       const size_t row = (size_t)tok;
-      const uint8_t byte = p.emb_qs[row * (p.hidden_size >> 1) + (c >> 5) * 16 + (c & 15)];
-      const int code = (c & 31) < 16 ? (byte & 15) : (byte >> 4);
-      const float d = __half2float(__ushort_as_half(p.emb_sc[row * (p.hidden_size >> 5) + (c >> 5)]));
-      v = __fmul_rn((float)(code - 8) * d, p.embed_scale);
+      if (p.emb_f16) {  // fp16 tied table
+        v = __fmul_rn(__half2float(__ushort_as_half(p.emb_f16[row * p.hidden_size + c])), p.embed_scale);
+      } else {
+        const uint8_t byte = p.emb_qs[row * (p.hidden_size >> 1) + (c >> 5) * 16 + (c & 15)];
+        const int code = (c & 31) < 16 ? (byte & 15) : (byte >> 4);
+        const float d = __half2float(__ushort_as_half(p.emb_sc[row * (p.hidden_size >> 5) + (c >> 5)]));
+        v = __fmul_rn((float)(code - 8) * d, p.embed_scale);
+      }
     }
     p.r_out[(size_t)j * p.hidden_size + c] = v;
     if (p.dump) p.dump[(size_t)j * p.dump_stride + c] = v;

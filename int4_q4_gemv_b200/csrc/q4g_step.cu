@@ -74,6 +74,7 @@ enum : int { PK_QKV = 0, PK_ATT = 1, PK_MRG = 2, PK_O = 3, PK_GU = 4, PK_DN = 5,
 struct SkShared {
   uint64_t full[kSkSlots];   // the stage's bytes landed
   uint64_t ready[kSkSlots];  // every compute warp is done with the stage
+  uint64_t pub;              // grid-count mode: the feeder stored the last outputs of a GEMV phase
   float red[kSkSlots][kSkMaxNC][kSkMaxR];  // GEMV chunk partials per slot
   float norm[2][kSkCompute];
   alignas(16) unsigned char cursor[512];  // the feeder's producer cursor (lane 0 only), a Cursor
@@ -139,9 +140,11 @@ Q4G_DEV void ld_tagged_wait(const uint64_t* p, int stride, int n, uint32_t tag, 
   }
   if (!miss) return;
   const uint64_t t0 = global_ns();
+  uint32_t sleep = P.poll_ns;  // doubling back-off: every CTA's threads poll, keep the L2 traffic low
   for (int it = 0; it < kSpinLimit && miss; ++it) {
     if (*abort_flag) return;
-    __nanosleep(P.poll_ns);
+    __nanosleep(sleep);
+    sleep = min(2 * sleep + 32, 2048u);
 #pragma unroll
     for (int i = 0; i < N; ++i) {
       if (miss & (1u << i)) {
@@ -417,6 +420,11 @@ Q4G_DEV bool sk_wait(uint64_t* bar, uint32_t phase, const StepKernelParams& P, v
   sk_abort(P, abort_flag);
   return false;
 }
+
+// Whether any lane of the warp has seen the CTA give up. Every lane of the warp must
+// call it: it reconverges lanes that waited for different lengths of time, so that
+// a guarded block holding warp collectives is entered by all lanes or by none.
+Q4G_DEV bool warp_aborted(volatile int* abort_flag) { return __any_sync(0xffffffffu, *abort_flag != 0); }
 
 // Thread 0 of the compute warps: wait until every CTA finished phase p.
 Q4G_DEV void wait_phase(const StepKernelParams& P, int p, volatile int* abort_flag) {
@@ -707,11 +715,11 @@ Q4G_DEV void attention_phase(const StepKernelParams& P, const AD& a, int l, SkSh
   const size_t rbytes = (size_t)HD * 2;
   for (int i = 0; i < n_st; ++i, ++T) {
     const int sl = T % kSkSlots;
-    if (!*abort_flag) sk_wait(&s.full[sl], (uint32_t)((T / kSkSlots) & 1), P, abort_flag);
+    if (!warp_aborted(abort_flag)) sk_wait(&s.full[sl], (uint32_t)((T / kSkSlots) & 1), P, abort_flag);
     const int ka = a.k0 + i * a.SK, kb = min(a.k1, ka + a.SK);
     const unsigned char* kbase = ring + (size_t)sl * kSkSlotBytes;
     const unsigned char* vbase = kbase + (size_t)a.SK * rbytes;
-    if (!*abort_flag) {
+    if (!warp_aborted(abort_flag)) {
       for (int j0 = ka + kg; j0 < kb; j0 += NKG * B) {
         float sc[B * RPW];
         bool valid[B];
@@ -970,6 +978,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) step_kernel(const StepKernelPar
   if (tid == 0) {
     s.abort_flag = 0;
     for (int i = 0; i < kSkSlots; ++i) mbar_init(&s.full[i], 1), mbar_init(&s.ready[i], kSkCompute);
+    mbar_init(&s.pub, 1);
     fence_mbar_init();
   }
   for (int i = tid; i < P.rope_pairs_sl; i += kSkThreads) s.rope_sl[i] = P.rope_sl[i];  // written before the launch
@@ -995,7 +1004,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) step_kernel(const StepKernelPar
     int T = 0;
     float best_v = -INFINITY;
     int best_i = 0x7fffffff;
-    for (int p = 0; p < cx.NP && !*abort_flag; ++p) {
+    for (int p = 0; p < cx.NP && !warp_aborted(abort_flag); ++p) {
       const int kind = phase_kind(p, cx.L);
       const int n = phase_stages(P, cx, p);
       GD g{};
@@ -1008,10 +1017,10 @@ __global__ void __launch_bounds__(kSkThreads, 1) step_kernel(const StepKernelPar
       }
       for (int i = 0; i < n; ++i, ++T) {
         const int sl = T % kSkSlots;
-        if (!sk_wait(&s.ready[sl], (uint32_t)((T / kSkSlots) & 1), P, abort_flag)) break;
+        sk_wait(&s.ready[sl], (uint32_t)((T / kSkSlots) & 1), P, abort_flag);  // a timeout sets the flag
         // compute warps that gave up still hand their slots back without having seen the
         // slot's fill complete: never refill such a slot (its barrier phase may be pending)
-        if (*abort_flag) break;
+        if (warp_aborted(abort_flag)) break;
         float val = 0.f;
         if (gemv && lane < g.R)
           for (int c = 0; c < g.NC; ++c) val += s.red[sl][c][lane];
@@ -1045,11 +1054,19 @@ __global__ void __launch_bounds__(kSkThreads, 1) step_kernel(const StepKernelPar
           }
         }
       }
-      if (*abort_flag) break;
-      if (trace && lane == 0 && gemv && n > 0) trace[4 * p + 3] = global_ns();
+      if (warp_aborted(abort_flag)) break;
+      if (gemv && n > 0) {
+        __syncwarp();
+        if (lane == 0) {
+          // grid-count mode: the compute warps count this CTA in on the way to the next
+          // phase (a fence there, not here: the feeder keeps streaming)
+          if (P.grid_sync) mbar_arrive(&s.pub);  // release of this warp's epilogue stores
+          if (trace) trace[4 * p + 3] = global_ns();
+        }
+      }
     }
     // head: per-CTA candidate, the last CTA picks the winner (lowest index on ties)
-    if (!*abort_flag) {
+    if (!warp_aborted(abort_flag)) {
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
         const float v2 = __shfl_xor_sync(0xffffffffu, best_v, o);
@@ -1084,16 +1101,34 @@ __global__ void __launch_bounds__(kSkThreads, 1) step_kernel(const StepKernelPar
   }
 
   // =================== compute warps ===================
-  // A phase starts as soon as this CTA is done with the previous one: its inputs
-  // are tagged words polled as they arrive. The only grid-wide wait is before the
-  // merge of a full-attention layer, which reads every CTA's partials.
+  // Tagged mode: a phase starts as soon as this CTA is done with the previous one;
+  // its inputs are tagged words polled as they arrive, and the only grid-wide wait
+  // is before the merge of a full-attention layer, which reads every CTA's
+  // partials. Grid-count mode: every phase starts once every CTA has counted
+  // itself done with the previous phase (the tagged reads then succeed at once).
   int T = 0;
+  uint32_t pubs = 0;     // completed phases of s.pub
+  bool publish = false;  // grid-count mode: the previous phase streamed GEMV stages here
+  int prev = -1;         // the previous phase this CTA ran
   for (int p = 0; p < cx.NP; ++p) {
     const int kind = phase_kind(p, cx.L);
     // sliding layers: the last CTA of each KV head merges the head's chunks inside
     // the attention phase, so there is no separate merge phase
     if (kind == PK_MRG && !P.layers[p / 6].full) continue;
     uint64_t* tr = trace ? trace + 4 * p : nullptr;
+    if (P.grid_sync && prev >= 0) {
+      if (tid == 0) {
+        if (publish) {  // the feeder's epilogue of the previous phase is done: count this CTA in
+          if (!*abort_flag) sk_wait(&s.pub, pubs & 1, P, abort_flag);
+          ++pubs;
+          signal_phase(P, prev);
+        }
+        wait_phase(P, prev, abort_flag);
+      }
+      compute_bar();  // every compute thread after thread 0's acquire
+    }
+    publish = false;
+    prev = p;
     if (tr && tid == 0) tr[0] = global_ns();
     if (kind == PK_ATT) {
       const int l = p / 6;
@@ -1115,7 +1150,11 @@ __global__ void __launch_bounds__(kSkThreads, 1) step_kernel(const StepKernelPar
           s.last = last;
         }
         compute_bar();
-        if (s.last && !*abort_flag) merge_head(P, a.hd, a.G, a.kv, a.nch, tag_of(cx.epoch, l + 1));
+        if (!warp_aborted(abort_flag) && s.last) merge_head(P, a.hd, a.G, a.kv, a.nch, tag_of(cx.epoch, l + 1));
+        if (P.grid_sync) {
+          compute_bar();
+          if (tid == 0) signal_phase(P, p);
+        }
       } else if (tid == 0) {
         signal_phase(P, p);  // the full layer's merge reads every CTA's partials
       }
@@ -1123,9 +1162,15 @@ __global__ void __launch_bounds__(kSkThreads, 1) step_kernel(const StepKernelPar
       continue;
     }
     if (kind == PK_MRG) {  // full layers
-      if (tid == 0) wait_phase(P, p - 1, abort_flag);
-      compute_bar();  // every compute thread after thread 0's acquire
-      if (!*abort_flag) merge_phase(P, p / 6, tag_of(cx.epoch, p / 6 + 1));
+      if (!P.grid_sync) {
+        if (tid == 0) wait_phase(P, p - 1, abort_flag);
+        compute_bar();  // every compute thread after thread 0's acquire
+      }
+      if (!warp_aborted(abort_flag)) merge_phase(P, p / 6, tag_of(cx.epoch, p / 6 + 1));
+      if (P.grid_sync) {
+        compute_bar();
+        if (tid == 0) signal_phase(P, p);
+      }
       if (tr && tid == 0) tr[2] = global_ns();
       continue;
     }
@@ -1139,7 +1184,11 @@ __global__ void __launch_bounds__(kSkThreads, 1) step_kernel(const StepKernelPar
       resid_gains(g, gains);
       resid_prologue(g, P, s, gains, abort_flag);  // ends with a compute barrier
     }
-    if (n == 0) continue;
+    if (n == 0) {
+      if (P.grid_sync && tid == 0) signal_phase(P, p);
+      continue;
+    }
+    publish = P.grid_sync != 0;
     const int nb = g.k >> 5, kh = g.k >> 1, c = warp % g.NC, grp = warp / g.NC;
     const int blk = 32 * c + lane;
     const bool act = warp < g.NC * g.G;
@@ -1171,8 +1220,8 @@ __global__ void __launch_bounds__(kSkThreads, 1) step_kernel(const StepKernelPar
     const int bq = min(blk, nb - 1);
     for (int i = 0; i < n; ++i, ++T) {
       const int sl = T % kSkSlots;
-      if (!*abort_flag) sk_wait(&s.full[sl], (uint32_t)((T / kSkSlots) & 1), P, abort_flag);
-      if (act && !*abort_flag) {
+      if (!warp_aborted(abort_flag)) sk_wait(&s.full[sl], (uint32_t)((T / kSkSlots) & 1), P, abort_flag);
+      if (!warp_aborted(abort_flag) && act) {
         const unsigned char* st = ring + (size_t)sl * kSkSlotBytes;
         const unsigned char* sq = st + (size_t)grp * 4 * kh + 16 * bq;
         const unsigned char* ss = st + (size_t)g.R * kh + (size_t)grp * 4 * 2 * nb + 2 * bq;

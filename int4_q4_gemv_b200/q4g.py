@@ -19,12 +19,13 @@ Q4G_OPT_GEMV_CHAIN = 7
 Q4G_OPT_TRACE = 8
 Q4G_OPT_STEP_KERNEL = 9
 Q4G_OPT_STEP_POLL_NS = 10
+Q4G_OPT_STEP_GRID_SYNC = 11
 KIND_NAMES = ["step_init", "qkv_gemv", "attn_sliding", "attn_full", "attn_combine", "o_gemv",
               "gate_up_gemv", "down_gemv", "head_gemv", "chain_gemv", "step_kernel"]
 
 EXPORTS = [
     "q4g_last_error", "q4g_status_string", "q4g_abi_version",
-    "q4g_q4_0_pack", "q4g_q4_0_unpack", "q4g_gemv",
+    "q4g_q4_0_pack", "q4g_q4_0_unpack", "q4g_gemv", "q4g_gemv_f16",
     "q4g_flash_decode_workspace_bytes", "q4g_flash_decode_ring", "q4g_flash_decode_linear",
     "q4g_model_create", "q4g_model_destroy", "q4g_model_check", "q4g_model_set_option",
     "q4g_cache_bytes", "q4g_cache_init", "q4g_cache_reset", "q4g_cache_destroy", "q4g_cache_layout",
@@ -46,7 +47,7 @@ class q4g_config(C.Structure):
         "n_layers", "hidden", "n_q_heads", "ffn", "vocab", "sl_kv_heads", "sl_head_dim", "window",
         "ring", "gl_kv_heads", "gl_head_dim", "full_every", "full_offset", "rope_pairs_full")] + \
         [(n, C.c_float) for n in ("rope_theta_sl", "rope_theta_gl", "rms_eps", "softcap",
-                                  "embed_scale")] + [("v_norm_sliding", C.c_int32)]
+                                  "embed_scale")] + [("v_norm_sliding", C.c_int32), ("head_fp16", C.c_int32)]
 
 
 class q4g_qtensor(C.Structure):
@@ -61,7 +62,7 @@ class q4g_layer_weights(C.Structure):
 
 class q4g_weights(C.Structure):
     _fields_ = [("layers", C.POINTER(q4g_layer_weights)), ("embed", q4g_qtensor),
-                ("norm_final", C.c_void_p)]
+                ("norm_final", C.c_void_p), ("embed_f16", C.c_void_p)]
 
 
 class q4g_launch_record(C.Structure):
@@ -95,6 +96,7 @@ def lib() -> C.CDLL:
             "q4g_q4_0_pack": (C.c_int, [vp, i64, i64, vp, vp, C.c_int, vp]),
             "q4g_q4_0_unpack": (C.c_int, [vp, vp, i64, i64, vp, C.c_int, vp]),
             "q4g_gemv": (C.c_int, [vp, vp, i64, i64, vp, i32, vp, vp]),
+            "q4g_gemv_f16": (C.c_int, [vp, i64, i64, vp, i32, vp, vp]),
             "q4g_flash_decode_workspace_bytes": (sz, [i32, i32]),
             "q4g_flash_decode_ring": (C.c_int, [vp, i32, i32, i32, vp, vp, i64, i64, i64, vp, vp, sz, vp]),
             "q4g_flash_decode_linear": (C.c_int, [vp, i32, i32, i32, vp, vp, i64, vp, vp, sz, vp]),
@@ -151,6 +153,10 @@ def q4g_q4_0_unpack(qs, scales, rows, k, w, on_device, stream):
 
 def q4g_gemv(qs, scales, n, k, x_f16, nrhs, y, stream):
     _call("q4g_gemv", qs, scales, n, k, x_f16, nrhs, y, stream)
+
+
+def q4g_gemv_f16(w16, n, k, x_f16, nrhs, y, stream):
+    _call("q4g_gemv_f16", w16, n, k, x_f16, nrhs, y, stream)
 
 
 Q4G_GEMV_AUTO, Q4G_GEMV_COLUMN_SPLIT, Q4G_GEMV_WARP_STREAM, Q4G_GEMV_REGISTER, Q4G_GEMV_STAGE = 0, 1, 2, 3, 4

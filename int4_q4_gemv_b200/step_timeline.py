@@ -60,9 +60,13 @@ def main() -> None:
     ap.add_argument("--steps", type=int, default=3)
     ap.add_argument("--json", action="store_true")
     ap.add_argument("--poll-ns", type=int, default=None, help="Q4G_OPT_STEP_POLL_NS (default: the library's)")
+    ap.add_argument("--grid-sync", type=int, choices=[0, 1], default=None,
+                    help="Q4G_OPT_STEP_GRID_SYNC (default: the library's)")
     a = ap.parse_args()
     cfg = dict(WL.B12, n_layers=a.layers)
-    g = S.SynthDecoder(cfg, seed=0)
+    g = S.SynthDecoder(cfg, seed=0, step_kernel=1)
+    if a.grid_sync is not None:
+        Q.q4g_model_set_option(g.handle, Q.Q4G_OPT_STEP_GRID_SYNC, a.grid_sync)
     if a.poll_ns is not None:
         Q.q4g_model_set_option(g.handle, Q.Q4G_OPT_STEP_POLL_NS, a.poll_ns)
     c = g.new_cache(a.context)

@@ -23,7 +23,7 @@ class OrConfig(C.Structure):
         "sl_kv_heads", "sl_head_dim", "window", "ring",
         "gl_kv_heads", "gl_head_dim", "full_every", "full_offset", "rope_pairs_full")] + \
         [(n, C.c_double) for n in ("rope_theta_sl", "rope_theta_gl", "rms_eps", "softcap",
-                                   "embed_scale")] + [("v_norm_sliding", C.c_int32)]
+                                   "embed_scale")] + [("v_norm_sliding", C.c_int32), ("head_fp16", C.c_int32)]
 
 
 def _p(a):
@@ -44,6 +44,8 @@ def lib():
             "or_q4_0_pack": (C.c_int, [vp, i64, i64, vp, vp]),
             "or_q4_0_unpack": (None, [vp, vp, i64, i64, vp]),
             "or_gemv": (None, [vp, vp, i64, i64, C.c_int, vp, vp]),
+            "or_gemv_f16": (None, [vp, i64, i64, C.c_int, vp, vp]),
+            "or_model_embed_f16": (vp, [vp]),
             "or_rmsnorm": (None, [vp, vp, i64, dbl, vp]),
             "or_rope": (None, [vp, i64, i64, dbl, i64]),
             "or_gelu_tanh": (dbl, [dbl]),
@@ -131,6 +133,17 @@ def gemv(qs, sc, x16):
     return y[0] if x16.ndim == 1 else y
 
 
+def gemv_f16(w16, x16):
+    """y = W @ x for fp16 weights W [n][k] and x as fp16 bits, shape [k] or [nrhs, k]."""
+    w16 = np.ascontiguousarray(w16, dtype=np.uint16)
+    x16 = np.ascontiguousarray(x16, dtype=np.uint16)
+    n, k = w16.shape
+    nrhs = 1 if x16.ndim == 1 else x16.shape[0]
+    y = np.empty((nrhs, n), dtype=np.float64)
+    lib().or_gemv_f16(_p(w16), n, k, nrhs, _p(x16), _p(y))
+    return y[0] if x16.ndim == 1 else y
+
+
 # ------------------------------------------------------------ elementwise --
 
 def rmsnorm(x, w=None, eps=1e-6):
@@ -215,6 +228,14 @@ class Model:
         q = np.ctypeslib.as_array(C.cast(qs, C.POINTER(C.c_uint8)), shape=(rows, k // 2)).copy()
         s = np.ctypeslib.as_array(C.cast(sc, C.POINTER(C.c_uint16)), shape=(rows, k // 32)).copy()
         return q, s
+
+    def embed_f16(self):
+        """The fp16 tied table (copy) when cfg["head_fp16"], else None."""
+        ptr = lib().or_model_embed_f16(self.h)
+        if not ptr:
+            return None
+        V, H = self.cfg["vocab"], self.cfg["hidden"]
+        return np.ctypeslib.as_array(C.cast(ptr, C.POINTER(C.c_uint16)), shape=(V, H)).copy()
 
     def close(self):
         if self.h:

@@ -160,6 +160,25 @@ void or_gemv(const uint8_t* qs, const uint16_t* scales, int64_t n, int64_t k, in
   free(xd);
 }
 
+/* y[n] = sum_k W[n][k] * x[k] for fp16 weights W (the fp16 tied head of
+ * [12b] "tiered-v3/": the bf16 -> fp16 cast of the table is exact, so the head
+ * reads the table's own values); x as fp16 bits; natural k order. */
+void or_gemv_f16(const uint16_t* w, int64_t n, int64_t k, int nrhs, const uint16_t* x16, double* y) {
+  double* xd = (double*)malloc(sizeof(double) * (size_t)(k * nrhs));
+  for (int64_t i = 0; i < k * nrhs; ++i) xd[i] = or_f16_to_double(x16[i]);
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < n; ++r) {
+    const uint16_t* row = w + r * k;
+    for (int j = 0; j < nrhs; ++j) {
+      const double* x = xd + (int64_t)j * k;
+      double acc = 0.0;
+      for (int64_t col = 0; col < k; ++col) acc += or_f16_to_double(row[col]) * x[col];
+      y[(int64_t)j * n + r] = acc;
+    }
+  }
+  free(xd);
+}
+
 /* ------------------------------------------------------------------------- */
 /* Elementwise pieces.                                                        */
 /* ------------------------------------------------------------------------- */
@@ -303,7 +322,8 @@ typedef struct {
 struct or_model {
   or_config cfg;
   layer_t* L;
-  qmat embed;
+  qmat embed;        /* q4_0 tied table (head_fp16 = 0) */
+  uint16_t* embed16; /* fp16 tied table [vocab][h] (head_fp16 = 1) */
   double* n_final;
   int n_sl, n_gl;
 };
@@ -392,7 +412,18 @@ or_model* or_model_create(const or_config* cfg, uint64_t seed, int variant, int 
                                                     0, 0.5f, 1.5f)
                          : 1.0;
   }
-  if (make_qmat(&m->embed, seed, DG_STREAM_EMBED, cfg->vocab, H)) {
+  if (cfg->head_fp16) {
+    /* the same N(0, 0.02) draws as the q4_0 table, kept at fp16 */
+    m->embed16 = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)cfg->vocab * (size_t)H);
+    if (!m->embed16) {
+      or_model_destroy(m);
+      return NULL;
+    }
+    uint64_t key = dg_key(seed, DG_STREAM_EMBED);
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < (int64_t)cfg->vocab * H; ++i)
+      m->embed16[i] = or_f16_from_double((double)dg_normal(key, (uint64_t)i, 0.02f));
+  } else if (make_qmat(&m->embed, seed, DG_STREAM_EMBED, cfg->vocab, H)) {
     or_model_destroy(m);
     return NULL;
   }
@@ -415,6 +446,7 @@ void or_model_destroy(or_model* m) {
   }
   free(m->L);
   free_qmat(&m->embed);
+  free(m->embed16);
   free(m->n_final);
   free(m);
 }
@@ -435,6 +467,8 @@ int64_t or_model_tensor(const or_model* m, int layer, int tensor, const uint8_t*
   *cols = q->cols;
   return q->rows;
 }
+
+const uint16_t* or_model_embed_f16(const or_model* m) { return m->embed16; }
 
 or_cache* or_cache_create(const or_model* m, int64_t capacity, int64_t ring_slots) {
   const or_config* c = &m->cfg;
@@ -539,10 +573,15 @@ int or_verify_block(or_model* m, or_cache* c, const int32_t* ids, const float* h
   for (int i = 0; i < K; ++i) {
     if (ids) {
       int64_t tok = ids[i];
-      const uint8_t* row = m->embed.qs + tok * (H / 2);
-      for (int64_t col = 0; col < H; ++col)
-        r[i * H + col] = (double)(code_at(row, col) - 8) *
-                         or_f16_to_double(m->embed.sc[tok * (H / 32) + col / 32]) * cfg->embed_scale;
+      if (cfg->head_fp16) {
+        for (int64_t col = 0; col < H; ++col)
+          r[i * H + col] = or_f16_to_double(m->embed16[tok * H + col]) * cfg->embed_scale;
+      } else {
+        const uint8_t* row = m->embed.qs + tok * (H / 2);
+        for (int64_t col = 0; col < H; ++col)
+          r[i * H + col] = (double)(code_at(row, col) - 8) *
+                           or_f16_to_double(m->embed.sc[tok * (H / 32) + col / 32]) * cfg->embed_scale;
+      }
     } else {
       for (int64_t col = 0; col < H; ++col) r[i * H + col] = (double)hidden_in[i * H + col];
     }
@@ -694,7 +733,10 @@ int or_verify_block(or_model* m, or_cache* c, const int32_t* ids, const float* h
     to_f16(tmp, H, x16 + i * H);
   }
   double* lg = (double*)malloc(sizeof(double) * (size_t)(K * V));
-  or_gemv(m->embed.qs, m->embed.sc, V, H, K, x16, lg);
+  if (cfg->head_fp16)
+    or_gemv_f16(m->embed16, V, H, K, x16, lg);
+  else
+    or_gemv(m->embed.qs, m->embed.sc, V, H, K, x16, lg);
   for (int i = 0; i < K; ++i) {
     int32_t best = 0;
     float bv = -INFINITY;

@@ -34,6 +34,7 @@ typedef struct {
   int32_t gl_kv_heads, gl_head_dim, full_every, full_offset, rope_pairs_full;
   double rope_theta_sl, rope_theta_gl, rms_eps, softcap, embed_scale;
   int32_t v_norm_sliding; /* 1: scale-free RMSNorm on sliding-layer V too */
+  int32_t head_fp16;      /* 1: the tied embedding / head is fp16 instead of q4_0 */
 } or_config;
 
 /* ---- IEEE binary16 ---- */
@@ -54,6 +55,9 @@ void or_q4_0_unpack(const uint8_t* qs, const uint16_t* scales, int64_t rows, int
 /* y[n] = sum_k dequant(W)[n][k] * x[k]; x as fp16 bits; natural k order. */
 void or_gemv(const uint8_t* qs, const uint16_t* scales, int64_t n, int64_t k, int nrhs,
              const uint16_t* x16, double* y);
+
+/* y[n] = sum_k W[n][k] * x[k] for fp16 weights W [n][k]; x as fp16 bits. */
+void or_gemv_f16(const uint16_t* w, int64_t n, int64_t k, int nrhs, const uint16_t* x16, double* y);
 
 /* ---- elementwise pieces (double) ---- */
 void or_rmsnorm(const double* x, const double* w /* NULL = scale-free */, int64_t n, double eps,
@@ -94,6 +98,10 @@ void or_model_destroy(or_model* m);
  * tensor: 0 wq, 1 wk, 2 wv, 3 wo, 4 wgate, 5 wup, 6 wdown, 100 embed. Returns rows (0 if absent). */
 int64_t or_model_tensor(const or_model* m, int layer, int tensor, const uint8_t** qs,
                         const uint16_t** scales, int64_t* cols);
+
+/* The fp16 tied table [vocab][h] when cfg.head_fp16 (NULL otherwise): fp16 of the
+ * same seeded N(0, 0.02) draws the q4_0 table is packed from. */
+const uint16_t* or_model_embed_f16(const or_model* m);
 
 or_cache* or_cache_create(const or_model* m, int64_t capacity, int64_t ring_slots /* 0: cfg.ring */);
 void or_cache_destroy(or_cache* c);

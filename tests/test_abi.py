@@ -40,7 +40,9 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert Q.q4g_abi_version() == 1
+    # version 2: q4g_config.head_fp16 and q4g_weights.embed_f16 (the fp16 tied head)
+    assert Q.q4g_abi_version() == 2
+    assert C.sizeof(Q.q4g_config) == 21 * 4 and C.sizeof(Q.q4g_weights) == 8 + 16 + 8 + 8
     assert lib.q4g_status_string(Q.Q4G_ERANGE) == b"Q4G_ERANGE"
 
 

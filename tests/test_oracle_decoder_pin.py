@@ -7,7 +7,7 @@ but every operation is a torch library call: rms_norm, complex-exponential
 rotation for RoPE, scaled_dot_product_attention over the linear history with an
 explicit window mask, gelu(approximate="tanh"), tanh. fp16 storage points use
 numpy's float16 conversion. Weights come from the oracle's (separately
-pinned) q4_0 unpack.
+pinned) q4_0 unpack; the fp16 tied table from the seeded draws rounded by numpy.
 """
 from __future__ import annotations
 
@@ -64,7 +64,12 @@ class TorchDecoder:
                 n_q=torch.from_numpy(DG.qk_gain(seed, s(DG.T_NORM_Q), hd, variant).astype(np.float64)),
                 n_k=torch.from_numpy(DG.qk_gain(seed, s(DG.T_NORM_K), hd, variant).astype(np.float64)),
                 scal=scal))
-        self.embed = torch.from_numpy(O.q4_0_unpack(*om.tensor(-1, 100)))
+        if cfg.get("head_fp16"):  # the N(0, 0.02) draws rounded to fp16 by numpy
+            V, H = cfg["vocab"], cfg["hidden"]
+            e = DG.normal(seed, DG.STREAM_EMBED, V * H, 0.02).astype(np.float16)
+            self.embed = torch.from_numpy(e.astype(np.float64).reshape(V, H))
+        else:
+            self.embed = torch.from_numpy(O.q4_0_unpack(*om.tensor(-1, 100)))
         self.n_final = gain(DG.STREAM_FINAL_NORM, cfg["hidden"])
         self.K = [[] for _ in range(L)]   # linear history of fp16 K per layer
         self.V = [[] for _ in range(L)]
@@ -104,11 +109,11 @@ class TorchDecoder:
         return torch.tanh((self.embed @ z) / c["softcap"]) * c["softcap"]
 
 
-@pytest.mark.parametrize("variant", [1, 2])
-def test_oracle_decoder_matches_torch_composition(variant):
+@pytest.mark.parametrize("variant,head_fp16", [(1, 0), (2, 0), (1, 1)])
+def test_oracle_decoder_matches_torch_composition(variant, head_fp16):
     """Variant 1: seeded gains and layer scalars; variant 2: unit q/k gains (a sharp
-    softmax, logits of order head_dim)."""
-    cfg = dict(WL.MICRO)
+    softmax, logits of order head_dim); head_fp16: the fp16 tied embedding / head."""
+    cfg = dict(WL.MICRO, head_fp16=head_fp16)
     seed, steps = 4, 40                      # 40 steps > 2 ring wraps at R = 16
     om = O.Model(cfg, seed=seed, variant=variant)
     cache = O.Cache(om, 64)
