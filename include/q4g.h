@@ -120,9 +120,9 @@ q4g_status q4g_gemv_f16(const uint16_t* w16, int64_t n, int64_t k, const uint16_
  *   Q4G_GEMV_REGISTER      plain streaming loads (any k % 32 == 0),
  *   Q4G_GEMV_STAGE         integer dot, every warp of a CTA on each 16-36 KB
  *                          stage of one contiguous bulk-copy stream, one warp
- *                          reducing and refilling (k % 256 == 0, <= 2
+ *                          reducing and refilling (k % 256 == 0, <= 4
  *                          activation rows, 16-byte aligned operands).
- * A kernel that cannot take a call falls back down this list (STAGE to AUTO). Affects launches
+ * A kernel that cannot take a call falls back to the automatic choice. Affects launches
  * made (and CUDA graphs captured) after the call. Q4G_EINVAL for other kinds. */
 #define Q4G_GEMV_AUTO 0
 #define Q4G_GEMV_COLUMN_SPLIT 1

@@ -1359,8 +1359,8 @@ __global__ void __launch_bounds__(kStageThreads, 1) gemv_q4_stage_kernel(const G
   uint64_t* ready = bars + kStageMaxSlots;  // [kStageMaxSlots]: every compute warp wrote its partials
   unsigned char* stages = reinterpret_cast<unsigned char*>(bars + 2 * kStageMaxSlots);
   __shared__ int s_abort, s_ticket;
-  __shared__ float s_bestv;
-  __shared__ int s_besti;
+  __shared__ float s_bestv[KRM];
+  __shared__ int s_besti[KRM];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_comp = NC * G;
@@ -1462,9 +1462,9 @@ __global__ void __launch_bounds__(kStageThreads, 1) gemv_q4_stage_kernel(const G
       // all own loads issued: start the next GEMV's weights towards L2
       if (issued == n_st) prefetch_next(p.next, blockIdx.x, gridDim.x);
     }
-    float best_v = -INFINITY;
+    float best_v = -INFINITY;  // of activation row j (head)
     int best_i = 0x7fffffff;
-    const int r = lane / KRM, j = lane % KRM;  // lanes l < R * KRM
+    const int r = lane / KRM, j = lane % KRM;  // lanes l < R * KRM <= 32
     int s = 0;
     uint32_t ph = 0;
     for (int t = 0; t < n_st; ++t) {
@@ -1506,32 +1506,35 @@ __global__ void __launch_bounds__(kStageThreads, 1) gemv_q4_stage_kernel(const G
     if (lane == 0) stamp(5);
     if (lane == 0 && p.trace_ends) p.trace_ends[blockIdx.x] = global_ns();
     if (p.epi == EPI_HEAD) {
+      // lanes with the same j (lane % KRM) hold row j's candidates
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
+      for (int o = 16; o >= KRM; o >>= 1) {
         const float v2 = __shfl_xor_sync(0xffffffffu, best_v, o);
         const int i2 = __shfl_xor_sync(0xffffffffu, best_i, o);
         if (v2 > best_v || (v2 == best_v && i2 < best_i)) best_v = v2, best_i = i2;
       }
-      if (lane == 0) s_bestv = best_v, s_besti = best_i;
+      if (lane < KRM) s_bestv[lane] = best_v, s_besti[lane] = best_i;
     }
   }
   if (p.epi == EPI_HEAD) {
     __syncthreads();
     if (tid == 0) {
-      p.am_val[blockIdx.x] = s_bestv;
-      p.am_idx[blockIdx.x] = s_besti;
+      for (int jj = 0; jj < p.kr; ++jj)
+        p.am_val[jj * gridDim.x + blockIdx.x] = s_bestv[jj], p.am_idx[jj * gridDim.x + blockIdx.x] = s_besti[jj];
       __threadfence();
       s_ticket = atomicAdd(p.counter, 1);
       if (s_ticket == (int)gridDim.x - 1) {
         __threadfence();
-        float v = -INFINITY;
-        int ix = 0x7fffffff;
-        for (int b = 0; b < (int)gridDim.x; ++b) {
-          const float vb = __ldcg(p.am_val + b);
-          const int ib = __ldcg(p.am_idx + b);
-          if (vb > v || (vb == v && ib < ix)) v = vb, ix = ib;
+        for (int jj = 0; jj < p.kr; ++jj) {
+          float v = -INFINITY;
+          int ix = 0x7fffffff;
+          for (int b = 0; b < (int)gridDim.x; ++b) {
+            const float vb = __ldcg(p.am_val + jj * gridDim.x + b);
+            const int ib = __ldcg(p.am_idx + jj * gridDim.x + b);
+            if (vb > v || (vb == v && ib < ix)) v = vb, ix = ib;
+          }
+          if (p.argmax_out) p.argmax_out[jj] = ix == 0x7fffffff ? 0 : ix;
         }
-        if (p.argmax_out) p.argmax_out[0] = ix == 0x7fffffff ? 0 : ix;
         *p.counter = 0;
       }
     }
@@ -1547,8 +1550,7 @@ __global__ void __launch_bounds__(kStageThreads, 1) gemv_q4_stage_kernel(const G
 // chunks, G row groups of RG rows, NS slots within the shared-memory budget.
 bool plan_stage(GemvParams& p, int& R, int& RG, bool forced) {
   const int k = p.k, nb = k >> 5;
-  if (k % 256 != 0 || p.kr > 2) return false;
-  if (p.epi == EPI_HEAD && p.kr != 1) return false;
+  if (k % 256 != 0 || p.kr > 4) return false;
   if (p.epi == EPI_GEGLU && (p.nseg != 2 || p.seg[0].rows != p.seg[1].rows || p.seg[0].rows % 8)) return false;
   if (p.pro == PRO_RESID && k > 8192) return false;
   for (int s = 0; s < p.nseg; ++s)
@@ -1558,7 +1560,7 @@ bool plan_stage(GemvParams& p, int& R, int& RG, bool forced) {
   (void)forced;
   const int NC = (nb + 31) / 32;
   if (NC > kStageCompute) return false;
-  const int krm = p.kr <= 1 ? 1 : 2;
+  const int krm = p.kr <= 1 ? 1 : p.kr <= 2 ? 2 : 4;
   const size_t row_bytes = (size_t)k / 2 + (size_t)k / 16;
   // Q4G_STAGE_ROWS (2, 4, 8, 16) forces the stage rows: a tuning switch
   static const int rows_env = getenv("Q4G_STAGE_ROWS") ? atoi(getenv("Q4G_STAGE_ROWS")) : 0;
@@ -1566,9 +1568,18 @@ bool plan_stage(GemvParams& p, int& R, int& RG, bool forced) {
   while (R > 2 && (size_t)R * row_bytes > 36 * 1024) R /= 2;
   if (rows_env == 2 || rows_env == 4 || rows_env == 8 || rows_env == 16) R = rows_env;
   if (p.epi == EPI_GEGLU) R = std::max(R, 4);
+  while (R * krm > 32) R /= 2;  // one reducer lane per (row, activation row)
   auto units = [&](int r) { return p.epi == EPI_GEGLU ? p.seg[0].rows / (r / 2) : (p.n_rows + r - 1) / r; };
   // keep every SM busy on small matrices
   while (R > 4 && units(R) < 2 * device_sm_count()) R /= 2;
+  // four activation rows: two rows per compute warp (the x digits of four rows
+  // take most of a lane's registers), so R <= 2 * (compute warps per chunk)
+  if (krm == 4) {
+    int gmax = kStageCompute / NC;
+    while (gmax & (gmax - 1)) --gmax;
+    while (R > 2 && R / 2 > gmax) R /= 2;
+    if (p.epi == EPI_GEGLU && R < 4) return false;
+  }
   int G = std::min(kStageCompute / NC, R == 16 ? 4 : R / 2);
   while (G > 1 && (G & (G - 1))) --G;  // power of two, divides R
   RG = R / G;
@@ -1627,10 +1638,17 @@ cudaError_t launch_stage_r(const GemvParams& p, cudaStream_t st, bool pdl) {
 
 template <int KRM>
 cudaError_t launch_stage_t(const GemvParams& p, int R, int RG, cudaStream_t st, bool pdl) {
-  if (R == 16) return launch_stage_r<KRM, 16, 4>(p, st, pdl);
-  if (R == 8) return RG == 4 ? launch_stage_r<KRM, 8, 4>(p, st, pdl) : launch_stage_r<KRM, 8, 2>(p, st, pdl);
-  if (R == 4) return RG == 4 ? launch_stage_r<KRM, 4, 4>(p, st, pdl) : launch_stage_r<KRM, 4, 2>(p, st, pdl);
-  return launch_stage_r<KRM, 2, 2>(p, st, pdl);
+  if constexpr (KRM == 4) {  // two rows per compute warp (plan_stage)
+    if (RG != 2 || R > 8) return cudaErrorInvalidValue;
+    if (R == 8) return launch_stage_r<4, 8, 2>(p, st, pdl);
+    if (R == 4) return launch_stage_r<4, 4, 2>(p, st, pdl);
+    return launch_stage_r<4, 2, 2>(p, st, pdl);
+  } else {
+    if (R == 16) return launch_stage_r<KRM, 16, 4>(p, st, pdl);
+    if (R == 8) return RG == 4 ? launch_stage_r<KRM, 8, 4>(p, st, pdl) : launch_stage_r<KRM, 8, 2>(p, st, pdl);
+    if (R == 4) return RG == 4 ? launch_stage_r<KRM, 4, 4>(p, st, pdl) : launch_stage_r<KRM, 4, 2>(p, st, pdl);
+    return launch_stage_r<KRM, 2, 2>(p, st, pdl);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -2107,6 +2125,7 @@ cudaError_t launch_gemv(const GemvParams& p_in, cudaStream_t st, bool pdl) {
     if (!p.err) p.err = device_error_word();
     if (!p.err) return cudaErrorInvalidValue;
     if (!p.wait_ns) p.wait_ns = 2000000000ull;
+    if (p.kr > 2) return launch_stage_t<4>(p, R, RG, st, pdl);
     return p.kr > 1 ? launch_stage_t<2>(p, R, RG, st, pdl) : launch_stage_t<1>(p, R, RG, st, pdl);
   }
   p = p_in;

@@ -205,9 +205,12 @@ def test_verify_single_pass_vs_oracle_two_pass(K):
         r = O.verify_block(p.orc, p.oc, pos, ids=ids[b], accepted=0, mode=0)
         O.verify_block(p.orc, p.oc, pos, ids=ids[b], accepted=n, mode=0, want_logits=False)
         torch.cuda.synchronize()
-        got = logits.cpu().numpy().astype(np.float64)
+        got32 = logits.cpu().numpy()
+        got = got32.astype(np.float64)
+        amh = am.cpu().numpy()
         for i in range(K):
             check_logits(got[i], r["logits"][i], f"block {b} row {i}")
+            assert amh[i] == int(np.argmax(got32[i])), f"block {b} row {i}: argmax output"
         pos += n
 
 
