@@ -92,10 +92,7 @@ def config_struct(cfg: dict) -> Q.q4g_config:
 class SynthDecoder:
     """The seeded synthetic decoder as a libq4g model (weights borrowed from torch)."""
 
-    def __init__(self, cfg: dict, seed: int = 0, variant: int = 0, device: str = "cuda",
-                 step_kernel: int | None = None):
-        """step_kernel: None keeps the library's default decode path; 1 / 0 selects the
-        persistent step kernel or one launch per kernel (Q4G_OPT_STEP_KERNEL)."""
+    def __init__(self, cfg: dict, seed: int = 0, variant: int = 0, device: str = "cuda"):
         self.cfg = dict(cfg)
         self.seed, self.variant, self.device = seed, variant, device
         c = self.cfg
@@ -158,8 +155,6 @@ class SynthDecoder:
         self._cfg_struct = config_struct(c)
         torch.cuda.synchronize()
         self.handle = Q.q4g_model_create(self._cfg_struct, self._w)
-        if step_kernel is not None:
-            Q.q4g_model_set_option(self.handle, Q.Q4G_OPT_STEP_KERNEL, int(step_kernel))
 
     def tensor(self, layer: int, name: str):
         """(qs, scales) torch tensors of one weight tensor (for byte comparisons)."""

@@ -109,13 +109,8 @@ q4g_status q4g_gemv_f16(const uint16_t* w16, int64_t n, int64_t k, const uint16_
 /* Process-wide choice of the q4_0 GEMV kernel, for tuning and tests (not on
  * the pages). All kernels compute the same operation within the same error
  * bound; the default picks per shape:
- *   Q4G_GEMV_AUTO          the stage kernel where it can take the call, else a
- *                          shape-based choice among the next three (default;
- *                          Q4G_GEMV_KERNEL=cs|ws|reg|stage in the environment
- *                          overrides it at first use),
- *   Q4G_GEMV_COLUMN_SPLIT  integer dot, x digits resident per chunk, one
- *                          contiguous bulk-copy stream per CTA (k % 256 == 0,
- *                          <= 2 activation rows, 16-byte aligned operands),
+ *   Q4G_GEMV_AUTO          the stage kernel where it can take the call, else the
+ *                          warp-streamed kernel, else the register kernel,
  *   Q4G_GEMV_WARP_STREAM   per-warp bulk-copy rings (k % 256 == 0),
  *   Q4G_GEMV_REGISTER      plain streaming loads (any k % 32 == 0),
  *   Q4G_GEMV_STAGE         integer dot, every warp of a CTA on each 16-36 KB
@@ -123,9 +118,9 @@ q4g_status q4g_gemv_f16(const uint16_t* w16, int64_t n, int64_t k, const uint16_
  *                          reducing and refilling (k % 256 == 0, <= 4
  *                          activation rows, 16-byte aligned operands).
  * A kernel that cannot take a call falls back to the automatic choice. Affects launches
- * made (and CUDA graphs captured) after the call. Q4G_EINVAL for other kinds. */
+ * made (and CUDA graphs captured) after the call. Q4G_EINVAL for other kinds
+ * (1 is retired). */
 #define Q4G_GEMV_AUTO 0
-#define Q4G_GEMV_COLUMN_SPLIT 1
 #define Q4G_GEMV_WARP_STREAM 2
 #define Q4G_GEMV_REGISTER 3
 #define Q4G_GEMV_STAGE 4
@@ -276,72 +271,30 @@ typedef enum {
                                  as one thread-block cluster and merge their partial
                                  softmax sums through distributed shared memory;
                                  0: split-KV with a merge through global memory */
-  Q4G_OPT_GEMV_CHAIN = 7,   /* [0] decode steps: O(l), gate|up(l), down(l) and QKV(l+1)
-                                 run as one persistent launch (one CTA per SM; a phase
-                                 starts when every CTA finished the previous one, a
-                                 bounded wait reported as Q4G_ETIMEOUT); 0: one launch
-                                 per GEMV */
-  Q4G_OPT_TRACE = 8,        /* [0] value = device uint64_t* [n_layers][32]: the GEMV
-                                 chain of layer l writes %globaltimer stamps (ns) of
-                                 its CTA 0 to row l: 0 start, 1 dependency wait done,
-                                 per phase i at 2 + 4i: inputs ready, x digits built,
-                                 last stage of CTA 0 done, producer done issuing;
-                                 18 end. With GEMV_CHAIN 0 the buffer must hold 1280
-                                 entries instead (1536 with the per-CTA ends): 256 each for gate|up, QKV, O and
-                                 down of layer 1 when they run on the column-split
-                                 or stage kernel, then 256 for layer 1's sliding
-                                 attention when it runs on the cluster kernel (0
-                                 entry, 1 dependency wait, 2 queries ready, 3 scan
+  Q4G_OPT_TRACE = 8         /* [0] value = device uint64_t* [1536]: %globaltimer stamps
+                                 (ns) of CTA 0 of layer 1's launches, 256 entries each:
+                                 gate|up at 0, QKV at 256, O at 512, down at 768 (per
+                                 GEMV launch: 0 entry, 1 dependency wait done, 2 x
+                                 digits built, 3 and 4 (fused norm prologue) first
+                                 loads used and second norm reduced, 5 last stage
+                                 reduced, 8 + t stage t issued, 72 + t stage t ready,
+                                 136 + t stage t reduced, t < 64); the sliding
+                                 attention at 1024 when it runs on the cluster kernel
+                                 (0 entry, 1 dependency wait, 2 queries ready, 3 scan
                                  done, 4 warps merged, 5 cluster synced, 6 output
-                                 written, 7 exit), then from entry 1280 when each
-                                 CTA of layer 1's gate|up finished its last stage
-                                 (stage kernel); per GEMV launch 0 entry, 1 dependency wait done,
-                                 2 x digits built, 3 and 4 (fused norm prologue)
-                                 first loads used and second norm reduced, 5 last
-                                 stage reduced (stage kernel), 8 + t
-                                 stage t issued, 72 + t stage t ready, 136 + t
-                                 stage t reduced (t < 64).
-                                 With the step kernel (Q4G_OPT_STEP_KERNEL) the
-                                 buffer holds 4 * (6 * n_layers + 1) + 2 entries
-                                 instead: per phase p (6 per layer: QKV, attention,
-                                 attention merge, O, gate|up, down; then the head)
-                                 at 4p, CTA 0's 0 phase start (every CTA finished
-                                 phase p - 1), 1 inputs ready (norm / queries /
-                                 x digits), 2 compute done, 3 outputs published
-                                 (GEMV phases); then the kernel's entry and exit.
-                                 Unwritten slots keep their contents. */
-  Q4G_OPT_STEP_KERNEL = 9,  /* [0] decode steps (one row) run as one persistent,
-                                 cooperative launch of one CTA per SM: every
-                                 layer's QKV, attention, attention merge, O,
-                                 gate|up and down, then the head, as phases that
-                                 start once every CTA finished the previous one
-                                 (a bounded wait, reported as Q4G_ETIMEOUT), while
-                                 each CTA's producer warp streams the weights and
-                                 K/V rows of the coming phases through one ring of
-                                 shared-memory stages. Used when the shapes fit
-                                 (hidden <= 4096, head dims 256 / 512); 0: one
-                                 launch per GEMV / attention kernel. Verify blocks
-                                 (K > 1 rows) always use the per-kernel path. */
-  Q4G_OPT_STEP_POLL_NS = 10, /* [64] step kernel: nanoseconds a thread first sleeps between
-                                 two polls of a phase counter or of tagged activation
-                                 words (0..100000; tagged words back off by doubling) */
-  Q4G_OPT_STEP_GRID_SYNC = 11 /* [1] step kernel: 1: every phase starts once every CTA
-                                 has counted itself done with the previous phase; 0: a
-                                 phase starts as soon as its own inputs (tagged words:
-                                 value and the step and layer that wrote it) have
-                                 arrived, with one grid-wide count per full-attention
-                                 layer only */
+                                 written, 7 exit); from 1280, when each CTA of layer
+                                 1's gate|up finished its last stage. Unwritten slots
+                                 keep their contents. Option values 7, 9, 10 and 11
+                                 are retired (Q4G_EINVAL). */
 } q4g_option;
 q4g_status q4g_model_set_option(q4g_model* m, q4g_option opt, intptr_t value);
 
 /* One kernel launch recorded in profile mode. kind: 0 step init, 1 QKV GEMV,
  * 2 sliding attention, 3 full attention, 4 attention combine, 5 O GEMV,
- * 6 gate|up GEMV, 7 down GEMV, 8 head GEMV, 9 GEMV chain (O, gate|up, down and
- * the next layer's QKV in one launch), 10 the persistent step kernel (the whole
- * step after step init). bytes: algorithmic HBM bytes of the launch (q4_0
- * weights 0.5625 B/weight + activations; attention: the live K/V rows,
- * 2 * head_dim * 2 B per key and KV head; the step kernel: its GEMVs' bytes,
- * the K/V rows are not included). */
+ * 6 gate|up GEMV, 7 down GEMV, 8 head GEMV. bytes: algorithmic HBM bytes of the
+ * launch (q4_0 weights 0.5625 B/weight, fp16 head weights 2 B/weight, plus
+ * activations; attention: the live K/V rows, 2 * head_dim * 2 B per key and KV
+ * head). */
 typedef struct {
   int32_t kind;
   int32_t layer;

@@ -111,20 +111,7 @@ struct q4g_model {
   float* part_ml;
   float* part_acc;
   // persistent step kernel: per-layer descriptors (device) and its partials / counters
-  StepLayer* step_layers = nullptr;
-  float* sk_part_ml = nullptr;
-  float* sk_part_acc = nullptr;
-  int32_t* sk_done = nullptr;
-  // its activations as tagged words (value | tag << 32) and the step number in the tags
-  uint64_t *sk_r[2] = {nullptr, nullptr}, *sk_qkv = nullptr, *sk_attn = nullptr, *sk_o = nullptr;
-  uint64_t *sk_act = nullptr, *sk_d = nullptr;
-  uint32_t* sk_epoch = nullptr;
-  uint32_t epoch = 0;
-  bool step_ok = false;  // the shapes fit the step kernel
-  uint32_t poll_ns = 64;  // step kernel: back-off between polls of a phase counter
-  int32_t step_grid_sync = 1;  // step kernel: grid counts between phases (0: tagged reads only)
-  // options
-  bool use_graph = true, use_pdl = true, attn_cluster = true, gemv_chain = false, use_step = false;
+  bool use_graph = true, use_pdl = true, attn_cluster = true;
   uint64_t* trace = nullptr;  // Q4G_OPT_TRACE
   float* dump = nullptr;
   // profile mode: events around every launch
@@ -275,19 +262,8 @@ extern "C" q4g_status q4g_model_create(const q4g_config* cfg, const q4g_weights*
     part = b > part ? b : part;
   }
   const size_t part_ml = part / 128 + 1024;  // (m, l) per row and chunk: hd >= 256
-  // head, attention, chain phases, the two-cluster ring attention merge, then the
-  // phase counters of the persistent step kernel
-  const int sk_counters = step_kernel_counters(c.n_layers, c.sl_kv_heads);
-  m->n_counters = 64 + kChainMaxPhases * c.n_layers + kRingSplitCounters + sk_counters;
-  StepKernelParams skp{};
-  skp.n_q = c.n_q_heads, skp.sl_nkv = c.sl_kv_heads, skp.gl_nkv = c.gl_kv_heads;
-  skp.sl_hd = c.sl_head_dim, skp.gl_hd = c.gl_head_dim, skp.hidden = c.hidden, skp.ffn = c.ffn;
-  skp.n_layers = c.n_layers, skp.rope_pairs_sl = c.sl_head_dim / 2, skp.rope_pairs_gl = c.rope_pairs_full;
-  {
-    char why[128];
-    m->step_ok = step_kernel_supported(skp, why, sizeof why);
-  }
-  const size_t sk_acc = step_kernel_partial_floats(skp, m->sm_count), sk_ml = step_kernel_ml_floats(skp, m->sm_count);
+  // head, attention, then the two-cluster ring attention merge
+  m->n_counters = 64 + kRingSplitCounters;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -312,12 +288,6 @@ extern "C" q4g_status q4g_model_create(const q4g_config* cfg, const q4g_weights*
   const size_t o_ifg = take(sizeof(double) * (m->gl.rope_pairs > 0 ? m->gl.rope_pairs : 1));
   const size_t o_pml = take(sizeof(float) * 2 * part_ml);
   const size_t o_pacc = take(sizeof(float) * part);
-  const size_t o_skml = take(sizeof(float) * sk_ml);
-  const size_t o_skacc = take(sizeof(float) * sk_acc);
-  const size_t o_layers = take(sizeof(StepLayer) * c.n_layers);
-  const size_t o_tr0 = take(8 * (size_t)H), o_tr1 = take(8 * (size_t)H), o_tqkv = take(8 * (size_t)qkv_max);
-  const size_t o_tattn = take(8 * (size_t)attn_max / 2), o_to = take(8 * (size_t)H);
-  const size_t o_tact = take(8 * (size_t)c.ffn / 2), o_td = take(8 * (size_t)H), o_epoch = take(sizeof(uint32_t));
   m->scratch_bytes = off;
   cudaError_t e = cudaMalloc(&m->scratch, off);
   if (e != cudaSuccess) {
@@ -344,46 +314,7 @@ extern "C" q4g_status q4g_model_create(const q4g_config* cfg, const q4g_weights*
   m->inv_freq_gl = (double*)(b + o_ifg);
   m->part_ml = (float*)(b + o_pml);
   m->part_acc = (float*)(b + o_pacc);
-  m->sk_part_ml = (float*)(b + o_skml);
-  m->sk_part_acc = (float*)(b + o_skacc);
-  m->sk_done = m->counters + (m->n_counters - sk_counters);
-  m->step_layers = (StepLayer*)(b + o_layers);
-  m->sk_r[0] = (uint64_t*)(b + o_tr0), m->sk_r[1] = (uint64_t*)(b + o_tr1), m->sk_qkv = (uint64_t*)(b + o_tqkv);
-  m->sk_attn = (uint64_t*)(b + o_tattn), m->sk_o = (uint64_t*)(b + o_to), m->sk_act = (uint64_t*)(b + o_tact);
-  m->sk_d = (uint64_t*)(b + o_td), m->sk_epoch = (uint32_t*)(b + o_epoch);
-  // the step kernel streams every tensor with bulk copies and reads the gains as
-  // float4: 16-byte aligned operands only (else the per-kernel path serves)
-  auto a16 = [](const void* ptr) { return aligned(ptr, 16); };
-  for (int l = 0; l < c.n_layers && m->step_ok; ++l) {
-    const q4g_layer_weights& W = m->layers[l];
-    const q4g_qtensor* ts[7] = {&W.wq, &W.wk, &W.wv, &W.wo, &W.wgate, &W.wup, &W.wdown};
-    for (int t = 0; t < 7; ++t)
-      if (!(t == 2 && m->full[l]) && (!a16(ts[t]->qs) || !a16(ts[t]->scales))) m->step_ok = false;
-    if (!a16(W.norm_in) || !a16(W.norm_post_attn) || !a16(W.norm_pre_ffn) || !a16(W.norm_post_ffn))
-      m->step_ok = false;
-  }
-  if (!a16(m->embed.qs) || !a16(m->embed.scales) || !a16(m->norm_final)) m->step_ok = false;
-  if (m->embed_f16) m->step_ok = false;  // the step kernel streams the q4_0 head only
   e = cudaMemset(m->scratch, 0, off);
-  {  // per-layer descriptors of the persistent step kernel
-    std::vector<StepLayer> sl(c.n_layers);
-    for (int l = 0; l < c.n_layers; ++l) {
-      const q4g_layer_weights& W = m->layers[l];
-      const q4g_qtensor* ts[7] = {&W.wq, &W.wk, &W.wv, &W.wo, &W.wgate, &W.wup, &W.wdown};
-      for (int t = 0; t < 7; ++t) {
-        const bool absent = t == 2 && m->full[l];
-        sl[l].q[t] = absent ? nullptr : ts[t]->qs;
-        sl[l].s[t] = absent ? nullptr : ts[t]->scales;
-      }
-      sl[l].norm_in = W.norm_in, sl[l].norm_post_attn = W.norm_post_attn, sl[l].norm_pre_ffn = W.norm_pre_ffn;
-      sl[l].norm_post_ffn = W.norm_post_ffn, sl[l].norm_q = W.norm_q, sl[l].norm_k = W.norm_k;
-      sl[l].layer_scalar = W.layer_scalar;
-      sl[l].full = m->full[l];
-      sl[l].ordinal = m->ordinal[l];
-    }
-    if (e == cudaSuccess)
-      e = cudaMemcpy(m->step_layers, sl.data(), sizeof(StepLayer) * sl.size(), cudaMemcpyHostToDevice);
-  }
   // RoPE inverse frequencies theta^(-2i/hd), in fp64 ("Gemma 4 12B" architecture:
   // dual RoPE; the full layers' frequencies are those of head dim 512, first pairs only)
   std::vector<double> fs(m->sl.rope_pairs), fg(m->gl.rope_pairs > 0 ? m->gl.rope_pairs : 1, 0.0);
@@ -437,11 +368,7 @@ extern "C" q4g_status q4g_model_set_option(q4g_model* m, q4g_option opt, intptr_
     case Q4G_OPT_PROFILE: m->profile = value != 0; break;
     case Q4G_OPT_TEST_STALL: m->stall_next = value != 0; break;
     case Q4G_OPT_ATTN_CLUSTER: m->attn_cluster = value != 0; break;
-    case Q4G_OPT_GEMV_CHAIN: m->gemv_chain = value != 0; break;
     case Q4G_OPT_TRACE: m->trace = (uint64_t*)value; break;
-    case Q4G_OPT_STEP_KERNEL: m->use_step = value != 0; break;
-    case Q4G_OPT_STEP_POLL_NS: m->poll_ns = (uint32_t)std::max<intptr_t>(0, std::min<intptr_t>(value, 100000)); break;
-    case Q4G_OPT_STEP_GRID_SYNC: m->step_grid_sync = value != 0; break;
     default: return fail(Q4G_EINVAL, "unknown option %d", (int)opt);
   }
   free_graphs(m);
@@ -756,18 +683,6 @@ cudaError_t debug_sync(cudaError_t e, const char* what, int layer, cudaStream_t 
   return e;
 }
 
-// Scale of the fraction of the next GEMV's per-warp ranges a kernel prefetches
-// into L2 once its own loads are in flight (Q4G_L2_PREFETCH, default 0: off;
-// measured slower, the prefetch traffic delays the attention kernels).
-float prefetch_scale() {
-  static float f = -1.f;
-  if (f < 0.f) {
-    const char* e = getenv("Q4G_L2_PREFETCH");
-    f = e ? (float)atof(e) : 0.0f;
-  }
-  return f;
-}
-
 // All kernels of one step after step_init (the part that is captured in a graph).
 cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0, float* logits,
                          int32_t* argmax, cudaStream_t st) {
@@ -775,7 +690,6 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
   const int H = cf.hidden, L = cf.n_layers;
   const bool pdl = m->use_pdl;
   const int64_t dstride = (int64_t)(L + 1) * H;
-  const float pf = prefetch_scale();
   cudaError_t e;
   float* rA = m->r[0];
   float* rB = m->r[1];
@@ -906,11 +820,6 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
     p.argmax_out = argmax ? argmax : m->argmax_buf;
     return p;
   };
-  auto next_of = [&](const GemvParams& q, float frac) {
-    return pf > 0.f ? gemv_next_desc(q, std::min(1.0f, frac * pf)) : NextGemv{};
-  };
-
-  bool qkv_done = false;  // QKV(l) already ran as the last phase of the previous chain
   for (int l = 0; l < L; ++l) {
     const q4g_layer_weights& W = m->layers[l];
     const bool full = m->full[l];
@@ -918,10 +827,9 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
     const int ord = m->ordinal[l];
     const GemvParams gate_up = gate_up_params(l);
     // separate launches: the timeline of layer 1's QKV and gate|up (CTA 0)
-    uint64_t* const trace_sep = m->trace && !m->gemv_chain && l == 1 ? m->trace : nullptr;
-    if (!qkv_done) {
+    uint64_t* const trace_sep = m->trace && l == 1 ? m->trace : nullptr;
+    {
       GemvParams p = qkv_params(l);
-      p.next = next_of(o_params(l, 0), 1.0f);
       p.trace = trace_sep ? trace_sep + kGemvTraceSlots : nullptr;
       if (l == 0 && m->stall_next) {
         p.stall_test = 1;
@@ -934,7 +842,6 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
     // (a4-a6) q/k/v epilogue, cache write, split-KV attention, combine
     {
       AttnParams p{};
-      p.next = next_of(gate_up, 0.15f);
       p.qkv = m->qkv;
       p.qkv_stride = S.qkv_cols;
       p.k_off = S.nq_cols;
@@ -967,7 +874,7 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
         p.trace = trace_sep ? trace_sep + 4 * kGemvTraceSlots : nullptr;
         if (S.nkv * kAttnCluster <= kRingSplitCounters) {
           p.ring_split = 2;
-          p.counters = m->counters + 64 + kChainMaxPhases * L;
+          p.counters = m->counters + 64;
         }
         p.cluster = kAttnCluster;
         p.n_chunks = kAttnCluster;
@@ -981,32 +888,10 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
       e = pr.done(debug_sync(launch_attention(p, st, pdl), "attention", l, st), full ? 3 : 2, l, kv_bytes);
       if (e != cudaSuccess) return e;
       if (full) {
-        p.next = NextGemv{};
         Prof pc(m, st);
         e = pc.done(debug_sync(launch_attn_combine(p, st, pdl), "combine", l, st), 4, l,
                     (double)kr * cf.n_q_heads * p.n_chunks * (S.hd + 2) * 4.0);
         if (e != cudaSuccess) return e;
-      }
-    }
-    // O(l), gate|up(l), down(l) and QKV(l+1) as one persistent chain launch
-    qkv_done = false;
-    if (kr == 1 && m->gemv_chain) {
-      ChainParams ch{};
-      ch.ph[0] = o_params(l, 0);
-      ch.ph[1] = gate_up;
-      ch.ph[2] = down_params(l, 0);
-      ch.n_ph = 3;
-      if (l + 1 < L) ch.ph[3] = qkv_params(l + 1), ch.n_ph = 4;
-      ch.done = m->counters + 64 + kChainMaxPhases * l;
-      ch.trace = m->trace ? m->trace + (size_t)kChainTraceSlots * l : nullptr;
-      if (plan_chain(ch)) {
-        double bytes = 0;
-        for (int i = 0; i < ch.n_ph; ++i) bytes += gemv_bytes(ch.ph[i].n_rows, ch.ph[i].k, 1, 4);
-        Prof pr(m, st);
-        e = pr.done(debug_sync(launch_gemv_chain(ch, st, pdl), "gemv_chain", l, st), 9, l, bytes);
-        if (e != cudaSuccess) return e;
-        qkv_done = ch.n_ph == 4;
-        continue;
       }
     }
     {
@@ -1014,7 +899,6 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
       const int maxr = gemv_max_rows(kin);
       for (int r0 = 0; r0 < kr; r0 += maxr) {
         GemvParams p = o_params(l, r0);
-        if (r0 + maxr >= kr) p.next = next_of(gate_up, 0.35f);
         p.trace = trace_sep && r0 == 0 ? trace_sep + 2 * kGemvTraceSlots : nullptr;
         Prof pr(m, st);
         e = pr.done(debug_sync(launch_gemv(p, st, pdl), "o_proj", l, st), 5, l, gemv_bytes(H, kin, p.kr, 4));
@@ -1023,7 +907,6 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
     }
     {
       GemvParams p = gate_up;
-      p.next = next_of(down_params(l, 0), 0.6f);
       p.trace = trace_sep;
       p.trace_ends = trace_sep ? trace_sep + 5 * kGemvTraceSlots : nullptr;
       Prof pr(m, st);
@@ -1034,8 +917,6 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
       const int maxr = gemv_max_rows(cf.ffn);
       for (int r0 = 0; r0 < kr; r0 += maxr) {
         GemvParams p = down_params(l, r0);
-        if (r0 + maxr >= kr && (l + 1 < L || !m->embed_f16))
-          p.next = l + 1 < L ? next_of(qkv_params(l + 1), 1.0f) : next_of(head_params(), 0.05f);
         p.trace = trace_sep && r0 == 0 ? trace_sep + 3 * kGemvTraceSlots : nullptr;
         Prof pr(m, st);
         e = pr.done(debug_sync(launch_gemv(p, st, pdl), "down", l, st), 7, l, gemv_bytes(H, cf.ffn, p.kr, 4));
@@ -1058,50 +939,6 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
   }
   return cudaSuccess;
 }
-
-// One decode step (one row) as the persistent step kernel.
-cudaError_t enqueue_step_kernel(q4g_model* m, const q4g_cache* c, float* logits, int32_t* argmax, cudaStream_t st) {
-  const q4g_config& cf = m->cfg;
-  StepKernelParams p{};
-  p.layers = m->step_layers;
-  p.n_layers = cf.n_layers, p.hidden = cf.hidden, p.n_q = cf.n_q_heads, p.ffn = cf.ffn, p.vocab = cf.vocab;
-  p.sl_nkv = cf.sl_kv_heads, p.sl_hd = cf.sl_head_dim, p.gl_nkv = cf.gl_kv_heads, p.gl_hd = cf.gl_head_dim;
-  p.window = cf.window, p.ring = cf.ring, p.capacity = c->capacity;
-  p.rope_pairs_sl = m->sl.rope_pairs, p.rope_pairs_gl = m->gl.rope_pairs, p.v_norm_sliding = cf.v_norm_sliding;
-  p.eps = cf.rms_eps, p.softcap = cf.softcap;
-  p.cache = c->buf;
-  p.ring_k_off = c->view.ring_k_offset, p.ring_v_off = c->view.ring_v_offset, p.ring_layer_bytes = c->view.ring_layer_bytes;
-  p.glob_k_off = c->view.global_k_offset, p.glob_v_off = c->view.global_v_offset;
-  p.glob_layer_bytes = c->view.global_layer_bytes;
-  p.emb_q = m->embed.qs, p.emb_s = m->embed.scales, p.norm_final = m->norm_final;
-  p.r0 = m->sk_r[0], p.r1 = m->sk_r[1], p.qkv = m->sk_qkv, p.attn = m->sk_attn, p.o = m->sk_o;
-  p.act = m->sk_act, p.d = m->sk_d, p.epoch = m->sk_epoch;
-  p.part_ml = m->sk_part_ml, p.part_acc = m->sk_part_acc;
-  p.rope_sl = m->rope_sl, p.rope_gl = m->rope_gl, p.pos_dev = m->pos_dev;
-  p.logits = logits, p.argmax_out = argmax ? argmax : m->argmax_buf;
-  p.am_val = m->am_val, p.am_idx = m->am_idx;
-  p.done = m->sk_done;
-  p.tickets = m->sk_done + step_kernel_phases(cf.n_layers) + 1;
-  p.dump = m->dump;
-  p.trace = m->trace;
-  p.poll_ns = m->poll_ns;
-  p.grid_sync = m->step_grid_sync;
-  if (m->stall_next) {
-    p.stall_test = 1;
-    p.wait_ns = 20000000ull;  // 20 ms
-  }
-  Prof pr(m, st);
-  double bytes = 0;
-  for (int l = 0; l < cf.n_layers; ++l) {
-    const LayerShape& S = m->full[l] ? m->gl : m->sl;
-    bytes += gemv_bytes(S.qkv_cols, cf.hidden, 1, 4) + gemv_bytes(cf.hidden, (int64_t)cf.n_q_heads * S.hd, 1, 4) +
-             gemv_bytes(2 * (int64_t)cf.ffn, cf.hidden, 1, 1) + gemv_bytes(cf.hidden, cf.ffn, 1, 4);
-  }
-  bytes += gemv_bytes(cf.vocab, cf.hidden, 1, logits ? 4 : 0);
-  return pr.done(debug_sync(launch_step_kernel(p, st), "step_kernel", -1, st), 10, -1, bytes);
-}
-
-bool use_step_kernel(const q4g_model* m, int kr) { return kr == 1 && m->use_step && m->step_ok; }
 
 q4g_status run_step(q4g_model* m, q4g_cache* c, int kr, int64_t pos0, const int32_t* ids_dev,
                     const int32_t* ids_host, const float* hidden, float* logits, int32_t* argmax,
@@ -1135,20 +972,12 @@ q4g_status run_step(q4g_model* m, q4g_cache* c, int kr, int64_t pos0, const int3
   sp.pos_dev = m->pos_dev;
   sp.counters = m->counters;
   sp.n_counters = m->n_counters;
-  if (use_step_kernel(m, kr)) {  // the layer-0 input as tagged words, and this step's number
-    sp.r_tagged = m->sk_r[0];
-    sp.epoch_dev = m->sk_epoch;
-    sp.epoch = ++m->epoch;  // never 0: the zeroed buffers carry tag 0
-    if (m->epoch >= (1u << 25) - 1) m->epoch = 0;  // epoch * 128 stays within 32 bits
-  }
   {
     Prof pr(m, st);
     CK(pr.done(launch_step_init(sp, st), 0, -1, (double)kr * cf.hidden * (4 + 0.5625)));
   }
-  const bool step_kernel = use_step_kernel(m, kr);
   if (!m->use_graph || m->profile || m->stall_next) {
-    cudaError_t e = step_kernel ? enqueue_step_kernel(m, c, logits, argmax, st)
-                                : enqueue_body(m, c, kr, pos0, logits, argmax, st);
+    cudaError_t e = enqueue_body(m, c, kr, pos0, logits, argmax, st);
     m->stall_next = false;
     CK(e);
     return Q4G_OK;
@@ -1161,8 +990,7 @@ q4g_status run_step(q4g_model* m, q4g_cache* c, int kr, int64_t pos0, const int3
     if (m->graphs.size() >= 16) free_graphs(m);
     cudaGraph_t graph = nullptr;
     CK(cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal));
-    cudaError_t e = step_kernel ? enqueue_step_kernel(m, c, logits, argmax, m->cap_stream)
-                                : enqueue_body(m, c, kr, pos0, logits, argmax, m->cap_stream);
+    cudaError_t e = enqueue_body(m, c, kr, pos0, logits, argmax, m->cap_stream);
     cudaError_t e2 = cudaStreamEndCapture(m->cap_stream, &graph);
     if (e != cudaSuccess) {
       if (graph) cudaGraphDestroy(graph);

@@ -24,7 +24,6 @@
 // rows to the cache; every CTA reads this block's own rows from shared memory.
 #include "q4g_common.cuh"
 #include "q4g_internal.h"
-#include "q4g_prefetch.cuh"
 
 namespace q4g {
 
@@ -164,11 +163,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
     load_tile(0, false, 0);
     cp_async_commit();
   }
-  // the next GEMV's first weights towards L2, one slice per CTA
-  if (tid == 0)
-    prefetch_next(p.next, ((long long)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x,
-                  (long long)gridDim.x * gridDim.y * gridDim.z);
-
   // ---- prologue: queries (and this block's K/V rows) into shared memory ----
   if (fused) {
     const int nvec = nrows + 2 * p.kr;

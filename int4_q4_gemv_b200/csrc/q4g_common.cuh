@@ -159,17 +159,6 @@ Q4G_DEV uint64_t policy_evict_first() {
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
   return pol;
 }
-// Asynchronous L2 prefetch of [p, p + bytes) (p 16-byte aligned; a tail below
-// 16 bytes is skipped). A hint: nothing waits for it.
-Q4G_DEV void l2_prefetch(const void* p, uint64_t bytes) {
-  const char* c = static_cast<const char*>(p);
-  while (bytes >= 16) {
-    const uint32_t n = (uint32_t)(bytes < 32768 ? bytes : 32768) & ~15u;
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(c), "r"(n) : "memory");
-    c += n;
-    bytes -= n;
-  }
-}
 Q4G_DEV uint64_t global_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -1,5 +1,4 @@
-// The integer block dot product of the q4_0 GEMV kernels and its helpers
-// (shared by the per-GEMV kernels and the persistent decode-step kernel).
+// The integer block dot product of the q4_0 GEMV kernels and its helpers.
 #pragma once
 
 #include "q4g_common.cuh"

@@ -39,7 +39,6 @@
 #include "q4g_common.cuh"
 #include "q4g_dot.cuh"
 #include "q4g_internal.h"
-#include "q4g_prefetch.cuh"
 
 #include <stdlib.h>
 
@@ -642,8 +641,6 @@ __global__ void __launch_bounds__(kWarpThreads, 1) gemv_q4_tma_kernel(const Gemv
     for (; issued < NS && issued < n_items; ++issued)
       issue_item(p, u_begin + issued / nchunk, issued % nchunk, wst + (size_t)issued * p.stage_bytes,
                  &wbar[issued], p.stall_test && u_begin == 0 && issued == 0, pol);  // the warp owning unit 0
-    // all own loads issued: start the next GEMV's weights towards L2
-    if (issued == n_items) prefetch_next(p.next, gw, tw);
   }
   __syncwarp();
 
@@ -736,7 +733,7 @@ __global__ void __launch_bounds__(kWarpThreads, 1) gemv_q4_tma_kernel(const Gemv
     if (lane == 0 && !abort_ && issued < n_items) {  // refill this stage
       issue_item(p, u_begin + issued / nchunk, issued % nchunk, wst + (size_t)s * p.stage_bytes, &wbar[s],
                  false, pol);
-      if (++issued == n_items) prefetch_next(p.next, gw, tw);
+      ++issued;
     }
     if (c != nchunk - 1) continue;
     // unit complete: the two row sums of every activation row
@@ -815,15 +812,6 @@ __global__ void __launch_bounds__(kWarpThreads, 1) gemv_q4_tma_kernel(const Gemv
 
 size_t tma_fixed_bytes(int dot, int krm, int k) {
   return x_region_bytes(dot, krm, k) + 64 * 4 + 2 * kWarps * 4 + 128 + kWarps * kMaxStages * 8;
-}
-
-int gemv_dot_kind() {
-  static int kind = -1;
-  if (kind < 0) {
-    const char* e = getenv("Q4G_GEMV_DOT");
-    kind = !e ? -1 : e[0] == 'h' ? DOT_FMA_HALF : e[0] == 'f' ? DOT_FMA : DOT_INT;
-  }
-  return kind;
 }
 
 template <int KRM, int DOT>
@@ -910,38 +898,8 @@ bool plan_tma(GemvParams& p, int& dot) {
 }
 
 // ---------------------------------------------------------------------------
-// Column-split integer GEMV (the default for k % 256 == 0, up to 2 activation
-// rows).
-//
-// Each CTA owns a contiguous, balanced range of units (R rows each, R = 8, 4
-// or 2; a GeGLU unit is R/2 gate rows and the same R/2 up rows) and streams it
-// in order through a ring of NS stages: one producer warp issues 2 (GeGLU: 4)
-// large 1-D bulk copies per stage (the unit's codes, then its scales), so every
-// SM reads one contiguous region, the access pattern that reaches the copy
-// bandwidth of HBM. The k columns are cut into NC chunks of 32 BPL blocks
-// (BPL = 2 for one activation row, else 1); consumer warp (g, c) owns chunk c
-// and takes the stages g, g + G, ... (G = 16 / NC groups). Lane l of that warp
-// holds the integer digits of x for blocks 32 BPL c + l + 32 b in registers
-// for the whole kernel (block_dot_int) and dots them with the R rows of every
-// stage it takes. The R partial sums of a
-// warp go to shared memory with a transposing butterfly; the last of the NC
-// warps to finish a stage adds the chunk partials in chunk order
-// (deterministic), runs the epilogue and hands the stage back, so the producer
-// only waits and refills.
+// Helpers of the bulk-copy ring (stage kernel).
 // ---------------------------------------------------------------------------
-constexpr int kCsMaxConsumers = 16;
-constexpr int kCsThreads = (kCsMaxConsumers + 1) * 32;
-constexpr int kCsMaxStages = 16;
-
-__host__ __device__ inline size_t cs_red_floats(int ns, int nc, int rows, int krm) {
-  return (size_t)ns * nc * rows * krm;
-}
-__host__ __device__ inline size_t cs_fixed_bytes(int krm, int k, int ns, int nc, int rows) {
-  const size_t nb = (size_t)k / 32;
-  const size_t red = (cs_red_floats(ns, nc, rows, krm) * 4 + 15) & ~(size_t)15;
-  return (size_t)krm * nb * (16 * kDigitQuads + 16) + 64 * 4 + red + 128 + 2 * kCsMaxStages * 8;
-}
-
 
 // Wait for `phase` of `bar` until done, until another warp gave up (flag set),
 // or until limit_ns pass (then this warp sets the flag and the error word).
@@ -956,31 +914,6 @@ Q4G_DEV bool cs_wait(uint64_t* bar, uint32_t phase, const GemvParams& p, volatil
   *abort_flag = 1;
   atomicOr(p.err, 1);
   return false;
-}
-
-// Several consumer groups share one ring, so a group can reach slot s for
-// stage t while the slot's previous fill (stage t - NS, another group's) is
-// still in flight; the mbarrier parity of fill t equals that of fill t - 2 NS,
-// so a parity wait alone could pass early. The producer therefore publishes
-// the stage number it issued into each slot (after the expect-tx arrive), and
-// a consumer first waits until slot s carries stage t: from then on the slot's
-// pending phase is fill t's and the parity wait is exact.
-Q4G_DEV bool wait_issued(volatile int* seq, int t, const GemvParams& p, volatile int* abort_flag) {
-  if (*seq == t) return true;
-  const uint64_t t0 = global_ns();
-  for (int it = 0; it < kSpinLimit; ++it) {
-    if (*seq == t) return true;
-    if (*abort_flag) return false;
-    if (global_ns() - t0 > p.wait_ns) break;
-    __nanosleep(32);
-  }
-  *abort_flag = 1;
-  atomicOr(p.err, 1);
-  return false;
-}
-Q4G_DEV void publish_issued(volatile int* seq, int t) {
-  __threadfence_block();
-  *seq = t;
 }
 
 // Issue the bulk copies of unit u into stage `st` ([R rows of codes][R rows of scales]).
@@ -1005,312 +938,6 @@ Q4G_DEV void cs_issue(const GemvParams& p, int u, unsigned char* st, uint64_t* b
     bulk_g2s_hint(st, sg->qs + (size_t)r0 * kh, qb, bar, pol);
     bulk_g2s_hint(st + (size_t)R * kh, sg->sc + (size_t)r0 * nb, sb, bar, pol);
   }
-}
-
-template <int KRM, int R, int BPL>
-__global__ void __launch_bounds__(kCsThreads, 1) gemv_q4_cs_kernel(const GemvParams p) {
-  extern __shared__ __align__(16) unsigned char cs_smem[];
-  const int k = p.k, nb = k >> 5, kh = k >> 1, NS = p.ns, NC = p.nchunk, G = p.groups;
-  uint4* dg = reinterpret_cast<uint4*>(cs_smem);                          // [KRM][kDigitQuads][nb]
-  int4* bc = reinterpret_cast<int4*>(dg + (size_t)KRM * kDigitQuads * nb);  // [KRM][nb]
-  float* misc = reinterpret_cast<float*>(bc + (size_t)KRM * nb);          // 64 floats
-  float* red = misc + 64;                                                 // [NS][NC][R][KRM]
-  const size_t red_bytes = (cs_red_floats(NS, NC, R, KRM) * 4 + 15) & ~(size_t)15;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(
-      ((uintptr_t)(reinterpret_cast<unsigned char*>(red) + red_bytes) + 127) & ~(uintptr_t)127);
-  uint64_t* full = bars;                    // [kCsMaxStages]
-  uint64_t* empty = bars + kCsMaxStages;    // [kCsMaxStages]
-  unsigned char* stages = reinterpret_cast<unsigned char*>(bars + 2 * kCsMaxStages);
-  __shared__ int s_abort, s_ticket;
-  __shared__ int s_cnt[kCsMaxStages];       // consumer warps done with a stage
-  __shared__ int s_seq[kCsMaxStages];       // stage number last issued into each slot
-  __shared__ float s_bestv[kCsMaxConsumers];
-  __shared__ int s_besti[kCsMaxConsumers];
-
-  // kCsThreads threads: consumer warps 0 .. NC*G-1, producer warp kCsMaxConsumers,
-  // the rest only help stage x
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n_cons = NC * G;
-  const bool producer = warp == kCsMaxConsumers;
-  const int u0 = (int)((long long)blockIdx.x * p.n_units / gridDim.x);
-  const int n_st = (int)((long long)(blockIdx.x + 1) * p.n_units / gridDim.x) - u0;
-  const size_t SB = (size_t)p.stage_bytes;
-  const uint64_t pol = policy_evict_first();
-  int issued = 0;
-  uint64_t* const tr = blockIdx.x == 0 ? p.trace : nullptr;
-  auto stamp = [&](int i) {
-    if (tr) tr[i] = global_ns();
-  };
-
-  if (tid == 0) stamp(0), s_abort = 0;
-  if (tid < kCsMaxStages) s_cnt[tid] = 0, s_seq[tid] = -1;
-  if (tid < kCsMaxConsumers) s_bestv[tid] = -INFINITY, s_besti[tid] = 0x7fffffff;
-  if (producer && lane == 0) {
-    for (int s = 0; s < NS; ++s) mbar_init(&full[s], 1), mbar_init(&empty[s], 1);
-    fence_mbar_init();
-    const int pre = p.prefetch_stages > 0 ? min(NS, p.prefetch_stages) : NS;
-    for (; issued < pre && issued < n_st; ++issued) {
-      cs_issue<R>(p, u0 + issued, stages + issued * SB, &full[issued],
-                  p.stall_test && u0 == 0 && issued == 0, pol);  // the CTA owning unit 0
-      if (issued < 64) stamp(8 + issued);
-    }
-  }
-  __syncthreads();  // s_seq initialised before the producer publishes
-  if (producer && lane == 0)
-    for (int i = 0; i < issued; ++i) publish_issued(&s_seq[i], i);
-  pdl_wait();
-  if (tid == 0) stamp(1);
-  stage_digits<KRM, kCsThreads>(p, dg, bc, misc);  // ends with __syncthreads
-  if (tid == 0) stamp(2);
-  pdl_launch_dependents();
-  volatile int* abort_flag = &s_abort;
-
-  if (warp < n_cons) {
-    // ---------------- consumer: chunk c, stages g, g + G, ... ----------------
-    // lane l holds blocks 32 BPL c + l + 32 b, b < BPL, of every row. A lane
-    // past the end of the row reads block nb - 1 with zero digits and a zero
-    // x scale, so the loop below has no branch.
-    const int c = warp % NC, g = warp / NC;
-    int qoff[BPL], soff[BPL];
-    uint4 xg[KRM][BPL][kDigitQuads];
-    int4 cv[KRM][BPL];
-    float xsc[KRM][BPL];
-#pragma unroll
-    for (int b = 0; b < BPL; ++b) {
-      const int blk = 32 * BPL * c + lane + 32 * b;
-      const bool has = blk < nb;
-      qoff[b] = 16 * min(blk, nb - 1);
-      soff[b] = 2 * min(blk, nb - 1);
-#pragma unroll
-      for (int j = 0; j < KRM; ++j) {
-        if (has && (KRM == 1 || j < p.kr)) {
-#pragma unroll
-          for (int q = 0; q < kDigitQuads; ++q) xg[j][b][q] = dg[(size_t)(j * kDigitQuads + q) * nb + blk];
-          cv[j][b] = bc[j * nb + blk];
-        } else {
-#pragma unroll
-          for (int q = 0; q < kDigitQuads; ++q) xg[j][b][q] = make_uint4(0, 0, 0, 0);
-          cv[j][b] = make_int4(0, 0, 0, 0);
-        }
-        xsc[j][b] = __int_as_float(cv[j][b].w);
-      }
-    }
-    float best_v = -INFINITY;
-    int best_i = 0x7fffffff;
-    int s = g % NS;
-    uint32_t ph = (uint32_t)((g / NS) & 1);
-    for (int t = g; t < n_st; t += G) {
-      if (!*abort_flag && wait_issued(&s_seq[s], t, p, abort_flag)) cs_wait(&full[s], ph, p, abort_flag);
-      if (c == 0 && lane == 0 && t < 64) stamp(72 + t);
-      const unsigned char* st = stages + s * SB;
-      const unsigned char* ss = st + R * kh;
-      float v[KRM][R];
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        float a[KRM];
-#pragma unroll
-        for (int j = 0; j < KRM; ++j) a[j] = 0.f;
-#pragma unroll
-        for (int b = 0; b < BPL; ++b) {
-          const uint4 qv = *reinterpret_cast<const uint4*>(st + r * kh + qoff[b]);
-          const float d = __half2float(*reinterpret_cast<const __half*>(ss + r * 2 * nb + soff[b]));
-#pragma unroll
-          for (int j = 0; j < KRM; ++j)
-            if (KRM == 1 || j < p.kr) a[j] = fmaf(d * xsc[j][b], block_dot_int(qv, xg[j][b], cv[j][b]), a[j]);
-        }
-#pragma unroll
-        for (int j = 0; j < KRM; ++j) v[j][r] = a[j];
-      }
-      float* rs = red + (size_t)s * NC * R * KRM;  // [NC][R][KRM] of this stage
-#pragma unroll
-      for (int j = 0; j < KRM; ++j) {
-        const float tot = cs_reduce_rows<R>(v[j], lane);
-        if ((lane & (32 / R - 1)) == 0) rs[((size_t)c * R + cs_row<R>(lane)) * KRM + j] = tot;
-      }
-      // the last of the NC warps of this stage adds the chunks in order, runs
-      // the epilogue and hands the stage back to the producer
-      __syncwarp();
-      int last = 0;
-      if (lane == 0) {
-        __threadfence_block();
-        last = atomicAdd(&s_cnt[s], 1) == NC - 1;
-      }
-      last = __shfl_sync(0xffffffffu, last, 0);
-      if (last) {
-        __threadfence_block();
-        const int u = u0 + t;
-        const int r = lane / KRM, j = lane % KRM;  // lanes l < R * KRM
-        float val = 0.f;
-        if (lane < R * KRM)
-          for (int cc = 0; cc < NC; ++cc) val += rs[((size_t)cc * R + r) * KRM + j];
-        if (p.epi == EPI_GEGLU) {
-          const float up = __shfl_sync(0xffffffffu, val, (lane + (R / 2) * KRM) & 31);
-          if (lane < (R / 2) * KRM && j < p.kr)
-            p.act[(size_t)j * p.act_stride + (size_t)(R / 2) * u + r] = __float2half_rn(gelu_tanh(val) * up);
-        } else if (lane < R * KRM && j < p.kr) {
-          const int row = R * u + r;
-          if (row < p.n_rows) {
-            if (p.epi == EPI_STORE) {
-              p.y[(size_t)j * p.y_stride + row] = val;
-            } else {
-              const float z = p.softcap * tanhf(val / p.softcap);
-              if (p.logits) p.logits[(size_t)j * p.logits_stride + row] = z;
-              if (z > best_v || (z == best_v && row < best_i)) best_v = z, best_i = row;
-            }
-          }
-        }
-        __syncwarp();
-        if (lane == 0) {
-          s_cnt[s] = 0;
-          mbar_arrive(&empty[s]);
-          if (t < 64) stamp(136 + t);
-        }
-      }
-      s += G;
-      while (s >= NS) s -= NS, ph ^= 1u;
-    }
-    if (p.epi == EPI_HEAD) {
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float v2 = __shfl_xor_sync(0xffffffffu, best_v, o);
-        const int i2 = __shfl_xor_sync(0xffffffffu, best_i, o);
-        if (v2 > best_v || (v2 == best_v && i2 < best_i)) best_v = v2, best_i = i2;
-      }
-      if (lane == 0) s_bestv[warp] = best_v, s_besti[warp] = best_i;
-    }
-  } else if (producer) {
-    // ---------------- producer: refill each stage once it is handed back ----------------
-    if (lane == 0) {
-      for (int t = issued; t < n_st; ++t) {
-        const int s = t % NS;
-        if (t >= NS && !*abort_flag) cs_wait(&empty[s], (uint32_t)(((t - NS) / NS) & 1), p, abort_flag);
-        if (*abort_flag) break;
-        cs_issue<R>(p, u0 + t, stages + s * SB, &full[s], false, pol);
-        publish_issued(&s_seq[s], t);
-        if (t < 64) stamp(8 + t);
-        issued = t + 1;
-      }
-    }
-  }
-  if (p.epi == EPI_HEAD) {
-    __syncthreads();
-    if (tid == 0) {
-      float bv = -INFINITY;
-      int bi = 0x7fffffff;
-      for (int w = 0; w < kCsMaxConsumers; ++w)
-        if (s_bestv[w] > bv || (s_bestv[w] == bv && s_besti[w] < bi)) bv = s_bestv[w], bi = s_besti[w];
-      p.am_val[blockIdx.x] = bv;
-      p.am_idx[blockIdx.x] = bi;
-      __threadfence();
-      s_ticket = atomicAdd(p.counter, 1);
-      if (s_ticket == (int)gridDim.x - 1) {
-        __threadfence();
-        float v = -INFINITY;
-        int ix = 0x7fffffff;
-        for (int b = 0; b < (int)gridDim.x; ++b) {
-          const float vb = __ldcg(p.am_val + b);
-          const int ib = __ldcg(p.am_idx + b);
-          if (vb > v || (vb == v && ib < ix)) v = vb, ix = ib;
-        }
-        if (p.argmax_out) p.argmax_out[0] = ix == 0x7fffffff ? 0 : ix;
-        *p.counter = 0;
-      }
-    }
-  }
-  // after a timeout, wait (bounded) for the copies still in flight
-  if (producer && lane == 0 && *abort_flag) {
-    for (int t = issued > NS ? issued - NS : 0; t < issued; ++t)
-      mbar_wait_bounded(&full[t % NS], (uint32_t)((t / NS) & 1), p.wait_ns);
-  }
-}
-
-// Plan of the column-split kernel: rows per stage R, chunks NC, groups G and
-// stages NS within the shared-memory budget.
-bool plan_cs(GemvParams& p, int& R, int& BPL, bool forced) {
-  const int k = p.k, nb = k >> 5;
-  if (k % 256 != 0 || p.kr > 2) return false;
-  // measured: the warp-streamed kernel is faster for long rows (k = 15360)
-  // and small matrices (3840 x 4096), where a stage carries less work
-  if (!forced && (k > 4096 || p.n_rows < 8192)) return false;
-  if (p.epi == EPI_HEAD && p.kr != 1) return false;
-  if (p.epi == EPI_GEGLU && (p.nseg != 2 || p.seg[0].rows != p.seg[1].rows || p.seg[0].rows % 4)) return false;
-  if (p.pro == PRO_RESID && k > 8192) return false;
-  for (int s = 0; s < p.nseg; ++s)
-    if (!aligned16(p.seg[s].qs) || !aligned16(p.seg[s].sc) || (s < p.nseg - 1 && p.seg[s].rows % 8))
-      return false;
-  if (p.pro == PRO_X16 && !aligned16(p.x)) return false;
-  // two blocks per lane when the digits of one row fit the registers
-  // (Q4G_GEMV_BPL=1 forces one, a tuning switch)
-  static const int bpl_env = getenv("Q4G_GEMV_BPL") ? atoi(getenv("Q4G_GEMV_BPL")) : 0;
-  BPL = p.kr <= 1 && bpl_env != 1 ? 2 : 1;
-  const int NC = (nb + 32 * BPL - 1) / (32 * BPL);
-  if (NC > kCsMaxConsumers) return false;
-  int G = kCsMaxConsumers / NC;
-  const int krm = p.kr <= 1 ? 1 : 2;
-  auto units = [&](int r) { return p.epi == EPI_GEGLU ? p.seg[0].rows / (r / 2) : (p.n_rows + r - 1) / r; };
-  // Q4G_CS_ROWS (2, 4, 8) and Q4G_CS_GROUPS cap the stage rows and the
-  // consumer groups: tuning switches
-  static const int rows_env = getenv("Q4G_CS_ROWS") ? atoi(getenv("Q4G_CS_ROWS")) : 0;
-  static const int groups_env = getenv("Q4G_CS_GROUPS") ? atoi(getenv("Q4G_CS_GROUPS")) : 0;
-  R = k <= 4096 ? 8 : k <= 8192 ? 4 : 2;
-  if (rows_env == 2 || rows_env == 4 || rows_env == 8) R = std::min(R, rows_env);
-  if (p.epi == EPI_GEGLU && (p.seg[0].rows % (R / 2))) return false;
-  while (R > 2 && units(R) < 6 * device_sm_count()) R /= 2;
-  const size_t budget = 220 * 1024, stage = (size_t)R * ((size_t)k / 2 + (size_t)k / 16);
-  int ns = 0;
-  for (int n = kCsMaxStages; n >= 1; --n)
-    if (cs_fixed_bytes(krm, k, n, NC, R) + (size_t)n * stage <= budget) {
-      ns = n;
-      break;
-    }
-  G = std::min(G, ns - 2);  // at least 2 stages in flight while G are consumed
-  if (groups_env > 0) G = std::min(G, groups_env);
-  // Q4G_CS_PREFETCH: stages issued before the dependency wait (0: all), a tuning switch
-  static const int prefetch_env = getenv("Q4G_CS_PREFETCH") ? atoi(getenv("Q4G_CS_PREFETCH")) : 0;
-  p.prefetch_stages = prefetch_env;
-  if (G < 1) return false;
-  p.ns = ns;
-  p.nchunk = NC;
-  p.groups = G;
-  p.stage_rows = R;
-  p.stage_bytes = (int)stage;
-  p.n_units = units(R);
-  return true;
-}
-
-template <int KRM, int R, int BPL>
-cudaError_t launch_cs_r(const GemvParams& p, cudaStream_t st, bool pdl) {
-  static size_t configured = 0;
-  const size_t smem = cs_fixed_bytes(KRM, p.k, p.ns, p.nchunk, R) + (size_t)p.ns * p.stage_bytes;
-  cudaError_t e;
-  if (smem > configured) {
-    e = cudaFuncSetAttribute(gemv_q4_cs_kernel<KRM, R, BPL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(gemv_q4_cs_kernel<KRM, R, BPL>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess) return e;
-    configured = smem;
-  }
-  int grid = device_sm_count();
-  if (grid > p.n_units) grid = p.n_units;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kCsThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, gemv_q4_cs_kernel<KRM, R, BPL>, p);
-}
-
-template <int KRM, int BPL>
-cudaError_t launch_cs_t(const GemvParams& p, int R, cudaStream_t st, bool pdl) {
-  if (R == 8) return launch_cs_r<KRM, 8, BPL>(p, st, pdl);
-  if (R == 4) return launch_cs_r<KRM, 4, BPL>(p, st, pdl);
-  return launch_cs_r<KRM, 2, BPL>(p, st, pdl);
 }
 
 // ---------------------------------------------------------------------------
@@ -1459,8 +1086,6 @@ __global__ void __launch_bounds__(kStageThreads, 1) gemv_q4_stage_kernel(const G
         cs_issue<R>(p, u0 + issued, stages + issued * SB, &full[issued], false, pol);
         if (issued < 64) stamp(8 + issued);
       }
-      // all own loads issued: start the next GEMV's weights towards L2
-      if (issued == n_st) prefetch_next(p.next, blockIdx.x, gridDim.x);
     }
     float best_v = -INFINITY;  // of activation row j (head)
     int best_i = 0x7fffffff;
@@ -1498,7 +1123,6 @@ __global__ void __launch_bounds__(kStageThreads, 1) gemv_q4_stage_kernel(const G
           cs_issue<R>(p, u0 + t + NS, stages + s * SB, &full[s], false, pol);
           if (t + NS < 64) stamp(8 + t + NS);
           issued = t + NS + 1;
-          if (issued == n_st) prefetch_next(p.next, blockIdx.x, gridDim.x);
         }
       }
       if (++s == NS) s = 0, ph ^= 1u;
@@ -1548,7 +1172,7 @@ __global__ void __launch_bounds__(kStageThreads, 1) gemv_q4_stage_kernel(const G
 
 // Plan of the stage kernel: R rows per stage (about 16-36 KB), NC = 32-block
 // chunks, G row groups of RG rows, NS slots within the shared-memory budget.
-bool plan_stage(GemvParams& p, int& R, int& RG, bool forced) {
+bool plan_stage(GemvParams& p, int& R, int& RG) {
   const int k = p.k, nb = k >> 5;
   if (k % 256 != 0 || p.kr > 4) return false;
   if (p.epi == EPI_GEGLU && (p.nseg != 2 || p.seg[0].rows != p.seg[1].rows || p.seg[0].rows % 8)) return false;
@@ -1557,16 +1181,12 @@ bool plan_stage(GemvParams& p, int& R, int& RG, bool forced) {
     if (!aligned16(p.seg[s].qs) || !aligned16(p.seg[s].sc) || (s < p.nseg - 1 && p.seg[s].rows % 16))
       return false;
   if (p.pro == PRO_X16 && (!aligned16(p.x) || (p.kr > 1 && p.x_stride % 8))) return false;
-  (void)forced;
   const int NC = (nb + 31) / 32;
   if (NC > kStageCompute) return false;
   const int krm = p.kr <= 1 ? 1 : p.kr <= 2 ? 2 : 4;
   const size_t row_bytes = (size_t)k / 2 + (size_t)k / 16;
-  // Q4G_STAGE_ROWS (2, 4, 8, 16) forces the stage rows: a tuning switch
-  static const int rows_env = getenv("Q4G_STAGE_ROWS") ? atoi(getenv("Q4G_STAGE_ROWS")) : 0;
   R = 16;
   while (R > 2 && (size_t)R * row_bytes > 36 * 1024) R /= 2;
-  if (rows_env == 2 || rows_env == 4 || rows_env == 8 || rows_env == 16) R = rows_env;
   if (p.epi == EPI_GEGLU) R = std::max(R, 4);
   while (R * krm > 32) R /= 2;  // one reducer lane per (row, activation row)
   auto units = [&](int r) { return p.epi == EPI_GEGLU ? p.seg[0].rows / (r / 2) : (p.n_rows + r - 1) / r; };
@@ -1594,10 +1214,8 @@ bool plan_stage(GemvParams& p, int& R, int& RG, bool forced) {
     }
   if (ns < 4) return false;
   // stages issued before the dependency wait: measured best at 2 (more delays
-  // the prologue's own loads behind the weight stream); Q4G_CS_PREFETCH
-  // overrides it (0: all), a tuning switch
-  static const int prefetch_env = getenv("Q4G_CS_PREFETCH") ? atoi(getenv("Q4G_CS_PREFETCH")) : 2;
-  p.prefetch_stages = prefetch_env;
+  // the prologue's own loads behind the weight stream)
+  p.prefetch_stages = 2;
   p.ns = ns;
   p.nchunk = NC;
   p.groups = G;
@@ -1651,358 +1269,11 @@ cudaError_t launch_stage_t(const GemvParams& p, int R, int RG, cudaStream_t st, 
   }
 }
 
-// ---------------------------------------------------------------------------
-// Chain of q4_0 GEMVs in one persistent launch (one activation row).
-//
-// The GEMVs between two attention kernels of a decode step -- O(l),
-// gate|up(l), down(l) and QKV(l+1) -- depend on each other only through their
-// activations, never through their weights. One cooperative launch of one CTA
-// per SM runs them as phases:
-//   * the producer warp streams this CTA's unit range of every phase, phase
-//     after phase, through one ring of NS stage slots (one or two bulk copies
-//     per operand), never waiting for activations, so HBM keeps streaming
-//     while the consumers cross from one phase to the next;
-//   * before a phase the consumer warps wait until every CTA has finished the
-//     previous phase (a grid-wide counter, bounded wait), then build the
-//     integer digits of x for their own 32-column block straight into
-//     registers (RMSNorm reductions over the CTA use a named barrier that the
-//     producer never joins);
-//   * each stage is consumed as in the column-split kernel: warp (g, c) takes
-//     chunk c of the stages g, g + G, ...; the last of the NC warps of a stage
-//     adds the chunk partials in chunk order and runs the epilogue; the warp
-//     that completes the CTA's last stage of a phase publishes it grid-wide.
-// ---------------------------------------------------------------------------
-constexpr int kChainConsumers = 16;
-constexpr int kChainThreads = (kChainConsumers + 1) * 32;
-constexpr int kChainStages = 5;         // ring slots
-constexpr int kChainSlotBytes = 36864;  // largest stage: 16 rows x 4096 or 8 rows x 8192 columns
-constexpr int kChainMaxRows = 16;       // rows per stage
+// Kernel choice (q4g_set_gemv_kernel): -1 automatic, 1 warp-streamed,
+// 2 register path, 3 stage kernel.
+std::atomic<int> g_kernel_choice{-1};
 
-Q4G_DEV void consumer_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kChainConsumers * 32) : "memory"); }
-
-Q4G_DEV int ld_acquire(const int32_t* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-// Integer digits (block_dot_int layout) of the 32 x values of block blk of
-// phase P's activation row, for one lane. PRO_RESID: the 512 consumer threads
-// first compute the normed row together (one round of loads, two reductions
-// over the consumer barrier in a fixed warp order) into the fp16 buffer xs;
-// every consumer warp calls this, warps without a block get zeros.
-constexpr int kChainMaxK = 8192;  // PRO_RESID rows
-
-Q4G_DEV void chain_digits(const GemvParams& P, int blk, bool has, float* s_norm, __half* xs,
-                          uint4 (&g)[kDigitQuads], int4& cv) {
-  const int k = P.k, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  constexpr int NT = kChainConsumers * 32;
-  uint4 xv[4];
-  if (P.pro == PRO_X16) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      xv[q] = has ? *reinterpret_cast<const uint4*>(P.x + (size_t)blk * 32 + 8 * q) : make_uint4(0, 0, 0, 0);
-  } else {
-    constexpr int R4 = kChainMaxK / (4 * NT);
-    const int n4 = k >> 2;
-    const float4* rin = reinterpret_cast<const float4*>(P.r_in);
-    const float4* dl = reinterpret_cast<const float4*>(P.delta);
-    const float4* wd = reinterpret_cast<const float4*>(P.w_delta);
-    const float4* wx = reinterpret_cast<const float4*>(P.w_x);
-    float4 rn[R4], dv[R4], wdv[R4], wxv[R4];
-    const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int i = 0; i < R4; ++i) {  // one round of loads
-      const int c4 = tid + i * NT;
-      const bool in = c4 < n4;
-      rn[i] = in ? rin[c4] : z4;
-      wxv[i] = in ? wx[c4] : z4;
-      dv[i] = in && dl ? dl[c4] : z4;
-      wdv[i] = in && dl ? wd[c4] : z4;
-    }
-    if (dl) {
-      float ss = 0.f;
-#pragma unroll
-      for (int i = 0; i < R4; ++i)
-        ss = fmaf(dv[i].x, dv[i].x, fmaf(dv[i].y, dv[i].y, fmaf(dv[i].z, dv[i].z, fmaf(dv[i].w, dv[i].w, ss))));
-      ss = warp_sum(ss);
-      if (lane == 0) s_norm[warp] = ss;
-      consumer_bar();
-      float tot = 0.f;
-#pragma unroll
-      for (int w = 0; w < kChainConsumers; ++w) tot += s_norm[w];
-      const float inv_d = rms_inv(tot, k, P.eps);
-#pragma unroll
-      for (int i = 0; i < R4; ++i) {
-        rn[i].x = __fmul_rn(__fadd_rn(rn[i].x, __fmul_rn(__fmul_rn(dv[i].x, inv_d), wdv[i].x)), P.scale);
-        rn[i].y = __fmul_rn(__fadd_rn(rn[i].y, __fmul_rn(__fmul_rn(dv[i].y, inv_d), wdv[i].y)), P.scale);
-        rn[i].z = __fmul_rn(__fadd_rn(rn[i].z, __fmul_rn(__fmul_rn(dv[i].z, inv_d), wdv[i].z)), P.scale);
-        rn[i].w = __fmul_rn(__fadd_rn(rn[i].w, __fmul_rn(__fmul_rn(dv[i].w, inv_d), wdv[i].w)), P.scale);
-      }
-    }
-    float ss2 = 0.f;
-#pragma unroll
-    for (int i = 0; i < R4; ++i) {
-      const int c4 = tid + i * NT;
-      ss2 = fmaf(rn[i].x, rn[i].x, fmaf(rn[i].y, rn[i].y, fmaf(rn[i].z, rn[i].z, fmaf(rn[i].w, rn[i].w, ss2))));
-      if (blockIdx.x == 0 && c4 < n4) {
-        reinterpret_cast<float4*>(P.r_out)[c4] = rn[i];
-        if (P.dump) reinterpret_cast<float4*>(P.dump)[c4] = rn[i];
-      }
-    }
-    ss2 = warp_sum(ss2);
-    if (lane == 0) s_norm[kChainConsumers + warp] = ss2;
-    consumer_bar();
-    float tot2 = 0.f;
-#pragma unroll
-    for (int w = 0; w < kChainConsumers; ++w) tot2 += s_norm[kChainConsumers + w];
-    const float inv_r = rms_inv(tot2, k, P.eps);
-#pragma unroll
-    for (int i = 0; i < R4; ++i) {
-      const int c4 = tid + i * NT;
-      if (c4 < n4) {
-        __half2* dst = reinterpret_cast<__half2*>(xs + 4 * c4);
-        dst[0] = __floats2half2_rn(__fmul_rn(__fmul_rn(rn[i].x, inv_r), wxv[i].x),
-                                   __fmul_rn(__fmul_rn(rn[i].y, inv_r), wxv[i].y));
-        dst[1] = __floats2half2_rn(__fmul_rn(__fmul_rn(rn[i].z, inv_r), wxv[i].z),
-                                   __fmul_rn(__fmul_rn(rn[i].w, inv_r), wxv[i].w));
-      }
-    }
-    consumer_bar();
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      xv[q] = has ? *reinterpret_cast<const uint4*>(xs + (size_t)blk * 32 + 8 * q) : make_uint4(0, 0, 0, 0);
-  }
-  lane_block_digits(xv, g, cv);
-  if (!has) cv = make_int4(0, 0, 0, 0);  // a lane without a block: zero digits and x scale
-}
-
-struct ChainShared {
-  alignas(16) __half xs[kChainMaxK];                    // the normed activation row (PRO_RESID), read as uint4
-  alignas(16) float red[kChainStages][kCsMaxConsumers][kChainMaxRows];  // [slot][chunk][row]
-  uint64_t full[kChainStages];   // the stage's bytes landed
-  uint64_t ready[kChainStages];  // every compute warp wrote its partials of the stage
-  float norm[2 * kChainConsumers];
-  int abort_flag;
-};
-
-Q4G_DEV void chain_issue_r(const GemvParams& P, int u, unsigned char* st, uint64_t* bar, uint64_t pol) {
-  if (P.stage_rows == 16) cs_issue<16>(P, u, st, bar, false, pol);
-  else if (P.stage_rows == 8) cs_issue<8>(P, u, st, bar, false, pol);
-  else cs_issue<4>(P, u, st, bar, false, pol);
-}
-
-// Units of phase P owned by this CTA.
-Q4G_DEV void chain_range(const GemvParams& P, int& u0, int& n_st) {
-  u0 = (int)((long long)blockIdx.x * P.n_units / gridDim.x);
-  n_st = (int)((long long)(blockIdx.x + 1) * P.n_units / gridDim.x) - u0;
-}
-
-// The GEMVs of one decode layer (O, gate|up, down, next QKV) in one persistent
-// launch, one CTA per SM, built like the stage kernel: one ring of
-// kChainStages slots runs through all phases in order, compute warp (c, g)
-// takes chunk c of row group g (4 rows) of every stage, and the reducer warp
-// adds the partials, runs the phase's epilogue and refills the slot with the
-// next stage of the whole sequence, which may belong to a later phase: the
-// weights keep streaming while the compute warps wait for the previous phase
-// to finish everywhere (a per-phase counter every CTA bumps once its last
-// stage of the phase is reduced) and build the next x digits. Every wait is
-// bounded; the launch is cooperative, so all CTAs are resident.
-__global__ void __launch_bounds__(kChainThreads, 1) gemv_q4_chain_kernel(const ChainParams c) {
-  extern __shared__ __align__(128) unsigned char chain_stages[];  // [kChainStages][kChainSlotBytes]
-  __shared__ __align__(16) ChainShared sh;
-  constexpr int RG = 4;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool reducer = warp == kChainConsumers;
-  const int NS = kChainStages;
-  const uint64_t pol = policy_evict_first();
-
-  if (tid == 0) {
-    sh.abort_flag = 0;
-    for (int s = 0; s < NS; ++s) mbar_init(&sh.full[s], 1), mbar_init(&sh.ready[s], kChainConsumers);
-    fence_mbar_init();
-  }
-  __syncthreads();
-  volatile int* abort_flag = &sh.abort_flag;
-  const bool tr = c.trace && blockIdx.x == 0;
-  auto stamp = [&](int slot) {
-    if (tr) c.trace[slot] = global_ns();
-  };
-  // GemvParams-shaped view for the bounded waits (err word and limit)
-  GemvParams wp{};
-  wp.err = c.err;
-  wp.wait_ns = c.wait_ns;
-  // the whole stage sequence of this CTA: phase ph holds global stages
-  // [base[ph], base[ph] + cnt[ph])
-  int base[kChainMaxPhases + 1], u0s[kChainMaxPhases];
-  base[0] = 0;
-  for (int ph = 0; ph < c.n_ph; ++ph) {
-    int n;
-    chain_range(c.ph[ph], u0s[ph], n);
-    base[ph + 1] = base[ph] + n;
-  }
-  const int total = base[c.n_ph];
-  auto issue = [&](int T) {  // global stage T into slot T % NS
-    int ph = 0;
-    while (T >= base[ph + 1]) ++ph;
-    chain_issue_r(c.ph[ph], u0s[ph] + T - base[ph], chain_stages + (size_t)(T % NS) * kChainSlotBytes,
-                  &sh.full[T % NS], pol);
-    if (T == base[ph + 1] - 1) stamp(2 + 4 * ph + 3);
-  };
-
-  if (reducer) {
-    // ---------------- reducer: partials -> epilogue, refill, phase counters ----------------
-    int issued = 0;
-    if (lane == 0)
-      for (; issued < NS && issued < total; ++issued) issue(issued);
-    int T = 0;
-    for (int ph = 0; ph < c.n_ph && !*abort_flag; ++ph) {
-      const GemvParams& P = c.ph[ph];
-      const int R = P.stage_rows, NC = P.nchunk;
-      for (int i = 0; i < base[ph + 1] - base[ph]; ++i, ++T) {
-        const int s = T % NS;
-        if (!*abort_flag) cs_wait(&sh.ready[s], (uint32_t)((T / NS) & 1), wp, abort_flag);
-        if (*abort_flag) break;
-        float val = 0.f;
-        if (lane < R)
-          for (int cc = 0; cc < NC; ++cc) val += sh.red[s][cc][lane];
-        const int u = u0s[ph] + i;
-        if (P.epi == EPI_GEGLU) {
-          const float up = __shfl_sync(0xffffffffu, val, (lane + R / 2) & 31);
-          if (lane < R / 2) P.act[(size_t)(R / 2) * u + lane] = __float2half_rn(gelu_tanh(val) * up);
-        } else if (lane < R && R * u + lane < P.n_rows) {
-          P.y[R * u + lane] = val;
-        }
-        __syncwarp();  // every lane read slot s's partials before the refill
-        if (lane == 0) {
-          if (T + NS < total) issue(T + NS), issued = T + NS + 1;
-          if (i == base[ph + 1] - base[ph] - 1) {
-            // this CTA's outputs of the phase, visible GPU-wide before the count
-            __threadfence();
-            atomicAdd(&c.done[ph], 1);
-            stamp(2 + 4 * ph + 2);
-          }
-        }
-      }
-      if (base[ph + 1] == base[ph] && lane == 0) {
-        __threadfence();
-        atomicAdd(&c.done[ph], 1);
-      }
-    }
-    // after a timeout, wait (bounded) for the copies still in flight
-    if (lane == 0 && *abort_flag)
-      for (int i = issued > NS ? issued - NS : 0; i < issued; ++i)
-        mbar_wait_bounded(&sh.full[i % NS], (uint32_t)((i / NS) & 1), c.wait_ns);
-    return;
-  }
-
-  // ---------------- compute warps ----------------
-  if (tid == 0) stamp(0);
-  pdl_wait();
-  if (tid == 0) stamp(1);
-  for (int ph = 0; ph < c.n_ph; ++ph) {
-    const GemvParams& P = c.ph[ph];
-    const int NC = P.nchunk, G = P.groups, R = P.stage_rows, nb = P.k >> 5, kh = P.k >> 1;
-    if (ph == c.n_ph - 1) pdl_launch_dependents();
-    // every CTA finished the previous phase: its outputs are this phase's input
-    if (ph > 0) {
-      if (tid == 0 && !*abort_flag) {
-        const uint64_t t0 = global_ns();
-        for (int it = 0;; ++it) {
-          if (ld_acquire(&c.done[ph - 1]) >= (int)gridDim.x) break;
-          if (it >= kSpinLimit || global_ns() - t0 > c.wait_ns) {
-            *abort_flag = 1;
-            atomicOr(c.err, 1);
-            break;
-          }
-          __nanosleep(64);
-        }
-      }
-      consumer_bar();  // orders every compute thread after thread 0's acquire
-    }
-    if (tid == 0) stamp(2 + 4 * ph);
-    const bool active = warp < NC * G;
-    const int cidx = warp % NC, g = warp / NC;
-    const int blk = 32 * cidx + lane;
-    const bool has = active && blk < nb;
-    uint4 xg[kDigitQuads];
-    int4 cv;
-    chain_digits(P, blk, has, sh.norm, sh.xs, xg, cv);
-    const float xsc = __int_as_float(cv.w);  // 0 for a lane without a block
-    if (tid == 0) stamp(2 + 4 * ph + 1);
-    const int bq = min(blk, nb - 1);
-    // after a timeout the loops run on without waiting or computing: every
-    // compute warp reaches every consumer barrier of the later phases
-    for (int T = base[ph]; T < base[ph + 1]; ++T) {
-      const int s = T % NS;
-      if (!*abort_flag) cs_wait(&sh.full[s], (uint32_t)((T / NS) & 1), wp, abort_flag);
-      if (active && !*abort_flag) {
-        const unsigned char* st = chain_stages + (size_t)s * kChainSlotBytes;
-        const unsigned char* sq = st + (size_t)g * RG * kh + 16 * bq;
-        const unsigned char* ss = st + (size_t)R * kh + (size_t)g * RG * 2 * nb + 2 * bq;
-        float v[RG];
-#pragma unroll
-        for (int r = 0; r < RG; ++r) {
-          const uint4 qv = *reinterpret_cast<const uint4*>(sq + r * kh);
-          const float d = __half2float(*reinterpret_cast<const __half*>(ss + r * 2 * nb));
-          v[r] = d * xsc * block_dot_int(qv, xg, cv);
-        }
-        const float tot = cs_reduce_rows<RG>(v, lane);
-        if ((lane & (32 / RG - 1)) == 0) sh.red[s][cidx][g * RG + cs_row<RG>(lane)] = tot;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh.ready[s]);  // release of the partials above
-    }
-  }
-  if (tid == 0) stamp(18);
-}
-
-// Plan of one chain phase: rows per stage within a slot, chunks, groups.
-bool plan_chain_phase(GemvParams& p) {
-  const int k = p.k, nb = k >> 5;
-  if (k % 256 != 0 || p.kr != 1 || p.epi == EPI_HEAD) return false;
-  if (p.epi == EPI_GEGLU && (p.nseg != 2 || p.seg[0].rows != p.seg[1].rows)) return false;
-  if (p.pro == PRO_RESID && k > kChainMaxK) return false;
-  for (int s = 0; s < p.nseg; ++s)
-    if (!aligned16(p.seg[s].qs) || !aligned16(p.seg[s].sc)) return false;
-  if (p.pro == PRO_X16 && !aligned16(p.x)) return false;
-  const int NC = (nb + 31) / 32;
-  if (NC > kChainConsumers) return false;
-  const size_t row_bytes = (size_t)k / 2 + (size_t)k / 16;
-  auto units = [&](int r) { return p.epi == EPI_GEGLU ? p.seg[0].rows / (r / 2) : (p.n_rows + r - 1) / r; };
-  // rows per stage: a multiple of the 4-row groups, within a slot and within
-  // the 16 compute warps
-  auto fits = [&](int r) { return (size_t)r * row_bytes <= (size_t)kChainSlotBytes && NC * (r / 4) <= kChainConsumers; };
-  int R = kChainMaxRows;
-  while (R > 4 && !fits(R)) R /= 2;
-  if (!fits(R)) return false;
-  while (R > 4 && units(R) < device_sm_count()) R /= 2;  // small matrices: more, smaller stages
-  if (p.epi == EPI_GEGLU && p.seg[0].rows % (R / 2)) return false;
-  for (int s = 0; s + 1 < p.nseg; ++s)
-    if (p.seg[s].rows % R) return false;  // no stage straddles two segments
-  p.stage_rows = R;
-  p.nchunk = NC;
-  p.groups = R / 4;
-  p.stage_bytes = (int)((size_t)R * row_bytes);
-  p.n_units = units(R);
-  return p.n_units >= 1;
-}
-
-// Kernel choice: Q4G_GEMV_KERNEL = "cs" (column-split) | "ws" (warp-streamed) |
-// "reg" (register path); default: cs where it plans, else ws, else reg.
-// -1 auto, 0 column-split, 1 warp-streamed, 2 register path; -2: not read yet
-std::atomic<int> g_kernel_choice{-2};
-
-int gemv_kernel_choice() {
-  int c = g_kernel_choice.load(std::memory_order_relaxed);
-  if (c == -2) {
-    const char* e = getenv("Q4G_GEMV_KERNEL");
-    c = !e ? -1 : e[0] == 'c' ? 0 : e[0] == 'w' ? 1 : e[0] == 's' ? 3 : 2;
-    int expected = -2;
-    if (!g_kernel_choice.compare_exchange_strong(expected, c)) c = expected;
-  }
-  return c;
-}
+int gemv_kernel_choice() { return g_kernel_choice.load(std::memory_order_relaxed); }
 
 template <int KRM>
 cudaError_t launch_t(const GemvParams& p, cudaStream_t st, bool pdl) {
@@ -2058,52 +1329,6 @@ int gemv_max_rows(int k) {
   return best;
 }
 
-NextGemv gemv_next_desc(const GemvParams& p_in, float frac) {
-  NextGemv nx{};
-  GemvParams p = p_in;
-  int dot = gemv_dot_kind(), R = 0, BPL = 1;
-  const int choice = gemv_kernel_choice();
-  GemvParams px = p_in;
-  int RG = 2;
-  if ((choice == 3 || choice == -1) && plan_stage(px, R, RG, choice == 3)) {
-    for (int s = 0; s < 3; ++s) nx.seg[s] = px.seg[s];
-    nx.nseg = px.nseg;
-    nx.k = px.k;
-    nx.n_units = px.n_units;
-    nx.unit_rows = R;
-    nx.geglu = px.epi == EPI_GEGLU;
-    nx.tw = std::min(device_sm_count(), px.n_units);
-    nx.frac = frac;
-    return nx;
-  }
-  px = p_in;
-  if (choice <= 0 && plan_cs(px, R, BPL, choice == 0)) {
-    // one stream per CTA: the first units of every CTA's range
-    for (int s = 0; s < 3; ++s) nx.seg[s] = px.seg[s];
-    nx.nseg = px.nseg;
-    nx.k = px.k;
-    nx.n_units = px.n_units;
-    nx.unit_rows = R;
-    nx.geglu = px.epi == EPI_GEGLU;
-    nx.tw = std::min(device_sm_count(), px.n_units);
-    nx.frac = frac;
-    return nx;
-  }
-  if (choice == 2 || !plan_tma(p, dot)) return nx;
-  int grid = device_sm_count();
-  const int min_units = (p.n_units + kWarps - 1) / kWarps;
-  if (grid > min_units) grid = min_units;
-  for (int s = 0; s < 3; ++s) nx.seg[s] = p.seg[s];
-  nx.nseg = p.nseg;
-  nx.k = p.k;
-  nx.n_units = p.n_units;
-  nx.unit_rows = 2;
-  nx.geglu = p.epi == EPI_GEGLU;
-  nx.tw = grid * kWarps;
-  nx.frac = frac;
-  return nx;
-}
-
 int32_t* device_error_word() {
   static int32_t* ptr[64];
   int dev = 0;
@@ -2120,8 +1345,8 @@ int32_t* device_error_word() {
 cudaError_t launch_gemv(const GemvParams& p_in, cudaStream_t st, bool pdl) {
   GemvParams p = p_in;
   const int choice = gemv_kernel_choice();
-  int R = 0, BPL = 1, RG = 2;
-  if ((choice == 3 || choice == -1) && plan_stage(p, R, RG, choice == 3)) {
+  int R = 0, RG = 2;
+  if ((choice == 3 || choice == -1) && plan_stage(p, R, RG)) {
     if (!p.err) p.err = device_error_word();
     if (!p.err) return cudaErrorInvalidValue;
     if (!p.wait_ns) p.wait_ns = 2000000000ull;
@@ -2129,15 +1354,7 @@ cudaError_t launch_gemv(const GemvParams& p_in, cudaStream_t st, bool pdl) {
     return p.kr > 1 ? launch_stage_t<2>(p, R, RG, st, pdl) : launch_stage_t<1>(p, R, RG, st, pdl);
   }
   p = p_in;
-  if (choice <= 0 && plan_cs(p, R, BPL, choice == 0)) {
-    if (!p.err) p.err = device_error_word();
-    if (!p.err) return cudaErrorInvalidValue;
-    if (!p.wait_ns) p.wait_ns = 2000000000ull;
-    if (p.kr > 1) return launch_cs_t<2, 1>(p, R, st, pdl);
-    return BPL == 2 ? launch_cs_t<1, 2>(p, R, st, pdl) : launch_cs_t<1, 1>(p, R, st, pdl);
-  }
-  p = p_in;
-  int dot = gemv_dot_kind();
+  int dot = -1;
   if (choice != 2 && plan_tma(p, dot)) {
     if (!p.err) p.err = device_error_word();
     if (!p.err) return cudaErrorInvalidValue;
@@ -2311,54 +1528,9 @@ cudaError_t launch_gemv_f16(const GemvParams& p, cudaStream_t st, bool pdl) {
 }
 
 bool set_gemv_kernel_choice(int kind) {
-  if (kind < 0 || kind > 4) return false;
+  if (kind < 0 || kind > 4 || kind == 1) return false;
   g_kernel_choice.store(kind - 1);
   return true;
-}
-
-bool plan_chain(ChainParams& c) {
-  if (c.n_ph < 1 || c.n_ph > kChainMaxPhases || gemv_kernel_choice() > 0) return false;
-  for (int i = 0; i < c.n_ph; ++i)
-    if (!plan_chain_phase(c.ph[i])) return false;
-  return true;
-}
-
-cudaError_t launch_gemv_chain(const ChainParams& c_in, cudaStream_t st, bool pdl) {
-  ChainParams c = c_in;
-  if (!c.err) c.err = device_error_word();
-  if (!c.err) return cudaErrorInvalidValue;
-  if (!c.wait_ns) c.wait_ns = 2000000000ull;
-  static bool configured = false;
-  const size_t smem = (size_t)kChainStages * kChainSlotBytes;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_q4_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(gemv_q4_chain_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
-  // one CTA per SM, and at least one unit of every phase per CTA
-  int grid = device_sm_count();
-  for (int i = 0; i < c.n_ph; ++i) grid = std::min(grid, c.ph[i].n_units);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kChainThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[2];
-  int na = 0;
-  attr[na].id = cudaLaunchAttributeCooperative;  // all CTAs resident: the phases wait on each other
-  attr[na].val.cooperative = 1;
-  ++na;
-  if (pdl) {
-    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[na].val.programmaticStreamSerializationAllowed = 1;
-    ++na;
-  }
-  cfg.attrs = attr;
-  cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, gemv_q4_chain_kernel, c);
 }
 
 int device_sm_count() {

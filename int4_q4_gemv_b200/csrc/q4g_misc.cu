@@ -85,10 +85,6 @@ __global__ void step_init_kernel(const StepParams p) {
     }
     p.r_out[(size_t)j * p.hidden_size + c] = v;
     if (p.dump) p.dump[(size_t)j * p.dump_stride + c] = v;
-    if (p.r_tagged && j == 0) {  // tag of this step's layer-0 input: epoch * 128 + 0
-      const uint64_t w = ((uint64_t)(p.epoch * 128u) << 32) | __float_as_uint(v);
-      asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p.r_tagged + c), "l"(w) : "memory");
-    }
     return;
   }
   // last block: tables and state
@@ -108,7 +104,6 @@ __global__ void step_init_kernel(const StepParams p) {
   }
   for (int t = threadIdx.x; t < p.n_counters; t += blockDim.x) p.counters[t] = 0;
   if (threadIdx.x == 0) *p.pos_dev = p.pos0;
-  if (threadIdx.x == 0 && p.epoch_dev) *p.epoch_dev = p.epoch;
 }
 
 }  // namespace

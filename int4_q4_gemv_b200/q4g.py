@@ -15,13 +15,9 @@ LIB_PATH = os.path.join(_HERE, "libq4g.so")
 Q4G_OK, Q4G_EINVAL, Q4G_ERANGE, Q4G_ENOMEM, Q4G_ECUDA, Q4G_ETIMEOUT = range(6)
 Q4G_OPT_CUDA_GRAPH, Q4G_OPT_PDL, Q4G_OPT_DUMP, Q4G_OPT_PROFILE, Q4G_OPT_TEST_STALL = 1, 2, 3, 4, 5
 Q4G_OPT_ATTN_CLUSTER = 6
-Q4G_OPT_GEMV_CHAIN = 7
 Q4G_OPT_TRACE = 8
-Q4G_OPT_STEP_KERNEL = 9
-Q4G_OPT_STEP_POLL_NS = 10
-Q4G_OPT_STEP_GRID_SYNC = 11
 KIND_NAMES = ["step_init", "qkv_gemv", "attn_sliding", "attn_full", "attn_combine", "o_gemv",
-              "gate_up_gemv", "down_gemv", "head_gemv", "chain_gemv", "step_kernel"]
+              "gate_up_gemv", "down_gemv", "head_gemv"]
 
 EXPORTS = [
     "q4g_last_error", "q4g_status_string", "q4g_abi_version",
@@ -159,7 +155,7 @@ def q4g_gemv_f16(w16, n, k, x_f16, nrhs, y, stream):
     _call("q4g_gemv_f16", w16, n, k, x_f16, nrhs, y, stream)
 
 
-Q4G_GEMV_AUTO, Q4G_GEMV_COLUMN_SPLIT, Q4G_GEMV_WARP_STREAM, Q4G_GEMV_REGISTER, Q4G_GEMV_STAGE = 0, 1, 2, 3, 4
+Q4G_GEMV_AUTO, Q4G_GEMV_WARP_STREAM, Q4G_GEMV_REGISTER, Q4G_GEMV_STAGE = 0, 2, 3, 4
 
 
 def q4g_set_gemv_kernel(kind):

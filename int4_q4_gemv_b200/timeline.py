@@ -36,7 +36,6 @@ def main() -> None:
     a = ap.parse_args()
     cfg = dict(WL.B12, n_layers=a.layers)
     g = S.SynthDecoder(cfg, seed=0)
-    Q.q4g_model_set_option(g.handle, Q.Q4G_OPT_STEP_KERNEL, 0)  # the per-kernel path's trace layout
     c = g.new_cache(a.context)
     S.fill_history(c)
     sp = S.stream_ptr()

@@ -55,9 +55,9 @@ def check_logits(got, ref, where=""):
 class Pair:
     """GPU model + cache and oracle model + cache on the same seeded recipe."""
 
-    def __init__(self, cfg, seed=0, variant=0, capacity=1024, step_kernel=None):
+    def __init__(self, cfg, seed=0, variant=0, capacity=1024):
         self.cfg = cfg
-        self.gpu = S.SynthDecoder(cfg, seed=seed, variant=variant, step_kernel=step_kernel)
+        self.gpu = S.SynthDecoder(cfg, seed=seed, variant=variant)
         self.gc = self.gpu.new_cache(capacity)
         self.orc = O.Model(cfg, seed=seed, variant=variant)
         self.oc = O.Cache(self.orc, capacity)
@@ -81,11 +81,9 @@ class Pair:
         return self.logits[0].cpu().numpy().astype(np.float64), int(self.am[0]), r["logits"], int(r["argmax"][0])
 
 
-@pytest.fixture(scope="module", params=[1, 0], ids=["step_kernel", "per_kernel"])
-def tiny(request):
-    """The tiny decoder on both decode paths: the persistent step kernel and one
-    launch per kernel."""
-    return Pair(WL.TINY, seed=0, variant=0, capacity=512, step_kernel=request.param)
+@pytest.fixture(scope="module")
+def tiny():
+    return Pair(WL.TINY, seed=0, variant=0, capacity=512)
 
 
 def test_tiny_weights_bitexact(tiny):
@@ -127,11 +125,10 @@ def test_tiny_config1_prefill_then_greedy(tiny):
     assert gpu_seq == ref_seq
 
 
-@pytest.mark.parametrize("step", [1, 0])
-def test_tiny_free_greedy_on_device_tokens(step):
+def test_tiny_free_greedy_on_device_tokens():
     """The GPU's own greedy loop (token read from the previous argmax on the device)
-    reproduces the oracle's greedy sequence, on both decode paths."""
-    p = Pair(WL.TINY, seed=3, variant=1, capacity=512, step_kernel=step)
+    reproduces the oracle's greedy sequence."""
+    p = Pair(WL.TINY, seed=3, variant=1, capacity=512)
     tok = torch.zeros(1, dtype=torch.int32, device="cuda")
     am = torch.zeros(64, dtype=torch.int32, device="cuda")
     ref_tok, seq_ref = 7, []
@@ -147,19 +144,15 @@ def test_tiny_free_greedy_on_device_tokens(step):
     assert am.cpu().tolist() == seq_ref
 
 
-@pytest.mark.parametrize("step,cluster,chain", [(1, 1, 0), (0, 1, 1), (0, 0, 0)])
-def test_wrap_heavy_ring_and_layer_dumps(step, cluster, chain):
+@pytest.mark.parametrize("cluster", [1, 0])
+def test_wrap_heavy_ring_and_layer_dumps(cluster):
     """300 positions through a ring of 64 slots (> 4 wraps), seeded gains and layer
-    scalars; residual stream compared after every layer. The persistent step
-    kernel, and the per-kernel path with both merges of the sliding-layer
-    attention chunks: in a thread-block cluster (8 CTAs per KV head, most of them
-    with no live key here) and through global memory; and the layer's GEMVs as
-    one persistent chain launch or one launch each."""
+    scalars; residual stream compared after every layer, with both merges of the
+    sliding-layer attention chunks: in a thread-block cluster (most CTAs with no
+    live key here) and through global memory."""
     cfg = WRAP
     p = Pair(cfg, seed=5, variant=1, capacity=320)
-    Q.q4g_model_set_option(p.gpu.handle, Q.Q4G_OPT_STEP_KERNEL, step)
     Q.q4g_model_set_option(p.gpu.handle, Q.Q4G_OPT_ATTN_CLUSTER, cluster)
-    Q.q4g_model_set_option(p.gpu.handle, Q.Q4G_OPT_GEMV_CHAIN, chain)
     L, H = cfg["n_layers"], cfg["hidden"]
     dump = torch.zeros((1, L + 1, H), dtype=torch.float32, device="cuda")
     Q.q4g_model_set_option(p.gpu.handle, Q.Q4G_OPT_DUMP, dump.data_ptr())
@@ -233,16 +226,13 @@ def test_capacity_invariance_and_graph_equivalence_bitwise():
     assert np.array_equal(outs[0], outs[2])
 
 
-@pytest.mark.parametrize("step", [1, 0])
-def test_bounded_wait_gives_up_and_reports_timeout(step):
+def test_bounded_wait_gives_up_and_reports_timeout():
     """Failure path without a fault: one pipeline stage of the step's first GEMV
     expects bytes that never arrive; its bounded wait gives up after 20 ms, the
     step completes, q4g_model_check reports Q4G_ETIMEOUT, and the next step on the
-    same context is clean and correct again (the persistent step kernel: every
-    CTA then gives up at its next phase boundary, also within 20 ms)."""
+    same context is clean and correct again."""
     cfg = WRAP
     p = Pair(cfg, seed=6, variant=0, capacity=64)
-    Q.q4g_model_set_option(p.gpu.handle, Q.Q4G_OPT_STEP_KERNEL, step)
     Q.q4g_model_set_option(p.gpu.handle, Q.Q4G_OPT_TEST_STALL, 1)
     Q.q4g_decode_step(p.gpu.handle, p.gc.handle, 3, 0, 0, 0, sp())
     with pytest.raises(Q.Q4GError) as e:
@@ -283,7 +273,6 @@ def test_trace_timeline_is_ordered():
     CTA, and the step's logits equal those of an untraced step."""
     cfg = WL.TINY
     g = S.SynthDecoder(cfg, seed=3, variant=0)
-    Q.q4g_model_set_option(g.handle, Q.Q4G_OPT_STEP_KERNEL, 0)
     c = g.new_cache(512)
     tr = torch.zeros(1536, dtype=torch.int64, device="cuda")
     lg = torch.empty((2, cfg["vocab"]), dtype=torch.float32, device="cuda")
@@ -314,15 +303,14 @@ def test_trace_timeline_is_ordered():
     assert n >= 1 and np.all(ends[:n] >= t[0]), n  # every CTA of gate|up, from CTA 0 up
 
 
-@pytest.mark.parametrize("step", [1, 0])
-def test_long_context_decode_vs_oracle_32k(step):
+def test_long_context_decode_vs_oracle_32k():
     """The 32K-context decode config on one period of the 12B shapes (5 sliding
     layers, 1 full layer, the 262,144-row head): both sides fill every ring slot and
     every global row from the same seeded history, then run the last two positions
-    of the context and compare logits and argmax, on both decode paths."""
+    of the context and compare logits and argmax."""
     cfg = dict(WL.B12, n_layers=WL.B12["full_every"])
     C = 32768
-    p = Pair(cfg, seed=4, variant=1, capacity=C, step_kernel=step)
+    p = Pair(cfg, seed=4, variant=1, capacity=C)
     S.fill_history(p.gc)
     O.fill_history(p.oc)
     ids = DG.uniform_int(4, DG.STREAM_PREFIX_IDS, 2, cfg["vocab"])

@@ -191,8 +191,7 @@ def test_flash_decode_linear_vs_oracle(n_q, length):
     assert np.all(np.abs(got - ref) <= 2e-3 * (1 + np.abs(ref)))
 
 
-@pytest.mark.parametrize("kind", [Q.Q4G_GEMV_COLUMN_SPLIT, Q.Q4G_GEMV_WARP_STREAM, Q.Q4G_GEMV_REGISTER,
-                                  Q.Q4G_GEMV_STAGE])
+@pytest.mark.parametrize("kind", [Q.Q4G_GEMV_WARP_STREAM, Q.Q4G_GEMV_REGISTER, Q.Q4G_GEMV_STAGE])
 @pytest.mark.parametrize("n,k,nrhs", [(3840, 15360, 1), (8192, 3840, 1), (1000, 1024, 2), (3840, 4096, 4),
                                       (260, 3840, 2), (77, 256, 1), (3840, 15360, 4), (1000, 8192, 8),
                                       (531, 3840, 3), (40, 256, 7)])
