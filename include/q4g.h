@@ -341,6 +341,8 @@ q4g_status q4g_cache_layout(const q4g_cache* c, q4g_cache_view* out);
  * pos on full layers). Sliding layers attend positions pos-W+1..pos, full layers
  * 0..pos. Writes softcapped fp32 logits [vocab] (if logits != NULL) and the
  * greedy argmax (lowest index on ties) to argmax[0] (if != NULL); device outputs.
+ * With logits and argmax both NULL (and no dump buffer set) the step only
+ * appends its K/V rows to the cache: the final norm and the head are skipped.
  * Q4G_ERANGE if pos < 0 or pos >= capacity or token outside [0, vocab).
  * The host owns the position counter; the cache holds contents only. */
 q4g_status q4g_decode_step(q4g_model* m, q4g_cache* c, int32_t token, int64_t pos, float* logits,
@@ -379,6 +381,19 @@ q4g_status q4g_decode_step_host(q4g_model* m, q4g_cache* c, int32_t token, int64
 q4g_status q4g_verify_block(q4g_model* m, q4g_cache* c, const int32_t* ids, int32_t K,
                             int64_t pos0, int32_t accepted_count, float* logits, int32_t* argmax,
                             q4g_stream_t stream);
+
+/* Chunked prefill ("Gemma-4-12B-CoreAI", tiered-v3/ section: a last-row-only
+ * prefill entry point at S = 64; "gemma-4-E4B-CoreAI", stable/ contract):
+ * tokens ids[0..S-1] (device) at positions pos0..pos0+S-1, 1 <= S <= 64, with
+ * exactly the result of S decode steps in order (row i attends what a decode
+ * step at pos0+i after rows 0..i-1 attends) up to the rounding of the
+ * multi-row GEMVs. Runs as passes of up to 4 rows, every row kept; only the
+ * last pass runs the head. Outputs the last row's logits [vocab] (if != NULL)
+ * and argmax[0] (if != NULL), device. No alignment precondition on pos0: every
+ * row is written to its own slot (pos mod R). Q4G_ERANGE: S outside 1..64,
+ * pos0 < 0, pos0 + S > capacity. */
+q4g_status q4g_prefill_chunk(q4g_model* m, q4g_cache* c, const int32_t* ids, int32_t S, int64_t pos0,
+                             float* logits, int32_t* argmax, q4g_stream_t stream);
 
 #ifdef __cplusplus
 }

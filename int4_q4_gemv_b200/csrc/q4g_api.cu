@@ -924,6 +924,7 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
       }
     }
   }
+  if (!logits && !argmax && !m->dump) return cudaSuccess;  // no output asked for: the step only fills the cache
   {
     GemvParams p = head_params();
     Prof pr(m, st);
@@ -1053,6 +1054,34 @@ extern "C" q4g_status q4g_verify_block(q4g_model* m, q4g_cache* c, const int32_t
   if (pos0 < 0 || pos0 + K > c->capacity) return fail(Q4G_ERANGE, "block outside [0, capacity)");
   if (accepted_count < 0 || accepted_count > K) return fail(Q4G_ERANGE, "accepted_count outside [0, K]");
   return run_step(m, c, K, pos0, ids, nullptr, nullptr, logits, argmax, (cudaStream_t)stream);
+}
+
+extern "C" q4g_status q4g_prefill_chunk(q4g_model* m, q4g_cache* c, const int32_t* ids, int32_t S, int64_t pos0,
+                                        float* logits, int32_t* argmax, q4g_stream_t stream) {
+  if (!m || !c || !ids) return fail(Q4G_EINVAL, "NULL argument");
+  if (S < 1 || S > kPrefillChunk) return fail(Q4G_ERANGE, "S must be 1..%d", kPrefillChunk);
+  if (pos0 < 0 || pos0 + S > c->capacity) return fail(Q4G_ERANGE, "chunk outside [0, capacity)");
+  if (logits && !aligned(logits, 4)) return fail(Q4G_EINVAL, "logits misaligned");
+  // blocks of up to 4 rows (the widest the stage GEMV takes), each one verify pass
+  // whose rows are all kept; the head runs for the last block only
+  const int kb = std::min(kPrefillBlock, m->cfg.ring - m->cfg.window);
+  const cudaStream_t st = (cudaStream_t)stream;
+  for (int b0 = 0; b0 < S; b0 += kb) {
+    const int n = std::min(kb, S - b0);
+    const bool last = b0 + n == S;
+    const bool out = last && (logits || argmax);
+    q4g_status r = run_step(m, c, n, pos0 + b0, ids + b0, nullptr, nullptr, out ? m->logits_buf : nullptr,
+                            out ? m->argmax_buf : nullptr, st);
+    if (r != Q4G_OK) return r;
+    if (out) {  // the chunk's last row
+      if (logits)
+        CK(cudaMemcpyAsync(logits, m->logits_buf + (size_t)(n - 1) * m->cfg.vocab, sizeof(float) * m->cfg.vocab,
+                           cudaMemcpyDeviceToDevice, st));
+      if (argmax)
+        CK(cudaMemcpyAsync(argmax, m->argmax_buf + (n - 1), sizeof(int32_t), cudaMemcpyDeviceToDevice, st));
+    }
+  }
+  return Q4G_OK;
 }
 
 extern "C" int32_t q4g_model_profile_read(q4g_model* m, q4g_launch_record* out, int32_t max,

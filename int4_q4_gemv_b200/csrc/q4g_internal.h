@@ -84,7 +84,9 @@ cudaError_t launch_gemv(const GemvParams& p, cudaStream_t st, bool pdl);
 // Q4G_GEMV_* kind; false if out of range
 bool set_gemv_kernel_choice(int kind);
 
-constexpr int kGemvTraceSlots = 256;  // one GEMV launch's timeline (GemvParams::trace)
+constexpr int kGemvTraceSlots = 256;
+constexpr int kPrefillChunk = 64;  // rows of one prefill call
+constexpr int kPrefillBlock = 4;   // rows per pass inside a prefill call  // one GEMV launch's timeline (GemvParams::trace)
 // Device address of the library's error word (bit 0: a bounded wait gave up).
 int32_t* device_error_word();
 

@@ -26,7 +26,7 @@ EXPORTS = [
     "q4g_model_create", "q4g_model_destroy", "q4g_model_check", "q4g_model_set_option",
     "q4g_cache_bytes", "q4g_cache_init", "q4g_cache_reset", "q4g_cache_destroy", "q4g_cache_layout",
     "q4g_decode_step", "q4g_decode_step_device_token", "q4g_decode_step_hidden",
-    "q4g_decode_step_host", "q4g_verify_block", "q4g_model_profile_read",
+    "q4g_decode_step_host", "q4g_verify_block", "q4g_prefill_chunk", "q4g_model_profile_read",
     "q4g_flash_decode_ring_noalloc", "q4g_set_gemv_kernel",
 ]
 Q4G_NOALLOC_SCRATCH_BYTES = 1 << 20
@@ -110,6 +110,7 @@ def lib() -> C.CDLL:
             "q4g_decode_step_hidden": (C.c_int, [vp, vp, vp, i64, vp, vp, vp]),
             "q4g_decode_step_host": (C.c_int, [vp, vp, i32, i64, vp, vp, vp]),
             "q4g_verify_block": (C.c_int, [vp, vp, vp, i32, i64, i32, vp, vp, vp]),
+            "q4g_prefill_chunk": (C.c_int, [vp, vp, vp, i32, i64, vp, vp, vp]),
             "q4g_model_profile_read": (i32, [vp, C.POINTER(q4g_launch_record), i32, vp]),
             "q4g_flash_decode_ring_noalloc": (C.c_int, [vp, i32, i32, i32, vp, vp, i64, i64, i64, vp, vp]),
             "q4g_set_gemv_kernel": (C.c_int, [i32]),
@@ -242,6 +243,10 @@ def q4g_decode_step_host(model, cache, token, pos, logits_host, argmax_host, str
 
 def q4g_verify_block(model, cache, ids, K, pos0, accepted_count, logits, argmax, stream):
     _call("q4g_verify_block", model, cache, ids, K, pos0, accepted_count, logits, argmax, stream)
+
+
+def q4g_prefill_chunk(model, cache, ids, S, pos0, logits, argmax, stream):
+    _call("q4g_prefill_chunk", model, cache, ids, S, pos0, logits, argmax, stream)
 
 
 def q4g_model_profile_read(model, stream, max_records: int = 1 << 16):
