@@ -338,6 +338,36 @@ def measure_verify(Q, S, DG, model, cfg, C, Kv, blocks, warm, seed, sp, stream):
     return ms, bpb, accepted
 
 
+def measure_prefill(Q, DG, model, cfg, n_tokens, seed, sp, stream):
+    """Chunked prefill of n_tokens seeded ids from position 0 into a fresh cache, in
+    64-token chunks (q4g_prefill_chunk, last row's logits of the last chunk); one
+    untimed pass first (graph capture), then the timed one on another cache."""
+    import numpy as np
+    import torch
+    V = cfg["vocab"]
+    ids = torch.from_numpy(DG.uniform_int(seed, DG.STREAM_PREFIX_IDS, n_tokens, V).astype(np.int32)).cuda()
+    lg = torch.empty(V, dtype=torch.float32, device="cuda")
+    am = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ms = None
+    for rep in range(2):
+        cache = model.new_cache(n_tokens)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for p0 in range(0, n_tokens, 64):
+            n = min(64, n_tokens - p0)
+            last = p0 + n == n_tokens
+            Q.q4g_prefill_chunk(model.handle, cache.handle, ids[p0:].data_ptr(), n, p0,
+                                lg.data_ptr() if last else 0, am.data_ptr() if last else 0, sp)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        Q.q4g_model_check(model.handle, sp)
+        cache.close()
+        del cache
+    return ms
+
+
 def time_rotating(fn, n_items, reps, stream):
     """Mean time of fn(i) over reps passes of i = 0..n_items-1 (CUDA events)."""
     import torch
@@ -591,6 +621,13 @@ def main():
             "accepted_tokens_per_s": accepted / (nb * msv / 1e3), "rows_per_s": Kv * 1e3 / msv,
             "bytes_per_block": bpb, "gbs": bpb / (msv / 1e3) / 1e9, "frac": bpb / (msv / 1e3) / 1e9 / peak,
             "accepted_count": "seeded U{0..4}", "history": "synthetic"}
+        npf = 1024
+        mspf = measure_prefill(Q, DG, model, cfg, npf, args.seed, sp, stream)
+        per_context["prefill_1024_c64"] = {
+            "kind": "prefill", "tokens": npf, "chunk": 64, "rows_per_pass": 4, "ms": mspf,
+            "tokens_per_s": npf / (mspf / 1e3),
+            "note": "64-token chunks from position 0 into a fresh cache, each as passes of 4 rows; "
+                    "the head only for the last chunk's last pass"}
         micro = microbench(Q, S, DG, WL, peak, sp, stream)
 
     cpu = None

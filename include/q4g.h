@@ -250,7 +250,9 @@ void q4g_model_destroy(q4g_model* m);
 
 /* Reports (and clears) the device-side error word that a bounded wait sets when
  * it gives up (Q4G_ETIMEOUT; every wait inside the kernels is limited in time,
- * 2 s by default) and any sticky CUDA error (Q4G_ECUDA). Synchronises `stream`. */
+ * 2 s by default) and any sticky CUDA error (Q4G_ECUDA). Synchronises `stream`.
+ * Diagnostics: with Q4G_DEBUG_SYNC set in the environment, eager (non-graph)
+ * steps synchronise after every launch and name the launch that failed. */
 q4g_status q4g_model_check(q4g_model* m, q4g_stream_t stream);
 
 /* Options (defaults in brackets): */

@@ -467,14 +467,12 @@ cudaError_t launch_ring_t(const AttnParams& p, cudaStream_t st, bool pdl) {
 }
 
 // CTAs per KV head: 16 (a non-portable cluster, twice the SMs on the scan) when
-// eight such clusters fit on the device at once, else 8; Q4G_ATTN_CLUSTER=8|16
-// forces it (a tuning switch).
+// eight such clusters fit on the device at once, else 8.
 int ring_cluster_size() {
   static int cl = 0;
   if (cl) return cl;
-  const char* env = getenv("Q4G_ATTN_CLUSTER");
-  int pick = env ? atoi(env) : 0;
-  if (pick != 8 && pick != 16) {
+  int pick = 0;
+  {
     pick = 8;
     AttnParams p{};
     p.n_kv = 8;

@@ -156,6 +156,8 @@ def _attn_ws(n_q, hd):
     (8, 2, 256, 512, 1531),        # tiny-config shape
     (4, 1, 64, 128, 0),            # a single live key
     (16, 8, 100, 160, 333),        # window not a multiple of the tile
+    (8, 8, 1024, 2048, 3001),      # one query row per KV head
+    (2, 2, 256, 512, 700),         # one row per head, few heads
 ])
 def test_flash_decode_ring_vs_oracle(n_q, n_kv, W, R, pos):
     hd = 256
@@ -173,7 +175,7 @@ def test_flash_decode_ring_vs_oracle(n_q, n_kv, W, R, pos):
     assert np.all(np.abs(got - ref) <= 2e-3 * (1 + np.abs(ref)))
 
 
-@pytest.mark.parametrize("n_q,length", [(16, 1), (16, 63), (16, 4096), (16, 20001), (8, 3000)])
+@pytest.mark.parametrize("n_q,length", [(16, 1), (16, 63), (16, 4096), (16, 20001), (8, 3000), (16, 131072)])
 def test_flash_decode_linear_vs_oracle(n_q, length):
     hd = 512
     rng = np.random.default_rng(length)
