@@ -89,6 +89,24 @@ def unit_normal(seed: int, stream: int, n: int, start: int = 0) -> np.ndarray:
     return ((s - 393210).astype(np.float32) * np.float32(1.0 / 65536.0)).astype(np.float32)
 
 
+def code8(seed: int, stream: int, n: int, start: int = 0) -> np.ndarray:
+    """Seeded int8 codes: 36 x the unit normal, rounded half to even in exact integer
+    arithmetic, clamped to [-127, 127] (the C header's dg_code8)."""
+    k = key(seed, stream)
+    idx = _indices(start, n)
+    s = np.zeros(n, dtype=np.int64)
+    mask = np.uint64(0xFFFF)
+    for j in range(3):
+        w = _word(k, idx, j)
+        for t in range(4):
+            s += ((w >> np.uint64(16 * t)) & mask).astype(np.int64)
+    t = 9 * (s - 393210)
+    q = t >> 14
+    r = t - q * 16384
+    q = q + ((r > 8192) | ((r == 8192) & ((q & 1) == 1))).astype(np.int64)
+    return np.clip(q, -127, 127).astype(np.int8)
+
+
 def normal(seed: int, stream: int, n: int, sigma: float, start: int = 0) -> np.ndarray:
     z = unit_normal(seed, stream, n, start)
     return (z * np.float32(sigma)).astype(np.float32)
@@ -125,6 +143,12 @@ def history_sigma(kv: int, hd: int) -> float:
     hd^(-1/4) (variants 0 and 1), whose elements have RMS hd^(-1/4); V rows are a
     scale-free RMSNorm, RMS 1."""
     return float(qk_gain_base(hd)) if kv == 0 else 1.0
+
+
+def history_scale8(kv: int, hd: int) -> np.float32:
+    """Row scale of the synthetic int8 K/V history: codes carry 36 per standard
+    deviation, so code x scale has the standard deviation history_sigma."""
+    return np.float32(np.float32(history_sigma(kv, hd)) / np.float32(36.0))
 
 
 def qk_gain_base(hd: int) -> np.float32:

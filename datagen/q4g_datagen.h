@@ -63,6 +63,25 @@ DG_FN float dg_unit_normal(uint64_t key, uint64_t i) {
   return (float)(s - 393210) * (1.0f / 65536.0f);
 }
 
+/* A seeded int8 code: 36 x the same Irwin-Hall(12) normal, rounded to the
+ * nearest integer (ties to even) in exact integer arithmetic, clamped to
+ * [-127, 127] (synthetic int8 K/V history; 36 codes per standard deviation). */
+DG_FN int dg_code8(uint64_t key, uint64_t i) {
+  int64_t s = 0;
+  for (unsigned j = 0; j < 3; ++j) {
+    uint64_t w = dg_word(key, i, j);
+    s += (int64_t)(w & 0xFFFFu);
+    s += (int64_t)((w >> 16) & 0xFFFFu);
+    s += (int64_t)((w >> 32) & 0xFFFFu);
+    s += (int64_t)((w >> 48) & 0xFFFFu);
+  }
+  const int64_t t = 9 * (s - 393210); /* 36 z = t / 2^14 exactly */
+  int64_t q = t >> 14;                /* floor */
+  const int64_t r = t - q * 16384;    /* 0 <= r < 2^14 */
+  if (r > 8192 || (r == 8192 && (q & 1))) q += 1;
+  return (int)(q > 127 ? 127 : (q < -127 ? -127 : q));
+}
+
 DG_FN float dg_normal(uint64_t key, uint64_t i, float sigma) {
 #ifdef __CUDA_ARCH__
   return __fmul_rn(dg_unit_normal(key, i), sigma);

@@ -23,6 +23,14 @@ __global__ void fill_uniform_int(int* out, long long n, unsigned long long key, 
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
     out[i] = (int)dg_uniform_int(key, (uint64_t)(start + i), (uint64_t)hi);
 }
+__global__ void fill_code8(int8_t* out, long long n, unsigned long long key, long long start) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+    out[i] = (int8_t)dg_code8(key, (uint64_t)(start + i));
+}
+__global__ void fill_const_f32(float* out, long long n, float v) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+    out[i] = v;
+}
 unsigned grid_for(long long n) {
   long long g = (n + 255) / 256;
   return (unsigned)(g > 65536 ? 65536 : (g < 1 ? 1 : g));
@@ -42,6 +50,15 @@ int dg_fill_normal_f16(void* out, long long n, unsigned long long seed, unsigned
 }
 int dg_fill_gain_f32(float* out, long long n, unsigned long long seed, unsigned long long stream, cudaStream_t st) {
   fill_gain_f32<<<grid_for(n), 256, 0, st>>>(out, n, dg_key(seed, stream));
+  return (int)cudaGetLastError();
+}
+int dg_fill_code8(void* out, long long n, unsigned long long seed, unsigned long long stream, long long start,
+                  cudaStream_t st) {
+  fill_code8<<<grid_for(n), 256, 0, st>>>((int8_t*)out, n, dg_key(seed, stream), start);
+  return (int)cudaGetLastError();
+}
+int dg_fill_const_f32(float* out, long long n, float v, cudaStream_t st) {
+  fill_const_f32<<<grid_for(n), 256, 0, st>>>(out, n, v);
   return (int)cudaGetLastError();
 }
 int dg_fill_uniform_int(int* out, long long n, unsigned long long seed, unsigned long long stream, long long hi,

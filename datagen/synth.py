@@ -34,6 +34,8 @@ def dglib():
             "dg_fill_normal_f16": [vp, ll, ull, ull, f, ll, vp],
             "dg_fill_gain_f32": [vp, ll, ull, ull, vp],
             "dg_fill_uniform_int": [vp, ll, ull, ull, ll, ll, vp],
+            "dg_fill_code8": [vp, ll, ull, ull, ll, vp],
+            "dg_fill_const_f32": [vp, ll, f, vp],
         }.items():
             fn = getattr(L, name)
             fn.restype = C.c_int
@@ -58,6 +60,16 @@ def fill_normal_f32(t: torch.Tensor, seed, stream_id, sigma, start=0):
 
 def fill_normal_f16(t: torch.Tensor, seed, stream_id, sigma, start=0):
     _ok(dglib().dg_fill_normal_f16(t.data_ptr(), t.numel(), seed, stream_id, sigma, start, stream_ptr()))
+
+
+def fill_code8(t: torch.Tensor, seed, stream_id, start=0):
+    assert t.dtype == torch.int8 and t.is_contiguous()
+    _ok(dglib().dg_fill_code8(t.data_ptr(), t.numel(), seed, stream_id, start, stream_ptr()))
+
+
+def fill_const(t: torch.Tensor, v: float):
+    assert t.dtype == torch.float32 and t.is_contiguous()
+    _ok(dglib().dg_fill_const_f32(t.data_ptr(), t.numel(), float(v), stream_ptr()))
 
 
 def fill_gain(t: torch.Tensor, seed, stream_id):
@@ -204,6 +216,22 @@ class SynthCache:
         n = v.gl_kv_heads * v.capacity * v.gl_head_dim
         return self.buf[off:off + 2 * n].view(torch.float16).view(v.gl_kv_heads, v.capacity, v.gl_head_dim)
 
+    def _i8(self, off, so, nkv, rows, hd):
+        codes = self.buf[off:off + nkv * rows * hd].view(torch.int8).view(nkv, rows, hd)
+        scales = self.buf[off + so:off + so + 4 * nkv * rows].view(torch.float32).view(nkv, rows)
+        return codes, scales
+
+    def ring_i8(self, i: int, kv: int):
+        """int8 cache: (codes [n_kv][R][hd] int8, scales [n_kv][R] fp32), views of the buffer."""
+        v = self.view
+        off = (v.ring_v_offset if kv else v.ring_k_offset) + i * v.ring_layer_bytes
+        return self._i8(off, v.ring_scale_offset, v.sl_kv_heads, v.ring, v.sl_head_dim)
+
+    def global_i8(self, i: int, kv: int):
+        v = self.view
+        off = (v.global_v_offset if kv else v.global_k_offset) + i * v.global_layer_bytes
+        return self._i8(off, v.global_scale_offset, v.gl_kv_heads, v.capacity, v.gl_head_dim)
+
     def close(self):
         if getattr(self, "handle", None):
             Q.q4g_cache_destroy(self.handle)
@@ -218,8 +246,22 @@ class SynthCache:
 
 def fill_history(cache: SynthCache, seed: int = 99):
     """Seeded fp16 K/V history in every ring slot and every global row, at the scale
-    the decoder writes (datagen.history_sigma: K ~ N(0, hd^(-1/2)), V ~ N(0, 1))."""
+    the decoder writes (datagen.history_sigma: K ~ N(0, hd^(-1/2)), V ~ N(0, 1)); for
+    an int8 cache, seeded codes (datagen.code8) with the row scale
+    datagen.history_scale8, the same standard deviations."""
     v = cache.view
+    if v.kv_int8:
+        for i in range(v.n_sliding):
+            for kv in (0, 1):
+                c, sc = cache.ring_i8(i, kv)
+                fill_code8(c, seed, DG.history_stream("ring", i, kv))
+                fill_const(sc, DG.history_scale8(kv, v.sl_head_dim))
+        for i in range(v.n_full):
+            for kv in (0, 1):
+                c, sc = cache.global_i8(i, kv)
+                fill_code8(c, seed, DG.history_stream("global", i, kv))
+                fill_const(sc, DG.history_scale8(kv, v.gl_head_dim))
+        return
     for i in range(v.n_sliding):
         for kv in (0, 1):
             fill_normal_f16(cache.ring(i, kv), seed, DG.history_stream("ring", i, kv),

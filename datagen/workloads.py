@@ -24,7 +24,7 @@ def decoder(n_layers, hidden, n_q_heads, ffn, vocab, sl_kv_heads, window, ring,
         gl_kv_heads=gl_kv_heads, gl_head_dim=gl_head_dim, full_every=full_every,
         full_offset=full_offset, rope_pairs_full=rope_pairs_full,
         rope_theta_sl=1.0e4, rope_theta_gl=1.0e6, rms_eps=_f32(1e-6), softcap=30.0,
-        embed_scale=_f32(math.sqrt(hidden)), v_norm_sliding=1, head_fp16=0)
+        embed_scale=_f32(math.sqrt(hidden)), v_norm_sliding=1, head_fp16=0, kv_int8=0)
 
 
 # Tiny 6-layer decoder (layers 0-4 sliding, layer 5 full): parity config.

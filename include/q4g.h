@@ -40,7 +40,7 @@
 extern "C" {
 #endif
 
-#define Q4G_ABI_VERSION 2
+#define Q4G_ABI_VERSION 3
 
 /* A CUDA stream (cudaStream_t / CUstream). NULL selects the legacy default stream. */
 typedef struct CUstream_st* q4g_stream_t;
@@ -151,6 +151,20 @@ q4g_status q4g_flash_decode_linear(const uint16_t* q, int32_t n_q, int32_t n_kv,
                                    const uint16_t* k, const uint16_t* v, int64_t len, uint16_t* out,
                                    void* workspace, size_t workspace_bytes, q4g_stream_t stream);
 
+/* The same two over int8 rows (the kv_int8 cache format): codes [.][hd] int8
+ * and one fp32 scale per row, scales laid out like the rows without head_dim
+ * (ring: [n_kv][ring]; linear: [len_capacity][n_kv]); value = code * scale.
+ * Codes 16-byte aligned, scales 4-byte aligned. Otherwise as above. */
+q4g_status q4g_flash_decode_ring_i8(const uint16_t* q, int32_t n_q, int32_t n_kv, int32_t head_dim,
+                                    const int8_t* k_codes, const float* k_scales, const int8_t* v_codes,
+                                    const float* v_scales, int64_t ring, int64_t window, int64_t pos,
+                                    uint16_t* out, void* workspace, size_t workspace_bytes,
+                                    q4g_stream_t stream);
+q4g_status q4g_flash_decode_linear_i8(const uint16_t* q, int32_t n_q, int32_t n_kv, int32_t head_dim,
+                                      const int8_t* k_codes, const float* k_scales, const int8_t* v_codes,
+                                      const float* v_scales, int64_t len, uint16_t* out, void* workspace,
+                                      size_t workspace_bytes, q4g_stream_t stream);
+
 /* Allocation-free variant of q4g_flash_decode_ring (no counterpart on the pages;
  * an integration convenience). It is for callers that cannot allocate device
  * memory at call time -- for example a program whose device memory belongs to a
@@ -210,6 +224,12 @@ typedef struct {
                               binary16, the "fp16 vocab path" of "Gemma-4-12B-CoreAI",
                               tiered-v3/ section): the head GEMV reads 2 B per weight
                               and the embedding row is the fp16 row times embed_scale */
+  int32_t kv_int8;         /* 0: K/V cache rows fp16; 1: int8 ("Gemma-4-12B-CoreAI",
+                              per-tier cost section: int8 KV), each row of head_dim
+                              codes with one fp32 scale: scale = amax / 127, code =
+                              clamp(rint(x / scale), -127, 127) for the row's fp16
+                              values x (both IEEE fp32 divisions), value = code *
+                              scale; see q4g_cache_view for the layout */
 } q4g_config;
 
 /* One q4_0 tensor in the layout above (device pointers, borrowed). */
@@ -311,9 +331,10 @@ int32_t q4g_model_profile_read(q4g_model* m, q4g_launch_record* out, int32_t max
                                q4g_stream_t stream);
 
 /* KV cache for up to `capacity` positions: per sliding layer a ring K and V of
- * [sl_kv_heads][ring][sl_head_dim] fp16 (slot = position mod ring); per full
- * layer K and V of [gl_kv_heads][capacity][gl_head_dim] fp16 indexed by absolute
- * position ("Gemma-4-12B-CoreAI": v5 section and "The per-tier cost"). The
+ * [sl_kv_heads][ring][sl_head_dim] (slot = position mod ring); per full layer K
+ * and V of [gl_kv_heads][capacity][gl_head_dim] indexed by absolute position
+ * ("Gemma-4-12B-CoreAI": v5 section and "The per-tier cost"); fp16 rows, or int8
+ * rows with scales (kv_int8, see q4g_cache_view). The
  * storage is a caller-owned device buffer of q4g_cache_bytes() bytes.
  * 1 <= capacity <= 2^30, else Q4G_ERANGE. */
 q4g_status q4g_cache_bytes(const q4g_model* m, int64_t capacity, size_t* bytes);
@@ -323,13 +344,18 @@ q4g_status q4g_cache_init(const q4g_model* m, int64_t capacity, void* dev_buf, s
 q4g_status q4g_cache_reset(q4g_cache* c, q4g_stream_t stream);
 void q4g_cache_destroy(q4g_cache* c); /* frees the handle, not the caller's buffer */
 
-/* Byte offsets inside the cache buffer, for snapshots and test access. */
+/* Byte offsets inside the cache buffer, for snapshots and test access. A layer's
+ * K (or V) region holds [n_kv][rows][hd] fp16 values, or with kv_int8 [n_kv][rows][hd]
+ * int8 codes followed, at scale_offset within the region, by [n_kv][rows] fp32
+ * scales (rows = ring for sliding layers, capacity for full layers). */
 typedef struct {
   int64_t capacity, ring;
   int32_t n_sliding, n_full, sl_kv_heads, sl_head_dim, gl_kv_heads, gl_head_dim;
   size_t ring_k_offset, ring_v_offset, ring_layer_bytes;       /* layer i at offset + i*bytes */
   size_t global_k_offset, global_v_offset, global_layer_bytes; /* full-layer ordinal i */
   size_t total_bytes;
+  int32_t kv_int8;
+  size_t ring_scale_offset, global_scale_offset; /* within a layer's K or V region (kv_int8) */
 } q4g_cache_view;
 q4g_status q4g_cache_layout(const q4g_cache* c, q4g_cache_view* out);
 

@@ -176,6 +176,7 @@ q4g_status validate_config(const q4g_config* c) {
   if (c->full_every < 0 || (c->full_every > 0 && (c->full_offset < 0 || c->full_offset >= c->full_every)))
     return fail(Q4G_EINVAL, "bad full_every / full_offset");
   if (c->head_fp16 != 0 && c->head_fp16 != 1) return fail(Q4G_EINVAL, "head_fp16 must be 0 or 1");
+  if (c->kv_int8 != 0 && c->kv_int8 != 1) return fail(Q4G_EINVAL, "kv_int8 must be 0 or 1");
   return Q4G_OK;
 }
 
@@ -376,13 +377,26 @@ extern "C" q4g_status q4g_model_set_option(q4g_model* m, q4g_option opt, intptr_
 }
 
 // --------------------------------------------------------------- cache ------
+namespace {
+size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
+// One layer's K (or V) region: fp16 rows, or int8 codes then the fp32 row scales.
+size_t kv_region_bytes(bool kv8, size_t rows, size_t hd, size_t* scale_offset) {
+  if (!kv8) {
+    if (scale_offset) *scale_offset = 0;
+    return up256(rows * hd * 2);
+  }
+  const size_t so = up256(rows * hd);
+  if (scale_offset) *scale_offset = so;
+  return up256(so + rows * sizeof(float));
+}
+}  // namespace
+
 extern "C" q4g_status q4g_cache_bytes(const q4g_model* m, int64_t capacity, size_t* bytes) {
   if (!m || !bytes) return fail(Q4G_EINVAL, "NULL argument");
   if (capacity < 1 || capacity > (int64_t)1 << 30) return fail(Q4G_ERANGE, "capacity must be in [1, 2^30]");
   const q4g_config& c = m->cfg;
-  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
-  const size_t ring = up((size_t)c.sl_kv_heads * c.ring * c.sl_head_dim * 2);
-  const size_t glob = up((size_t)c.gl_kv_heads * capacity * c.gl_head_dim * 2);
+  const size_t ring = kv_region_bytes(c.kv_int8, (size_t)c.sl_kv_heads * c.ring, c.sl_head_dim, nullptr);
+  const size_t glob = kv_region_bytes(c.kv_int8, (size_t)c.gl_kv_heads * capacity, c.gl_head_dim, nullptr);
   *bytes = 2 * ring * m->n_sl + 2 * glob * m->n_gl;
   return Q4G_OK;
 }
@@ -399,7 +413,6 @@ extern "C" q4g_status q4g_cache_init(const q4g_model* m, int64_t capacity, void*
   q4g_cache* c = new (std::nothrow) q4g_cache();
   if (!c) return fail(Q4G_ENOMEM, "cache handle");
   const q4g_config& cf = m->cfg;
-  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
   c->m = m;
   c->capacity = capacity;
   c->buf = (char*)dev_buf;
@@ -412,8 +425,11 @@ extern "C" q4g_status q4g_cache_init(const q4g_model* m, int64_t capacity, void*
   v.sl_head_dim = cf.sl_head_dim;
   v.gl_kv_heads = cf.gl_kv_heads;
   v.gl_head_dim = cf.gl_head_dim;
-  v.ring_layer_bytes = up((size_t)cf.sl_kv_heads * cf.ring * cf.sl_head_dim * 2);
-  v.global_layer_bytes = up((size_t)cf.gl_kv_heads * capacity * cf.gl_head_dim * 2);
+  v.kv_int8 = cf.kv_int8;
+  v.ring_layer_bytes = kv_region_bytes(cf.kv_int8, (size_t)cf.sl_kv_heads * cf.ring, cf.sl_head_dim,
+                                       &v.ring_scale_offset);
+  v.global_layer_bytes = kv_region_bytes(cf.kv_int8, (size_t)cf.gl_kv_heads * capacity, cf.gl_head_dim,
+                                         &v.global_scale_offset);
   v.ring_k_offset = 0;
   v.ring_v_offset = v.ring_layer_bytes * m->n_sl;
   v.global_k_offset = 2 * v.ring_layer_bytes * m->n_sl;
@@ -567,10 +583,13 @@ extern "C" size_t q4g_flash_decode_workspace_bytes(int32_t n_q_heads, int32_t he
 }
 
 namespace {
-q4g_status flash_standalone(const uint16_t* q, int32_t n_q, int32_t n_kv, int32_t hd, const uint16_t* kc,
-                            const uint16_t* vc, int64_t rows, bool ring, int64_t window, int64_t pos,
-                            uint16_t* out, void* ws, size_t ws_bytes, cudaStream_t st) {
+q4g_status flash_standalone(const uint16_t* q, int32_t n_q, int32_t n_kv, int32_t hd, const void* kc,
+                            const void* vc, const float* ks, const float* vs, int64_t rows, bool ring,
+                            int64_t window, int64_t pos, uint16_t* out, void* ws, size_t ws_bytes,
+                            cudaStream_t st) {
   if (!q || !kc || !vc || !out || !ws) return fail(Q4G_EINVAL, "NULL pointer");
+  const bool kv8 = ks != nullptr || vs != nullptr;
+  if (kv8 && (!ks || !vs || !aligned(ks, 4) || !aligned(vs, 4))) return fail(Q4G_EINVAL, "scales NULL or misaligned");
   if (hd != 256 && hd != 512) return fail(Q4G_EINVAL, "head_dim must be 256 or 512");
   if (n_q < 1 || n_kv < 1 || n_q % n_kv) return fail(Q4G_EINVAL, "n_q must be a positive multiple of n_kv");
   if (!aligned(q, 16) || !aligned(kc, 16) || !aligned(vc, 16) || !aligned(out, 16) || !aligned(ws, 256))
@@ -578,8 +597,11 @@ q4g_status flash_standalone(const uint16_t* q, int32_t n_q, int32_t n_kv, int32_
   if (ws_bytes < q4g_flash_decode_workspace_bytes(n_q, hd)) return fail(Q4G_EINVAL, "workspace too small");
   AttnParams p{};
   p.q16 = reinterpret_cast<const __half*>(q);
-  p.k_cache = reinterpret_cast<__half*>(const_cast<uint16_t*>(kc));
-  p.v_cache = reinterpret_cast<__half*>(const_cast<uint16_t*>(vc));
+  p.k_cache = reinterpret_cast<__half*>(const_cast<void*>(kc));
+  p.v_cache = reinterpret_cast<__half*>(const_cast<void*>(vc));
+  p.kv8 = kv8;
+  p.k_scale = const_cast<float*>(ks);
+  p.v_scale = const_cast<float*>(vs);
   p.cache_rows = rows;
   p.ring = ring;
   p.window = window;
@@ -617,8 +639,21 @@ extern "C" q4g_status q4g_flash_decode_ring(const uint16_t* q, int32_t n_q, int3
   if (ring < 1 || window < 1 || window > ring) return fail(Q4G_EINVAL, "need 1 <= window <= ring");
   if (ring > ((int64_t)1 << 30)) return fail(Q4G_ERANGE, "ring > 2^30");
   if (pos < 0) return fail(Q4G_ERANGE, "pos < 0");
-  return flash_standalone(q, n_q, n_kv, head_dim, k_ring, v_ring, ring, true, window, pos, out, workspace,
-                          workspace_bytes, (cudaStream_t)stream);
+  return flash_standalone(q, n_q, n_kv, head_dim, k_ring, v_ring, nullptr, nullptr, ring, true, window, pos, out,
+                          workspace, workspace_bytes, (cudaStream_t)stream);
+}
+
+extern "C" q4g_status q4g_flash_decode_ring_i8(const uint16_t* q, int32_t n_q, int32_t n_kv, int32_t head_dim,
+                                               const int8_t* k_codes, const float* k_scales, const int8_t* v_codes,
+                                               const float* v_scales, int64_t ring, int64_t window, int64_t pos,
+                                               uint16_t* out, void* workspace, size_t workspace_bytes,
+                                               q4g_stream_t stream) {
+  if (ring < 1 || window < 1 || window > ring) return fail(Q4G_EINVAL, "need 1 <= window <= ring");
+  if (ring > ((int64_t)1 << 30)) return fail(Q4G_ERANGE, "ring > 2^30");
+  if (pos < 0) return fail(Q4G_ERANGE, "pos < 0");
+  if (!k_scales || !v_scales) return fail(Q4G_EINVAL, "NULL pointer");
+  return flash_standalone(q, n_q, n_kv, head_dim, k_codes, v_codes, k_scales, v_scales, ring, true, window, pos,
+                          out, workspace, workspace_bytes, (cudaStream_t)stream);
 }
 
 extern "C" q4g_status q4g_flash_decode_linear(const uint16_t* q, int32_t n_q, int32_t n_kv, int32_t head_dim,
@@ -627,17 +662,44 @@ extern "C" q4g_status q4g_flash_decode_linear(const uint16_t* q, int32_t n_q, in
   if (len < 1 || len > ((int64_t)1 << 30)) return fail(Q4G_ERANGE, "len must be in [1, 2^30]");
   // linear cache [len][n_kv][hd] is addressed as [n_kv][rows][hd] with rows = len only when n_kv == 1
   if (n_kv != 1) return fail(Q4G_EINVAL, "the linear entry point takes one KV head ([len][hd] cache)");
-  return flash_standalone(q, n_q, n_kv, head_dim, k, v, len, false, 0, len - 1, out, workspace,
+  return flash_standalone(q, n_q, n_kv, head_dim, k, v, nullptr, nullptr, len, false, 0, len - 1, out, workspace,
                           workspace_bytes, (cudaStream_t)stream);
+}
+
+extern "C" q4g_status q4g_flash_decode_linear_i8(const uint16_t* q, int32_t n_q, int32_t n_kv, int32_t head_dim,
+                                                 const int8_t* k_codes, const float* k_scales,
+                                                 const int8_t* v_codes, const float* v_scales, int64_t len,
+                                                 uint16_t* out, void* workspace, size_t workspace_bytes,
+                                                 q4g_stream_t stream) {
+  if (len < 1 || len > ((int64_t)1 << 30)) return fail(Q4G_ERANGE, "len must be in [1, 2^30]");
+  if (n_kv != 1) return fail(Q4G_EINVAL, "the linear entry point takes one KV head ([len][hd] cache)");
+  if (!k_scales || !v_scales) return fail(Q4G_EINVAL, "NULL pointer");
+  return flash_standalone(q, n_q, n_kv, head_dim, k_codes, v_codes, k_scales, v_scales, len, false, 0, len - 1, out,
+                          workspace, workspace_bytes, (cudaStream_t)stream);
 }
 
 // --------------------------------------------------------------- decode -----
 namespace {
 
-__half* ring_k(const q4g_cache* c, int i) { return (__half*)(c->buf + c->view.ring_k_offset + i * c->view.ring_layer_bytes); }
-__half* ring_v(const q4g_cache* c, int i) { return (__half*)(c->buf + c->view.ring_v_offset + i * c->view.ring_layer_bytes); }
-__half* glob_k(const q4g_cache* c, int i) { return (__half*)(c->buf + c->view.global_k_offset + i * c->view.global_layer_bytes); }
-__half* glob_v(const q4g_cache* c, int i) { return (__half*)(c->buf + c->view.global_v_offset + i * c->view.global_layer_bytes); }
+char* ring_reg(const q4g_cache* c, int i, int kv) {
+  return c->buf + (kv ? c->view.ring_v_offset : c->view.ring_k_offset) + i * c->view.ring_layer_bytes;
+}
+char* glob_reg(const q4g_cache* c, int i, int kv) {
+  return c->buf + (kv ? c->view.global_v_offset : c->view.global_k_offset) + i * c->view.global_layer_bytes;
+}
+// Cache rows of one layer into p (fp16 values, or int8 codes and their scales).
+void bind_cache(AttnParams& p, const q4g_cache* c, bool full, int ord) {
+  char* k = full ? glob_reg(c, ord, 0) : ring_reg(c, ord, 0);
+  char* v = full ? glob_reg(c, ord, 1) : ring_reg(c, ord, 1);
+  p.k_cache = (__half*)k;
+  p.v_cache = (__half*)v;
+  p.kv8 = c->view.kv_int8;
+  if (p.kv8) {
+    const size_t so = full ? c->view.global_scale_offset : c->view.ring_scale_offset;
+    p.k_scale = (float*)(k + so);
+    p.v_scale = (float*)(v + so);
+  }
+}
 
 // Profile mode: an event before and after each launch on the launching stream.
 cudaEvent_t next_event(q4g_model* m) {
@@ -852,8 +914,7 @@ cudaError_t enqueue_body(q4g_model* m, const q4g_cache* c, int kr, int64_t pos0,
       p.rope = full ? m->rope_gl : m->rope_sl;
       p.rope_pairs = S.rope_pairs;
       p.eps = cf.rms_eps;
-      p.k_cache = full ? glob_k(c, ord) : ring_k(c, ord);
-      p.v_cache = full ? glob_v(c, ord) : ring_v(c, ord);
+      bind_cache(p, c, full, ord);
       p.cache_rows = full ? c->capacity : cf.ring;
       p.ring = full ? 0 : 1;
       p.window = cf.window;

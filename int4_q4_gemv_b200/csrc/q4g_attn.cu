@@ -61,6 +61,9 @@ Q4G_DEV void cp_async16(void* dst, const void* src, bool valid) {
                "r"(valid ? 16 : 0));
 }
 Q4G_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+Q4G_DEV void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(saddr(dst)), "l"(src) : "memory");
+}
 
 template <int N>
 Q4G_DEV void cp_async_wait() {
@@ -77,19 +80,65 @@ struct Smem {
   __half plo[MROWS][TK + 8];
   __half kloc[kMaxRows][HD];
   __half vloc[kMaxRows][HD];
+  alignas(16) int8_t kloc8[kMaxRows][HD];  // int8 cache: the block's rows as stored
+  alignas(16) int8_t vloc8[kMaxRows][HD];
+  float klocs[kMaxRows], vlocs[kMaxRows];
+  float ks[2][TK], vs[2][TK];  // int8 cache: the tile's row scales (0 for no key)
   int32_t kidx[2][TK];  // slot (ring) or position (linear); -1: no key
   float red[8][MROWS];
   float m_run[MROWS], l_run[MROWS], scale[MROWS];
   int ticket;
 };
 
+// int8 cache: a tile of TK code rows staged at the end of an fp16 tile's storage
+// (byte offset kStage8 of sm.k or sm.v) becomes the fp16 tile (exact: |code| <=
+// 127). The fp16 rows of the first TK/2 keys end below the staging area; those of
+// the other keys overlap it, so their codes are read into registers before any
+// of them is written. Ends with __syncthreads.
+template <int HD>
+Q4G_DEV void convert_tile8(__half (*dst)[HD + 8], const int8_t* stage, int tid) {
+  constexpr int CPR8 = HD / 16;                  // 16-code pieces per row
+  constexpr int NHALF = (TK / 2) * CPR8;         // pieces of half a tile
+  constexpr int NPER = NHALF / kThreads;
+  static_assert(NHALF % kThreads == 0, "whole pieces per thread");
+  auto put = [&](int key, int part, uint4 u) {
+    const int8_t* c = reinterpret_cast<const int8_t*>(&u);
+    __half2 h[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) h[i] = __floats2half2_rn((float)c[2 * i], (float)c[2 * i + 1]);
+    uint4* d = reinterpret_cast<uint4*>(&dst[key][part * 16]);
+    d[0] = *reinterpret_cast<const uint4*>(&h[0]);
+    d[1] = *reinterpret_cast<const uint4*>(&h[4]);
+  };
+#pragma unroll
+  for (int i = 0; i < NPER; ++i) {
+    const int c = tid + i * kThreads, key = c / CPR8, part = c - key * CPR8;
+    put(key, part, *reinterpret_cast<const uint4*>(stage + (size_t)key * HD + part * 16));
+  }
+  uint4 u[NPER];
+#pragma unroll
+  for (int i = 0; i < NPER; ++i) {
+    const int c = tid + i * kThreads, key = TK / 2 + c / CPR8, part = c % CPR8;
+    u[i] = *reinterpret_cast<const uint4*>(stage + (size_t)key * HD + part * 16);
+  }
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < NPER; ++i) {
+    const int c = tid + i * kThreads, key = TK / 2 + c / CPR8, part = c % CPR8;
+    put(key, part, u[i]);
+  }
+  __syncthreads();
+}
+
 // CL > 0: the grid's y dimension is one cluster of CL CTAs (n_chunks == CL);
 // the chunk partials are merged through distributed shared memory.
-template <int HD, int CL>
+template <int HD, int CL, bool KV8>
 __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   Smem<HD>& sm = *reinterpret_cast<Smem<HD>*>(smem_raw);
   constexpr int LD = Smem<HD>::LD;
+  constexpr size_t kStage8 = sizeof(sm.k) - (size_t)TK * HD;  // int8 staging inside sm.k / sm.v
+  static_assert(kStage8 >= (size_t)(TK / 2) * LD * 2, "staging above the first half tile");
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int kv = blockIdx.x, chunk = blockIdx.y, mg = blockIdx.z;
   const int G = p.n_q / p.n_kv;
@@ -125,7 +174,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
 
   const __half* kc = p.k_cache + (size_t)kv * p.cache_rows * HD;
   const __half* vc = p.v_cache + (size_t)kv * p.cache_rows * HD;
+  const int8_t* kc8 = reinterpret_cast<const int8_t*>(p.k_cache) + (size_t)kv * p.cache_rows * HD;
+  const int8_t* vc8 = reinterpret_cast<const int8_t*>(p.v_cache) + (size_t)kv * p.cache_rows * HD;
+  const float* ksc = KV8 ? p.k_scale + (size_t)kv * p.cache_rows : nullptr;
+  const float* vsc = KV8 ? p.v_scale + (size_t)kv * p.cache_rows : nullptr;
   constexpr int CPR = HD / 8;  // 16-byte chunks per row
+  constexpr int CPR8 = HD / 16;  // 16-byte chunks per int8 row
 
   // mode 0: cache rows only (the block's own rows do not exist yet);
   // 1: the block's own rows only, from shared memory; 2: both
@@ -135,6 +189,37 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
     if (kpart && tid < TK && mode != 1) {
       const int a = a0 + tid;
       sm.kidx[buf][tid] = a < a_end ? key_row(a) : -1;
+    }
+    if (KV8) {
+      int8_t* dst8 = reinterpret_cast<int8_t*>(kpart ? &sm.k[0][0] : &sm.v[0][0]) + kStage8;
+      const int8_t* src8 = kpart ? kc8 : vc8;
+      for (int c = tid; c < TK * CPR8; c += kThreads) {
+        const int key = c / CPR8, part = c - key * CPR8;
+        const int a = a0 + key;
+        const bool in = a < a_end;
+        const int loc = in ? key_is_local(a) : -1;
+        if (loc >= 0) {
+          if (mode != 0)
+            *reinterpret_cast<uint4*>(dst8 + (size_t)key * HD + part * 16) =
+                *reinterpret_cast<const uint4*>((kpart ? sm.kloc8[loc] : sm.vloc8[loc]) + part * 16);
+        } else if (mode != 1) {
+          const int8_t* s8 = in ? src8 + (size_t)key_row(a) * HD + part * 16 : src8;
+          cp_async16(dst8 + (size_t)key * HD + part * 16, s8, in);
+        }
+      }
+      if (tid < TK) {  // the rows' scales
+        const int a = a0 + tid;
+        const bool in = a < a_end;
+        const int loc = in ? key_is_local(a) : -1;
+        float* sd = kpart ? &sm.ks[buf][tid] : &sm.vs[buf][tid];
+        if (loc >= 0) {
+          if (mode != 0) *sd = kpart ? sm.klocs[loc] : sm.vlocs[loc];
+        } else if (mode != 1) {
+          if (in) cp_async4(sd, (kpart ? ksc : vsc) + key_row(a));
+          else *sd = 0.f;
+        }
+      }
+      return;
     }
     __half(*dst)[LD] = kpart ? sm.k : sm.v;
     const __half* src = kpart ? kc : vc;
@@ -212,6 +297,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
         dst[i] = __float2half_rn(a);
         dst[HD / 2 + i] = __float2half_rn(b);
       }
+      if (KV8 && kind != 0) {  // the row as the int8 cache stores it
+        __syncwarp();
+        kv_quantize_row_warp<HD>(kind == 1 ? sm.kloc[j] : sm.vloc[j], kind == 1 ? sm.kloc8[j] : sm.vloc8[j],
+                                 kind == 1 ? &sm.klocs[j] : &sm.vlocs[j], lane);
+      }
     }
   } else {
     for (int c = tid; c < nrows * CPR; c += kThreads) {
@@ -231,7 +321,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
   if (tid < MROWS) sm.m_run[tid] = -INFINITY, sm.l_run[tid] = 0.f;
   __syncthreads();
 
-  if (fused && p.write_kv && chunk == 0 && mg == 0) {
+  if (KV8 && fused && p.write_kv && chunk == 0 && mg == 0) {
+    int8_t* k8 = reinterpret_cast<int8_t*>(p.k_cache);
+    int8_t* v8 = reinterpret_cast<int8_t*>(p.v_cache);
+    for (int c = tid; c < p.kr * CPR8; c += kThreads) {
+      const int j = c / CPR8, part = c - j * CPR8;
+      const int64_t pos = pos0 + j;
+      const int64_t row = p.ring ? (int64_t)wrap(qlm - (p.kr - 1 - j), R) : pos;
+      *reinterpret_cast<uint4*>(k8 + ((size_t)kv * p.cache_rows + row) * HD + part * 16) =
+          *reinterpret_cast<const uint4*>(&sm.kloc8[j][part * 16]);
+      *reinterpret_cast<uint4*>(v8 + ((size_t)kv * p.cache_rows + row) * HD + part * 16) =
+          *reinterpret_cast<const uint4*>(&sm.vloc8[j][part * 16]);
+      if (part == 0) {
+        p.k_scale[(size_t)kv * p.cache_rows + row] = sm.klocs[j];
+        p.v_scale[(size_t)kv * p.cache_rows + row] = sm.vlocs[j];
+      }
+    }
+  } else if (fused && p.write_kv && chunk == 0 && mg == 0) {
     for (int c = tid; c < p.kr * CPR; c += kThreads) {
       const int j = c / CPR, part = c - j * CPR;
       const int64_t pos = pos0 + j;
@@ -264,6 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
     }
     cp_async_wait<1>();
     __syncthreads();
+    if (KV8) convert_tile8<HD>(sm.k, reinterpret_cast<const int8_t*>(&sm.k[0][0]) + kStage8, tid);
 
     // scores S[row][key] for key n-tile `warp`
     float s[2][4];
@@ -314,6 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
             }
           }
           float& v = s[mt][hh * 2 + e];
+          if (KV8) v *= sm.ks[buf][key];  // q . (code * scale)
           v = live ? v : -INFINITY;
           mx = fmaxf(mx, v);
         }
@@ -349,6 +457,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
           pv[e] = (v == -INFINITY) ? 0.f : __expf(v - mrow);
           sum += pv[e];
         }
+        if (KV8) {  // p * (code * scale): the V scale joins P; the row sum keeps p
+          pv[0] *= sm.vs[buf][warp * 8 + t4 * 2];
+          pv[1] *= sm.vs[buf][warp * 8 + t4 * 2 + 1];
+        }
         ph = __floats2half2_rn(pv[0], pv[1]);
         const float2 phf = __half22float2(ph);
         pl = __floats2half2_rn(pv[0] - phf.x, pv[1] - phf.y);
@@ -361,6 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
     }
     cp_async_wait<1>();  // V tile of this step (the next K may still fly)
     __syncthreads();
+    if (KV8) convert_tile8<HD>(sm.v, reinterpret_cast<const int8_t*>(&sm.v[0][0]) + kStage8, tid);
     if (tid < MROWS) {
       float sum = 0.f;
 #pragma unroll
@@ -580,15 +693,15 @@ __global__ void __launch_bounds__(kCombineThreads) attn_combine_kernel(const Att
   }
 }
 
-template <int HD, int CL>
-cudaError_t launch_attn_t(const AttnParams& p, cudaStream_t st, bool pdl) {
+template <int HD, int CL, bool KV8>
+cudaError_t launch_attn_kv(const AttnParams& p, cudaStream_t st, bool pdl) {
   static bool configured = false;
   const size_t smem = sizeof(Smem<HD>);
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel<HD, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(attn_kernel<HD, CL, KV8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(attn_kernel<HD, CL>, cudaFuncAttributePreferredSharedMemoryCarveout,
+    e = cudaFuncSetAttribute(attn_kernel<HD, CL, KV8>, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     configured = true;
@@ -615,7 +728,11 @@ cudaError_t launch_attn_t(const AttnParams& p, cudaStream_t st, bool pdl) {
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, attn_kernel<HD, CL>, p);
+  return cudaLaunchKernelEx(&cfg, attn_kernel<HD, CL, KV8>, p);
+}
+template <int HD, int CL>
+cudaError_t launch_attn_t(const AttnParams& p, cudaStream_t st, bool pdl) {
+  return p.kv8 ? launch_attn_kv<HD, CL, true>(p, st, pdl) : launch_attn_kv<HD, CL, false>(p, st, pdl);
 }
 
 template <int HD>

@@ -49,11 +49,16 @@ struct RingSmem {
   alignas(16) __half q[ROWS][HD];      // queries after norm and RoPE (fp16, as stored)
   alignas(16) __half kloc[kMaxRows][HD];  // the block's own K rows
   alignas(16) __half vloc[kMaxRows][HD];  // the block's own V rows
+  alignas(16) int8_t kloc8[kMaxRows][HD];  // int8 cache: the same rows as stored
+  alignas(16) int8_t vloc8[kMaxRows][HD];
+  float klocs[kMaxRows], vlocs[kMaxRows];
+  float kvs[kRingWarps][kRingKeysPerWarp][2];  // int8 cache: each warp's row scales
   float pm[kRingWarps][ROWS], pl[kRingWarps][ROWS];
   float cacc[ROWS][HD];                // CTA partial, relative to cm
   float cm[ROWS], cl[ROWS];
   union alignas(16) {  // read and written 16 bytes at a time
     __half kv[kRingWarps][kRingKeysPerWarp][2][HD];  // scan: each warp's K and V rows
+    int8_t kv8[kRingWarps][kRingKeysPerWarp][2][HD];  // scan, int8 cache
     float part[kRingWarps][ROWS][HD];                // merge: warp partial sums of p * v
   };
 };
@@ -68,6 +73,20 @@ static_assert(sizeof(RingSmem<256, 4>) <= 227 * 1024, "shared memory of one CTA"
 Q4G_DEV void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
                : "memory");
+}
+Q4G_DEV void cp_async8(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
+               : "memory");
+}
+Q4G_DEV void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
+               : "memory");
+}
+// 8 int8 codes (one 8-byte piece) as floats
+Q4G_DEV void unpack8_i8(const uint2 u, float* f) {
+  const int8_t* c = reinterpret_cast<const int8_t*>(&u);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) f[i] = (float)c[i];
 }
 
 // Sum v[0..N) over the 32 lanes (N a power of two <= 32) and give every lane
@@ -146,7 +165,7 @@ Q4G_DEV void norm_rope_vec(const AttnParams& p, const float* src, const float* g
 
 // Code size is kept small on purpose: every SM runs one CTA of this kernel per
 // layer, so its instructions are fetched cold; the loop over key groups is rolled.
-template <int HD, int ROWS, int CL, int S>
+template <int HD, int ROWS, int CL, int S, bool KV8>
 __global__ void __launch_bounds__(kRingThreads, 1) attn_ring_kernel(const AttnParams p) {
   static_assert(HD == 256, "one 16-byte piece per lane and row");
   constexpr int B = ROWS <= 2 ? 4 : 2;  // keys per group
@@ -180,13 +199,28 @@ __global__ void __launch_bounds__(kRingThreads, 1) attn_ring_kernel(const AttnPa
 
   // lane l holds dims 8l .. 8l+7 of every row; every cached key of the warp
   // (wa1 - wa0 <= kRingKeysPerWarp, checked on the host) goes to shared memory
-  const __half* kcache = p.k_cache + (size_t)kv * R * HD + lane * 8;
-  const __half* vcache = p.v_cache + (size_t)kv * R * HD + lane * 8;
+  if (!KV8) {
+    const __half* kcache = p.k_cache + (size_t)kv * R * HD + lane * 8;
+    const __half* vcache = p.v_cache + (size_t)kv * R * HD + lane * 8;
 #pragma unroll 1
-  for (int a = max(wa0, first_cached); a < wa1; ++a) {
-    const size_t off = (size_t)wrap(qlm - a, R) * HD;
-    cp_async16(&sm.kv[warp][a - wa0][0][lane * 8], kcache + off);
-    cp_async16(&sm.kv[warp][a - wa0][1][lane * 8], vcache + off);
+    for (int a = max(wa0, first_cached); a < wa1; ++a) {
+      const size_t off = (size_t)wrap(qlm - a, R) * HD;
+      cp_async16(&sm.kv[warp][a - wa0][0][lane * 8], kcache + off);
+      cp_async16(&sm.kv[warp][a - wa0][1][lane * 8], vcache + off);
+    }
+  } else {  // int8 rows: 8 codes per lane, and the rows' scales
+    const int8_t* kcache = reinterpret_cast<const int8_t*>(p.k_cache) + (size_t)kv * R * HD + lane * 8;
+    const int8_t* vcache = reinterpret_cast<const int8_t*>(p.v_cache) + (size_t)kv * R * HD + lane * 8;
+#pragma unroll 1
+    for (int a = max(wa0, first_cached); a < wa1; ++a) {
+      const size_t row = (size_t)wrap(qlm - a, R);
+      cp_async8(&sm.kv8[warp][a - wa0][0][lane * 8], kcache + row * HD);
+      cp_async8(&sm.kv8[warp][a - wa0][1][lane * 8], vcache + row * HD);
+      if (lane == 0) {
+        cp_async4(&sm.kvs[warp][a - wa0][0], p.k_scale + (size_t)kv * R + row);
+        cp_async4(&sm.kvs[warp][a - wa0][1], p.v_scale + (size_t)kv * R + row);
+      }
+    }
   }
   asm volatile("cp.async.commit_group;" ::: "memory");
 
@@ -205,6 +239,11 @@ __global__ void __launch_bounds__(kRingThreads, 1) attn_ring_kernel(const AttnPa
       norm_rope_vec<HD>(p, p.qkv + (size_t)j * p.qkv_stride + col,
                         kind == 0 ? p.w_q : kind == 1 ? p.w_k : nullptr, kind != 2 || p.v_norm != 0,
                         kind != 2, j, dst, lane);
+      if (KV8 && kind != 0) {  // the row as the int8 cache stores it
+        __syncwarp();
+        kv_quantize_row_warp<HD>(dst, kind == 1 ? sm.kloc8[j] : sm.vloc8[j], kind == 1 ? &sm.klocs[j] : &sm.vlocs[j],
+                                 lane);
+      }
     }
   } else {
     for (int c = tid; c < nr * HD / 8; c += kRingThreads) {
@@ -215,13 +254,30 @@ __global__ void __launch_bounds__(kRingThreads, 1) attn_ring_kernel(const AttnPa
   }
   __syncthreads();
   if (fused && p.write_kv && gchunk == 0) {
-    for (int c = tid; c < p.kr * HD / 8; c += kRingThreads) {
-      const int j = c / (HD / 8), part = c - j * (HD / 8);
-      const size_t row = (size_t)wrap(qlm - (p.kr - 1 - j), R);
-      *reinterpret_cast<uint4*>(p.k_cache + ((size_t)kv * R + row) * HD + part * 8) =
-          *reinterpret_cast<const uint4*>(&sm.kloc[j][part * 8]);
-      *reinterpret_cast<uint4*>(p.v_cache + ((size_t)kv * R + row) * HD + part * 8) =
-          *reinterpret_cast<const uint4*>(&sm.vloc[j][part * 8]);
+    if (!KV8) {
+      for (int c = tid; c < p.kr * HD / 8; c += kRingThreads) {
+        const int j = c / (HD / 8), part = c - j * (HD / 8);
+        const size_t row = (size_t)wrap(qlm - (p.kr - 1 - j), R);
+        *reinterpret_cast<uint4*>(p.k_cache + ((size_t)kv * R + row) * HD + part * 8) =
+            *reinterpret_cast<const uint4*>(&sm.kloc[j][part * 8]);
+        *reinterpret_cast<uint4*>(p.v_cache + ((size_t)kv * R + row) * HD + part * 8) =
+            *reinterpret_cast<const uint4*>(&sm.vloc[j][part * 8]);
+      }
+    } else {
+      int8_t* k8 = reinterpret_cast<int8_t*>(p.k_cache);
+      int8_t* v8 = reinterpret_cast<int8_t*>(p.v_cache);
+      for (int c = tid; c < p.kr * HD / 16; c += kRingThreads) {
+        const int j = c / (HD / 16), part = c - j * (HD / 16);
+        const size_t row = (size_t)wrap(qlm - (p.kr - 1 - j), R);
+        *reinterpret_cast<uint4*>(k8 + ((size_t)kv * R + row) * HD + part * 16) =
+            *reinterpret_cast<const uint4*>(&sm.kloc8[j][part * 16]);
+        *reinterpret_cast<uint4*>(v8 + ((size_t)kv * R + row) * HD + part * 16) =
+            *reinterpret_cast<const uint4*>(&sm.vloc8[j][part * 16]);
+        if (part == 0) {
+          p.k_scale[(size_t)kv * R + row] = sm.klocs[j];
+          p.v_scale[(size_t)kv * R + row] = sm.vlocs[j];
+        }
+      }
     }
   }
   pdl_launch_dependents();
@@ -259,25 +315,43 @@ __global__ void __launch_bounds__(kRingThreads, 1) attn_ring_kernel(const AttnPa
   }
 #pragma unroll 1
   for (int a0 = wa0; a0 < wa1; a0 += B) {
-    uint4 kb[B], vb[B];
+    uint4 kb[B], vb[B];  // fp16: 8 values; int8: 8 codes in .x/.y
+    float ksc[B], vsc[B];  // int8: the rows' scales
 #pragma unroll
     for (int i = 0; i < B; ++i) {
       const int a = a0 + i;
+      ksc[i] = vsc[i] = 0.f;
       if (a >= wa1) {
         kb[i] = vb[i] = make_uint4(0, 0, 0, 0);
-      } else if (a < first_cached) {  // the block's own rows, from the prologue
-        kb[i] = *reinterpret_cast<const uint4*>(&sm.kloc[p.kr - 1 - a][lane * 8]);
-        vb[i] = *reinterpret_cast<const uint4*>(&sm.vloc[p.kr - 1 - a][lane * 8]);
+      } else if (!KV8) {
+        if (a < first_cached) {  // the block's own rows, from the prologue
+          kb[i] = *reinterpret_cast<const uint4*>(&sm.kloc[p.kr - 1 - a][lane * 8]);
+          vb[i] = *reinterpret_cast<const uint4*>(&sm.vloc[p.kr - 1 - a][lane * 8]);
+        } else {
+          kb[i] = *reinterpret_cast<const uint4*>(&sm.kv[warp][a - wa0][0][lane * 8]);
+          vb[i] = *reinterpret_cast<const uint4*>(&sm.kv[warp][a - wa0][1][lane * 8]);
+        }
       } else {
-        kb[i] = *reinterpret_cast<const uint4*>(&sm.kv[warp][a - wa0][0][lane * 8]);
-        vb[i] = *reinterpret_cast<const uint4*>(&sm.kv[warp][a - wa0][1][lane * 8]);
+        uint2 k2, v2;
+        if (a < first_cached) {
+          k2 = *reinterpret_cast<const uint2*>(&sm.kloc8[p.kr - 1 - a][lane * 8]);
+          v2 = *reinterpret_cast<const uint2*>(&sm.vloc8[p.kr - 1 - a][lane * 8]);
+          ksc[i] = sm.klocs[p.kr - 1 - a], vsc[i] = sm.vlocs[p.kr - 1 - a];
+        } else {
+          k2 = *reinterpret_cast<const uint2*>(&sm.kv8[warp][a - wa0][0][lane * 8]);
+          v2 = *reinterpret_cast<const uint2*>(&sm.kv8[warp][a - wa0][1][lane * 8]);
+          ksc[i] = sm.kvs[warp][a - wa0][0], vsc[i] = sm.kvs[warp][a - wa0][1];
+        }
+        kb[i] = make_uint4(k2.x, k2.y, 0, 0);
+        vb[i] = make_uint4(v2.x, v2.y, 0, 0);
       }
     }
     float s[B * ROWS];
 #pragma unroll
     for (int i = 0; i < B; ++i) {
       float kf[8];
-      unpack8(kb[i], kf);
+      if (KV8) unpack8_i8(make_uint2(kb[i].x, kb[i].y), kf);
+      else unpack8(kb[i], kf);
 #pragma unroll
       for (int r = 0; r < ROWS; ++r) {
         float t = 0.f;
@@ -287,6 +361,12 @@ __global__ void __launch_bounds__(kRingThreads, 1) attn_ring_kernel(const AttnPa
       }
     }
     warp_allreduce_vec<B * ROWS>(s, lane);
+    if (KV8) {  // q . (code * scale) = scale * (q . code)
+#pragma unroll
+      for (int i = 0; i < B; ++i)
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) s[i * ROWS + r] *= ksc[i];
+    }
 #pragma unroll
     for (int r = 0; r < ROWS; ++r) {
       if (r >= nr) continue;
@@ -309,10 +389,12 @@ __global__ void __launch_bounds__(kRingThreads, 1) attn_ring_kernel(const AttnPa
         const float sv = s[i * ROWS + r];
         const float pv = sv == -INFINITY ? 0.f : __expf(sv - mx);
         float vf[8];
-        unpack8(vb[i], vf);
+        if (KV8) unpack8_i8(make_uint2(vb[i].x, vb[i].y), vf);
+        else unpack8(vb[i], vf);
         l[r] += pv;
+        const float pw = KV8 ? pv * vsc[i] : pv;  // p * (code * scale)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[r][e] = fmaf(pv, vf[e], acc[r][e]);
+        for (int e = 0; e < 8; ++e) acc[r][e] = fmaf(pw, vf[e], acc[r][e]);
       }
     }
   }
@@ -422,11 +504,11 @@ __global__ void __launch_bounds__(kRingThreads, 1) attn_ring_kernel(const AttnPa
   if (tid == 0) p.counters[kv * CL + chunk] = 0;  // ready for the next layer
 }
 
-template <int HD, int ROWS, int CL, int S>
+template <int HD, int ROWS, int CL, int S, bool KV8 = false>
 cudaError_t configure_ring() {
   static bool configured = false;
   if (configured) return cudaSuccess;
-  auto kern = attn_ring_kernel<HD, ROWS, CL, S>;
+  auto kern = attn_ring_kernel<HD, ROWS, CL, S, KV8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)sizeof(RingSmem<HD, ROWS>));
   if (e == cudaSuccess && CL > 8) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
@@ -457,13 +539,13 @@ cudaLaunchConfig_t ring_config(const AttnParams& p, cudaStream_t st, bool pdl, c
   return cfg;
 }
 
-template <int HD, int ROWS, int CL, int S>
+template <int HD, int ROWS, int CL, int S, bool KV8>
 cudaError_t launch_ring_t(const AttnParams& p, cudaStream_t st, bool pdl) {
-  cudaError_t e = configure_ring<HD, ROWS, CL, S>();
+  cudaError_t e = configure_ring<HD, ROWS, CL, S, KV8>();
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[2];
   const cudaLaunchConfig_t cfg = ring_config<HD, ROWS, CL, S>(p, st, pdl, attr);
-  return cudaLaunchKernelEx(&cfg, attn_ring_kernel<HD, ROWS, CL, S>, p);
+  return cudaLaunchKernelEx(&cfg, attn_ring_kernel<HD, ROWS, CL, S, KV8>, p);
 }
 
 // CTAs per KV head: 16 (a non-portable cluster, twice the SMs on the scan) when
@@ -480,7 +562,7 @@ int ring_cluster_size() {
     cudaLaunchAttribute attr[2];
     if (configure_ring<256, 2, 16, 1>() == cudaSuccess) {
       const cudaLaunchConfig_t cfg = ring_config<256, 2, 16, 1>(p, 0, false, attr);
-      if (cudaOccupancyMaxActiveClusters(&n, attn_ring_kernel<256, 2, 16, 1>, &cfg) == cudaSuccess && n >= 8)
+      if (cudaOccupancyMaxActiveClusters(&n, attn_ring_kernel<256, 2, 16, 1, false>, &cfg) == cudaSuccess && n >= 8)
         pick = 16;
     }
     cudaGetLastError();  // a refused query leaves no error behind
@@ -512,12 +594,30 @@ bool ring_split_fits(int n_kv) {
     if (configure_ring<256, 2, 4, 4>() == cudaSuccess) {
       const cudaLaunchConfig_t cfg = ring_config<256, 2, 4, 4>(p, 0, false, attr);
       int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, attn_ring_kernel<256, 2, 4, 4>, &cfg) == cudaSuccess) max_clusters = n;
+      if (cudaOccupancyMaxActiveClusters(&n, attn_ring_kernel<256, 2, 4, 4, false>, &cfg) == cudaSuccess) max_clusters = n;
     }
     cudaGetLastError();
   }
   return n_kv * 4 <= max_clusters;
 }
+
+namespace {
+template <bool KV8>
+cudaError_t launch_ring_rows(const AttnParams& p, bool split, bool wide, cudaStream_t st, bool pdl) {
+  switch (ring_decode_rows(p)) {
+    case 1:
+      return split ? launch_ring_t<256, 1, 4, 4, KV8>(p, st, pdl)
+             : wide ? launch_ring_t<256, 1, 16, 1, KV8>(p, st, pdl) : launch_ring_t<256, 1, 8, 1, KV8>(p, st, pdl);
+    case 2:
+      return split ? launch_ring_t<256, 2, 4, 4, KV8>(p, st, pdl)
+             : wide ? launch_ring_t<256, 2, 16, 1, KV8>(p, st, pdl) : launch_ring_t<256, 2, 8, 1, KV8>(p, st, pdl);
+    case 4:
+      return split ? launch_ring_t<256, 4, 4, 4, KV8>(p, st, pdl)
+             : wide ? launch_ring_t<256, 4, 16, 1, KV8>(p, st, pdl) : launch_ring_t<256, 4, 8, 1, KV8>(p, st, pdl);
+    default: return cudaErrorInvalidValue;
+  }
+}
+}  // namespace
 
 cudaError_t launch_attention_ring(const AttnParams& p, cudaStream_t st, bool pdl) {
   // 16 CTAs per KV head (four clusters of 4, merged through the caller's
@@ -526,18 +626,8 @@ cudaError_t launch_attention_ring(const AttnParams& p, cudaStream_t st, bool pdl
   // 16 or 8
   const bool split = p.ring_split == 2 && ring_split_fits(p.n_kv);
   const bool wide = !split && ring_cluster_size() == 16;
-  switch (ring_decode_rows(p)) {
-    case 1:
-      return split ? launch_ring_t<256, 1, 4, 4>(p, st, pdl)
-             : wide ? launch_ring_t<256, 1, 16, 1>(p, st, pdl) : launch_ring_t<256, 1, 8, 1>(p, st, pdl);
-    case 2:
-      return split ? launch_ring_t<256, 2, 4, 4>(p, st, pdl)
-             : wide ? launch_ring_t<256, 2, 16, 1>(p, st, pdl) : launch_ring_t<256, 2, 8, 1>(p, st, pdl);
-    case 4:
-      return split ? launch_ring_t<256, 4, 4, 4>(p, st, pdl)
-             : wide ? launch_ring_t<256, 4, 16, 1>(p, st, pdl) : launch_ring_t<256, 4, 8, 1>(p, st, pdl);
-    default: return cudaErrorInvalidValue;
-  }
+  if (p.kv8) return launch_ring_rows<true>(p, split, wide, st, pdl);
+  return launch_ring_rows<false>(p, split, wide, st, pdl);
 }
 
 }  // namespace q4g

@@ -217,6 +217,31 @@ Q4G_DEV float warp_max(float v) {
   return v;
 }
 
+// int8 KV row ("Gemma-4-12B-CoreAI", per-tier cost section: int8 K/V) from an fp16
+// row in shared memory, by one warp: scale = amax / 127 and code = clamp(rint(x /
+// scale), -127, 127), both IEEE fp32 divisions (round to nearest even); an
+// all-zero row has scale 0 and codes 0.
+template <int HD>
+Q4G_DEV void kv_quantize_row_warp(const __half* x, int8_t* codes, float* scale, int lane) {
+  constexpr int E = HD / 32;
+  float v[E];
+  float amax = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    v[e] = __half2float(x[lane * E + e]);
+    amax = fmaxf(amax, fabsf(v[e]));
+  }
+  amax = warp_max(amax);
+  const float s = __fdiv_rn(amax, 127.0f);
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    int c = 0;
+    if (s != 0.f) c = min(max(__float2int_rn(__fdiv_rn(v[e], s)), -127), 127);
+    codes[lane * E + e] = (int8_t)c;
+  }
+  if (lane == 0) *scale = s;
+}
+
 // Block-wide sum for blockDim.x == NT; `red` holds >= 32 floats. All threads
 // receive the result. Summation order is fixed.
 template <int NT = kThreads>

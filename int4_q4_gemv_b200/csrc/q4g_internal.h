@@ -106,6 +106,11 @@ struct AttnParams {
   // cache
   __half* k_cache;       // ring: [n_kv][R][hd]; linear: [n_kv][cap][hd]
   __half* v_cache;
+  // int8 cache (kv8 = 1): codes [n_kv][rows][hd] at k_cache / v_cache (as int8)
+  // with one fp32 scale per row, [n_kv][rows] at k_scale / v_scale
+  int32_t kv8;
+  float* k_scale;
+  float* v_scale;
   int64_t cache_rows;    // R (ring) or capacity (linear)
   int32_t ring;          // 1: ring addressing with the implied-position window test
   int64_t window;

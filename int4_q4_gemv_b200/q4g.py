@@ -23,6 +23,7 @@ EXPORTS = [
     "q4g_last_error", "q4g_status_string", "q4g_abi_version",
     "q4g_q4_0_pack", "q4g_q4_0_unpack", "q4g_gemv", "q4g_gemv_f16",
     "q4g_flash_decode_workspace_bytes", "q4g_flash_decode_ring", "q4g_flash_decode_linear",
+    "q4g_flash_decode_ring_i8", "q4g_flash_decode_linear_i8",
     "q4g_model_create", "q4g_model_destroy", "q4g_model_check", "q4g_model_set_option",
     "q4g_cache_bytes", "q4g_cache_init", "q4g_cache_reset", "q4g_cache_destroy", "q4g_cache_layout",
     "q4g_decode_step", "q4g_decode_step_device_token", "q4g_decode_step_hidden",
@@ -43,7 +44,8 @@ class q4g_config(C.Structure):
         "n_layers", "hidden", "n_q_heads", "ffn", "vocab", "sl_kv_heads", "sl_head_dim", "window",
         "ring", "gl_kv_heads", "gl_head_dim", "full_every", "full_offset", "rope_pairs_full")] + \
         [(n, C.c_float) for n in ("rope_theta_sl", "rope_theta_gl", "rms_eps", "softcap",
-                                  "embed_scale")] + [("v_norm_sliding", C.c_int32), ("head_fp16", C.c_int32)]
+                                  "embed_scale")] + [("v_norm_sliding", C.c_int32), ("head_fp16", C.c_int32),
+                                                     ("kv_int8", C.c_int32)]
 
 
 class q4g_qtensor(C.Structure):
@@ -71,7 +73,8 @@ class q4g_cache_view(C.Structure):
                                   "gl_kv_heads", "gl_head_dim")] + \
         [(n, C.c_size_t) for n in ("ring_k_offset", "ring_v_offset", "ring_layer_bytes",
                                    "global_k_offset", "global_v_offset", "global_layer_bytes",
-                                   "total_bytes")]
+                                   "total_bytes")] + \
+        [("kv_int8", C.c_int32), ("ring_scale_offset", C.c_size_t), ("global_scale_offset", C.c_size_t)]
 
 
 _lib = None
@@ -96,6 +99,9 @@ def lib() -> C.CDLL:
             "q4g_flash_decode_workspace_bytes": (sz, [i32, i32]),
             "q4g_flash_decode_ring": (C.c_int, [vp, i32, i32, i32, vp, vp, i64, i64, i64, vp, vp, sz, vp]),
             "q4g_flash_decode_linear": (C.c_int, [vp, i32, i32, i32, vp, vp, i64, vp, vp, sz, vp]),
+            "q4g_flash_decode_ring_i8": (C.c_int, [vp, i32, i32, i32, vp, vp, vp, vp, i64, i64, i64, vp, vp, sz,
+                                                   vp]),
+            "q4g_flash_decode_linear_i8": (C.c_int, [vp, i32, i32, i32, vp, vp, vp, vp, i64, vp, vp, sz, vp]),
             "q4g_model_create": (C.c_int, [C.POINTER(q4g_config), C.POINTER(q4g_weights), C.POINTER(vp)]),
             "q4g_model_destroy": (None, [vp]),
             "q4g_model_check": (C.c_int, [vp, vp]),
@@ -174,6 +180,18 @@ def q4g_flash_decode_ring(q, n_q, n_kv, head_dim, k_ring, v_ring, ring, window, 
 
 def q4g_flash_decode_linear(q, n_q, n_kv, head_dim, k, v, length, out, ws, ws_bytes, stream):
     _call("q4g_flash_decode_linear", q, n_q, n_kv, head_dim, k, v, length, out, ws, ws_bytes, stream)
+
+
+def q4g_flash_decode_ring_i8(q, n_q, n_kv, head_dim, k_codes, k_scales, v_codes, v_scales, ring, window, pos,
+                             out, ws, ws_bytes, stream):
+    _call("q4g_flash_decode_ring_i8", q, n_q, n_kv, head_dim, k_codes, k_scales, v_codes, v_scales, ring, window,
+          pos, out, ws, ws_bytes, stream)
+
+
+def q4g_flash_decode_linear_i8(q, n_q, n_kv, head_dim, k_codes, k_scales, v_codes, v_scales, length, out, ws,
+                               ws_bytes, stream):
+    _call("q4g_flash_decode_linear_i8", q, n_q, n_kv, head_dim, k_codes, k_scales, v_codes, v_scales, length, out,
+          ws, ws_bytes, stream)
 
 
 def q4g_flash_decode_ring_noalloc(q, n_q, n_kv, head_dim, k_ring, v_ring, ring, window, pos, out, stream):

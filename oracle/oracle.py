@@ -23,7 +23,8 @@ class OrConfig(C.Structure):
         "sl_kv_heads", "sl_head_dim", "window", "ring",
         "gl_kv_heads", "gl_head_dim", "full_every", "full_offset", "rope_pairs_full")] + \
         [(n, C.c_double) for n in ("rope_theta_sl", "rope_theta_gl", "rms_eps", "softcap",
-                                   "embed_scale")] + [("v_norm_sliding", C.c_int32), ("head_fp16", C.c_int32)]
+                                   "embed_scale")] + [("v_norm_sliding", C.c_int32), ("head_fp16", C.c_int32),
+                                                       ("kv_int8", C.c_int32)]
 
 
 def _p(a):
@@ -53,6 +54,12 @@ def lib():
             "or_attn_ring": (None, [vp, C.c_int, C.c_int, C.c_int, vp, vp, i64, i64, i64, vp]),
             "or_attn_linear": (None, [vp, C.c_int, C.c_int, C.c_int, vp, vp, i64, vp]),
             "or_ring_implied_positions": (None, [i64, i64, i64, vp]),
+            "or_attn_ring_i8": (None, [vp, C.c_int, C.c_int, C.c_int, vp, vp, vp, vp, i64, i64, i64, vp]),
+            "or_attn_linear_i8": (None, [vp, C.c_int, C.c_int, C.c_int, vp, vp, vp, vp, i64, vp]),
+            "or_kv_quantize_row": (None, [vp, C.c_int, vp, vp]),
+            "or_fill_code8": (None, [vp, i64, u64, u64, i64]),
+            "or_cache_ring_i8": (vp, [vp, C.c_int, C.c_int, C.POINTER(vp)]),
+            "or_cache_global_i8": (vp, [vp, C.c_int, C.c_int, C.POINTER(vp)]),
             "or_model_create": (vp, [C.POINTER(OrConfig), u64, C.c_int, C.c_int]),
             "or_model_destroy": (None, [vp]),
             "or_model_tensor": (i64, [vp, C.c_int, C.c_int, C.POINTER(vp), C.POINTER(vp),
@@ -194,6 +201,39 @@ def attn_linear(q16, kc, vc, length):
     return out
 
 
+def attn_ring_i8(q16, k8, ks, v8, vs, R, W, q):
+    """int8 rows: k8/v8 [n_kv][R][hd] codes, ks/vs [n_kv][R] fp32 scales."""
+    q16 = np.ascontiguousarray(q16, dtype=np.uint16)
+    k8, v8 = (np.ascontiguousarray(a, dtype=np.int8) for a in (k8, v8))
+    ks, vs = (np.ascontiguousarray(a, dtype=np.float32) for a in (ks, vs))
+    n_q, hd = q16.shape
+    out = np.empty((n_q, hd), dtype=np.float64)
+    lib().or_attn_ring_i8(_p(q16), n_q, k8.shape[0], hd, _p(k8), _p(ks), _p(v8), _p(vs), int(R), int(W),
+                          int(q), _p(out))
+    return out
+
+
+def attn_linear_i8(q16, k8, ks, v8, vs, length):
+    """int8 rows: k8/v8 [L][n_kv][hd] codes, ks/vs [L][n_kv] fp32 scales; keys 0..length-1."""
+    q16 = np.ascontiguousarray(q16, dtype=np.uint16)
+    k8, v8 = (np.ascontiguousarray(a, dtype=np.int8) for a in (k8, v8))
+    ks, vs = (np.ascontiguousarray(a, dtype=np.float32) for a in (ks, vs))
+    n_q, hd = q16.shape
+    out = np.empty((n_q, hd), dtype=np.float64)
+    lib().or_attn_linear_i8(_p(q16), n_q, k8.shape[1], hd, _p(k8), _p(ks), _p(v8), _p(vs), int(length),
+                            _p(out))
+    return out
+
+
+def kv_quantize_row(x16):
+    """int8 KV row of fp16 bits x16 [hd]: (codes int8 [hd], scale float32)."""
+    x16 = np.ascontiguousarray(x16, dtype=np.uint16)
+    codes = np.empty(x16.size, dtype=np.int8)
+    sc = np.zeros(1, dtype=np.float32)
+    lib().or_kv_quantize_row(_p(x16), x16.size, _p(codes), _p(sc))
+    return codes, sc[0]
+
+
 def ring_implied_positions(R, W, q):
     out = np.empty(int(R), dtype=np.int64)
     lib().or_ring_implied_positions(int(R), int(W), int(q), _p(out))
@@ -271,6 +311,23 @@ class Cache:
         shape = (cfg["gl_kv_heads"], self.capacity, cfg["gl_head_dim"])
         return np.ctypeslib.as_array(C.cast(ptr, C.POINTER(C.c_uint16)), shape=shape)
 
+    def _i8(self, fn, index, kv, rows, nkv, hd):
+        sp = C.c_void_p()
+        ptr = fn(self.h, index, kv, C.byref(sp))
+        codes = np.ctypeslib.as_array(C.cast(ptr, C.POINTER(C.c_int8)), shape=(nkv, rows, hd))
+        scales = np.ctypeslib.as_array(C.cast(sp, C.POINTER(C.c_float)), shape=(nkv, rows))
+        return codes, scales
+
+    def ring_i8(self, sl_index: int, kv: int):
+        """int8 cache: (codes [n_kv][R][hd] int8, scales [n_kv][R] fp32), views."""
+        cfg = self.model.cfg
+        return self._i8(lib().or_cache_ring_i8, sl_index, kv, self.R, cfg["sl_kv_heads"], cfg["sl_head_dim"])
+
+    def global_i8(self, gl_index: int, kv: int):
+        cfg = self.model.cfg
+        return self._i8(lib().or_cache_global_i8, gl_index, kv, self.capacity, cfg["gl_kv_heads"],
+                        cfg["gl_head_dim"])
+
     def close(self):
         if self.h:
             lib().or_cache_destroy(self.h)
@@ -281,6 +338,12 @@ class Cache:
             self.close()
         except Exception:
             pass
+
+
+def fill_code8(out: np.ndarray, seed: int, stream: int, start: int = 0):
+    """Seeded int8 codes from the C header (datagen's dg_code8)."""
+    assert out.dtype == np.int8 and out.flags["C_CONTIGUOUS"]
+    lib().or_fill_code8(_p(out), out.size, seed, stream, start)
 
 
 def fill_normal_f16(out: np.ndarray, seed: int, stream: int, sigma: float = 1.0, start: int = 0):
@@ -295,6 +358,15 @@ def fill_history(cache: Cache, seed: int = 99):
     cfg = cache.model.cfg
     n_sl = sum(1 for l in range(cfg["n_layers"]) if not _is_full(cfg, l))
     n_gl = cfg["n_layers"] - n_sl
+    if cfg.get("kv_int8"):  # seeded codes and the constant row scale (datagen.code8)
+        for kind, n, hd, get in (("ring", n_sl, cfg["sl_head_dim"], cache.ring_i8),
+                                 ("global", n_gl, cfg["gl_head_dim"], cache.global_i8)):
+            for i in range(n):
+                for kv in (0, 1):
+                    codes, scales = get(i, kv)
+                    codes[...] = DG.code8(seed, DG.history_stream(kind, i, kv), codes.size).reshape(codes.shape)
+                    scales[...] = DG.history_scale8(kv, hd)
+        return
     for i in range(n_sl):
         for kv in (0, 1):
             fill_normal_f16(cache.ring(i, kv), seed, DG.history_stream("ring", i, kv),

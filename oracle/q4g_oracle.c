@@ -225,14 +225,26 @@ static inline int64_t pmod(int64_t a, int64_t m) {
 /* description), keys taken in ascending position.                           */
 /* ------------------------------------------------------------------------- */
 
-/* One head: n keys given as pointers, in the order they are summed. */
-static void attend_one(const double* q, int hd, const uint16_t* const* keys,
-                       const uint16_t* const* vals, int64_t n, double* out) {
+/* A cache row: fp16 values (h), or int8 codes c with the row's scale s, whose
+ * value is c[d] * s ("Gemma-4-12B-CoreAI", per-tier cost section: int8 KV). */
+typedef struct {
+  const uint16_t* h;
+  const int8_t* c;
+  float s;
+} kvrow;
+
+static inline double kv_at(const kvrow* r, int d) {
+  return r->h ? or_f16_to_double(r->h[d]) : (double)r->c[d] * (double)r->s;
+}
+
+/* One head: n keys given as rows, in the order they are summed. */
+static void attend_one(const double* q, int hd, const kvrow* keys, const kvrow* vals, int64_t n,
+                       double* out) {
   double* s = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
   double mx = -INFINITY;
   for (int64_t t = 0; t < n; ++t) {
     double acc = 0.0;
-    for (int d = 0; d < hd; ++d) acc += q[d] * or_f16_to_double(keys[t][d]);
+    for (int d = 0; d < hd; ++d) acc += q[d] * kv_at(&keys[t], d);
     s[t] = acc;
     if (acc > mx) mx = acc;
   }
@@ -243,9 +255,32 @@ static void attend_one(const double* q, int hd, const uint16_t* const* keys,
   }
   for (int d = 0; d < hd; ++d) out[d] = 0.0;
   for (int64_t t = 0; t < n; ++t)
-    for (int d = 0; d < hd; ++d) out[d] += s[t] * or_f16_to_double(vals[t][d]);
+    for (int d = 0; d < hd; ++d) out[d] += s[t] * kv_at(&vals[t], d);
   for (int d = 0; d < hd; ++d) out[d] /= l;
   free(s);
+}
+
+/* int8 KV row: s = amax / 127 (fp32 division; amax = largest |x| of the fp16
+ * row), code = clamp(rint(x / s), -127, 127) with x / s an fp32 division and
+ * rint to nearest even; an all-zero row has s = 0 and codes 0. */
+void or_kv_quantize_row(const uint16_t* x16, int hd, int8_t* codes, float* scale) {
+  float amax = 0.0f;
+  for (int d = 0; d < hd; ++d) {
+    const float v = fabsf((float)or_f16_to_double(x16[d]));
+    if (v > amax) amax = v;
+  }
+  const float s = amax / 127.0f;
+  *scale = s;
+  for (int d = 0; d < hd; ++d) {
+    if (s == 0.0f) {
+      codes[d] = 0;
+      continue;
+    }
+    float q = rintf((float)or_f16_to_double(x16[d]) / s);
+    if (q > 127.0f) q = 127.0f;
+    if (q < -127.0f) q = -127.0f;
+    codes[d] = (int8_t)q;
+  }
 }
 
 void or_ring_implied_positions(int64_t R, int64_t W, int64_t q, int64_t* out) {
@@ -255,14 +290,15 @@ void or_ring_implied_positions(int64_t R, int64_t W, int64_t q, int64_t* out) {
   }
 }
 
-void or_attn_ring(const uint16_t* q16, int n_q, int n_kv, int hd, const uint16_t* kc,
-                  const uint16_t* vc, int64_t R, int64_t W, int64_t q, double* out) {
+static void attn_ring_any(const uint16_t* q16, int n_q, int n_kv, int hd, const uint16_t* kc,
+                          const uint16_t* vc, const int8_t* k8, const float* ks, const int8_t* v8,
+                          const float* vs, int64_t R, int64_t W, int64_t q, double* out) {
   int G = n_q / n_kv;
 #pragma omp parallel for schedule(static)
   for (int h = 0; h < n_q; ++h) {
     int g = h / G;
-    const uint16_t** keys = (const uint16_t**)malloc(sizeof(void*) * (size_t)R);
-    const uint16_t** vals = (const uint16_t**)malloc(sizeof(void*) * (size_t)R);
+    kvrow* keys = (kvrow*)calloc((size_t)R, sizeof(kvrow));
+    kvrow* vals = (kvrow*)calloc((size_t)R, sizeof(kvrow));
     double* qd = (double*)malloc(sizeof(double) * (size_t)hd);
     for (int d = 0; d < hd; ++d) qd[d] = or_f16_to_double(q16[(int64_t)h * hd + d]);
     int64_t n = 0;
@@ -270,8 +306,13 @@ void or_attn_ring(const uint16_t* q16, int n_q, int n_kv, int hd, const uint16_t
       int64_t j = pmod(q - a, R);
       int64_t p = q - pmod(q - j, R);
       if (p < 0 || q - p >= W) continue;
-      keys[n] = kc + ((int64_t)g * R + j) * hd;
-      vals[n] = vc + ((int64_t)g * R + j) * hd;
+      const int64_t row = (int64_t)g * R + j;
+      if (kc) {
+        keys[n].h = kc + row * hd, vals[n].h = vc + row * hd;
+      } else {
+        keys[n].c = k8 + row * hd, keys[n].s = ks[row];
+        vals[n].c = v8 + row * hd, vals[n].s = vs[row];
+      }
       ++n;
     }
     attend_one(qd, hd, keys, vals, n, out + (int64_t)h * hd);
@@ -281,25 +322,48 @@ void or_attn_ring(const uint16_t* q16, int n_q, int n_kv, int hd, const uint16_t
   }
 }
 
-void or_attn_linear(const uint16_t* q16, int n_q, int n_kv, int hd, const uint16_t* kc,
-                    const uint16_t* vc, int64_t len, double* out) {
+static void attn_linear_any(const uint16_t* q16, int n_q, int n_kv, int hd, const uint16_t* kc,
+                            const uint16_t* vc, const int8_t* k8, const float* ks, const int8_t* v8,
+                            const float* vs, int64_t len, double* out) {
   int G = n_q / n_kv;
 #pragma omp parallel for schedule(static)
   for (int h = 0; h < n_q; ++h) {
     int g = h / G;
-    const uint16_t** keys = (const uint16_t**)malloc(sizeof(void*) * (size_t)(len > 0 ? len : 1));
-    const uint16_t** vals = (const uint16_t**)malloc(sizeof(void*) * (size_t)(len > 0 ? len : 1));
+    kvrow* keys = (kvrow*)calloc((size_t)(len > 0 ? len : 1), sizeof(kvrow));
+    kvrow* vals = (kvrow*)calloc((size_t)(len > 0 ? len : 1), sizeof(kvrow));
     double* qd = (double*)malloc(sizeof(double) * (size_t)hd);
     for (int d = 0; d < hd; ++d) qd[d] = or_f16_to_double(q16[(int64_t)h * hd + d]);
     for (int64_t p = 0; p < len; ++p) {
-      keys[p] = kc + (p * n_kv + g) * hd;
-      vals[p] = vc + (p * n_kv + g) * hd;
+      const int64_t row = p * n_kv + g;
+      if (kc) {
+        keys[p].h = kc + row * hd, vals[p].h = vc + row * hd;
+      } else {
+        keys[p].c = k8 + row * hd, keys[p].s = ks[row];
+        vals[p].c = v8 + row * hd, vals[p].s = vs[row];
+      }
     }
     attend_one(qd, hd, keys, vals, len, out + (int64_t)h * hd);
     free(keys);
     free(vals);
     free(qd);
   }
+}
+
+void or_attn_ring(const uint16_t* q16, int n_q, int n_kv, int hd, const uint16_t* kc,
+                  const uint16_t* vc, int64_t R, int64_t W, int64_t q, double* out) {
+  attn_ring_any(q16, n_q, n_kv, hd, kc, vc, NULL, NULL, NULL, NULL, R, W, q, out);
+}
+void or_attn_ring_i8(const uint16_t* q16, int n_q, int n_kv, int hd, const int8_t* k8, const float* ks,
+                     const int8_t* v8, const float* vs, int64_t R, int64_t W, int64_t q, double* out) {
+  attn_ring_any(q16, n_q, n_kv, hd, NULL, NULL, k8, ks, v8, vs, R, W, q, out);
+}
+void or_attn_linear(const uint16_t* q16, int n_q, int n_kv, int hd, const uint16_t* kc,
+                    const uint16_t* vc, int64_t len, double* out) {
+  attn_linear_any(q16, n_q, n_kv, hd, kc, vc, NULL, NULL, NULL, NULL, len, out);
+}
+void or_attn_linear_i8(const uint16_t* q16, int n_q, int n_kv, int hd, const int8_t* k8, const float* ks,
+                       const int8_t* v8, const float* vs, int64_t len, double* out) {
+  attn_linear_any(q16, n_q, n_kv, hd, NULL, NULL, k8, ks, v8, vs, len, out);
 }
 
 /* ------------------------------------------------------------------------- */
@@ -331,7 +395,10 @@ struct or_model {
 struct or_cache {
   int64_t capacity, R;
   int n_sl, n_gl, sl_kv, gl_kv, hd_s, hd_g;
-  uint16_t **ringK, **ringV, **glK, **glV;
+  int kv8;                              /* int8 rows with one fp32 scale each */
+  uint16_t **ringK, **ringV, **glK, **glV;  /* fp16 rows (kv8 = 0) */
+  int8_t **ringK8, **ringV8, **glK8, **glV8;  /* int8 codes (kv8 = 1) */
+  float **ringKs, **ringVs, **glKs, **glVs;   /* per-row scales (kv8 = 1) */
 };
 
 static int layer_is_full(const or_config* c, int l) {
@@ -470,6 +537,46 @@ int64_t or_model_tensor(const or_model* m, int layer, int tensor, const uint8_t*
 
 const uint16_t* or_model_embed_f16(const or_model* m) { return m->embed16; }
 
+/* Allocate every layer's rows, zeroed, or as a copy of src's (copy != 0). */
+static void* alloc_copy(size_t bytes, const void* from) {
+  void* p = calloc(bytes ? bytes : 1, 1);
+  if (from) memcpy(p, from, bytes);
+  return p;
+}
+static void cache_alloc(or_cache* k, int copy, const or_cache* src) {
+  const size_t nsl = (size_t)k->n_sl + 1, ngl = (size_t)k->n_gl + 1;
+  const size_t rrows = (size_t)k->sl_kv * (size_t)k->R, grows = (size_t)k->gl_kv * (size_t)k->capacity;
+  const size_t rvals = rrows * (size_t)k->hd_s, gvals = grows * (size_t)k->hd_g;
+  k->ringK = (uint16_t**)calloc(nsl, sizeof(void*)), k->ringV = (uint16_t**)calloc(nsl, sizeof(void*));
+  k->glK = (uint16_t**)calloc(ngl, sizeof(void*)), k->glV = (uint16_t**)calloc(ngl, sizeof(void*));
+  k->ringK8 = (int8_t**)calloc(nsl, sizeof(void*)), k->ringV8 = (int8_t**)calloc(nsl, sizeof(void*));
+  k->glK8 = (int8_t**)calloc(ngl, sizeof(void*)), k->glV8 = (int8_t**)calloc(ngl, sizeof(void*));
+  k->ringKs = (float**)calloc(nsl, sizeof(void*)), k->ringVs = (float**)calloc(nsl, sizeof(void*));
+  k->glKs = (float**)calloc(ngl, sizeof(void*)), k->glVs = (float**)calloc(ngl, sizeof(void*));
+  for (int i = 0; i < k->n_sl; ++i) {
+    if (!k->kv8) {
+      k->ringK[i] = (uint16_t*)alloc_copy(rvals * 2, copy ? src->ringK[i] : NULL);
+      k->ringV[i] = (uint16_t*)alloc_copy(rvals * 2, copy ? src->ringV[i] : NULL);
+    } else {
+      k->ringK8[i] = (int8_t*)alloc_copy(rvals, copy ? src->ringK8[i] : NULL);
+      k->ringV8[i] = (int8_t*)alloc_copy(rvals, copy ? src->ringV8[i] : NULL);
+      k->ringKs[i] = (float*)alloc_copy(rrows * sizeof(float), copy ? src->ringKs[i] : NULL);
+      k->ringVs[i] = (float*)alloc_copy(rrows * sizeof(float), copy ? src->ringVs[i] : NULL);
+    }
+  }
+  for (int i = 0; i < k->n_gl; ++i) {
+    if (!k->kv8) {
+      k->glK[i] = (uint16_t*)alloc_copy(gvals * 2, copy ? src->glK[i] : NULL);
+      k->glV[i] = (uint16_t*)alloc_copy(gvals * 2, copy ? src->glV[i] : NULL);
+    } else {
+      k->glK8[i] = (int8_t*)alloc_copy(gvals, copy ? src->glK8[i] : NULL);
+      k->glV8[i] = (int8_t*)alloc_copy(gvals, copy ? src->glV8[i] : NULL);
+      k->glKs[i] = (float*)alloc_copy(grows * sizeof(float), copy ? src->glKs[i] : NULL);
+      k->glVs[i] = (float*)alloc_copy(grows * sizeof(float), copy ? src->glVs[i] : NULL);
+    }
+  }
+}
+
 or_cache* or_cache_create(const or_model* m, int64_t capacity, int64_t ring_slots) {
   const or_config* c = &m->cfg;
   or_cache* k = (or_cache*)calloc(1, sizeof(or_cache));
@@ -481,57 +588,54 @@ or_cache* or_cache_create(const or_model* m, int64_t capacity, int64_t ring_slot
   k->gl_kv = c->gl_kv_heads;
   k->hd_s = c->sl_head_dim;
   k->hd_g = c->gl_head_dim;
-  k->ringK = (uint16_t**)calloc((size_t)k->n_sl + 1, sizeof(void*));
-  k->ringV = (uint16_t**)calloc((size_t)k->n_sl + 1, sizeof(void*));
-  k->glK = (uint16_t**)calloc((size_t)k->n_gl + 1, sizeof(void*));
-  k->glV = (uint16_t**)calloc((size_t)k->n_gl + 1, sizeof(void*));
-  size_t rs = (size_t)(k->sl_kv * k->R * k->hd_s), gs = (size_t)(k->gl_kv * capacity * k->hd_g);
-  for (int i = 0; i < k->n_sl; ++i) {
-    k->ringK[i] = (uint16_t*)calloc(rs, 2);
-    k->ringV[i] = (uint16_t*)calloc(rs, 2);
-  }
-  for (int i = 0; i < k->n_gl; ++i) {
-    k->glK[i] = (uint16_t*)calloc(gs, 2);
-    k->glV[i] = (uint16_t*)calloc(gs, 2);
-  }
+  k->kv8 = c->kv_int8 != 0;
+  cache_alloc(k, 0, NULL);
   return k;
 }
 
 void or_cache_destroy(or_cache* c) {
   if (!c) return;
-  for (int i = 0; i < c->n_sl; ++i) free(c->ringK[i]), free(c->ringV[i]);
-  for (int i = 0; i < c->n_gl; ++i) free(c->glK[i]), free(c->glV[i]);
+  for (int i = 0; i < c->n_sl; ++i) {
+    free(c->ringK[i]), free(c->ringV[i]), free(c->ringK8[i]), free(c->ringV8[i]);
+    free(c->ringKs[i]), free(c->ringVs[i]);
+  }
+  for (int i = 0; i < c->n_gl; ++i) {
+    free(c->glK[i]), free(c->glV[i]), free(c->glK8[i]), free(c->glV8[i]);
+    free(c->glKs[i]), free(c->glVs[i]);
+  }
   free(c->ringK), free(c->ringV), free(c->glK), free(c->glV);
+  free(c->ringK8), free(c->ringV8), free(c->glK8), free(c->glV8);
+  free(c->ringKs), free(c->ringVs), free(c->glKs), free(c->glVs);
   free(c);
 }
 
 or_cache* or_cache_clone(const or_cache* c) {
   or_cache* k = (or_cache*)malloc(sizeof(or_cache));
   *k = *c;
-  k->ringK = (uint16_t**)calloc((size_t)k->n_sl + 1, sizeof(void*));
-  k->ringV = (uint16_t**)calloc((size_t)k->n_sl + 1, sizeof(void*));
-  k->glK = (uint16_t**)calloc((size_t)k->n_gl + 1, sizeof(void*));
-  k->glV = (uint16_t**)calloc((size_t)k->n_gl + 1, sizeof(void*));
-  size_t rs = (size_t)(k->sl_kv * k->R * k->hd_s) * 2, gs = (size_t)(k->gl_kv * k->capacity * k->hd_g) * 2;
-  for (int i = 0; i < k->n_sl; ++i) {
-    k->ringK[i] = (uint16_t*)malloc(rs), memcpy(k->ringK[i], c->ringK[i], rs);
-    k->ringV[i] = (uint16_t*)malloc(rs), memcpy(k->ringV[i], c->ringV[i], rs);
-  }
-  for (int i = 0; i < k->n_gl; ++i) {
-    k->glK[i] = (uint16_t*)malloc(gs), memcpy(k->glK[i], c->glK[i], gs);
-    k->glV[i] = (uint16_t*)malloc(gs), memcpy(k->glV[i], c->glV[i], gs);
-  }
+  cache_alloc(k, 1, c);
   return k;
 }
 
 uint16_t* or_cache_ring(or_cache* c, int sl_index, int kv) {
-  if (sl_index < 0 || sl_index >= c->n_sl) return NULL;
+  if (c->kv8 || sl_index < 0 || sl_index >= c->n_sl) return NULL;
   return kv ? c->ringV[sl_index] : c->ringK[sl_index];
 }
 
 uint16_t* or_cache_global(or_cache* c, int gl_index, int kv) {
-  if (gl_index < 0 || gl_index >= c->n_gl) return NULL;
+  if (c->kv8 || gl_index < 0 || gl_index >= c->n_gl) return NULL;
   return kv ? c->glV[gl_index] : c->glK[gl_index];
+}
+
+int8_t* or_cache_ring_i8(or_cache* c, int sl_index, int kv, float** scales) {
+  if (!c->kv8 || sl_index < 0 || sl_index >= c->n_sl) return NULL;
+  *scales = kv ? c->ringVs[sl_index] : c->ringKs[sl_index];
+  return kv ? c->ringV8[sl_index] : c->ringK8[sl_index];
+}
+
+int8_t* or_cache_global_i8(or_cache* c, int gl_index, int kv, float** scales) {
+  if (!c->kv8 || gl_index < 0 || gl_index >= c->n_gl) return NULL;
+  *scales = kv ? c->glVs[gl_index] : c->glKs[gl_index];
+  return kv ? c->glV8[gl_index] : c->glK8[gl_index];
 }
 
 /* ------------------------------------------------------------------------- */
@@ -568,6 +672,11 @@ int or_verify_block(or_model* m, or_cache* c, const int32_t* ids, const float* h
   double* gg = (double*)malloc(sizeof(double) * (size_t)(K * F));
   double* uu = (double*)malloc(sizeof(double) * (size_t)(K * F));
   double* hv = (double*)malloc(sizeof(double) * (size_t)hdmax);
+  /* int8 KV: this block's rows as stored (codes and one scale per row) */
+  int8_t* k8 = (int8_t*)malloc((size_t)(K * kvmax * hdmax));
+  int8_t* v8 = (int8_t*)malloc((size_t)(K * kvmax * hdmax));
+  float* k8s = (float*)malloc(sizeof(float) * (size_t)(K * kvmax));
+  float* v8s = (float*)malloc(sizeof(float) * (size_t)(K * kvmax));
 
   /* a1: embedding (tied table, dequantised, times the embedding scale) */
   for (int i = 0; i < K; ++i) {
@@ -598,6 +707,11 @@ int or_verify_block(or_model* m, or_cache* c, const int32_t* ids, const float* h
     const double theta = full ? cfg->rope_theta_gl : cfg->rope_theta_sl;
     uint16_t* cK = full ? c->glK[L->ordinal] : c->ringK[L->ordinal];
     uint16_t* cV = full ? c->glV[L->ordinal] : c->ringV[L->ordinal];
+    int8_t* cK8 = full ? c->glK8[L->ordinal] : c->ringK8[L->ordinal];
+    int8_t* cV8 = full ? c->glV8[L->ordinal] : c->ringV8[L->ordinal];
+    float* cKs = full ? c->glKs[L->ordinal] : c->ringKs[L->ordinal];
+    float* cVs = full ? c->glVs[L->ordinal] : c->ringVs[L->ordinal];
+    const int64_t crows = full ? c->capacity : R; /* rows per KV head in this layer's cache */
 
     /* a2: pre-attention RMSNorm, stored fp16 */
     for (int i = 0; i < K; ++i) {
@@ -638,15 +752,30 @@ int or_verify_block(or_model* m, or_cache* c, const int32_t* ids, const float* h
       }
     }
 
+    /* int8 KV: each fp16 row becomes codes and a scale before it is stored or read */
+    if (c->kv8)
+      for (int64_t t = 0; t < K * nkv; ++t) {
+        or_kv_quantize_row(k16 + t * hd, (int)hd, k8 + t * hd, &k8s[t]);
+        or_kv_quantize_row(v16 + t * hd, (int)hd, v8 + t * hd, &v8s[t]);
+      }
+    /* store row i of this block into its cache row */
+#define STORE_ROW(i)                                                                        \
+  for (int64_t g = 0; g < nkv; ++g) {                                                       \
+    const int64_t pos = pos0 + (i);                                                         \
+    const int64_t crow = g * crows + (full ? pos : pmod(pos, R));                           \
+    const int64_t t = (i) * nkv + g;                                                        \
+    if (c->kv8) {                                                                           \
+      memcpy(cK8 + crow * hd, k8 + t * hd, (size_t)hd), cKs[crow] = k8s[t];                 \
+      memcpy(cV8 + crow * hd, v8 + t * hd, (size_t)hd), cVs[crow] = v8s[t];                 \
+    } else {                                                                                \
+      memcpy(cK + crow * hd, k16 + t * hd, 2 * (size_t)hd);                                 \
+      memcpy(cV + crow * hd, v16 + t * hd, 2 * (size_t)hd);                                 \
+    }                                                                                       \
+  }
     /* write rows into the cache: mode 1 writes every row before attention */
     int64_t nwrite_before = mode == 1 ? K : 0;
     for (int64_t i = 0; i < nwrite_before; ++i) {
-      int64_t pos = pos0 + i;
-      for (int64_t g = 0; g < nkv; ++g) {
-        int64_t off = full ? (g * c->capacity + pos) * hd : (g * R + pmod(pos, R)) * hd;
-        memcpy(cK + off, k16 + (i * nkv + g) * hd, 2 * (size_t)hd);
-        memcpy(cV + off, v16 + (i * nkv + g) * hd, 2 * (size_t)hd);
-      }
+      STORE_ROW(i)
     }
 
     /* a5/a6: attention */
@@ -655,10 +784,18 @@ int or_verify_block(or_model* m, or_cache* c, const int32_t* ids, const float* h
       for (int64_t h = 0; h < Hq; ++h) {
         int64_t qpos = pos0 + i, g = h / G;
         int64_t nmax = full ? qpos + 1 : (W < R ? R : W);
-        const uint16_t** keys = (const uint16_t**)malloc(sizeof(void*) * (size_t)nmax);
-        const uint16_t** vals = (const uint16_t**)malloc(sizeof(void*) * (size_t)nmax);
+        kvrow* keys = (kvrow*)calloc((size_t)nmax, sizeof(kvrow));
+        kvrow* vals = (kvrow*)calloc((size_t)nmax, sizeof(kvrow));
         double* qd = (double*)malloc(sizeof(double) * (size_t)hd);
         for (int64_t d = 0; d < hd; ++d) qd[d] = or_f16_to_double(q16[(i * Hq + h) * hd + d]);
+        /* cache row crow, or row t of this block */
+#define CACHE_ROW(n, crow)                                                    \
+  if (c->kv8) {                                                               \
+    keys[n].c = cK8 + (crow) * hd, keys[n].s = cKs[crow];                     \
+    vals[n].c = cV8 + (crow) * hd, vals[n].s = cVs[crow];                     \
+  } else {                                                                    \
+    keys[n].h = cK + (crow) * hd, vals[n].h = cV + (crow) * hd;               \
+  }
         int64_t n = 0;
         if (mode == 1 && !full) {
           /* the ring read literally: every slot, implied position, window test */
@@ -666,8 +803,7 @@ int or_verify_block(or_model* m, or_cache* c, const int32_t* ids, const float* h
             int64_t j = pmod(qpos - a, R);
             int64_t p = qpos - pmod(qpos - j, R);
             if (p < 0 || qpos - p >= W) continue;
-            keys[n] = cK + (g * R + j) * hd;
-            vals[n] = cV + (g * R + j) * hd;
+            CACHE_ROW(n, g * R + j)
             ++n;
           }
         } else {
@@ -675,16 +811,20 @@ int or_verify_block(or_model* m, or_cache* c, const int32_t* ids, const float* h
           int64_t p_lo = full ? 0 : (qpos - W + 1 > 0 ? qpos - W + 1 : 0);
           for (int64_t p = p_lo; p <= qpos; ++p) {
             if (mode == 0 && p >= pos0) { /* this block's own rows */
-              keys[n] = k16 + ((p - pos0) * nkv + g) * hd;
-              vals[n] = v16 + ((p - pos0) * nkv + g) * hd;
+              const int64_t t = (p - pos0) * nkv + g;
+              if (c->kv8) {
+                keys[n].c = k8 + t * hd, keys[n].s = k8s[t];
+                vals[n].c = v8 + t * hd, vals[n].s = v8s[t];
+              } else {
+                keys[n].h = k16 + t * hd, vals[n].h = v16 + t * hd;
+              }
             } else {
-              int64_t off = full ? (g * c->capacity + p) * hd : (g * R + pmod(p, R)) * hd;
-              keys[n] = cK + off;
-              vals[n] = cV + off;
+              CACHE_ROW(n, g * crows + (full ? p : pmod(p, R)))
             }
             ++n;
           }
         }
+#undef CACHE_ROW
         attend_one(qd, (int)hd, keys, vals, n, att + (i * Hq + h) * hd);
         free(keys), free(vals), free(qd);
       }
@@ -693,13 +833,9 @@ int or_verify_block(or_model* m, or_cache* c, const int32_t* ids, const float* h
     /* mode 0 commits the accepted rows after the block is evaluated */
     if (mode == 0)
       for (int64_t i = 0; i < accepted; ++i) {
-        int64_t pos = pos0 + i;
-        for (int64_t g = 0; g < nkv; ++g) {
-          int64_t off = full ? (g * c->capacity + pos) * hd : (g * R + pmod(pos, R)) * hd;
-          memcpy(cK + off, k16 + (i * nkv + g) * hd, 2 * (size_t)hd);
-          memcpy(cV + off, v16 + (i * nkv + g) * hd, 2 * (size_t)hd);
-        }
+        STORE_ROW(i)
       }
+#undef STORE_ROW
 
     /* a7/a8: output projection, post-attention norm, residual */
     or_gemv(L->wo.qs, L->wo.sc, H, Hq * hd, K, x16, tmp);
@@ -754,7 +890,7 @@ int or_verify_block(or_model* m, or_cache* c, const int32_t* ids, const float* h
   if (logits) memcpy(logits, lg, sizeof(double) * (size_t)(K * V));
   free(lg);
   free(r), free(tmp), free(x16), free(qp), free(kp), free(vp), free(q16), free(k16), free(v16);
-  free(att), free(gg), free(uu), free(hv);
+  free(att), free(gg), free(uu), free(hv), free(k8), free(v8), free(k8s), free(v8s);
   return 0;
 }
 
@@ -791,4 +927,9 @@ void or_fill_normal_f16(uint16_t* out, int64_t n, uint64_t seed, uint64_t stream
 #pragma omp parallel for schedule(static)
   for (int64_t i = 0; i < n; ++i)
     out[i] = or_f16_from_double((double)dg_normal(key, (uint64_t)(start + i), sigma));
+}
+
+void or_fill_code8(int8_t* out, int64_t n, uint64_t seed, uint64_t stream, int64_t start) {
+  const uint64_t key = dg_key(seed, stream);
+  for (int64_t i = 0; i < n; ++i) out[i] = (int8_t)dg_code8(key, (uint64_t)(start + i));
 }

@@ -35,6 +35,8 @@ typedef struct {
   double rope_theta_sl, rope_theta_gl, rms_eps, softcap, embed_scale;
   int32_t v_norm_sliding; /* 1: scale-free RMSNorm on sliding-layer V too */
   int32_t head_fp16;      /* 1: the tied embedding / head is fp16 instead of q4_0 */
+  int32_t kv_int8;        /* 1: K/V cache rows stored as int8 codes with one fp32 scale per
+                             row ("Gemma-4-12B-CoreAI", per-tier cost section) */
 } or_config;
 
 /* ---- IEEE binary16 ---- */
@@ -75,12 +77,25 @@ void or_attn_ring(const uint16_t* q16, int n_q, int n_kv, int hd, const uint16_t
 /* Linear cache: K/V [L][n_kv][hd]; keys 0..len-1 all live. */
 void or_attn_linear(const uint16_t* q16, int n_q, int n_kv, int hd, const uint16_t* kc,
                     const uint16_t* vc, int64_t len, double* out);
+/* The same over int8 K/V rows: codes [rows][hd] with one fp32 scale per row
+ * (value = code * scale); rows indexed as in the fp16 versions. */
+void or_attn_ring_i8(const uint16_t* q16, int n_q, int n_kv, int hd, const int8_t* k8, const float* ks,
+                     const int8_t* v8, const float* vs, int64_t R, int64_t W, int64_t q, double* out);
+void or_attn_linear_i8(const uint16_t* q16, int n_q, int n_kv, int hd, const int8_t* k8, const float* ks,
+                       const int8_t* v8, const float* vs, int64_t len, double* out);
+/* int8 KV row from an fp16 row x16[hd]: scale = amax / 127 (fp32 division,
+ * amax = largest |x|), code = clamp(rint(x / scale), -127, 127) (fp32
+ * division, round to nearest even); an all-zero row: scale 0, codes 0. */
+void or_kv_quantize_row(const uint16_t* x16, int hd, int8_t* codes, float* scale);
 /* Live-slot mask of the ring for query position q: mask[j] = implied position or -1. */
 void or_ring_implied_positions(int64_t R, int64_t W, int64_t q, int64_t* out);
 
 /* Seeded N(0, sigma) rounded to fp16 (datagen definition): synthetic history. */
 void or_fill_normal_f16(uint16_t* out, int64_t n, uint64_t seed, uint64_t stream, float sigma,
                         int64_t start);
+
+/* Seeded int8 codes (datagen definition dg_code8): synthetic int8 history. */
+void or_fill_code8(int8_t* out, int64_t n, uint64_t seed, uint64_t stream, int64_t start);
 
 /* ---- model ---- */
 typedef struct or_model or_model;
@@ -111,6 +126,11 @@ or_cache* or_cache_clone(const or_cache* c);
  * global layer index = full-layer ordinal; K/V [n_kv][capacity][hd] fp16. */
 uint16_t* or_cache_ring(or_cache* c, int sl_index, int kv /*0 K, 1 V*/);
 uint16_t* or_cache_global(or_cache* c, int gl_index, int kv);
+/* The same for a kv_int8 model's cache: codes [n_kv][rows][hd] int8, and
+ * *scales [n_kv][rows] fp32 (the fp16 accessors return NULL then, and these
+ * return NULL for an fp16 cache). */
+int8_t* or_cache_ring_i8(or_cache* c, int sl_index, int kv, float** scales);
+int8_t* or_cache_global_i8(or_cache* c, int gl_index, int kv, float** scales);
 
 /* Verify block of K rows at absolute positions pos0..pos0+K-1 (decode = K 1).
  * mode 0 (reference protocol): row i attends the positions

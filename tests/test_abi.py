@@ -40,9 +40,11 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    # version 2: q4g_config.head_fp16 and q4g_weights.embed_f16 (the fp16 tied head)
-    assert Q.q4g_abi_version() == 2
-    assert C.sizeof(Q.q4g_config) == 21 * 4 and C.sizeof(Q.q4g_weights) == 8 + 16 + 8 + 8
+    # version 2: q4g_config.head_fp16 and q4g_weights.embed_f16 (the fp16 tied head);
+    # version 3: q4g_config.kv_int8 and the int8 fields of q4g_cache_view
+    assert Q.q4g_abi_version() == 3
+    assert C.sizeof(Q.q4g_config) == 22 * 4 and C.sizeof(Q.q4g_weights) == 8 + 16 + 8 + 8
+    assert C.sizeof(Q.q4g_cache_view) == 16 + 6 * 4 + 7 * 8 + 8 + 2 * 8
     assert lib.q4g_status_string(Q.Q4G_ERANGE) == b"Q4G_ERANGE"
 
 

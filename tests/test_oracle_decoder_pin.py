@@ -27,6 +27,16 @@ def _h(x: torch.Tensor) -> torch.Tensor:
     return torch.from_numpy(x.numpy().astype(np.float16).astype(np.float64))
 
 
+def _q8(x: torch.Tensor) -> torch.Tensor:
+    """Rows of fp16 values through the int8 KV format, in torch ops: per row a
+    float32 scale amax / 127, codes round-half-even(x / scale) clamped to
+    [-127, 127] (float32 division), value = code * scale."""
+    xf = x.to(torch.float32)
+    s = xf.abs().amax(dim=-1, keepdim=True) / torch.tensor(127.0, dtype=torch.float32)
+    c = torch.where(s > 0, torch.round(xf / torch.where(s > 0, s, torch.ones_like(s))), torch.zeros_like(xf))
+    return c.clamp(-127, 127).to(torch.float64) * s.to(torch.float64)
+
+
 def _rope(x: torch.Tensor, rot: int, theta: float, pos: int) -> torch.Tensor:
     hd = x.shape[-1]
     half = hd // 2
@@ -90,6 +100,8 @@ class TorchDecoder:
             q = _h(_rope(F.rms_norm(q, (hd,), Ly["n_q"], eps), rot, theta, pos))
             k = _h(_rope(F.rms_norm(kraw, (hd,), Ly["n_k"], eps), rot, theta, pos))
             v = _h(F.rms_norm(vsrc, (hd,), None, eps))
+            if c.get("kv_int8"):
+                k, v = _q8(k), _q8(v)
             self.K[l].append(k)
             self.V[l].append(v)
             Kh = torch.stack(self.K[l], dim=1)             # [nkv, L, hd]
@@ -109,11 +121,12 @@ class TorchDecoder:
         return torch.tanh((self.embed @ z) / c["softcap"]) * c["softcap"]
 
 
-@pytest.mark.parametrize("variant,head_fp16", [(1, 0), (2, 0), (1, 1)])
-def test_oracle_decoder_matches_torch_composition(variant, head_fp16):
+@pytest.mark.parametrize("variant,head_fp16,kv_int8", [(1, 0, 0), (2, 0, 0), (1, 1, 0), (1, 0, 1)])
+def test_oracle_decoder_matches_torch_composition(variant, head_fp16, kv_int8):
     """Variant 1: seeded gains and layer scalars; variant 2: unit q/k gains (a sharp
-    softmax, logits of order head_dim); head_fp16: the fp16 tied embedding / head."""
-    cfg = dict(WL.MICRO, head_fp16=head_fp16)
+    softmax, logits of order head_dim); head_fp16: the fp16 tied embedding / head;
+    kv_int8: K/V rows stored as int8 with a per-row scale."""
+    cfg = dict(WL.MICRO, head_fp16=head_fp16, kv_int8=kv_int8)
     seed, steps = 4, 40                      # 40 steps > 2 ring wraps at R = 16
     om = O.Model(cfg, seed=seed, variant=variant)
     cache = O.Cache(om, 64)
