@@ -109,12 +109,14 @@ def weight_bytes(cfg) -> float:
 
 def kv_bytes(cfg, q) -> float:
     """Live K/V bytes read at query position q: per sliding layer K and V of
-    min(q + 1, W) positions, per full layer K and V of q + 1 positions (fp16)."""
+    min(q + 1, W) positions, per full layer K and V of q + 1 positions (fp16 rows of
+    2 * hd bytes; int8 rows of hd bytes plus a 4-byte scale)."""
     from datagen import workloads as WL
     n_sl = sum(1 for l in range(cfg["n_layers"]) if not WL.layer_is_full(cfg, l))
     n_gl = cfg["n_layers"] - n_sl
-    sl = n_sl * min(q + 1, cfg["window"]) * cfg["sl_kv_heads"] * cfg["sl_head_dim"] * 2 * 2
-    gl = n_gl * (q + 1) * cfg["gl_kv_heads"] * cfg["gl_head_dim"] * 2 * 2
+    row = (lambda hd: hd + 4) if cfg.get("kv_int8") else (lambda hd: 2 * hd)
+    sl = n_sl * min(q + 1, cfg["window"]) * cfg["sl_kv_heads"] * row(cfg["sl_head_dim"]) * 2
+    gl = n_gl * (q + 1) * cfg["gl_kv_heads"] * row(cfg["gl_head_dim"]) * 2
     return float(sl + gl)
 
 
@@ -621,6 +623,20 @@ def main():
             "accepted_tokens_per_s": accepted / (nb * msv / 1e3), "rows_per_s": Kv * 1e3 / msv,
             "bytes_per_block": bpb, "gbs": bpb / (msv / 1e3) / 1e9, "frac": bpb / (msv / 1e3) / 1e9 / peak,
             "accepted_count": "seeded U{0..4}", "history": "synthetic"}
+        # the int8 KV cache (kv_int8): the same weights under a second model handle
+        m8 = model.sibling(kv_int8=1)
+        ms8, bpt8 = measure_context(Q, S, m8, m8.cfg, 32768, 50, 4, sp, stream)
+        per_context["32768_kv_int8"] = {"kind": "decode", "kv": "int8", "tokens_per_s": 1e3 / ms8,
+                                        "ms_per_step": ms8, "bytes_per_token": bpt8,
+                                        "gbs": bpt8 / (ms8 / 1e3) / 1e9, "frac": bpt8 / (ms8 / 1e3) / 1e9 / peak,
+                                        "steps": 50, "history": "synthetic"}
+        msv8, bpb8, acc8 = measure_verify(Q, S, DG, m8, m8.cfg, 131072, Kv, nb, 2, args.seed, sp, stream)
+        per_context["131072_verify_k4_kv_int8"] = {
+            "kind": "verify", "kv": "int8", "k": Kv, "blocks": nb, "blocks_per_s": 1e3 / msv8,
+            "ms_per_block": msv8, "accepted_tokens_per_s": acc8 / (nb * msv8 / 1e3), "rows_per_s": Kv * 1e3 / msv8,
+            "bytes_per_block": bpb8, "gbs": bpb8 / (msv8 / 1e3) / 1e9, "frac": bpb8 / (msv8 / 1e3) / 1e9 / peak,
+            "accepted_count": "seeded U{0..4}", "history": "synthetic"}
+        m8.close()
         npf = 1024
         mspf = measure_prefill(Q, DG, model, cfg, npf, args.seed, sp, stream)
         per_context["prefill_1024_c64"] = {

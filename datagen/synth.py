@@ -183,6 +183,36 @@ class SynthDecoder:
     def new_cache(self, capacity: int) -> "SynthCache":
         return SynthCache(self, capacity)
 
+    def sibling(self, **overrides) -> "SynthSibling":
+        """A second model handle over the same weights with some configuration
+        fields changed (for example kv_int8=1)."""
+        return SynthSibling(self, overrides)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            Q.q4g_model_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class SynthSibling:
+    """A model handle that borrows a SynthDecoder's weights (which must outlive it)."""
+
+    def __init__(self, parent: SynthDecoder, overrides: dict):
+        self.parent = parent
+        self.cfg = dict(parent.cfg, **overrides)
+        self.device = parent.device
+        self._cfg_struct = config_struct(self.cfg)
+        self.handle = Q.q4g_model_create(self._cfg_struct, parent._w)
+
+    def new_cache(self, capacity: int) -> "SynthCache":
+        return SynthCache(self, capacity)
+
     def close(self):
         if getattr(self, "handle", None):
             Q.q4g_model_destroy(self.handle)
