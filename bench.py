@@ -12,9 +12,10 @@ flush is needed between steps.
 
 Besides the headline context the line carries:
   * per_context: 32K decode over seeded synthetic history and the 128K verify config
-    (K = 4 draft rows, seeded accepted counts) in blocks/s, each with its HBM fraction;
-  * roofline: the dominant kernel (the persistent step kernel: the whole step after
-    its init launch) timed with CUDA events around its launches;
+    (K = 4 draft rows, seeded accepted counts) in blocks/s, each with its HBM fraction,
+    the same two with the int8 KV cache, and 1,024 tokens of chunked prefill;
+  * roofline: the dominant kernel (the q4_0 GEMV), its time inside the timed graph
+    step taken as its share of a profile pass with CUDA events around every launch;
   * microbench: the four q4_0 GEMV shapes (seeds 1-4) and flash-decode alone (hd 256
     ring, hd 512 linear at 4K..128K), each rotated over copies larger than L2;
   * cpu_baseline: the oracle on the host cores, all threads and one thread.

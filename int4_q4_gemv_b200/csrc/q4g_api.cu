@@ -110,7 +110,6 @@ struct q4g_model {
   double* inv_freq_gl;
   float* part_ml;
   float* part_acc;
-  // persistent step kernel: per-layer descriptors (device) and its partials / counters
   bool use_graph = true, use_pdl = true, attn_cluster = true;
   uint64_t* trace = nullptr;  // Q4G_OPT_TRACE
   float* dump = nullptr;

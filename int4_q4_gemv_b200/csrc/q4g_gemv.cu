@@ -5,25 +5,23 @@
 // with w(r,c) = (code - 8) * d(r, c/32), x fp16, fp32 accumulation.
 //
 // Kernels (one operation, chosen per call; see launch_gemv):
-//   * stage kernel (default): one CTA per SM streams a contiguous range of
-//     16-36 KB row stages through a bulk-copy ring; every compute warp works on
-//     every stage (a column chunk of a row group), with the integer block dot
-//     (16-bit block fixed-point x, dp4a over the raw nibble codes); a reducer
-//     warp adds the chunk partials in a fixed order, runs the epilogue and
-//     refills the slot;
-//   * column-split kernel: the same dot, consumer groups on alternate stages;
+//   * stage kernel (default, 1-4 activation rows): one CTA per SM streams a
+//     contiguous range of 16-36 KB row stages through a bulk-copy ring; every
+//     compute warp works on every stage (a column chunk of a row group), with the
+//     integer block dot (16-bit block fixed-point x, dp4a over the raw nibble
+//     codes); a reducer warp adds the chunk partials in a fixed order, runs the
+//     epilogue and refills the slot;
 //   * warp-streamed kernel: each warp streams its own row pairs through its own
-//     ring, fp16 nibble unpacking with mixed-precision FMAs (also the fallback
-//     for more than two activation rows);
+//     ring, fp16 nibble unpacking with mixed-precision FMAs (the fallback for 5-8
+//     activation rows);
 //   * register kernel (below): plain streaming loads, any k % 32 == 0;
-//   * chain kernel: O, gate|up, down and the next QKV of a layer in one
-//     cooperative launch built like the stage kernel.
+//   * fp16 GEMV (end of the file): the fp16 tied head.
 // The fused prologues (RMSNorm, residual, layer scalar) and epilogues (store,
 // GeGLU, softcap + logits + argmax) are shared by all of them. The first weight
 // loads of every kernel are issued before griddepcontrol.wait, so with
 // programmatic dependent launch they overlap the previous kernel's tail.
 //
-// Register kernel, work decomposition (one launch, persistent over 16-row units):
+// Register kernel, work decomposition (one launch, each CTA looping over 16-row units):
 //   * a CTA (8 warps) owns a contiguous, balanced range of 16-row units;
 //   * warp w owns columns blocks [w*NB/8, (w+1)*NB/8) of every unit (NB = k/32);
 //   * a warp step covers 4 rows x 8 consecutive blocks: lane (r4 = lane/8,
@@ -944,7 +942,7 @@ Q4G_DEV void cs_issue(const GemvParams& p, int u, unsigned char* st, uint64_t* b
 // Stage kernel: every compute warp works on every stage.
 //
 // One CTA per SM streams a contiguous range of R-row stages through a ring of
-// NS shared-memory slots (same stage layout as the column-split kernel). The R
+// NS shared-memory slots ([R rows of codes][R rows of scales] per slot). The R
 // rows of a stage form G groups of RG rows and the columns NC chunks of 32
 // blocks; compute warp (c, g) takes chunk c of group g, so the NC * G warps go
 // through the ring together, in order. A warp sums its RG rows over its lanes,
