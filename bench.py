@@ -78,6 +78,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=None,
                     help="fewer layers of the same shapes (profiling captures of a small case)")
+    ap.add_argument("--kv-int8", action="store_true",
+                    help="the headline run with the int8 KV cache (kv_int8 = 1)")
     ap.add_argument("--quick", action="store_true",
                     help="the headline context only (no other contexts, no microbenchmarks)")
     return ap.parse_args()
@@ -471,6 +473,8 @@ def main():
     cfg = dict(WL.B12)
     if args.layers:
         cfg["n_layers"] = args.layers
+    if args.kv_int8:
+        cfg["kv_int8"] = 1
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -666,6 +670,7 @@ def main():
                                    f"context {C}, batch 1, greedy decode",
                        "context": C, "global_batch": world, "seq_len": C,
                        "parallelism": f"replicas{world}", "prefix": args.prefix,
+                       "kv_cache": "int8" if args.kv_int8 else "fp16",
                        "l2": "inputs larger than L2 (6.7 GB of weights read per step)"},
             "hbm": {"bytes_per_token": bytes_per_tok, "gbs_per_gpu": gbs, "peak_gbs": peak,
                     "frac": gbs / peak, "peak_kind": peak_kind},
