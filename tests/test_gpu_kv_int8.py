@@ -199,3 +199,56 @@ def test_12b_period_int8_32k_decode_and_128k_verify():
             _check(lg[i].cpu().numpy().astype(np.float64), r["logits"][i], f"128K block {b} row {i}")
         pos += int(acc[b])
     Q.q4g_model_check(g.handle, sp())
+
+
+def test_tiny_int8_verify_eight_rows_after_handoff():
+    """A verify block of K = 8 rows (32 query rows per KV head on the tensor-core
+    ring path) over a handed-off int8 history, against the oracle's two-pass protocol,
+    and the argmax output of every row."""
+    cfg = dict(WL.TINY, kv_int8=1)
+    seed, V, K = 9, cfg["vocab"], 8
+    g = S.SynthDecoder(cfg, seed=seed, variant=1)
+    om = O.Model(cfg, seed=seed, variant=1)
+    gc, oc = g.new_cache(512), O.Cache(om, 512)
+    ids = DG.uniform_int(seed, DG.STREAM_PREFIX_IDS, 280, V)
+    for pos in range(270):
+        Q.q4g_decode_step(g.handle, gc.handle, int(ids[pos]), pos, 0, 0, sp())
+    torch.cuda.synchronize()
+    _handoff_i8(gc, oc)
+    blk = DG.uniform_int(seed, DG.STREAM_DRAFT_IDS, K, V).astype(np.int32)
+    ids_d = torch.from_numpy(blk).cuda()
+    lg = torch.empty((K, V), dtype=torch.float32, device="cuda")
+    am = torch.empty(K, dtype=torch.int32, device="cuda")
+    Q.q4g_verify_block(g.handle, gc.handle, ids_d.data_ptr(), K, 270, K, lg.data_ptr(), am.data_ptr(), sp())
+    r = O.verify_block(om, oc, 270, ids=blk, accepted=0, mode=0)
+    torch.cuda.synchronize()
+    got32 = lg.cpu().numpy()
+    for i in range(K):
+        _check(got32[i].astype(np.float64), r["logits"][i], f"row {i}")
+        assert int(am[i]) == int(np.argmax(got32[i]))
+    Q.q4g_model_check(g.handle, sp())
+
+
+def test_int8_capacity_and_graph_invariance_bitwise():
+    """With int8 rows the logits do not depend on the cache capacity (512 or 1536),
+    nor on graph replay against eager launches."""
+    cfg = dict(WL.TINY, kv_int8=1)
+    V = cfg["vocab"]
+    g = S.SynthDecoder(cfg, seed=2, variant=1)
+    caches = [g.new_cache(512), g.new_cache(1536), g.new_cache(512)]
+    ids = DG.uniform_int(2, DG.STREAM_PREFIX_IDS, 300, V)
+    lg = torch.empty((3, V), dtype=torch.float32, device="cuda")
+    for pos in range(300):
+        want = pos % 50 == 49
+        for j, c in enumerate(caches):
+            eager = j == 2
+            if eager:
+                Q.q4g_model_set_option(g.handle, Q.Q4G_OPT_CUDA_GRAPH, 0)
+            Q.q4g_decode_step(g.handle, c.handle, int(ids[pos]), pos, lg[j].data_ptr() if want else 0, 0, sp())
+            if eager:
+                Q.q4g_model_set_option(g.handle, Q.Q4G_OPT_CUDA_GRAPH, 1)
+        if want:
+            torch.cuda.synchronize()
+            assert torch.equal(lg[0], lg[1]), f"capacity, pos {pos}"
+            assert torch.equal(lg[0], lg[2]), f"graph vs eager, pos {pos}"
+    Q.q4g_model_check(g.handle, sp())
