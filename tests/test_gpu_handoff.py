@@ -235,6 +235,55 @@ def test_tiny_unit_qk_gains_single_step():
     Q.q4g_model_check(g.handle, sp())
 
 
+def test_12b_period_unit_qk_gains_single_step():
+    """Unit q/k norm gains on one period of the 12B shapes (5 sliding layers of hd 256,
+    one full layer of hd 512, the 262,144-row head): a GPU-written 300-token history
+    handed to the oracle, then one step, compared with the bound max(2e-2, 2 x the
+    oracle's own spread) on the logits and every layer's residual. This is the sharp
+    softmax the 16-bit block fixed-point x of the integer dot has to survive."""
+    cfg = dict(WL.B12, n_layers=WL.B12["full_every"])
+    g = S.SynthDecoder(cfg, seed=12, variant=2)
+    gc = g.new_cache(4096)
+    pos = 300
+    ids = DG.uniform_int(12, DG.STREAM_PREFIX_IDS, pos + 1, cfg["vocab"])
+    for p in range(pos):
+        Q.q4g_decode_step(g.handle, gc.handle, int(ids[p]), p, 0, 0, sp())
+    torch.cuda.synchronize()
+    om = O.Model(cfg, seed=12, variant=2)
+    oc = O.Cache(om, 4096)
+    handoff(gc, oc)
+    tok = int(ids[pos])
+    sp_logits, sp_layers = oracle_spread(om, oc, cfg, pos, tok, trials=2)
+    print(f"oracle spread under 1e-6 input noise: logits {sp_logits:.3g}, layers {np.round(sp_layers, 4)}")
+    L, H, V = cfg["n_layers"], cfg["hidden"], cfg["vocab"]
+    dump = torch.zeros((1, L + 1, H), dtype=torch.float32, device="cuda")
+    logits = torch.empty(V, dtype=torch.float32, device="cuda")
+    am = torch.empty(1, dtype=torch.int32, device="cuda")
+    Q.q4g_model_set_option(g.handle, Q.Q4G_OPT_DUMP, dump.data_ptr())
+    Q.q4g_decode_step(g.handle, gc.handle, tok, pos, logits.data_ptr(), am.data_ptr(), sp())
+    r = O.decode_step(om, oc, pos, token=tok, want_dump=True)
+    torch.cuda.synchronize()
+    Q.q4g_model_set_option(g.handle, Q.Q4G_OPT_DUMP, 0)
+    got, ref = logits.cpu().numpy().astype(np.float64), r["logits"][0]
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    bound = max(TOL, 2 * sp_logits)
+    err = float(np.max(np.abs(got - ref))) / rms
+    print(f"GPU vs oracle: logits {err:.3g} (bound {bound:.3g})")
+    assert err <= bound
+    a_ref, a_got = int(np.argmax(ref.astype(np.float32))), int(am[0])
+    if a_ref != a_got:
+        assert float(ref[a_ref] - ref[a_got]) <= bound * rms
+    d = dump[0].cpu().numpy().astype(np.float64)
+    for l in range(L + 1):
+        ref_l = r["dump"][0, l]
+        e = float(np.max(np.abs(d[l] - ref_l)) / np.sqrt(np.mean(ref_l ** 2)))
+        assert e <= max(TOL, 2 * sp_layers[l]), f"layer {l - 1}: {e}"
+    Q.q4g_model_check(g.handle, sp())
+    gc.close()
+    g.close()
+    om.close()
+
+
 # ------------------------------------------------------- 12B-class, 48 layers ----
 
 @pytest.fixture(scope="module")
