@@ -172,10 +172,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
     return a >= (int)pos0 ? a - (int)pos0 : -1;
   };
 
-  const __half* kc = p.k_cache + (size_t)kv * p.cache_rows * HD;
-  const __half* vc = p.v_cache + (size_t)kv * p.cache_rows * HD;
-  const int8_t* kc8 = reinterpret_cast<const int8_t*>(p.k_cache) + (size_t)kv * p.cache_rows * HD;
-  const int8_t* vc8 = reinterpret_cast<const int8_t*>(p.v_cache) + (size_t)kv * p.cache_rows * HD;
   const float* ksc = KV8 ? p.k_scale + (size_t)kv * p.cache_rows : nullptr;
   const float* vsc = KV8 ? p.v_scale + (size_t)kv * p.cache_rows : nullptr;
   constexpr int CPR = HD / 8;  // 16-byte chunks per row
@@ -183,6 +179,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
 
   // mode 0: cache rows only (the block's own rows do not exist yet);
   // 1: the block's own rows only, from shared memory; 2: both
+  constexpr int kRowBytes = KV8 ? HD : HD * 2;
+  constexpr int CPRB = kRowBytes / 16;      // 16-byte pieces per row
+  constexpr int KPP = kThreads / CPRB;      // keys per pass of the CTA
+  static_assert(kThreads % CPRB == 0 && TK % KPP == 0, "whole rows per pass");
+  const int my_part = tid % CPRB, my_key = tid / CPRB;  // a thread's piece in every pass
   auto load_tile = [&](int t, bool kpart, int mode) {
     const int buf = t & 1;
     const int a0 = a_begin + t * TK;
@@ -190,53 +191,52 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
       const int a = a0 + tid;
       sm.kidx[buf][tid] = a < a_end ? key_row(a) : -1;
     }
-    if (KV8) {
-      int8_t* dst8 = reinterpret_cast<int8_t*>(kpart ? &sm.k[0][0] : &sm.v[0][0]) + kStage8;
-      const int8_t* src8 = kpart ? kc8 : vc8;
-      for (int c = tid; c < TK * CPR8; c += kThreads) {
-        const int key = c / CPR8, part = c - key * CPR8;
-        const int a = a0 + key;
-        const bool in = a < a_end;
-        const int loc = in ? key_is_local(a) : -1;
-        if (loc >= 0) {
-          if (mode != 0)
-            *reinterpret_cast<uint4*>(dst8 + (size_t)key * HD + part * 16) =
-                *reinterpret_cast<const uint4*>((kpart ? sm.kloc8[loc] : sm.vloc8[loc]) + part * 16);
-        } else if (mode != 1) {
-          const int8_t* s8 = in ? src8 + (size_t)key_row(a) * HD + part * 16 : src8;
-          cp_async16(dst8 + (size_t)key * HD + part * 16, s8, in);
-        }
+    if (KV8 && tid < TK) {  // the rows' scales
+      const int a = a0 + tid;
+      const bool in = a < a_end;
+      const int loc = in ? key_is_local(a) : -1;
+      float* sd = kpart ? &sm.ks[buf][tid] : &sm.vs[buf][tid];
+      if (loc >= 0) {
+        if (mode != 0) *sd = kpart ? sm.klocs[loc] : sm.vlocs[loc];
+      } else if (mode != 1) {
+        if (in) cp_async4(sd, (kpart ? ksc : vsc) + key_row(a));
+        else *sd = 0.f;
       }
-      if (tid < TK) {  // the rows' scales
-        const int a = a0 + tid;
-        const bool in = a < a_end;
-        const int loc = in ? key_is_local(a) : -1;
-        float* sd = kpart ? &sm.ks[buf][tid] : &sm.vs[buf][tid];
-        if (loc >= 0) {
-          if (mode != 0) *sd = kpart ? sm.klocs[loc] : sm.vlocs[loc];
-        } else if (mode != 1) {
-          if (in) cp_async4(sd, (kpart ? ksc : vsc) + key_row(a));
-          else *sd = 0.f;
-        }
+    }
+    unsigned char* dst = reinterpret_cast<unsigned char*>(kpart ? &sm.k[0][0] : &sm.v[0][0]);
+    if (KV8) dst += kStage8;
+    constexpr size_t kDstRow = KV8 ? HD : (size_t)LD * 2;  // bytes between staged rows
+    const unsigned char* src = reinterpret_cast<const unsigned char*>(kpart ? p.k_cache : p.v_cache) +
+                               (size_t)kv * p.cache_rows * kRowBytes;
+    // CTA-uniform: keys past the chunk's end, or the block's own rows, in this tile?
+    const bool tail = a0 + TK > a_end;
+    const bool own = fused && (p.ring ? a0 < p.kr : (a0 + TK > (int)pos0 && a0 < (int)pos0 + p.kr));
+    if (!tail && !own) {  // every key a cache row: no per-piece tests
+      if (mode == 1) return;
+      // kept rolled: the unrolled form issues each thread's copies as one burst,
+      // which measured 15-25% slower at 2-7 tiles per CTA (and no faster elsewhere)
+#pragma unroll 1
+      for (int i = 0; i < TK / KPP; ++i) {
+        const int key = my_key + i * KPP;
+        cp_async16(dst + key * kDstRow + my_part * 16, src + (size_t)key_row(a0 + key) * kRowBytes + my_part * 16,
+                   true);
       }
       return;
     }
-    __half(*dst)[LD] = kpart ? sm.k : sm.v;
-    const __half* src = kpart ? kc : vc;
-    for (int c = tid; c < TK * CPR; c += kThreads) {
-      const int key = c / CPR, part = c - key * CPR;
+    for (int i = 0; i < TK / KPP; ++i) {
+      const int key = my_key + i * KPP;
       const int a = a0 + key;
       const bool in = a < a_end;
       const int loc = in ? key_is_local(a) : -1;
+      unsigned char* d = dst + key * kDstRow + my_part * 16;
       if (loc >= 0) {
         if (mode != 0) {
-          const __half* l = kpart ? sm.kloc[loc] : sm.vloc[loc];
-          *reinterpret_cast<uint4*>(&dst[key][part * 8]) =
-              *reinterpret_cast<const uint4*>(l + part * 8);
+          const void* l = KV8 ? (const void*)(kpart ? sm.kloc8[loc] : sm.vloc8[loc])
+                              : (const void*)(kpart ? sm.kloc[loc] : sm.vloc[loc]);
+          *reinterpret_cast<uint4*>(d) = reinterpret_cast<const uint4*>(l)[my_part];
         }
-      } else if (mode != 1) {
-        const __half* s = in ? src + (size_t)key_row(a) * HD + part * 8 : src;
-        cp_async16(&dst[key][part * 8], s, in);
+      } else if (mode != 1) {  // a cache row, or zeros for no key
+        cp_async16(d, in ? src + (size_t)key_row(a) * kRowBytes + my_part * 16 : src, in);
       }
     }
   };
@@ -373,19 +373,26 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
     if (KV8) convert_tile8<HD>(sm.k, reinterpret_cast<const int8_t*>(&sm.k[0][0]) + kStage8, tid);
 
     // scores S[row][key] for key n-tile `warp`
+    // (even and odd k steps accumulate separately: two independent mma chains)
     float s[2][4];
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt) {
+      float s1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 4; ++c) s[mt][c] = 0.f;
       if (mt < mtiles) {
 #pragma unroll 4
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          uint32_t a[4], b[2];
-          ldsm_x4(a, &sm.q[mt * 16 + (lane & 15)][kk * 16 + (lane >> 4) * 8]);
-          ldsm_x2(b, &sm.k[warp * 8 + (lane & 7)][kk * 16 + ((lane >> 3) & 1) * 8]);
-          mma16816(s[mt], a, b);
+        for (int kk = 0; kk < HD / 16; kk += 2) {
+          uint32_t a0[4], b0[2], a1[4], b1[2];
+          ldsm_x4(a0, &sm.q[mt * 16 + (lane & 15)][kk * 16 + (lane >> 4) * 8]);
+          ldsm_x2(b0, &sm.k[warp * 8 + (lane & 7)][kk * 16 + ((lane >> 3) & 1) * 8]);
+          ldsm_x4(a1, &sm.q[mt * 16 + (lane & 15)][(kk + 1) * 16 + (lane >> 4) * 8]);
+          ldsm_x2(b1, &sm.k[warp * 8 + (lane & 7)][(kk + 1) * 16 + ((lane >> 3) & 1) * 8]);
+          mma16816(s[mt], a0, b0);
+          mma16816(s1, a1, b1);
         }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) s[mt][c] += s1[c];
       }
     }
     __syncthreads();  // K tile consumed
@@ -394,9 +401,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
     }
     cp_async_commit();
 
-    // mask and per-tile row maxima
+    // mask and per-tile row maxima (rows of unused m-tiles are never read)
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt) {
+      if (mt >= mtiles) break;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         const int lr = mt * 16 + g4 + hh * 8;  // local query row
@@ -444,6 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
     // probabilities (fp16 hi + lo) and per-tile row sums
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt) {
+      if (mt >= mtiles) break;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         const int lr = mt * 16 + g4 + hh * 8;
@@ -515,7 +524,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
     // ---- merge the CL chunk partials of this KV head through DSMEM ----
     __syncthreads();  // every warp is done with the K tile, reused below
     float* pacc = reinterpret_cast<float*>(&sm.k[0][0]);  // [nrows][HD] unnormalised partial
-    for (int mt = 0; mt < mtiles; ++mt) {
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {  // constant bounds: oacc stays in registers
+      if (mt >= mtiles) break;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         const int lr = mt * 16 + g4 + hh * 8;
@@ -558,7 +569,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnParams p) {
 
   // ---- partials ----
   const int nq_rows = p.kr * p.n_q;
-  for (int mt = 0; mt < mtiles; ++mt) {
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt) {  // constant bounds: oacc stays in registers
+    if (mt >= mtiles) break;
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       const int lr = mt * 16 + g4 + hh * 8;
