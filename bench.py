@@ -413,6 +413,19 @@ def microbench(Q, S, DG, WL, peak, sp, stream):
         b = wbytes + k * 2 + n * 4
         out["gemv"].append({"shape": name, "rows": n, "cols": k, "seeds": [1, 2, 3, 4], "copies": len(mats),
                             "us": ms * 1e3, "gbs": b / (ms / 1e3) / 1e9, "frac": b / (ms / 1e3) / 1e9 / peak})
+        # the same matrices against 4 activation rows (a verify block of K = 4): weights read once
+        try:
+            x4 = torch.empty(4 * k, dtype=torch.float16, device="cuda")
+            S.fill_normal_f16(x4, seed0, DG.stream_bench_x(seed0), 1.0)
+            y4 = torch.empty(4 * n, dtype=torch.float32, device="cuda")
+            ms4 = time_rotating(lambda i: Q.q4g_gemv(mats[i][0].data_ptr(), mats[i][1].data_ptr(), n, k,
+                                                     x4.data_ptr(), 4, y4.data_ptr(), sp), len(mats), 4, stream)
+            b4 = wbytes + 4 * k * 2 + 4 * n * 4
+            out.setdefault("gemv_rows4", []).append(
+                {"shape": name, "activation_rows": 4, "us": ms4 * 1e3, "gbs": b4 / (ms4 / 1e3) / 1e9,
+                 "frac": b4 / (ms4 / 1e3) / 1e9 / peak, "vs_rows1": ms / ms4})
+        except Exception as e:  # a microbenchmark never costs the bench line
+            out.setdefault("gemv_rows4", []).append({"shape": name, "error": str(e)[:200]})
         del mats
         torch.cuda.empty_cache()
     # flash-decode alone: 16 query heads over an hd 256 ring (8 KV heads, W 1024, R 2048, full window)
