@@ -148,7 +148,12 @@ int8_t* or_cache_global_i8(or_cache* c, int gl_index, int kv, float** scales);
  * and after every layer; kv_dump (may be NULL): per layer [K][2][hdmax] the
  * fp16 K and V rows of KV head 0 (hdmax = larger head dim, hd entries used);
  * vraw_dump (may be NULL): per layer [K][hdmax] the raw k_proj output of KV
- * head 0 (double). Returns 0 or -1. */
+ * head 0 (double). Returns 0 or -1.
+ * Parity unpinned as a whole: the pages print no worked example, expected logits
+ * or per-layer values for a decode step, so this composition is pinned only
+ * through its parts (q4_0 pack and unpack, GEMV, RMSNorm, RoPE, ring indexing,
+ * attention, GeGLU, softcap: each against a closed form, a library routine or
+ * brute force) and through a recomposition of those parts from torch primitives. */
 int or_verify_block(or_model* m, or_cache* c, const int32_t* ids, const float* hidden_in, int K,
                     int64_t pos0, int accepted, int mode, double* logits, int32_t* argmax,
                     double* dump, uint16_t* kv_dump, double* vraw_dump);
