@@ -22,6 +22,9 @@ BUILD_DIR = os.path.join(ROOT, "_build")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-Xptxas", "-warn-spills"]
+# the library's objects are compiled with ptxas's resource report, kept per source file
+# beside the object (registers, stack frame, spills of every kernel: kernel_resources())
+RES_FLAGS = ["-Xptxas", "-v"]
 
 
 def _nvcc() -> str:
@@ -56,10 +59,17 @@ def build(force: bool = False, verbose: bool = False) -> str:
     for s in srcs:
         o = os.path.join(BUILD_DIR, os.path.basename(s) + ".o")
         objs.append(o)
-        if force or _stale(o, [s] + headers):
-            jobs.append([nvcc, *ARCH, *FLAGS, "-c", s, "-o", o])
+        if force or _stale(o, [s] + headers) or not os.path.exists(o + ".resources.txt"):
+            jobs.append((o, [nvcc, *ARCH, *FLAGS, *RES_FLAGS, "-c", s, "-o", o]))
+
+    def compile_one(job):
+        o, cmd = job
+        log = _run(cmd, verbose)
+        with open(o + ".resources.txt", "w") as f:
+            f.write(log)
+
     with ThreadPoolExecutor(max_workers=min(8, len(jobs) or 1)) as ex:
-        list(ex.map(lambda c: _run(c, verbose), jobs))
+        list(ex.map(compile_one, jobs))
     if force or jobs or _stale(LIB, objs):
         _run([nvcc, *ARCH, "-shared", "-cudart", "static", "-o", LIB + ".tmp", *objs], verbose)
         os.replace(LIB + ".tmp", LIB)
@@ -68,6 +78,38 @@ def build(force: bool = False, verbose: bool = False) -> str:
         _run([nvcc, *ARCH, *FLAGS, "-shared", "-cudart", "static", "-o", DG_LIB + ".tmp", DG_SRC], verbose)
         os.replace(DG_LIB + ".tmp", DG_LIB)
     return LIB
+
+
+def kernel_resources() -> dict:
+    """Per kernel of libq4g.so, from the ptxas reports of the last build: demangled
+    name -> {"registers", "stack", "spill_stores", "spill_loads"} (bytes, per thread)."""
+    import re
+    text = ""
+    for f in sorted(glob.glob(os.path.join(BUILD_DIR, "*.o.resources.txt"))):
+        with open(f) as fh:
+            text += fh.read()
+    out, cur = {}, None
+    for line in text.splitlines():
+        m = re.search(r"Function properties for (\S+)", line)
+        if m:
+            cur = m.group(1)
+            out[cur] = {}
+            continue
+        m = re.search(r"(\d+) bytes stack frame, (\d+) bytes spill stores, (\d+) bytes spill loads", line)
+        if m and cur is not None:
+            out[cur].update(stack=int(m.group(1)), spill_stores=int(m.group(2)), spill_loads=int(m.group(3)))
+            continue
+        m = re.search(r"Used (\d+) registers", line)
+        if m and cur is not None:
+            out[cur]["registers"] = int(m.group(1))
+            cur = None
+    names = list(out)
+    try:  # demangle in one call
+        r = subprocess.run(["c++filt"], input="\n".join(names), capture_output=True, text=True, check=True)
+        pretty = r.stdout.splitlines()
+    except (OSError, subprocess.CalledProcessError):
+        pretty = names
+    return {p: out[n] for n, p in zip(names, pretty) if len(pretty) == len(names)} or out
 
 
 if __name__ == "__main__":
